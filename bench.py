@@ -1,0 +1,419 @@
+#!/usr/bin/env python
+"""Benchmark of the Infini-attention forward on B200: tokens/s and roofline fraction.
+
+One step = one full forward (every segment's local attention, memory retrieval, gate and
+memory update) over one batch of the workload's synthetic inputs, through the C ABI.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Prints ONE JSON line on rank 0.  Under torchrun (N > 1) every rank runs its own batch of
+the workload on its own GPU (independent problems: no data-path collective, weak
+scaling); step time is the max over ranks.
+
+Timing: W untimed warm-up steps, then K steps each bracketed by CUDA events on the launch
+stream, with a 256 MiB write (larger than the 126 MB L2) before every step, outside the
+events, so each step starts with a cold L2.  The library's launch trace (CUDA events
+around each of its kernels, on the same stream) gives the dominant kernel's device time
+for the roofline and the launch count.  ``--impl reference`` times the fp64 CPU oracle
+instead, on bounded samples of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from compressive_memory_long_b200 import workloads as wl  # noqa: E402
+
+METRIC = "Infini-attention fwd tokens/s at 1 B200; % of bf16 TC peak or HBM roofline"
+DEFAULT_WORKLOAD = "hf_repro_n64"
+FLUSH_BYTES = 256 << 20
+
+# Measured roofline denominators of this GPU pool (measured copy bandwidth and
+# cuBLAS bf16 GEMM); used when the measured-peaks file is absent.
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from an ncu
+# capture, keyed by (workload, kernel).  Absent: no capture of the current kernel.
+NCU_TRAFFIC_BYTES: dict = {}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        p = json.load(open(path))
+        return p, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---- algorithmic work per kernel (flops and bytes; snapshots and re-reads excluded) ----
+
+def algorithmic(w: wl.Workload, kernel: str):
+    """(flops, bytes) one launch of ``kernel`` does on workload ``w``.
+
+    segment kernel: local causal attention 2 d N (N + 1) + retrieval 2 N d^2 flops per
+    (b, h, segment); bytes = q, k, v read once and out written once.
+    state kernels: update 2 N d^2 (linear) or 4 N d^2 (delta) flops per (b, kv head,
+    segment); bytes = k, v read once plus M/z read and written once.
+    """
+    e = w.elem_bytes
+    B, H, Hkv, L, N, d, S = w.B, w.H, w.Hkv, w.L, w.N, w.d, w.S
+    state_bytes = 2 * B * Hkv * (d * d + d) * 4
+    if kernel.startswith("segment"):
+        flops = B * H * S * (2 * d * N * (N + 1) + 2 * N * d * d)
+        byts = (2 * H + 2 * Hkv) * B * L * d * e
+    elif kernel in ("linear_increments", "delta_chain", "linear_fused", "delta_fused"):
+        per = 2 if w.rule == "linear" else 4
+        flops = B * Hkv * S * per * N * d * d
+        byts = 2 * B * Hkv * L * d * e + state_bytes
+    else:   # scan / init: pure state traffic
+        flops = 0
+        byts = state_bytes
+    return flops, byts
+
+
+# ---- clocks during the timed region (NVML) ----
+
+class ClockSampler:
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._period = period_s
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            uuid = torch.cuda.get_device_properties(device_index).uuid
+            self._h = None
+            for i in range(pynvml.nvmlDeviceGetCount()):
+                h = pynvml.nvmlDeviceGetHandleByIndex(i)
+                u = pynvml.nvmlDeviceGetUUID(h)
+                u = u.decode() if isinstance(u, bytes) else u
+                if u.replace("GPU-", "") == str(uuid).replace("GPU-", ""):
+                    self._h = h
+            if self._h is None:
+                self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception as ex:   # NVML missing: report no clocks rather than fail the run
+            self._nv = None
+            self.error = repr(ex)
+
+    def _sample(self):
+        nv = self._nv
+        self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+        mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+        for bit, name in self.REASONS.items():
+            if mask & bit:
+                self.reasons.add(name)
+
+    def _run(self):
+        while not self._stop.is_set():
+            self._sample()
+            time.sleep(self._period)
+
+    def __enter__(self):
+        if self._nv is not None:
+            self._sample()
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self._nv is not None:
+            self._stop.set()
+            self._t.join()
+            self._sample()
+
+    def summary(self):
+        if self._nv is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+
+
+# ---- distributed plumbing ----
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ---- CPU oracle samples (the baseline leg and the reference arm) ----
+
+def oracle_sample(w: wl.Workload, seconds: float):
+    """Time the fp64 oracle on a bounded sample of ``w``.
+
+    Small workloads: the whole workload, repeated until about ``seconds`` have passed.
+    Large ones: chain (b=0, kv head 0) with its G query heads over the first n segments,
+    n sized to about ``seconds`` of work (one query head of H covers 1/H of a token).
+    Returns (token-equivalents per second, seconds timed, description).
+    """
+    import oracle
+    st = wl.has_initial_state(w)
+
+    if w.B * w.H * w.L * w.d <= (1 << 22):
+        q, k, v, beta, M0, z0 = wl.host_inputs(w)
+        reps, dt = 0, 0.0
+        while reps == 0 or dt < seconds:
+            t0 = time.perf_counter()
+            oracle.infini_attn_fwd(q, k, v, beta, M0 if st else None, z0 if st else None,
+                                   N=w.N, rule=w.rule)
+            dt += time.perf_counter() - t0
+            reps += 1
+        return w.B * w.L * reps / dt, dt, f"whole workload x {reps}"
+
+    def run(n_seg):
+        rows = n_seg * w.N
+        q, k, v, beta, M0, z0 = wl.host_slices(w, 0, 0, rows=rows)
+        t0 = time.perf_counter()
+        oracle.infini_attn_fwd(q, k, v, beta, M0 if st else None, z0 if st else None, N=w.N,
+                               rule=w.rule)
+        return rows * w.G / w.H, time.perf_counter() - t0
+
+    n = 1
+    tok, dt = run(n)
+    if dt < 0.5 * seconds and w.S > 1:
+        n = int(min(w.S, max(2, round(seconds / max(dt, 1e-6)))))
+        tok, dt = run(n)
+    desc = (f"chain (b=0, kv head 0) with its {w.G} query head(s) of {w.H}, first {n} of "
+            f"{w.S} segments ({n * w.N} tokens)")
+    return tok / dt, dt, desc
+
+
+def run_reference(args, w: wl.Workload):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    per_step = min(20.0, max(2.0, 150.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_sample(w, per_step)
+    vals, secs = [], 0.0
+    desc = ""
+    for _ in range(args.steps):
+        v, dt, desc = oracle_sample(w, per_step)
+        vals.append(v)
+        secs += dt
+    value = float(statistics.mean(vals))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000.0 * secs / max(1, args.steps), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_of(w),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_of(w: wl.Workload):
+    return {"workload": w.name, "B": w.B, "H": w.H, "Hkv": w.Hkv, "d": w.d, "N": w.N,
+            "S": w.S, "L": w.L, "rule": w.rule, "activations": w.dtype,
+            "l2": "256 MiB write before every step (L2 flushed)",
+            "description": w.description}
+
+
+# ---- our arm ----
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(wl.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="CPU-oracle sample size for cpu_baseline (0 disables)")
+    args = ap.parse_args()
+    w = wl.WORKLOADS[args.workload]
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    if args.impl == "reference":
+        return run_reference(args, w)
+
+    world, rank, local = dist_env()
+    if world != args.gpus:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    from compressive_memory_long_b200 import binding
+
+    host = wl.torch_inputs(w, pin_memory=True)
+    t = {k: (None if x is None else x.to(dev, non_blocking=True)) for k, x in host.items()}
+    out = torch.empty_like(t["q"])
+    M_out = torch.empty((w.B, w.Hkv, w.d, w.d), dtype=torch.float32, device=dev)
+    z_out = torch.empty((w.B, w.Hkv, w.d), dtype=torch.float32, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    fwd = binding.infini_attn_fwd if w.dtype == "bf16" else binding.infini_attn_fwd_f32
+
+    def step():
+        fwd(t["q"], t["k"], t["v"], t["beta"], t["M0"], t["z0"], out, M_out, z_out, w.N,
+            w.rule, stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+
+    # ---- timed region (device time; trace on for per-kernel events) ----
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    binding.infini_attn_trace_report()     # drop anything recorded before
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    binding.infini_attn_trace_enable(True)
+    with ClockSampler(local) as clocks:
+        for i in range(args.steps):
+            flush.zero_()
+            starts[i].record(stream)
+            step()
+            ends[i].record(stream)
+        torch.cuda.synchronize(dev)
+    binding.infini_attn_trace_enable(False)
+    barrier(world)
+    trace = binding.infini_attn_trace_report()
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = max_over_ranks(float(sum(step_ms)), world, dev)
+    launches = int(sum_over_ranks(float(sum(v["launches"] for k, v in trace.items()
+                                            if isinstance(v, dict))), world, dev))
+    tokens = w.tokens * args.steps * world
+    value = tokens / (total_ms / 1000.0)
+
+    # ---- dominant kernel roofline ----
+    peaks, peak_src = load_peaks()
+    kernels = {k: v for k, v in trace.items() if isinstance(v, dict)}
+    dom = max(kernels, key=lambda k: kernels[k]["ms"])
+    dom_ms = kernels[dom]["ms"] / kernels[dom]["launches"]
+    dom_ms = max_over_ranks(dom_ms, world, dev)
+    flops, byts = algorithmic(w, dom)
+    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    if flops > 0 and flops / byts > ridge:
+        achieved = flops / (dom_ms / 1e3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"]}
+    else:
+        achieved = byts / (dom_ms / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"]}
+    roof["traffic"] = NCU_TRAFFIC_BYTES.get((w.name, dom))
+    roof.update({"kernel": dom, "kernel_ms": dom_ms, "peak_source": f"{peak_src} (burst)",
+                 "algorithmic_flops": flops, "algorithmic_bytes": byts,
+                 "kernel_share": kernels[dom]["ms"] / sum(v["ms"] for v in kernels.values())})
+
+    # ---- end to end through the public call with host buffers ----
+    out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    M_h = torch.empty(M_out.shape, dtype=torch.float32, pin_memory=True)
+    z_h = torch.empty(z_out.shape, dtype=torch.float32, pin_memory=True)
+    h2d = sum(x.numel() * x.element_size() for x in host.values() if x is not None)
+    d2h = sum(x.numel() * x.element_size() for x in (out_h, M_h, z_h))
+    e_starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    e_ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+
+    def e2e_step(i=None):
+        if i is not None:
+            e_starts[i].record(stream)
+        for kname, x in host.items():
+            if x is not None:
+                t[kname].copy_(x, non_blocking=True)
+        step()
+        out_h.copy_(out, non_blocking=True)
+        M_h.copy_(M_out, non_blocking=True)
+        z_h.copy_(z_out, non_blocking=True)
+        if i is not None:
+            e_ends[i].record(stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        e2e_step()
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    for i in range(args.steps):
+        flush.zero_()
+        e2e_step(i)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    e2e_ms = max_over_ranks(float(sum(s.elapsed_time(e) for s, e in zip(e_starts, e_ends))),
+                            world, dev)
+
+    # ---- CPU oracle baseline (rank 0, single GPU only) ----
+    cpu = None
+    if rank == 0 and world == 1 and args.cpu_seconds > 0:
+        v, dt, desc = oracle_sample(w, args.cpu_seconds)
+        cpu = {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+               "sample": desc + f"; {dt:.1f} s on 1 host core (fp64, single-threaded C)"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
+            "data": "synthetic", "config": config_of(w),
+            "roofline": roof, "cpu_baseline": cpu,
+            "e2e": {"value": w.tokens * args.steps * world / (e2e_ms / 1000.0),
+                    "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches, "kernels": kernels,
+            "clocks": clocks.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,155 @@
+"""Thin ctypes binding of ``libinfini_attn.so`` (argument marshalling only).
+
+Every step of the forward runs in the CUDA library; torch supplies device memory and the
+current stream, nothing else.  There is no CPU fallback: if the library is missing or
+fails to load, importing this module raises.
+
+Names mirror the C ABI in ``include/infini_attn.h``:
+``infini_attn_fwd`` (bf16), ``infini_attn_fwd_f32``, ``infini_attn_workspace_bytes``,
+``infini_attn_status_string``, ``infini_attn_version``; ``forward`` allocates the outputs
+and picks the entry point from q's dtype.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+from . import build as _build
+
+LINEAR = 0
+DELTA = 1
+RULES = {"linear": LINEAR, "delta": DELTA, LINEAR: LINEAR, DELTA: DELTA}
+
+STATUS = {0: "INFINI_OK", 1: "INFINI_ERR_INVALID_ARG", 2: "INFINI_ERR_UNSUPPORTED",
+          3: "INFINI_ERR_CUDA", 4: "INFINI_ERR_OOM", 5: "INFINI_ERR_TIMEOUT"}
+
+#: C functions and their (argtypes, restype), exactly as include/infini_attn.h declares them
+_P, _I64, _I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+_FWD_ARGS = [_P] * 9 + [_I64] * 6 + [_I, _P]
+SIGNATURES = {
+    "infini_attn_fwd": (_FWD_ARGS, _I),
+    "infini_attn_fwd_f32": (_FWD_ARGS, _I),
+    "infini_attn_workspace_bytes": ([_I64] * 5, _I64),
+    "infini_attn_status_string": ([_I], ctypes.c_char_p),
+    "infini_attn_version": ([], _I),
+    "infini_attn_trace_enable": ([_I], _I),
+    "infini_attn_trace_report": ([ctypes.c_char_p, _I64], _I64),
+}
+
+
+class InfiniError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{STATUS.get(status, status)}: {msg}")
+        self.status = status
+
+
+def _load():
+    path = _build.LIB
+    if not os.path.exists(path) and os.environ.get("INFINI_NO_AUTOBUILD") != "1":
+        _build.build()
+    lib = ctypes.CDLL(path)
+    for name, (args, res) in SIGNATURES.items():
+        f = getattr(lib, name)
+        f.argtypes = args
+        f.restype = res
+    return lib
+
+
+LIB = _load()
+
+
+def infini_attn_status_string(status: int) -> str:
+    return LIB.infini_attn_status_string(status).decode()
+
+
+def infini_attn_version() -> int:
+    return LIB.infini_attn_version()
+
+
+def infini_attn_workspace_bytes(B, Hkv, L, N, d) -> int:
+    return LIB.infini_attn_workspace_bytes(B, Hkv, L, N, d)
+
+
+def infini_attn_trace_enable(on: bool) -> bool:
+    return bool(LIB.infini_attn_trace_enable(1 if on else 0))
+
+
+def infini_attn_trace_report() -> dict:
+    """Per-kernel launches and total device milliseconds since the last report."""
+    import json
+    n = LIB.infini_attn_trace_report(None, 0)
+    buf = ctypes.create_string_buffer(int(n) + 64)
+    LIB.infini_attn_trace_report(buf, len(buf))
+    return json.loads(buf.value.decode())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _call(fn, q, k, v, beta, M0, z0, out, M_out, z_out, N, rule, stream):
+    B, H, L, d = q.shape
+    Hkv = k.shape[1]
+    rc = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(M0), _ptr(z0), _ptr(out), _ptr(M_out),
+            _ptr(z_out), B, H, Hkv, L, int(N), d, RULES[rule], _stream_handle(stream))
+    if rc != 0:
+        raise InfiniError(rc, infini_attn_status_string(rc))
+
+
+def infini_attn_fwd(q, k, v, beta, M0, z0, out, M_out, z_out, N, rule, stream=None):
+    """bf16 entry point; all tensors preallocated, contiguous, on one CUDA device."""
+    _call(LIB.infini_attn_fwd, q, k, v, beta, M0, z0, out, M_out, z_out, N, rule, stream)
+
+
+def infini_attn_fwd_f32(q, k, v, beta, M0, z0, out, M_out, z_out, N, rule, stream=None):
+    """fp32 entry point; all tensors preallocated, contiguous, on one CUDA device."""
+    _call(LIB.infini_attn_fwd_f32, q, k, v, beta, M0, z0, out, M_out, z_out, N, rule, stream)
+
+
+def _check(t, name, dtype, shape, device):
+    if t is None:
+        return
+    if not isinstance(t, torch.Tensor) or t.device != device or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor on {device}")
+    if t.dtype != dtype or tuple(t.shape) != tuple(shape) or not t.is_contiguous():
+        raise ValueError(f"{name}: expected contiguous {dtype} {tuple(shape)}, got "
+                         f"{t.dtype} {tuple(t.shape)}")
+
+
+def forward(q, k, v, beta, M0=None, z0=None, *, N: int, rule="linear", out=None,
+            M_out=None, z_out=None, stream=None):
+    """Allocate outputs (unless given) and run the forward on q's device and dtype.
+
+    q [B,H,L,d], k/v [B,Hkv,L,d] (bf16 or fp32), beta [H] fp32, M0 [B,Hkv,d,d] / z0
+    [B,Hkv,d] fp32 or None.  Returns (out, M_out, z_out).
+    """
+    B, H, L, d = q.shape
+    Hkv = k.shape[1]
+    dev = q.device
+    _check(q, "q", q.dtype, (B, H, L, d), dev)
+    _check(k, "k", q.dtype, (B, Hkv, L, d), dev)
+    _check(v, "v", q.dtype, (B, Hkv, L, d), dev)
+    _check(beta, "beta", torch.float32, (H,), dev)
+    _check(M0, "M0", torch.float32, (B, Hkv, d, d), dev)
+    _check(z0, "z0", torch.float32, (B, Hkv, d), dev)
+    if out is None:
+        out = torch.empty_like(q)
+    if M_out is None:
+        M_out = torch.empty((B, Hkv, d, d), dtype=torch.float32, device=dev)
+    if z_out is None:
+        z_out = torch.empty((B, Hkv, d), dtype=torch.float32, device=dev)
+    if q.dtype == torch.bfloat16:
+        infini_attn_fwd(q, k, v, beta, M0, z0, out, M_out, z_out, N, rule, stream)
+    elif q.dtype == torch.float32:
+        infini_attn_fwd_f32(q, k, v, beta, M0, z0, out, M_out, z_out, N, rule, stream)
+    else:
+        raise ValueError(f"unsupported activation dtype {q.dtype}")
+    return out, M_out, z_out

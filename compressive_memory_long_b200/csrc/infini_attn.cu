@@ -1,0 +1,300 @@
+// Host side of the C ABI declared in include/infini_attn.h: argument checks, workspace,
+// kernel selection and launches.  No torch types cross this boundary.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <stdio.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <atomic>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "infini_attn.h"
+#include "simt_kernels.cuh"
+
+namespace infini {
+namespace {
+
+struct Problem {
+    int64_t B, H, Hkv, L, N, d, S;
+    int rule;
+};
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// [a, a+na) and [b, b+nb) overlap without being the same range
+bool partial_overlap(const void *a, int64_t na, const void *b, int64_t nb)
+{
+    if (!a || !b) return false;
+    const uintptr_t a0 = (uintptr_t)a, a1 = a0 + (uintptr_t)na;
+    const uintptr_t b0 = (uintptr_t)b, b1 = b0 + (uintptr_t)nb;
+    if (a0 == b0 && na == nb) return false;
+    return a0 < b1 && b0 < a1;
+}
+
+bool ranges_overlap(const void *a, int64_t na, const void *b, int64_t nb)
+{
+    if (!a || !b) return false;
+    const uintptr_t a0 = (uintptr_t)a, a1 = a0 + (uintptr_t)na;
+    const uintptr_t b0 = (uintptr_t)b, b1 = b0 + (uintptr_t)nb;
+    return a0 < b1 && b0 < a1;
+}
+
+int check_args(const void *q, const void *k, const void *v, const float *beta, const float *M0,
+               const float *z0, const void *out, const float *M_out, const float *z_out,
+               int64_t B, int64_t H, int64_t Hkv, int64_t L, int64_t N, int64_t d, int rule,
+               int64_t esize, Problem *pb)
+{
+    if (!q || !k || !v || !beta || !out || !M_out || !z_out) return INFINI_ERR_INVALID_ARG;
+    if (B <= 0 || H <= 0 || Hkv <= 0 || L <= 0 || N <= 0 || d <= 0) return INFINI_ERR_INVALID_ARG;
+    if (H % Hkv != 0 || L % N != 0) return INFINI_ERR_INVALID_ARG;
+    if (rule != INFINI_UPDATE_LINEAR && rule != INFINI_UPDATE_DELTA) return INFINI_ERR_INVALID_ARG;
+    // keep every element count far inside int64 and every grid inside 2^31 CTAs
+    if (B > (1 << 20) || H > (1 << 16) || L > ((int64_t)1 << 34) ||
+        B * H * L > ((int64_t)1 << 40))
+        return INFINI_ERR_INVALID_ARG;
+    const void *ptrs[] = {q, k, v, beta, M0, z0, out, M_out, z_out};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return INFINI_ERR_INVALID_ARG;
+    const int64_t mbytes = B * Hkv * d * d * 4, zbytes = B * Hkv * d * 4;
+    if (partial_overlap(M0, mbytes, M_out, mbytes) || partial_overlap(z0, zbytes, z_out, zbytes))
+        return INFINI_ERR_INVALID_ARG;
+    const int64_t obytes = B * H * L * d * esize, kvbytes = B * Hkv * L * d * esize;
+    if (ranges_overlap(out, obytes, q, obytes) || ranges_overlap(out, obytes, k, kvbytes) ||
+        ranges_overlap(out, obytes, v, kvbytes) || ranges_overlap(out, obytes, M_out, mbytes) ||
+        ranges_overlap(out, obytes, z_out, zbytes) || ranges_overlap(M_out, mbytes, z_out, zbytes))
+        return INFINI_ERR_INVALID_ARG;
+    if (d != 32 && d != 64 && d != 128) return INFINI_ERR_UNSUPPORTED;
+    if (N % 64 != 0) return INFINI_ERR_UNSUPPORTED;
+    pb->B = B; pb->H = H; pb->Hkv = Hkv; pb->L = L; pb->N = N; pb->d = d; pb->S = L / N;
+    pb->rule = rule;
+    return INFINI_OK;
+}
+
+// Raise a kernel's dynamic shared-memory limit once per (kernel, device).  Setting the
+// same value twice is harmless, so racing first calls need no lock.
+template <auto Kernel>
+bool opt_in_smem(size_t bytes)
+{
+    static std::atomic<uint64_t> done_mask{0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    const uint64_t bit = 1ull << (dev & 63);
+    if (done_mask.load(std::memory_order_relaxed) & bit) return true;
+    if (cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) !=
+        cudaSuccess)
+        return false;
+    done_mask.fetch_or(bit);
+    return true;
+}
+
+// ---- opt-in launch tracing: a pair of CUDA events on the launch stream around every
+// kernel this library enqueues, read back (and cleared) by infini_attn_trace_report ----
+namespace trace {
+struct Rec {
+    const char *name;
+    cudaEvent_t a, b;
+};
+std::mutex mu;
+std::vector<Rec> recs;
+std::atomic<int> enabled{0};
+
+struct Scope {
+    Rec r{};
+    bool on;
+    cudaStream_t st;
+    Scope(const char *name, cudaStream_t s) : on(enabled.load() != 0), st(s)
+    {
+        if (!on) return;
+        r.name = name;
+        if (cudaEventCreate(&r.a) != cudaSuccess || cudaEventCreate(&r.b) != cudaSuccess) {
+            on = false;
+            return;
+        }
+        cudaEventRecord(r.a, st);
+    }
+    ~Scope()
+    {
+        if (!on) return;
+        cudaEventRecord(r.b, st);
+        std::lock_guard<std::mutex> g(mu);
+        recs.push_back(r);
+    }
+};
+}  // namespace trace
+
+#define TRACED(name, st) trace::Scope trace_scope_##__LINE__(name, st)
+
+template <typename T, int D>
+int launch_all(const Problem &p, const T *q, const T *k, const T *v, const float *beta,
+               const float *M0, const float *z0, T *out, float *M_out, float *z_out,
+               float *snapM, float *snapZ, cudaStream_t st)
+{
+    const int64_t chains = p.B * p.Hkv;
+    const int S = (int)p.S, N = (int)p.N;
+    const int64_t per = (int64_t)D * D + D;
+    const unsigned state_grid = (unsigned)((chains * per + 255) / 256);
+    if (p.rule == INFINI_UPDATE_LINEAR) {
+        {
+            TRACED("linear_increments", st);
+            k_linear_increments<T, D><<<(unsigned)(chains * S), 256, 0, st>>>(k, v, snapM, snapZ,
+                                                                             p.L, N, S);
+        }
+        {
+            TRACED("linear_scan", st);
+            k_linear_scan<<<state_grid, 256, 0, st>>>(snapM, snapZ, M0, z0, M_out, z_out, S, D,
+                                                      chains);
+        }
+    } else {
+        constexpr int CB = 16;
+        {
+            TRACED("state_init", st);
+            k_state_init<<<state_grid, 256, 0, st>>>(M0, z0, snapM, snapZ, S, D, chains);
+        }
+        {
+            TRACED("delta_chain", st);
+            k_delta_chain<T, D, CB><<<(unsigned)(chains * (D / CB)), 256, 0, st>>>(
+                k, v, snapM, snapZ, M_out, z_out, p.L, N, S);
+        }
+    }
+    const size_t smem = SimtSegSmem<D>::bytes;
+    if (!opt_in_smem<k_segment_simt<T, D>>(smem)) return INFINI_ERR_CUDA;
+    const int64_t ctas = p.B * p.H * p.S * (p.N / 64);
+    {
+        TRACED("segment_simt", st);
+        k_segment_simt<T, D><<<(unsigned)ctas, 256, smem, st>>>(q, k, v, beta, snapM, snapZ, out,
+                                                               p.L, N, S, (int)p.H, (int)p.Hkv);
+    }
+    return cudaGetLastError() == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
+}
+
+template <typename T>
+int forward(const void *q, const void *k, const void *v, const float *beta, const float *M0,
+            const float *z0, void *out, float *M_out, float *z_out, int64_t B, int64_t H,
+            int64_t Hkv, int64_t L, int64_t N, int64_t d, int rule, infini_stream_t stream)
+{
+    Problem p;
+    int rc = check_args(q, k, v, beta, M0, z0, out, M_out, z_out, B, H, Hkv, L, N, d, rule,
+                        (int64_t)sizeof(T), &p);
+    if (rc != INFINI_OK) return rc;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaGetLastError();   // clear a stale error left by someone else's launch
+
+    const int64_t nM = p.B * p.Hkv * p.S * p.d * p.d, nZ = p.B * p.Hkv * p.S * p.d;
+    void *ws = nullptr;
+    if (cudaMallocAsync(&ws, (size_t)(nM + nZ) * sizeof(float), st) != cudaSuccess) {
+        cudaGetLastError();
+        return INFINI_ERR_OOM;
+    }
+    float *snapM = static_cast<float *>(ws), *snapZ = snapM + nM;
+    const T *tq = static_cast<const T *>(q), *tk = static_cast<const T *>(k),
+            *tv = static_cast<const T *>(v);
+    T *to = static_cast<T *>(out);
+    switch (p.d) {
+    case 32: rc = launch_all<T, 32>(p, tq, tk, tv, beta, M0, z0, to, M_out, z_out, snapM, snapZ, st); break;
+    case 64: rc = launch_all<T, 64>(p, tq, tk, tv, beta, M0, z0, to, M_out, z_out, snapM, snapZ, st); break;
+    default: rc = launch_all<T, 128>(p, tq, tk, tv, beta, M0, z0, to, M_out, z_out, snapM, snapZ, st); break;
+    }
+    if (cudaFreeAsync(ws, st) != cudaSuccess && rc == INFINI_OK) rc = INFINI_ERR_CUDA;
+    return rc;
+}
+
+}  // namespace
+}  // namespace infini
+
+extern "C" {
+
+int infini_attn_fwd(const void *q, const void *k, const void *v, const float *beta,
+                    const float *M0, const float *z0, void *out, float *M_out, float *z_out,
+                    int64_t B, int64_t H, int64_t Hkv, int64_t L, int64_t N, int64_t d,
+                    int update_rule, infini_stream_t stream)
+{
+    return infini::forward<__nv_bfloat16>(q, k, v, beta, M0, z0, out, M_out, z_out, B, H, Hkv,
+                                          L, N, d, update_rule, stream);
+}
+
+int infini_attn_fwd_f32(const void *q, const void *k, const void *v, const float *beta,
+                        const float *M0, const float *z0, void *out, float *M_out,
+                        float *z_out, int64_t B, int64_t H, int64_t Hkv, int64_t L, int64_t N,
+                        int64_t d, int update_rule, infini_stream_t stream)
+{
+    return infini::forward<float>(q, k, v, beta, M0, z0, out, M_out, z_out, B, H, Hkv, L, N, d,
+                                  update_rule, stream);
+}
+
+int64_t infini_attn_workspace_bytes(int64_t B, int64_t Hkv, int64_t L, int64_t N, int64_t d)
+{
+    if (B <= 0 || Hkv <= 0 || L <= 0 || N <= 0 || d <= 0 || L % N != 0) return 0;
+    return B * Hkv * (L / N) * (d * d + d) * (int64_t)sizeof(float);
+}
+
+const char *infini_attn_status_string(int status)
+{
+    switch (status) {
+    case INFINI_OK: return "ok";
+    case INFINI_ERR_INVALID_ARG: return "invalid argument";
+    case INFINI_ERR_UNSUPPORTED: return "unsupported shape (d must be 32, 64 or 128; N a multiple of 64)";
+    case INFINI_ERR_CUDA: return "CUDA error";
+    case INFINI_ERR_OOM: return "workspace allocation failed";
+    case INFINI_ERR_TIMEOUT: return "bounded device wait timed out";
+    default: return "unknown status";
+    }
+}
+
+int infini_attn_version(void) { return 100; }
+
+int infini_attn_trace_enable(int on)
+{
+    const int prev = infini::trace::enabled.exchange(on ? 1 : 0);
+    return prev;
+}
+
+int64_t infini_attn_trace_report(char *buf, int64_t len)
+{
+    using namespace infini::trace;
+    std::vector<Rec> taken;
+    {
+        std::lock_guard<std::mutex> g(mu);
+        taken.swap(recs);
+    }
+    // aggregate per kernel name, in first-seen order
+    std::vector<std::string> names;
+    std::vector<int64_t> count;
+    std::vector<double> ms;
+    bool ok = true;
+    for (const Rec &r : taken) {
+        float t = 0.f;
+        if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&t, r.a, r.b) != cudaSuccess)
+            ok = false;
+        cudaEventDestroy(r.a);
+        cudaEventDestroy(r.b);
+        size_t i = 0;
+        while (i < names.size() && names[i] != r.name) ++i;
+        if (i == names.size()) {
+            names.emplace_back(r.name);
+            count.push_back(0);
+            ms.push_back(0.0);
+        }
+        count[i] += 1;
+        ms[i] += t;
+    }
+    std::string js = "{";
+    for (size_t i = 0; i < names.size(); ++i) {
+        char item[160];
+        snprintf(item, sizeof(item), "%s\"%s\": {\"launches\": %lld, \"ms\": %.6f}", i ? ", " : "",
+                 names[i].c_str(), (long long)count[i], ms[i]);
+        js += item;
+    }
+    js += ok ? "}" : ", \"error\": true}";
+    if (buf && len > 0) {
+        const size_t n = js.size() < (size_t)(len - 1) ? js.size() : (size_t)(len - 1);
+        memcpy(buf, js.data(), n);
+        buf[n] = 0;
+    }
+    return (int64_t)js.size() + 1;
+}
+
+}  // extern "C"

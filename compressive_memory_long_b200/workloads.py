@@ -113,15 +113,19 @@ def _round(x: np.ndarray, w: Workload) -> np.ndarray:
     return t.to(torch.float32).numpy()
 
 
-def qkv_slice(w: Workload, tensor: str, b: int, head: int) -> np.ndarray:
-    """[L, d] float32 values (already rounded to the input dtype) of one head."""
+def qkv_slice(w: Workload, tensor: str, b: int, head: int, rows: Optional[int] = None) -> np.ndarray:
+    """[L, d] float32 values (already rounded to the input dtype) of one head.
+
+    ``rows``: draw only the first ``rows`` tokens (the same values as the full draw's
+    prefix: the generator fills row by row)."""
     assert tensor in ("q", "k", "v")
-    x = _rng(w, tensor, b, head).standard_normal((w.L, w.d), dtype=np.float32)
+    n_rows = w.L if rows is None else rows
+    x = _rng(w, tensor, b, head).standard_normal((n_rows, w.d), dtype=np.float32)
     x = x / np.float32(math.sqrt(w.d))
     if tensor == "k" and w.k_boost_frac > 0.0:
         n = int(round(w.L * w.k_boost_frac))
-        rows = _rng(w, "kboost", b, head).choice(w.L, size=n, replace=False)
-        x[rows] *= np.float32(w.k_boost)
+        sel = _rng(w, "kboost", b, head).choice(w.L, size=n, replace=False)
+        x[sel[sel < n_rows]] *= np.float32(w.k_boost)
     return _round(np.ascontiguousarray(x), w)
 
 
@@ -152,14 +156,15 @@ def has_initial_state(w: Workload) -> bool:
     return w.M0_dist is not None or w.z0_dist is not None
 
 
-def host_slices(w: Workload, b: int, kvh: int):
+def host_slices(w: Workload, b: int, kvh: int, rows: Optional[int] = None):
     """float32 inputs of one (batch, kv head) and its G query heads, for the oracle.
 
-    Returns q [1,G,L,d], k [1,1,L,d], v [1,1,L,d], beta [G], M0 [1,1,d,d], z0 [1,1,d].
+    Returns q [1,G,L,d], k [1,1,L,d], v [1,1,L,d], beta [G], M0 [1,1,d,d], z0 [1,1,d]
+    (L replaced by ``rows`` when given: the first ``rows`` tokens only).
     """
-    q = np.stack([qkv_slice(w, "q", b, kvh * w.G + g) for g in range(w.G)])[None]
-    k = qkv_slice(w, "k", b, kvh)[None, None]
-    v = qkv_slice(w, "v", b, kvh)[None, None]
+    q = np.stack([qkv_slice(w, "q", b, kvh * w.G + g, rows) for g in range(w.G)])[None]
+    k = qkv_slice(w, "k", b, kvh, rows)[None, None]
+    v = qkv_slice(w, "v", b, kvh, rows)[None, None]
     bt = beta(w)[kvh * w.G:(kvh + 1) * w.G]
     M0, z0 = initial_state(w, b, kvh)
     return q, k, v, bt, M0[None, None], z0[None, None]

@@ -1,0 +1,118 @@
+/*
+ * infini_attn.h -- C ABI of the B200 (sm_100a) Infini-attention forward library.
+ *
+ * What is computed (AI Wiki "Infini-Attention", "What happens inside the Infini-attention
+ * block?" and "How does the compressive memory work?"; the Hugging Face reproduction
+ * analysis, "Infini-Attention Mechanism", steps 1-6):
+ *
+ *   The length-L sequence of every (batch b, query head h) is cut into S = L / N segments of
+ *   N tokens, processed in order.  For segment s and query row q_t:
+ *     A_dot = causal softmax(q_t K_s^T / sqrt(d)) V_s     keys of segment s only, j <= t
+ *     A_mem = sigma(q_t) M_{s-1} / (sigma(q_t) . z_{s-1}) sigma(x) = ELU(x) + 1; 0 while the
+ *                                                          denominator is exactly 0
+ *     out_t = g_h A_mem + (1 - g_h) A_dot                  g_h = 1 / (1 + exp(-beta[h]))
+ *   After the segment the memory of its key/value head advances:
+ *     linear: M_s = M_{s-1} + sigma(K_s)^T V_s
+ *     delta : M_s = M_{s-1} + sigma(K_s)^T (V_s - sigma(K_s) M_{s-1} / (sigma(K_s) z_{s-1}))
+ *             (one batch update per segment; a row whose denominator is 0 predicts 0)
+ *     both  : z_s = z_{s-1} + sum_t sigma(K_{s,t})
+ *   Query head h reads key/value head h / (H / Hkv) (grouped-query attention).
+ *
+ * Layouts: row-major, contiguous, on the device:
+ *   q, out  [B, H,   L, d]        k, v  [B, Hkv, L, d]        beta [H] float
+ *   M0, M_out [B, Hkv, d, d] float (row = key feature, column = value feature)
+ *   z0, z_out [B, Hkv, d]    float
+ *
+ * Conventions shared by every entry point:
+ *   - All pointers are DEVICE pointers owned by the caller; the library keeps none of them
+ *     after the call returns.  Every pointer must be 16-byte aligned.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = the legacy default stream) and
+ *     runs asynchronously: results are valid once that stream has synchronised.
+ *   - M0 / z0 may be NULL (an empty memory: zeros).  M_out / z_out may alias M0 / z0
+ *     exactly (in-place state update); a partial overlap is INFINI_ERR_INVALID_ARG.  out
+ *     must not overlap any input.
+ *   - Preconditions not checked: z0 >= 0 elementwise (sigma > 0 then makes a zero
+ *     denominator mean an empty memory); inputs finite.
+ *   - On an argument error nothing is launched and nothing is written.  Nothing aborts,
+ *     throws or traps; every failure is an int status below.
+ *   - Scratch: the call allocates its workspace (per-segment memory snapshots,
+ *     B * Hkv * S * (d*d + d) * 4 bytes) with cudaMallocAsync on `stream` and frees it with
+ *     cudaFreeAsync on the same stream.
+ */
+#ifndef INFINI_ATTN_H
+#define INFINI_ATTN_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define INFINI_API __attribute__((visibility("default")))
+#else
+#define INFINI_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t, declared without the CUDA headers. */
+typedef struct CUstream_st *infini_stream_t;
+
+enum {
+    INFINI_UPDATE_LINEAR = 0, /* M += sigma(K)^T V                      */
+    INFINI_UPDATE_DELTA = 1   /* M += sigma(K)^T (V - sigma(K) M / den) */
+};
+
+enum {
+    INFINI_OK = 0,
+    INFINI_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size, L % N != 0, bad rule,
+                                   partial overlap of a state output with its input        */
+    INFINI_ERR_UNSUPPORTED = 2, /* valid but not built: d not in {32, 64, 128}, N % 64 != 0 */
+    INFINI_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed                      */
+    INFINI_ERR_OOM = 4,         /* the workspace allocation failed                           */
+    INFINI_ERR_TIMEOUT = 5      /* reserved: a bounded device wait gave up                   */
+};
+
+/*
+ * Infini-attention forward, bf16 activations (q, k, v, out are __nv_bfloat16; arithmetic
+ * in fp32, memory M / z in fp32, out rounded to nearest-even).
+ *
+ *   B, H, Hkv : batch, query heads, key/value heads (H % Hkv == 0)
+ *   L, N, d   : sequence length, segment length (L % N == 0), head dimension
+ *   update_rule : INFINI_UPDATE_LINEAR or INFINI_UPDATE_DELTA
+ * Returns INFINI_OK or an error status.
+ */
+INFINI_API int infini_attn_fwd(const void *q, const void *k, const void *v, const float *beta,
+                    const float *M0, const float *z0, void *out, float *M_out, float *z_out,
+                    int64_t B, int64_t H, int64_t Hkv, int64_t L, int64_t N, int64_t d,
+                    int update_rule, infini_stream_t stream);
+
+/* The same operation with fp32 activations (q, k, v, out are float); identical parameters. */
+INFINI_API int infini_attn_fwd_f32(const void *q, const void *k, const void *v, const float *beta,
+                        const float *M0, const float *z0, void *out, float *M_out,
+                        float *z_out, int64_t B, int64_t H, int64_t Hkv, int64_t L, int64_t N,
+                        int64_t d, int update_rule, infini_stream_t stream);
+
+/* Bytes of workspace one call allocates for these sizes (0 on invalid sizes). */
+INFINI_API int64_t infini_attn_workspace_bytes(int64_t B, int64_t Hkv, int64_t L, int64_t N, int64_t d);
+
+/* Static, NUL-terminated description of a status code. */
+INFINI_API const char *infini_attn_status_string(int status);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+INFINI_API int infini_attn_version(void);
+
+/*
+ * Launch tracing (off by default).  While enabled, every kernel this library enqueues is
+ * bracketed by two CUDA events recorded on the call's stream.  The report synchronises
+ * on those events, writes a JSON object {"<kernel>": {"launches": n, "ms": total}, ...}
+ * (NUL-terminated, truncated to len - 1 bytes) into buf, clears the records and returns
+ * the size the full report needs.  enable returns the previous setting.
+ */
+INFINI_API int infini_attn_trace_enable(int on);
+INFINI_API int64_t infini_attn_trace_report(char *buf, int64_t len);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* INFINI_ATTN_H */

@@ -1,0 +1,86 @@
+"""The C-ABI boundary on the host: the library loads, exports every symbol the header
+declares with the declared signature, and rejects bad arguments before any CUDA call
+(these calls pass fake device addresses that argument checking never dereferences)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from compressive_memory_long_b200 import binding, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    names = []
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            names += re.findall(r"INFINI_API\s+[\w\s\*]+?\b(infini_\w+)\s*\(", src)
+    return names
+
+
+def test_library_exports_every_declared_symbol():
+    names = declared_functions()
+    assert "infini_attn_fwd" in names and "infini_attn_fwd_f32" in names
+    lib = ctypes.CDLL(build.LIB)
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in include/ but not exported"
+        assert n in binding.SIGNATURES, f"{n} has no binding"
+
+
+def test_status_strings_and_version():
+    for s in range(6):
+        assert binding.infini_attn_status_string(s)
+    assert "unknown" in binding.infini_attn_status_string(99)
+    assert binding.infini_attn_version() >= 100
+
+
+def test_workspace_bytes():
+    assert binding.infini_attn_workspace_bytes(2, 8, 1024, 64, 64) == 2 * 8 * 16 * (64 * 64 + 64) * 4
+    assert binding.infini_attn_workspace_bytes(1, 1, 100, 64, 64) == 0
+    assert binding.infini_attn_workspace_bytes(0, 1, 64, 64, 64) == 0
+
+
+BASE = 1 << 40      # fake, 16-byte aligned, never dereferenced
+
+
+def call(entry="infini_attn_fwd", B=1, H=2, Hkv=2, L=128, N=64, d=64, rule=0, **ptr):
+    """Call an entry point with disjoint fake device ranges; override any pointer."""
+    gap = 1 << 32
+    p = {name: BASE + i * gap for i, name in enumerate(
+        ["q", "k", "v", "beta", "M0", "z0", "out", "M_out", "z_out"])}
+    p.update(ptr)
+    f = getattr(binding.LIB, entry)
+    args = [None if p[n] is None else ctypes.c_void_p(p[n]) for n in
+            ["q", "k", "v", "beta", "M0", "z0", "out", "M_out", "z_out"]]
+    return f(*args, B, H, Hkv, L, N, d, rule, None)
+
+
+INVALID, UNSUPPORTED = 1, 2
+
+
+@pytest.mark.parametrize("entry", ["infini_attn_fwd", "infini_attn_fwd_f32"])
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=None), INVALID), (dict(k=None), INVALID), (dict(v=None), INVALID),
+    (dict(beta=None), INVALID), (dict(out=None), INVALID), (dict(M_out=None), INVALID),
+    (dict(z_out=None), INVALID),
+    (dict(B=0), INVALID), (dict(H=0), INVALID), (dict(L=-64), INVALID), (dict(N=0), INVALID),
+    (dict(d=0), INVALID), (dict(H=3, Hkv=2), INVALID), (dict(L=100, N=64), INVALID),
+    (dict(rule=2), INVALID), (dict(rule=-1), INVALID),
+    (dict(q=BASE + 8), INVALID), (dict(M_out=BASE + (7 << 32) + 4), INVALID),
+    (dict(M_out=(1 << 40) + (4 << 32) + 64), INVALID),     # partial overlap with M0
+    (dict(z_out=(1 << 40) + (5 << 32) + 16), INVALID),     # partial overlap with z0
+    (dict(out=BASE), INVALID),                             # out on top of q
+    (dict(d=48), UNSUPPORTED), (dict(d=256), UNSUPPORTED), (dict(L=96, N=32), UNSUPPORTED),
+])
+def test_argument_errors(entry, kw, status):
+    assert call(entry, **kw) == status
+
+
+def test_python_binding_checks_shapes():
+    import torch
+    q = torch.zeros(1, 2, 64, 32)
+    with pytest.raises(ValueError):
+        binding.forward(q, q, q, torch.zeros(2), N=64)     # CPU tensors are refused

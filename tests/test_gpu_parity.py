@@ -1,0 +1,159 @@
+"""GPU path vs the fp64 CPU oracle, element by element, through the C ABI.
+
+Tolerances (max relative error per (batch, head) slice, max |x - r| / max |r|):
+1e-4 for fp32 activations, 2e-2 for bf16 activations with fp32 accumulation; the same
+bounds hold for out, M_out and z_out.  Full-size workloads are checked on sampled
+(batch, kv head) chains: the oracle runs each sampled chain's memory over every segment
+and computes outputs on sampled segments.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from compressive_memory_long_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"f32": 1e-4, "bf16": 2e-2}
+
+
+def rel_err(got, ref):
+    """max over leading (batch, head) slices of max|x - r| / max|r|."""
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    g = got.reshape(got.shape[0] * got.shape[1], -1)
+    r = ref.reshape(g.shape)
+    num = np.abs(g - r).max(axis=1)
+    den = np.maximum(np.abs(r).max(axis=1), 1e-30)
+    return float((num / den).max())
+
+
+def to_dev(t):
+    return {k: (None if x is None else x.cuda()) for k, x in t.items()}
+
+
+def run_gpu(w, t=None):
+    from compressive_memory_long_b200 import binding
+    t = to_dev(wl.torch_inputs(w) if t is None else t)
+    out, M, z = binding.forward(t["q"], t["k"], t["v"], t["beta"], t["M0"], t["z0"], N=w.N,
+                                rule=w.rule)
+    torch.cuda.synchronize()
+    return out, M, z
+
+
+def check_full(w):
+    out, M, z = run_gpu(w)
+    q, k, v, beta, M0, z0 = wl.host_inputs(w)
+    ro, rM, rz = oracle.infini_attn_fwd(q, k, v, beta, M0 if wl.has_initial_state(w) else None,
+                                        z0 if wl.has_initial_state(w) else None, N=w.N,
+                                        rule=w.rule)
+    errs = (rel_err(out.float().cpu(), ro), rel_err(M.cpu(), rM), rel_err(z.cpu()[:, :, None], rz[:, :, None]))
+    tol = TOL[w.dtype]
+    assert max(errs) <= tol, f"{w.name}: out/M/z rel err {errs} > {tol}"
+    return errs
+
+
+def check_sampled(w, chains, segs):
+    out, M, z = run_gpu(w)
+    out_c, M_c, z_c = out.cpu(), M.cpu(), z.cpu()
+    del out, M, z
+    torch.cuda.empty_cache()
+    tol = TOL[w.dtype]
+    for (b, kvh) in chains:
+        q, k, v, beta, M0, z0 = wl.host_slices(w, b, kvh)
+        st = wl.has_initial_state(w)
+        ro, rM, rz = oracle.infini_attn_fwd(q, k, v, beta, M0 if st else None,
+                                            z0 if st else None, N=w.N, rule=w.rule,
+                                            seg_out=segs)
+        heads = slice(kvh * w.G, (kvh + 1) * w.G)
+        for s in segs:
+            rows = slice(s * w.N, (s + 1) * w.N)
+            e = rel_err(out_c[b:b + 1, heads, rows].float(), ro[:, :, rows])
+            assert e <= tol, f"{w.name} chain {(b, kvh)} segment {s}: out rel err {e}"
+        eM = rel_err(M_c[b:b + 1, kvh:kvh + 1], rM)
+        ez = rel_err(z_c[b:b + 1, kvh:kvh + 1, None], rz[:, :, None])
+        assert max(eM, ez) <= tol, f"{w.name} chain {(b, kvh)}: M/z rel err {eM}, {ez}"
+
+
+@pytest.mark.parametrize("name", ["fp32_linear_small", "hf_repro_n64"])
+def test_small_workloads_full(name):
+    check_full(wl.WORKLOADS[name])
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("rule", ["linear", "delta"])
+@pytest.mark.parametrize("d", [32, 64, 128])
+def test_shapes_and_rules(dtype, rule, d):
+    """Several q tiles per segment, several segments, GQA, a nonzero initial state."""
+    w = wl.Workload("t", B=2, H=4, Hkv=2, d=d, N=192, S=3, dtype=dtype, rule=rule, seed=11,
+                    beta_dist=("normal", 0.0, 1.5), M0_dist=("uniform", 0.0, 0.1),
+                    z0_dist=("uniform", 1.0, 2.0))
+    check_full(w)
+
+
+@pytest.mark.parametrize("rule", ["linear", "delta"])
+def test_gqa8b_sampled(rule):
+    w = wl.WORKLOADS["gqa8b_n2048_delta"].replace(rule=rule)
+    check_sampled(w, chains=[(0, 3)], segs=[0, 1, 15])
+
+
+def test_stream1m_sampled():
+    w = wl.WORKLOADS["stream1m_n2048_delta"]
+    check_sampled(w, chains=[(0, 7)], segs=[0, 1, 511])
+
+
+def test_batched_sampled():
+    w = wl.WORKLOADS["batched_n1024_linear"]
+    check_sampled(w, chains=[(0, 0), (15, 31)], segs=[0, 3, 7])
+
+
+# ---- properties of the boundary on the device ---------------------------------------
+
+def test_null_state_equals_zero_state():
+    from compressive_memory_long_b200 import binding
+    w = wl.WORKLOADS["hf_repro_n64"].replace(rule="delta", S=3)
+    t = to_dev(wl.torch_inputs(w))
+    a = binding.forward(t["q"], t["k"], t["v"], t["beta"], None, None, N=w.N, rule=w.rule)
+    Z = torch.zeros(w.B, w.Hkv, w.d, w.d, device="cuda")
+    zz = torch.zeros(w.B, w.Hkv, w.d, device="cuda")
+    b = binding.forward(t["q"], t["k"], t["v"], t["beta"], Z, zz, N=w.N, rule=w.rule)
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+
+
+@pytest.mark.parametrize("rule", ["linear", "delta"])
+def test_in_place_state_and_streaming_split(rule):
+    """Running [0, L1) then [L1, L) with the state updated in place (M_out is M0) gives the
+    single-call result; only (M, z) carries between calls."""
+    from compressive_memory_long_b200 import binding
+    w = wl.Workload("split", B=1, H=4, Hkv=2, d=64, N=128, S=4, dtype="bf16", rule=rule,
+                    seed=12, beta_dist=("normal", 0.0, 1.0), M0_dist=("uniform", 0.0, 0.1),
+                    z0_dist=("uniform", 1.0, 2.0))
+    t = to_dev(wl.torch_inputs(w))
+    full, Mf, zf = binding.forward(t["q"], t["k"], t["v"], t["beta"], t["M0"], t["z0"], N=w.N,
+                                   rule=rule)
+    M, z = t["M0"].clone(), t["z0"].clone()
+    L1 = 2 * w.N
+    halves = []
+    for sl in (slice(0, L1), slice(L1, w.L)):
+        qs, ks, vs = (t[n][:, :, sl].contiguous() for n in ("q", "k", "v"))
+        o, _, _ = binding.forward(qs, ks, vs, t["beta"], M, z, N=w.N, rule=rule, M_out=M,
+                                  z_out=z)
+        halves.append(o)
+    torch.cuda.synchronize()
+    assert torch.equal(torch.cat(halves, dim=2), full)
+    assert torch.allclose(M, Mf, rtol=1e-6, atol=1e-6) and torch.allclose(z, zf, rtol=1e-6)
+
+
+def test_device_argument_errors():
+    from compressive_memory_long_b200 import binding
+    q = torch.zeros(1, 2, 100, 64, dtype=torch.bfloat16, device="cuda")
+    beta = torch.zeros(2, device="cuda")
+    with pytest.raises(binding.InfiniError) as e:
+        binding.forward(q, q, q, beta, N=64)
+    assert e.value.status == 1
+    q = torch.zeros(1, 2, 128, 48, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(binding.InfiniError) as e:
+        binding.forward(q, q, q, beta, N=64)
+    assert e.value.status == 2

@@ -272,3 +272,11 @@ def test_workload_slices_are_reproducible():
     w2 = wl.WORKLOADS["hf_repro_n64"]
     x = wl.qkv_slice(w2, "v", 1, 3)
     assert np.array_equal(x, torch.from_numpy(x).to(torch.bfloat16).float().numpy())
+
+
+def test_workload_prefix_draw():
+    """A bounded sample (the first rows of a slice) equals the full draw's prefix."""
+    w = wl.WORKLOADS["hf_repro_n64"].replace(k_boost_frac=0.05, k_boost=4.0)
+    for t in ("q", "k", "v"):
+        full = wl.qkv_slice(w, t, 1, 2)
+        np.testing.assert_array_equal(wl.qkv_slice(w, t, 1, 2, rows=192), full[:192])
