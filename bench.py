@@ -311,7 +311,6 @@ def main():
     # ---- timed region (device time; trace on for per-kernel events) ----
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    binding.infini_attn_trace_report()     # drop anything recorded before
     barrier(world)
     torch.cuda.synchronize(dev)
     binding.infini_attn_trace_enable(True)

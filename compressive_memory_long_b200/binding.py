@@ -34,6 +34,7 @@ SIGNATURES = {
     "infini_attn_workspace_bytes": ([_I64] * 5, _I64),
     "infini_attn_status_string": ([_I], ctypes.c_char_p),
     "infini_attn_version": ([], _I),
+    "infini_attn_device_status": ([_P], _I),
     "infini_attn_trace_enable": ([_I], _I),
     "infini_attn_trace_report": ([ctypes.c_char_p, _I64], _I64),
 }
@@ -70,6 +71,11 @@ def infini_attn_version() -> int:
 
 def infini_attn_workspace_bytes(B, Hkv, L, N, d) -> int:
     return LIB.infini_attn_workspace_bytes(B, Hkv, L, N, d)
+
+
+def infini_attn_device_status(stream=None) -> int:
+    """Synchronise the stream; INFINI_ERR_TIMEOUT (5) if a bounded device wait gave up."""
+    return LIB.infini_attn_device_status(_stream_handle(stream))
 
 
 def infini_attn_trace_enable(on: bool) -> bool:

@@ -14,6 +14,9 @@
 
 #include "infini_attn.h"
 #include "simt_kernels.cuh"
+#include "tc_segment.cuh"
+
+#include <cudaTypedefs.h>
 
 namespace infini {
 namespace {
@@ -99,7 +102,11 @@ struct Rec {
     cudaEvent_t a, b;
 };
 std::mutex mu;
-std::vector<Rec> recs;
+std::vector<Rec> recs;                  // launches not yet folded into the table
+std::vector<std::string> names;         // accumulated table: kernel, launches, device ms
+std::vector<int64_t> counts;
+std::vector<double> ms;
+bool failed = false;
 std::atomic<int> enabled{0};
 
 struct Scope {
@@ -126,12 +133,73 @@ struct Scope {
 };
 }  // namespace trace
 
-#define TRACED(name, st) trace::Scope trace_scope_##__LINE__(name, st)
+#define TRACED(name, st) trace::Scope trace_scope(name, st)
+
+// ---- TMA tensor maps (driver entry point fetched through the runtime: no libcuda link) ----
+using EncodeTiledFn = PFN_cuTensorMapEncodeTiled_v12000;
+
+EncodeTiledFn encode_tiled()
+{
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// bf16 tensor [d2][d1][d0] (d0 contiguous) read as boxes of box1 rows x 64 columns with the
+// 128-byte swizzle.  Every box starts at a column multiple of 64 (128 bytes).
+bool make_map_bf16_3d(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1, uint64_t d2,
+                      uint32_t box1)
+{
+    EncodeTiledFn fn = encode_tiled();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {d0, d1, d2};
+    cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+    cuuint32_t box[3] = {64, box1, 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
+              es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The tensor-core segment kernel covers bf16 activations, d in {64, 128}, N % 128 == 0.
+template <typename T>
+bool use_tc(const Problem &p)
+{
+    return sizeof(T) == 2 && (p.d == 64 || p.d == 128) && p.N % 128 == 0;
+}
+
+template <int D>
+int launch_segment_tc(const Problem &p, const __nv_bfloat16 *q, const __nv_bfloat16 *k,
+                      const __nv_bfloat16 *v, const float *beta, const __nv_bfloat16 *snapMb,
+                      const float *snapZ, __nv_bfloat16 *out, cudaStream_t st)
+{
+    using C = tc::SegCfg<D>;
+    CUtensorMap mq, mk, mv, mm;
+    if (!make_map_bf16_3d(&mq, q, D, p.L, p.B * p.H, 128) ||
+        !make_map_bf16_3d(&mk, k, D, p.L, p.B * p.Hkv, 128) ||
+        !make_map_bf16_3d(&mv, v, D, p.L, p.B * p.Hkv, 128) ||
+        !make_map_bf16_3d(&mm, snapMb, D, D, p.B * p.Hkv * p.S, D))
+        return INFINI_ERR_CUDA;
+    if (!opt_in_smem<tc::k_segment_tc<D>>(C::ALLOC)) return INFINI_ERR_CUDA;
+    tc::SegArgs a{beta, snapZ, out, p.L, (int)p.N, (int)p.S, (int)p.H, (int)p.Hkv};
+    const int64_t ctas = p.B * p.H * p.S * (p.N / 128);
+    TRACED("segment_tc", st);
+    tc::k_segment_tc<D><<<(unsigned)ctas, 256, C::ALLOC, st>>>(mq, mk, mv, mm, a);
+    return INFINI_OK;
+}
 
 template <typename T, int D>
 int launch_all(const Problem &p, const T *q, const T *k, const T *v, const float *beta,
                const float *M0, const float *z0, T *out, float *M_out, float *z_out,
-               float *snapM, float *snapZ, cudaStream_t st)
+               float *snapM, float *snapZ, __nv_bfloat16 *snapMb, cudaStream_t st)
 {
     const int64_t chains = p.B * p.Hkv;
     const int S = (int)p.S, N = (int)p.N;
@@ -145,19 +213,26 @@ int launch_all(const Problem &p, const T *q, const T *k, const T *v, const float
         }
         {
             TRACED("linear_scan", st);
-            k_linear_scan<<<state_grid, 256, 0, st>>>(snapM, snapZ, M0, z0, M_out, z_out, S, D,
-                                                      chains);
+            k_linear_scan<<<state_grid, 256, 0, st>>>(snapM, snapZ, snapMb, M0, z0, M_out, z_out,
+                                                      S, D, chains);
         }
     } else {
         constexpr int CB = 16;
         {
             TRACED("state_init", st);
-            k_state_init<<<state_grid, 256, 0, st>>>(M0, z0, snapM, snapZ, S, D, chains);
+            k_state_init<<<state_grid, 256, 0, st>>>(M0, z0, snapM, snapZ, snapMb, S, D, chains);
         }
         {
             TRACED("delta_chain", st);
             k_delta_chain<T, D, CB><<<(unsigned)(chains * (D / CB)), 256, 0, st>>>(
-                k, v, snapM, snapZ, M_out, z_out, p.L, N, S);
+                k, v, snapM, snapZ, snapMb, M_out, z_out, p.L, N, S);
+        }
+    }
+    if constexpr (sizeof(T) == 2 && (D == 64 || D == 128)) {
+        if (snapMb) {
+            const int rc = launch_segment_tc<D>(p, q, k, v, beta, snapMb, snapZ, out, st);
+            if (rc != INFINI_OK) return rc;
+            return cudaGetLastError() == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
         }
     }
     const size_t smem = SimtSegSmem<D>::bytes;
@@ -184,19 +259,22 @@ int forward(const void *q, const void *k, const void *v, const float *beta, cons
     cudaGetLastError();   // clear a stale error left by someone else's launch
 
     const int64_t nM = p.B * p.Hkv * p.S * p.d * p.d, nZ = p.B * p.Hkv * p.S * p.d;
+    const bool tc_path = use_tc<T>(p);
+    const size_t bytes = (size_t)(nM + nZ) * sizeof(float) + (tc_path ? (size_t)nM * 2 : 0);
     void *ws = nullptr;
-    if (cudaMallocAsync(&ws, (size_t)(nM + nZ) * sizeof(float), st) != cudaSuccess) {
+    if (cudaMallocAsync(&ws, bytes, st) != cudaSuccess) {
         cudaGetLastError();
         return INFINI_ERR_OOM;
     }
     float *snapM = static_cast<float *>(ws), *snapZ = snapM + nM;
+    __nv_bfloat16 *snapMb = tc_path ? reinterpret_cast<__nv_bfloat16 *>(snapZ + nZ) : nullptr;
     const T *tq = static_cast<const T *>(q), *tk = static_cast<const T *>(k),
             *tv = static_cast<const T *>(v);
     T *to = static_cast<T *>(out);
     switch (p.d) {
-    case 32: rc = launch_all<T, 32>(p, tq, tk, tv, beta, M0, z0, to, M_out, z_out, snapM, snapZ, st); break;
-    case 64: rc = launch_all<T, 64>(p, tq, tk, tv, beta, M0, z0, to, M_out, z_out, snapM, snapZ, st); break;
-    default: rc = launch_all<T, 128>(p, tq, tk, tv, beta, M0, z0, to, M_out, z_out, snapM, snapZ, st); break;
+    case 32: rc = launch_all<T, 32>(p, tq, tk, tv, beta, M0, z0, to, M_out, z_out, snapM, snapZ, snapMb, st); break;
+    case 64: rc = launch_all<T, 64>(p, tq, tk, tv, beta, M0, z0, to, M_out, z_out, snapM, snapZ, snapMb, st); break;
+    default: rc = launch_all<T, 128>(p, tq, tk, tv, beta, M0, z0, to, M_out, z_out, snapM, snapZ, snapMb, st); break;
     }
     if (cudaFreeAsync(ws, st) != cudaSuccess && rc == INFINI_OK) rc = INFINI_ERR_CUDA;
     return rc;
@@ -228,7 +306,10 @@ int infini_attn_fwd_f32(const void *q, const void *k, const void *v, const float
 int64_t infini_attn_workspace_bytes(int64_t B, int64_t Hkv, int64_t L, int64_t N, int64_t d)
 {
     if (B <= 0 || Hkv <= 0 || L <= 0 || N <= 0 || d <= 0 || L % N != 0) return 0;
-    return B * Hkv * (L / N) * (d * d + d) * (int64_t)sizeof(float);
+    const int64_t S = L / N;
+    int64_t bytes = B * Hkv * S * (d * d + d) * (int64_t)sizeof(float);
+    if ((d == 64 || d == 128) && N % 128 == 0) bytes += B * Hkv * S * d * d * 2;   // bf16 copies
+    return bytes;
 }
 
 const char *infini_attn_status_string(int status)
@@ -246,49 +327,68 @@ const char *infini_attn_status_string(int status)
 
 int infini_attn_version(void) { return 100; }
 
+int infini_attn_device_status(infini_stream_t stream)
+{
+    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return INFINI_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, infini::tc::g_wait_status, sizeof(int)) != cudaSuccess)
+        return INFINI_ERR_CUDA;
+    if (v == 0) return INFINI_OK;
+    const int zero = 0;
+    cudaMemcpyToSymbol(infini::tc::g_wait_status, &zero, sizeof(int));
+    return INFINI_ERR_TIMEOUT;
+}
+
 int infini_attn_trace_enable(int on)
 {
-    const int prev = infini::trace::enabled.exchange(on ? 1 : 0);
-    return prev;
+    using namespace infini::trace;
+    std::lock_guard<std::mutex> g(mu);
+    if (on) {   // a new trace: drop pending records and the accumulated table
+        for (const Rec &r : recs) {
+            cudaEventDestroy(r.a);
+            cudaEventDestroy(r.b);
+        }
+        recs.clear();
+        names.clear();
+        counts.clear();
+        ms.clear();
+        failed = false;
+    }
+    return enabled.exchange(on ? 1 : 0);
 }
 
 int64_t infini_attn_trace_report(char *buf, int64_t len)
 {
     using namespace infini::trace;
-    std::vector<Rec> taken;
-    {
-        std::lock_guard<std::mutex> g(mu);
-        taken.swap(recs);
-    }
-    // aggregate per kernel name, in first-seen order
-    std::vector<std::string> names;
-    std::vector<int64_t> count;
-    std::vector<double> ms;
-    bool ok = true;
-    for (const Rec &r : taken) {
+    std::lock_guard<std::mutex> g(mu);
+    // fold pending records into the per-kernel table (first-seen order)
+    for (const Rec &r : recs) {
         float t = 0.f;
         if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&t, r.a, r.b) != cudaSuccess)
-            ok = false;
+            failed = true;
         cudaEventDestroy(r.a);
         cudaEventDestroy(r.b);
         size_t i = 0;
         while (i < names.size() && names[i] != r.name) ++i;
         if (i == names.size()) {
             names.emplace_back(r.name);
-            count.push_back(0);
+            counts.push_back(0);
             ms.push_back(0.0);
         }
-        count[i] += 1;
+        counts[i] += 1;
         ms[i] += t;
     }
+    recs.clear();
     std::string js = "{";
     for (size_t i = 0; i < names.size(); ++i) {
         char item[160];
         snprintf(item, sizeof(item), "%s\"%s\": {\"launches\": %lld, \"ms\": %.6f}", i ? ", " : "",
-                 names[i].c_str(), (long long)count[i], ms[i]);
+                 names[i].c_str(), (long long)counts[i], ms[i]);
         js += item;
     }
-    js += ok ? "}" : ", \"error\": true}";
+    if (failed) js += names.empty() ? "\"error\": true" : ", \"error\": true";
+    js += "}";
     if (buf && len > 0) {
         const size_t n = js.size() < (size_t)(len - 1) ? js.size() : (size_t)(len - 1);
         memcpy(buf, js.data(), n);

@@ -89,9 +89,12 @@ k_linear_increments(const T *__restrict__ k, const T *__restrict__ v, float *__r
 // One thread per state element; each thread reads its M0 element before writing the same
 // element of M_out, so exact aliasing of M_out with M0 is safe.
 // ---------------------------------------------------------------------------------------
+// snapMb, when not NULL, receives bf16 copies of the M snapshots (the operand layout of
+// the tensor-core segment kernel); the fp32 M snapshots are then not written back.
 __global__ void __launch_bounds__(256)
-k_linear_scan(float *__restrict__ snapM, float *__restrict__ snapZ, const float *M0,
-              const float *z0, float *M_out, float *z_out, int S, int D, int64_t chains)
+k_linear_scan(float *__restrict__ snapM, float *__restrict__ snapZ,
+              __nv_bfloat16 *__restrict__ snapMb, const float *M0, const float *z0,
+              float *M_out, float *z_out, int S, int D, int64_t chains)
 {
     const int64_t per = (int64_t)D * D + D;
     const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -102,10 +105,19 @@ k_linear_scan(float *__restrict__ snapM, float *__restrict__ snapZ, const float 
         const int64_t o = chain * D * D + e;
         float run = M0 ? M0[o] : 0.f;
         float *p = snapM + chain * S * (int64_t)D * D + e;
-        for (int s = 0; s < S; ++s) {
-            const float x = p[(int64_t)s * D * D];
-            p[(int64_t)s * D * D] = run;
-            run += x;
+        if (snapMb) {
+            __nv_bfloat16 *pb = snapMb + chain * S * (int64_t)D * D + e;
+            for (int s = 0; s < S; ++s) {
+                const float x = p[(int64_t)s * D * D];
+                pb[(int64_t)s * D * D] = __float2bfloat16_rn(run);
+                run += x;
+            }
+        } else {
+            for (int s = 0; s < S; ++s) {
+                const float x = p[(int64_t)s * D * D];
+                p[(int64_t)s * D * D] = run;
+                run += x;
+            }
         }
         M_out[o] = run;
     } else {
@@ -128,7 +140,8 @@ k_linear_scan(float *__restrict__ snapM, float *__restrict__ snapZ, const float 
 // ---------------------------------------------------------------------------------------
 __global__ void __launch_bounds__(256)
 k_state_init(const float *M0, const float *z0, float *__restrict__ snapM,
-             float *__restrict__ snapZ, int S, int D, int64_t chains)
+             float *__restrict__ snapZ, __nv_bfloat16 *__restrict__ snapMb, int S, int D,
+             int64_t chains)
 {
     const int64_t per = (int64_t)D * D + D;
     const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -136,7 +149,9 @@ k_state_init(const float *M0, const float *z0, float *__restrict__ snapM,
     const int64_t chain = idx / per;
     int64_t e = idx % per;
     if (e < (int64_t)D * D) {
-        snapM[chain * S * (int64_t)D * D + e] = M0 ? M0[chain * D * D + e] : 0.f;
+        const float m = M0 ? M0[chain * D * D + e] : 0.f;
+        snapM[chain * S * (int64_t)D * D + e] = m;
+        if (snapMb) snapMb[chain * S * (int64_t)D * D + e] = __float2bfloat16_rn(m);
     } else {
         e -= (int64_t)D * D;
         snapZ[chain * S * (int64_t)D + e] = z0 ? z0[chain * D + e] : 0.f;
@@ -155,7 +170,8 @@ k_state_init(const float *M0, const float *z0, float *__restrict__ snapM,
 template <typename T, int D, int CB>
 __global__ void __launch_bounds__(256)
 k_delta_chain(const T *__restrict__ k, const T *__restrict__ v, float *__restrict__ snapM,
-              float *__restrict__ snapZ, float *M_out, float *z_out, int64_t L, int N, int S)
+              float *__restrict__ snapZ, __nv_bfloat16 *__restrict__ snapMb, float *M_out,
+              float *z_out, int64_t L, int N, int S)
 {
     constexpr int TK = 32, NBLK = D / CB, PER = D * CB / 256;
     static_assert(PER >= 1 && (D * CB) % 256 == 0, "column block too small");
@@ -178,8 +194,14 @@ k_delta_chain(const T *__restrict__ k, const T *__restrict__ v, float *__restric
 
     for (int s = 0; s < S; ++s) {
         if (s > 0) {
-            float *dst = chainM + (int64_t)s * D * D;
-            for (int i = tid; i < D * CB; i += 256) dst[(i / CB) * D + cb + i % CB] = sM[i / CB][i % CB];
+            if (snapMb) {
+                __nv_bfloat16 *dst = snapMb + (chain * S + s) * (int64_t)D * D;
+                for (int i = tid; i < D * CB; i += 256)
+                    dst[(i / CB) * D + cb + i % CB] = __float2bfloat16_rn(sM[i / CB][i % CB]);
+            } else {
+                float *dst = chainM + (int64_t)s * D * D;
+                for (int i = tid; i < D * CB; i += 256) dst[(i / CB) * D + cb + i % CB] = sM[i / CB][i % CB];
+            }
             if (cb == 0)
                 for (int i = tid; i < D; i += 256) chainZ[(int64_t)s * D + i] = sz[i];
         }

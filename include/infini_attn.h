@@ -35,8 +35,8 @@
  *     denominator mean an empty memory); inputs finite.
  *   - On an argument error nothing is launched and nothing is written.  Nothing aborts,
  *     throws or traps; every failure is an int status below.
- *   - Scratch: the call allocates its workspace (per-segment memory snapshots,
- *     B * Hkv * S * (d*d + d) * 4 bytes) with cudaMallocAsync on `stream` and frees it with
+ *   - Scratch: the call allocates its workspace (per-segment memory snapshots; the size
+ *     is infini_attn_workspace_bytes) with cudaMallocAsync on `stream` and frees it with
  *     cudaFreeAsync on the same stream.
  */
 #ifndef INFINI_ATTN_H
@@ -69,7 +69,7 @@ enum {
     INFINI_ERR_UNSUPPORTED = 2, /* valid but not built: d not in {32, 64, 128}, N % 64 != 0 */
     INFINI_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed                      */
     INFINI_ERR_OOM = 4,         /* the workspace allocation failed                           */
-    INFINI_ERR_TIMEOUT = 5      /* reserved: a bounded device wait gave up                   */
+    INFINI_ERR_TIMEOUT = 5      /* a bounded device wait gave up (infini_attn_device_status) */
 };
 
 /*
@@ -95,6 +95,15 @@ INFINI_API int infini_attn_fwd_f32(const void *q, const void *k, const void *v, 
 /* Bytes of workspace one call allocates for these sizes (0 on invalid sizes). */
 INFINI_API int64_t infini_attn_workspace_bytes(int64_t B, int64_t Hkv, int64_t L, int64_t N, int64_t d);
 
+/*
+ * Synchronises `stream`, then reports whether a bounded wait inside a kernel of this
+ * library gave up since the last check: INFINI_ERR_TIMEOUT (and the record is cleared),
+ * INFINI_OK, or INFINI_ERR_CUDA if the synchronisation itself failed.  A kernel whose wait
+ * gave up stops early and leaves part of its outputs unwritten.  The record is sticky:
+ * until it is read here, later launches of the waiting kernels return without work.
+ */
+INFINI_API int infini_attn_device_status(infini_stream_t stream);
+
 /* Static, NUL-terminated description of a status code. */
 INFINI_API const char *infini_attn_status_string(int status);
 
@@ -103,10 +112,12 @@ INFINI_API int infini_attn_version(void);
 
 /*
  * Launch tracing (off by default).  While enabled, every kernel this library enqueues is
- * bracketed by two CUDA events recorded on the call's stream.  The report synchronises
- * on those events, writes a JSON object {"<kernel>": {"launches": n, "ms": total}, ...}
- * (NUL-terminated, truncated to len - 1 bytes) into buf, clears the records and returns
- * the size the full report needs.  enable returns the previous setting.
+ * bracketed by two CUDA events recorded on the call's stream.  infini_attn_trace_enable(1)
+ * starts a new trace (clearing the previous one); it returns the previous setting.
+ * infini_attn_trace_report synchronises on the recorded events, adds them to a per-kernel
+ * table and writes it as JSON, {"<kernel>": {"launches": n, "ms": total}, ...}
+ * (NUL-terminated, truncated to len - 1 bytes; buf may be NULL), and returns the size
+ * the full report needs.  Reporting does not clear the table.
  */
 INFINI_API int infini_attn_trace_enable(int on);
 INFINI_API int64_t infini_attn_trace_report(char *buf, int64_t len);

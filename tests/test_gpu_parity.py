@@ -157,3 +157,34 @@ def test_device_argument_errors():
     with pytest.raises(binding.InfiniError) as e:
         binding.forward(q, q, q, beta, N=64)
     assert e.value.status == 2
+
+
+# ---- the tensor-core segment kernel (bf16, d in {64, 128}, N % 128 == 0) --------------
+
+@pytest.mark.parametrize("rule", ["linear", "delta"])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("N,S", [(128, 3), (256, 2), (384, 2)])
+def test_tensor_core_segment_kernel(rule, d, N, S):
+    """Several 128-row q tiles (diagonal and off-diagonal key tiles), GQA, nonzero state;
+    checks that the tensor-core kernel is the one that ran and that no wait gave up."""
+    from compressive_memory_long_b200 import binding
+    w = wl.Workload("tc", B=2, H=4, Hkv=2, d=d, N=N, S=S, dtype="bf16", rule=rule, seed=21,
+                    beta_dist=("normal", 0.0, 1.5), M0_dist=("uniform", 0.0, 0.1),
+                    z0_dist=("uniform", 1.0, 2.0))
+    binding.infini_attn_trace_enable(True)
+    check_full(w)
+    binding.infini_attn_trace_enable(False)
+    assert "segment_tc" in binding.infini_attn_trace_report()
+    assert binding.infini_attn_device_status() == 0
+
+
+def test_tensor_core_first_segment_empty_memory():
+    """z0 = 0: the first segment's retrieval is exactly 0, so with beta -> +inf the first
+    segment's output is exactly 0 and later segments are not."""
+    from compressive_memory_long_b200 import binding
+    w = wl.Workload("tc0", B=1, H=2, Hkv=2, d=128, N=256, S=2, dtype="bf16", rule="delta",
+                    seed=22, beta_dist=("normal", 40.0, 0.0))
+    out, _, _ = run_gpu(w)
+    assert torch.count_nonzero(out[:, :, :256]) == 0
+    assert torch.count_nonzero(out[:, :, 256:]) > 0
+    assert binding.infini_attn_device_status() == 0
