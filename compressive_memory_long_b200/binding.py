@@ -31,6 +31,7 @@ _FWD_ARGS = [_P] * 9 + [_I64] * 6 + [_I, _P]
 SIGNATURES = {
     "infini_attn_fwd": (_FWD_ARGS, _I),
     "infini_attn_fwd_f32": (_FWD_ARGS, _I),
+    "infini_attn_fwd_noalloc": (_FWD_ARGS, _I),
     "infini_attn_workspace_bytes": ([_I64] * 5, _I64),
     "infini_attn_status_string": ([_I], ctypes.c_char_p),
     "infini_attn_version": ([], _I),
@@ -118,6 +119,16 @@ def infini_attn_fwd(q, k, v, beta, M0, z0, out, M_out, z_out, N, rule, stream=No
 def infini_attn_fwd_f32(q, k, v, beta, M0, z0, out, M_out, z_out, N, rule, stream=None):
     """fp32 entry point; all tensors preallocated, contiguous, on one CUDA device."""
     _call(LIB.infini_attn_fwd_f32, q, k, v, beta, M0, z0, out, M_out, z_out, N, rule, stream)
+
+
+def infini_attn_fwd_noalloc(q, k, v, beta, M0, z0, out, M_out, z_out, N, rule, stream=None):
+    """bf16 entry point that allocates nothing (workspace: the library's fixed device array
+    of NOALLOC_SCRATCH_BYTES); all tensors preallocated, contiguous, on one CUDA device."""
+    _call(LIB.infini_attn_fwd_noalloc, q, k, v, beta, M0, z0, out, M_out, z_out, N, rule, stream)
+
+
+#: size of the fixed device array infini_attn_fwd_noalloc uses as its workspace
+NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
 def _check(t, name, dtype, shape, device):

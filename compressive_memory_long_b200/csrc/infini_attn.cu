@@ -18,6 +18,13 @@
 
 #include <cudaTypedefs.h>
 
+// Workspace of infini_attn_fwd_noalloc: a file-scope device array used instead of a
+// per-call allocation.  Every GPU that loads the library holds it until the process exits.
+// In host code the name is only a host-side stand-in for the symbol, never a device
+// address: the address comes from cudaGetSymbolAddress, looked up once per device with that
+// device current (noalloc_scratch_address below).
+static __device__ __align__(256) unsigned char g_noalloc_scratch[INFINI_NOALLOC_SCRATCH_BYTES];
+
 namespace infini {
 namespace {
 
@@ -280,10 +287,75 @@ int forward(const void *q, const void *k, const void *v, const float *beta, cons
     return rc;
 }
 
+// ---- allocation-free variant of the bf16 forward (workspace: g_noalloc_scratch) ----------
+constexpr size_t kNoAllocScratchBytes = (size_t)INFINI_NOALLOC_SCRATCH_BYTES;
+
+// Device address of g_noalloc_scratch on the current device (nullptr on failure).
+void *noalloc_scratch_address()
+{
+    constexpr int kMaxDevices = 64;
+    static std::atomic<void *> addr[kMaxDevices];
+    static std::mutex setup_mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    void *a = addr[dev].load(std::memory_order_acquire);
+    if (a) return a;
+    std::lock_guard<std::mutex> g(setup_mu);
+    a = addr[dev].load(std::memory_order_acquire);
+    if (a) return a;
+    if (cudaGetSymbolAddress(&a, g_noalloc_scratch) != cudaSuccess || a == nullptr) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    addr[dev].store(a, std::memory_order_release);
+    return a;
+}
+
+int forward_noalloc(const void *q, const void *k, const void *v, const float *beta,
+                    const float *M0, const float *z0, void *out, float *M_out, float *z_out,
+                    int64_t B, int64_t H, int64_t Hkv, int64_t L, int64_t N, int64_t d, int rule,
+                    infini_stream_t stream)
+{
+    using T = __nv_bfloat16;
+    Problem p;
+    int rc = check_args(q, k, v, beta, M0, z0, out, M_out, z_out, B, H, Hkv, L, N, d, rule,
+                        (int64_t)sizeof(T), &p);
+    if (rc != INFINI_OK) return rc;
+    const int64_t nM = p.B * p.Hkv * p.S * p.d * p.d, nZ = p.B * p.Hkv * p.S * p.d;
+    const bool tc_path = use_tc<T>(p);
+    const size_t bytes = (size_t)(nM + nZ) * sizeof(float) + (tc_path ? (size_t)nM * 2 : 0);
+    if (bytes > kNoAllocScratchBytes) return INFINI_ERR_UNSUPPORTED;
+    void *ws = noalloc_scratch_address();
+    if (!ws) return INFINI_ERR_CUDA;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaGetLastError();
+    // Nothing in the array needs to start at zero: every snapshot slot a kernel reads was
+    // written earlier in the same call (increments / initial state, then the scan or chain).
+    float *snapM = static_cast<float *>(ws), *snapZ = snapM + nM;
+    T *snapMb = tc_path ? reinterpret_cast<T *>(snapZ + nZ) : nullptr;
+    const T *tq = static_cast<const T *>(q), *tk = static_cast<const T *>(k),
+            *tv = static_cast<const T *>(v);
+    T *to = static_cast<T *>(out);
+    switch (p.d) {
+    case 32: return launch_all<T, 32>(p, tq, tk, tv, beta, M0, z0, to, M_out, z_out, snapM, snapZ, snapMb, st);
+    case 64: return launch_all<T, 64>(p, tq, tk, tv, beta, M0, z0, to, M_out, z_out, snapM, snapZ, snapMb, st);
+    default: return launch_all<T, 128>(p, tq, tk, tv, beta, M0, z0, to, M_out, z_out, snapM, snapZ, snapMb, st);
+    }
+}
+
 }  // namespace
 }  // namespace infini
 
 extern "C" {
+
+int infini_attn_fwd_noalloc(const void *q, const void *k, const void *v, const float *beta,
+                            const float *M0, const float *z0, void *out, float *M_out,
+                            float *z_out, int64_t B, int64_t H, int64_t Hkv, int64_t L,
+                            int64_t N, int64_t d, int update_rule, infini_stream_t stream)
+{
+    return infini::forward_noalloc(q, k, v, beta, M0, z0, out, M_out, z_out, B, H, Hkv, L, N, d,
+                                   update_rule, stream);
+}
 
 int infini_attn_fwd(const void *q, const void *k, const void *v, const float *beta,
                     const float *M0, const float *z0, void *out, float *M_out, float *z_out,

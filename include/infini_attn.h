@@ -92,6 +92,37 @@ INFINI_API int infini_attn_fwd_f32(const void *q, const void *k, const void *v, 
                         float *z_out, int64_t B, int64_t H, int64_t Hkv, int64_t L, int64_t N,
                         int64_t d, int update_rule, infini_stream_t stream);
 
+/*
+ * Allocation-free variant of infini_attn_fwd (bf16 activations); same parameters, same
+ * results.  The pages have no counterpart to this entry point: it exists for callers that
+ * may not allocate device memory while they run, for example a serving loop whose device
+ * memory is planned and handed out by its own allocator up front (a stream-ordered
+ * allocation there could fail when that allocator holds nearly all of HBM, or stall the
+ * loop while the driver's pool grows), or a host program that gives plugins buffers but
+ * no allocation rights.  This call makes no cudaMalloc / cudaFree / cudaMallocAsync /
+ * cudaFreeAsync call and calls no allocating library routine.
+ *
+ *   - Its workspace is a fixed device array of INFINI_NOALLOC_SCRATCH_BYTES inside the
+ *     library; every GPU that loads the library holds that array until the process exits.
+ *     A problem whose workspace (infini_attn_workspace_bytes) exceeds it is rejected with
+ *     INFINI_ERR_UNSUPPORTED, before anything is launched.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call before any
+ *     stream capture begins.
+ *   - All calls on a device share that device's one array, which keeps the last call's
+ *     contents.  Calls on the same device that overlap on the GPU (issued on different
+ *     streams or from different host threads without ordering between them) race and
+ *     corrupt each other's results: order them on one stream or with events.  Calls on
+ *     different devices do not interfere.  Nothing in the array has to start at zero: each
+ *     call writes every workspace byte it reads before reading it.
+ */
+#define INFINI_NOALLOC_SCRATCH_BYTES (16ull << 20)
+INFINI_API int infini_attn_fwd_noalloc(const void *q, const void *k, const void *v,
+                                       const float *beta, const float *M0, const float *z0,
+                                       void *out, float *M_out, float *z_out, int64_t B,
+                                       int64_t H, int64_t Hkv, int64_t L, int64_t N, int64_t d,
+                                       int update_rule, infini_stream_t stream);
+
 /* Bytes of workspace one call allocates for these sizes (0 on invalid sizes). */
 INFINI_API int64_t infini_attn_workspace_bytes(int64_t B, int64_t Hkv, int64_t L, int64_t N, int64_t d);
 
