@@ -72,7 +72,7 @@ def algorithmic(w: wl.Workload, kernel: str):
     if kernel.startswith("segment"):
         flops = B * H * S * (2 * d * N * (N + 1) + 2 * N * d * d)
         byts = (2 * H + 2 * Hkv) * B * L * d * e
-    elif kernel in ("linear_increments", "delta_chain", "linear_fused", "delta_fused"):
+    elif kernel.startswith(("linear_increments", "linear_state", "delta_chain")):
         per = 2 if w.rule == "linear" else 4
         flops = B * Hkv * S * per * N * d * d
         byts = 2 * B * Hkv * L * d * e + state_bytes

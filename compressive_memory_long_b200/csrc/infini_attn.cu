@@ -15,6 +15,9 @@
 #include "infini_attn.h"
 #include "simt_kernels.cuh"
 #include "tc_segment.cuh"
+#include "tc_segment2.cuh"
+#include "tc_delta.cuh"
+#include "tc_linear.cuh"
 
 #include <cudaTypedefs.h>
 
@@ -160,20 +163,57 @@ EncodeTiledFn encode_tiled()
     return fn;
 }
 
-// bf16 tensor [d2][d1][d0] (d0 contiguous) read as boxes of box1 rows x 64 columns with the
-// 128-byte swizzle.  Every box starts at a column multiple of 64 (128 bytes).
+// bf16 tensor [d2][d1][d0] (d0 contiguous) read as boxes of box1 rows x box0 columns.
+// With the 128-byte swizzle box0 is 64 (128 bytes) and every box starts at a column multiple
+// of 64; unswizzled boxes start at column multiples of 8 (16 bytes).
 bool make_map_bf16_3d(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1, uint64_t d2,
-                      uint32_t box1)
+                      uint32_t box1, uint32_t box0 = 64, bool swizzle128 = true)
 {
     EncodeTiledFn fn = encode_tiled();
     if (!fn) return false;
     cuuint64_t dims[3] = {d0, d1, d2};
     cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
-    cuuint32_t box[3] = {64, box1, 1};
+    cuuint32_t box[3] = {box0, box1, 1};
     cuuint32_t es[3] = {1, 1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
-              es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D>
+int launch_linear_state_tc(const Problem &p, const __nv_bfloat16 *k, const __nv_bfloat16 *v,
+                           const float *M0, const float *z0, float *snapZ, __nv_bfloat16 *snapMb,
+                           float *M_out, float *z_out, cudaStream_t st)
+{
+    using C = tc::LinCfg<D>;
+    CUtensorMap mk, mv;
+    if (!make_map_bf16_3d(&mk, k, D, p.L, p.B * p.Hkv, 128) ||
+        !make_map_bf16_3d(&mv, v, D, p.L, p.B * p.Hkv, 128))
+        return INFINI_ERR_CUDA;
+    if (!opt_in_smem<tc::k_linear_state_tc<D>>(C::ALLOC)) return INFINI_ERR_CUDA;
+    tc::LinArgs a{M0, z0, snapZ, snapMb, M_out, z_out, (int)p.N, (int)p.S};
+    TRACED("linear_state_tc", st);
+    tc::k_linear_state_tc<D><<<(unsigned)(p.B * p.Hkv), 256, C::ALLOC, st>>>(mk, mv, a);
+    return INFINI_OK;
+}
+
+template <int D>
+int launch_delta_chain_tc(const Problem &p, const __nv_bfloat16 *k, const __nv_bfloat16 *v,
+                          const float *snapM, float *snapZ, __nv_bfloat16 *snapMb, float *M_out,
+                          float *z_out, cudaStream_t st)
+{
+    using C = tc::ChainCfg;
+    CUtensorMap mk, mv;
+    if (!make_map_bf16_3d(&mk, k, D, p.L, p.B * p.Hkv, 128) ||
+        !make_map_bf16_3d(&mv, v, D, p.L, p.B * p.Hkv, 128, C::CB, false))
+        return INFINI_ERR_CUDA;
+    if (!opt_in_smem<tc::k_delta_chain_tc<D>>(C::ALLOC)) return INFINI_ERR_CUDA;
+    tc::ChainArgs a{snapM, snapZ, snapZ, snapMb, M_out, z_out, (int)p.N, (int)p.S};
+    const int64_t ctas = p.B * p.Hkv * (D / C::CB);
+    TRACED("delta_chain_tc", st);
+    tc::k_delta_chain_tc<D><<<(unsigned)ctas, 256, C::ALLOC, st>>>(mk, mv, a);
+    return INFINI_OK;
 }
 
 // The tensor-core segment kernel covers bf16 activations, d in {64, 128}, N % 128 == 0.
@@ -195,8 +235,16 @@ int launch_segment_tc(const Problem &p, const __nv_bfloat16 *q, const __nv_bfloa
         !make_map_bf16_3d(&mv, v, D, p.L, p.B * p.Hkv, 128) ||
         !make_map_bf16_3d(&mm, snapMb, D, D, p.B * p.Hkv * p.S, D))
         return INFINI_ERR_CUDA;
-    if (!opt_in_smem<tc::k_segment_tc<D>>(C::ALLOC)) return INFINI_ERR_CUDA;
     tc::SegArgs a{beta, snapZ, out, p.L, (int)p.N, (int)p.S, (int)p.H, (int)p.Hkv};
+    if (p.N % 256 == 0) {   // two query tiles per CTA share every key/value tile
+        using C2 = tc::Seg2Cfg<D>;
+        if (!opt_in_smem<tc::k_segment_tc2<D>>(C2::ALLOC)) return INFINI_ERR_CUDA;
+        const int64_t ctas = p.B * p.H * p.S * (p.N / 256);
+        TRACED("segment_tc", st);
+        tc::k_segment_tc2<D><<<(unsigned)ctas, C2::THREADS, C2::ALLOC, st>>>(mq, mk, mv, mm, a);
+        return INFINI_OK;
+    }
+    if (!opt_in_smem<tc::k_segment_tc<D>>(C::ALLOC)) return INFINI_ERR_CUDA;
     const int64_t ctas = p.B * p.H * p.S * (p.N / 128);
     TRACED("segment_tc", st);
     tc::k_segment_tc<D><<<(unsigned)ctas, 256, C::ALLOC, st>>>(mq, mk, mv, mm, a);
@@ -212,7 +260,16 @@ int launch_all(const Problem &p, const T *q, const T *k, const T *v, const float
     const int S = (int)p.S, N = (int)p.N;
     const int64_t per = (int64_t)D * D + D;
     const unsigned state_grid = (unsigned)((chains * per + 255) / 256);
-    if (p.rule == INFINI_UPDATE_LINEAR) {
+    bool linear_tc = false;
+    if constexpr (sizeof(T) == 2 && (D == 64 || D == 128)) {
+        if (p.rule == INFINI_UPDATE_LINEAR && snapMb) {
+            const int rc = launch_linear_state_tc<D>(p, k, v, M0, z0, snapZ, snapMb, M_out, z_out, st);
+            if (rc != INFINI_OK) return rc;
+            linear_tc = true;
+        }
+    }
+    if (linear_tc) {
+    } else if (p.rule == INFINI_UPDATE_LINEAR) {
         {
             TRACED("linear_increments", st);
             k_linear_increments<T, D><<<(unsigned)(chains * S), 256, 0, st>>>(k, v, snapM, snapZ,
@@ -229,7 +286,16 @@ int launch_all(const Problem &p, const T *q, const T *k, const T *v, const float
             TRACED("state_init", st);
             k_state_init<<<state_grid, 256, 0, st>>>(M0, z0, snapM, snapZ, snapMb, S, D, chains);
         }
-        {
+        bool done = false;
+        if constexpr (sizeof(T) == 2 && (D == 64 || D == 128)) {
+            if (snapMb) {
+                const int rc = launch_delta_chain_tc<D>(p, k, v, snapM, snapZ, snapMb, M_out,
+                                                        z_out, st);
+                if (rc != INFINI_OK) return rc;
+                done = true;
+            }
+        }
+        if (!done) {
             TRACED("delta_chain", st);
             k_delta_chain<T, D, CB><<<(unsigned)(chains * (D / CB)), 256, 0, st>>>(
                 k, v, snapM, snapZ, snapMb, M_out, z_out, p.L, N, S);

@@ -174,7 +174,9 @@ def test_tensor_core_segment_kernel(rule, d, N, S):
     binding.infini_attn_trace_enable(True)
     check_full(w)
     binding.infini_attn_trace_enable(False)
-    assert "segment_tc" in binding.infini_attn_trace_report()
+    report = binding.infini_attn_trace_report()
+    assert "segment_tc" in report
+    assert ("delta_chain_tc" if rule == "delta" else "linear_state_tc") in report
     assert binding.infini_attn_device_status() == 0
 
 
