@@ -42,17 +42,38 @@ def build(force: bool = False) -> str:
 _lib = None
 
 
+def _bind(path: str):
+    lib = ctypes.CDLL(path)
+    f = lib.oracle_infini_attn_fwd
+    P = ctypes.c_void_p
+    I64 = ctypes.c_int64
+    f.argtypes = [P, P, P, P, P, P, P, P, P, I64, I64, I64, I64, I64, I64, ctypes.c_int, P]
+    f.restype = ctypes.c_int
+    return lib
+
+
 def _load():
     global _lib
     if _lib is None:
-        lib = ctypes.CDLL(build())
-        f = lib.oracle_infini_attn_fwd
-        P = ctypes.c_void_p
-        I64 = ctypes.c_int64
-        f.argtypes = [P, P, P, P, P, P, P, P, P, I64, I64, I64, I64, I64, I64, ctypes.c_int, P]
-        f.restype = ctypes.c_int
-        _lib = lib
+        _lib = _bind(build())
     return _lib
+
+
+def source() -> str:
+    with open(_SRC) as fh:
+        return fh.read()
+
+
+def compile_variant(src: str, out_dir: str) -> str:
+    """Compile a modified copy of the oracle source (used by the tests that plant mistakes
+    in the oracle to show its pins catch them).  Returns the shared-library path."""
+    c_path = os.path.join(out_dir, "variant.c")
+    so_path = os.path.join(out_dir, "libvariant.so")
+    with open(c_path, "w") as fh:
+        fh.write(src)
+    subprocess.check_call(["gcc", "-O2", "-fPIC", "-shared", "-std=c11", "-fno-fast-math",
+                           "-ffp-contract=off", "-o", so_path, c_path, "-lm"])
+    return so_path
 
 
 def _f32(a):
@@ -67,7 +88,7 @@ def _ptr(a):
 
 
 def infini_attn_fwd(q, k, v, beta, M0=None, z0=None, *, N: int, rule="linear",
-                    seg_out=None, out=None):
+                    seg_out=None, out=None, lib_path=None):
     """Run the oracle.
 
     q [B,H,L,d], k/v [B,Hkv,L,d], beta [H], M0 [B,Hkv,d,d] or None, z0 [B,Hkv,d] or None.
@@ -75,6 +96,7 @@ def infini_attn_fwd(q, k, v, beta, M0=None, z0=None, *, N: int, rule="linear",
     ``seg_out``: optional iterable of segment indices whose outputs are computed (all
     segments' memory updates always run).  ``out``: optional float64 array to fill
     (rows of segments not in ``seg_out`` keep its contents; default zeros).
+    ``lib_path``: run a variant compiled by ``compile_variant`` instead of the oracle.
     Returns (out [B,H,L,d], M_out [B,Hkv,d,d], z_out [B,Hkv,d]).
     """
     q, k, v, beta, M0, z0 = (_f32(x) for x in (q, k, v, beta, M0, z0))
@@ -95,7 +117,8 @@ def infini_attn_fwd(q, k, v, beta, M0=None, z0=None, *, N: int, rule="linear",
     assert out.dtype == np.float64 and out.shape == (B, H, L, d) and out.flags.c_contiguous
     M_out = np.zeros((B, Hkv, d, d), dtype=np.float64)
     z_out = np.zeros((B, Hkv, d), dtype=np.float64)
-    rc = _load().oracle_infini_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(M0),
+    lib = _load() if lib_path is None else _bind(lib_path)
+    rc = lib.oracle_infini_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(M0),
                                         _ptr(z0), _ptr(out), _ptr(M_out), _ptr(z_out),
                                         B, H, Hkv, L, N, d, _RULES[rule], _ptr(mask))
     if rc != 0:
