@@ -69,6 +69,10 @@ def algorithmic(w: wl.Workload, kernel: str):
     e = w.elem_bytes
     B, H, Hkv, L, N, d, S = w.B, w.H, w.Hkv, w.L, w.N, w.d, w.S
     state_bytes = 2 * B * Hkv * (d * d + d) * 4
+    if kernel == "small_fused":     # the whole forward in one launch
+        f1, b1 = algorithmic(w, "segment")
+        f2, b2 = algorithmic(w, "linear_state")
+        return f1 + f2, b1 + state_bytes
     if kernel.startswith("segment"):
         flops = B * H * S * (2 * d * N * (N + 1) + 2 * N * d * d)
         byts = (2 * H + 2 * Hkv) * B * L * d * e

@@ -18,6 +18,7 @@
 #include "tc_segment2.cuh"
 #include "tc_delta.cuh"
 #include "tc_linear.cuh"
+#include "tc_small.cuh"
 
 #include <cudaTypedefs.h>
 
@@ -116,8 +117,36 @@ std::vector<Rec> recs;                  // launches not yet folded into the tabl
 std::vector<std::string> names;         // accumulated table: kernel, launches, device ms
 std::vector<int64_t> counts;
 std::vector<double> ms;
+std::vector<cudaEvent_t> pool;          // events ready for reuse (each belongs to one device)
+std::vector<int> pool_dev;
 bool failed = false;
 std::atomic<int> enabled{0};
+
+// An event of the current device from the pool, or a new one.
+bool take_event(cudaEvent_t *e)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    {
+        std::lock_guard<std::mutex> g(mu);
+        for (size_t i = pool.size(); i-- > 0;)
+            if (pool_dev[i] == dev) {
+                *e = pool[i];
+                pool.erase(pool.begin() + i);
+                pool_dev.erase(pool_dev.begin() + i);
+                return true;
+            }
+    }
+    return cudaEventCreate(e) == cudaSuccess;
+}
+
+void give_event(cudaEvent_t e)
+{
+    int dev = 0;
+    cudaGetDevice(&dev);
+    pool.push_back(e);          // callers hold mu
+    pool_dev.push_back(dev);
+}
 
 struct Scope {
     Rec r{};
@@ -127,7 +156,7 @@ struct Scope {
     {
         if (!on) return;
         r.name = name;
-        if (cudaEventCreate(&r.a) != cudaSuccess || cudaEventCreate(&r.b) != cudaSuccess) {
+        if (!take_event(&r.a) || !take_event(&r.b)) {
             on = false;
             return;
         }
@@ -204,8 +233,21 @@ int launch_delta_chain_tc(const Problem &p, const __nv_bfloat16 *k, const __nv_b
                           float *z_out, cudaStream_t st)
 {
     using C = tc::ChainCfg;
+    // sigma(K) once per token, into the workspace after the bf16 snapshots
+    __nv_bfloat16 *sk = snapMb + p.B * p.Hkv * p.S * (int64_t)D * D;
+    const int64_t n8 = p.B * p.Hkv * p.L * (int64_t)D / 8;
+    {
+        int sms = 148;
+        int dev = 0;
+        if (cudaGetDevice(&dev) == cudaSuccess)
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        const int64_t want = (n8 + 255) / 256;
+        const unsigned grid = (unsigned)(want < (int64_t)sms * 16 ? want : (int64_t)sms * 16);
+        TRACED("sigma_keys", st);
+        tc::k_sigma_bf16<<<grid, 256, 0, st>>>(k, sk, n8);
+    }
     CUtensorMap mk, mv;
-    if (!make_map_bf16_3d(&mk, k, D, p.L, p.B * p.Hkv, 128) ||
+    if (!make_map_bf16_3d(&mk, sk, D, p.L, p.B * p.Hkv, 128) ||
         !make_map_bf16_3d(&mv, v, D, p.L, p.B * p.Hkv, 128, C::CB, false))
         return INFINI_ERR_CUDA;
     if (!opt_in_smem<tc::k_delta_chain_tc<D>>(C::ALLOC)) return INFINI_ERR_CUDA;
@@ -223,6 +265,40 @@ bool use_tc(const Problem &p)
     return sizeof(T) == 2 && (p.d == 64 || p.d == 128) && p.N % 128 == 0;
 }
 
+// One launch for 64-token segments under the additive rule (bf16, d = 64, MHA).
+template <typename T>
+bool use_small_fused(const Problem &p)
+{
+    return sizeof(T) == 2 && p.d == 64 && p.N == 64 && p.rule == INFINI_UPDATE_LINEAR &&
+           p.H == p.Hkv && p.L % 128 == 0;
+}
+
+// Workspace of one call: fp32 snapshots (M, z) for every segment, bf16 copies of M for the
+// tensor-core kernels, and room for the fused path's flags; an upper bound for every path.
+// Layout: [fp32 snapshots M | z][bf16 copies of M][sigma(K) in bf16][flags of the fused path].
+int64_t workspace_bytes(int64_t B, int64_t Hkv, int64_t S, int64_t N, int64_t d)
+{
+    const int64_t units = B * Hkv * S;
+    return units * (d * d + d) * 4 + units * d * d * 2 + units * N * d * 2 + units * 4 + 256;
+}
+
+// The two-tile kernel redistributes registers with setmaxnreg; its split assumes the
+// register count per thread it was compiled with.  Checked once per kernel: a mismatch
+// would leave the growing warpgroups waiting forever, so the one-tile kernel runs instead.
+template <int D>
+bool seg2_registers_match()
+{
+    static const bool ok = [] {
+        cudaFuncAttributes fa;
+        if (cudaFuncGetAttributes(&fa, tc::k_segment_tc2<D>) != cudaSuccess) {
+            cudaGetLastError();
+            return false;
+        }
+        return fa.numRegs == tc::Seg2Cfg<D>::REGS;
+    }();
+    return ok;
+}
+
 template <int D>
 int launch_segment_tc(const Problem &p, const __nv_bfloat16 *q, const __nv_bfloat16 *k,
                       const __nv_bfloat16 *v, const float *beta, const __nv_bfloat16 *snapMb,
@@ -236,7 +312,7 @@ int launch_segment_tc(const Problem &p, const __nv_bfloat16 *q, const __nv_bfloa
         !make_map_bf16_3d(&mm, snapMb, D, D, p.B * p.Hkv * p.S, D))
         return INFINI_ERR_CUDA;
     tc::SegArgs a{beta, snapZ, out, p.L, (int)p.N, (int)p.S, (int)p.H, (int)p.Hkv};
-    if (p.N % 256 == 0) {   // two query tiles per CTA share every key/value tile
+    if (p.N % 256 == 0 && seg2_registers_match<D>()) {   // two query tiles per CTA
         using C2 = tc::Seg2Cfg<D>;
         if (!opt_in_smem<tc::k_segment_tc2<D>>(C2::ALLOC)) return INFINI_ERR_CUDA;
         const int64_t ctas = p.B * p.H * p.S * (p.N / 256);
@@ -251,11 +327,44 @@ int launch_segment_tc(const Problem &p, const __nv_bfloat16 *q, const __nv_bfloa
     return INFINI_OK;
 }
 
+int launch_small_fused(const Problem &p, const __nv_bfloat16 *q, const __nv_bfloat16 *k,
+                       const __nv_bfloat16 *v, const float *beta, const float *M0,
+                       const float *z0, __nv_bfloat16 *out, float *M_out, float *z_out,
+                       void *ws, cudaStream_t st)
+{
+    using C = tc::SmallCfg;
+    const int64_t chains = p.B * p.Hkv, U = p.L / 128, units = chains * U;
+    // workspace: ticket + flags (zeroed here), then the published aggregates / prefixes
+    int *ticket = static_cast<int *>(ws);
+    int *flags = ticket + 64;
+    const size_t head = ((size_t)(64 + units) * 4 + 255) / 256 * 256;
+    float *agg = reinterpret_cast<float *>(static_cast<char *>(ws) + head);
+    float *incl = agg + units * C::D * C::ROW;
+    if (cudaMemsetAsync(ws, 0, (size_t)(64 + units) * 4, st) != cudaSuccess) return INFINI_ERR_CUDA;
+    CUtensorMap mq, mk, mv;
+    if (!make_map_bf16_3d(&mq, q, C::D, p.L, p.B * p.H, 128) ||
+        !make_map_bf16_3d(&mk, k, C::D, p.L, chains, 128) ||
+        !make_map_bf16_3d(&mv, v, C::D, p.L, chains, 128))
+        return INFINI_ERR_CUDA;
+    if (!opt_in_smem<tc::k_small_linear_fused>(C::ALLOC)) return INFINI_ERR_CUDA;
+    tc::SmallArgs a{beta, M0, z0, out, M_out, z_out, ticket, flags, agg, incl, p.L, (int)U, (int)p.H};
+    TRACED("small_fused", st);
+    tc::k_small_linear_fused<<<(unsigned)units, 256, C::ALLOC, st>>>(mq, mk, mv, a);
+    return INFINI_OK;
+}
+
 template <typename T, int D>
 int launch_all(const Problem &p, const T *q, const T *k, const T *v, const float *beta,
                const float *M0, const float *z0, T *out, float *M_out, float *z_out,
                float *snapM, float *snapZ, __nv_bfloat16 *snapMb, cudaStream_t st)
 {
+    if constexpr (sizeof(T) == 2 && D == 64) {
+        if (use_small_fused<T>(p)) {
+            const int rc = launch_small_fused(p, q, k, v, beta, M0, z0, out, M_out, z_out, snapM, st);
+            if (rc != INFINI_OK) return rc;
+            return cudaGetLastError() == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
+        }
+    }
     const int64_t chains = p.B * p.Hkv;
     const int S = (int)p.S, N = (int)p.N;
     const int64_t per = (int64_t)D * D + D;
@@ -319,6 +428,35 @@ int launch_all(const Problem &p, const T *q, const T *k, const T *v, const float
     return cudaGetLastError() == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
 }
 
+// The library's own stream-ordered pool on the current device.  Its release threshold keeps
+// freed workspace mapped between calls, so a steady stream of same-sized calls does not
+// return memory to the driver and map it again every time.
+cudaMemPool_t workspace_pool()
+{
+    constexpr int kMaxDevices = 64;
+    static cudaMemPool_t pools[kMaxDevices];
+    static std::mutex mu_pool;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> g(mu_pool);
+    if (!pools[dev]) {
+        cudaMemPoolProps props = {};
+        props.allocType = cudaMemAllocationTypePinned;
+        props.handleTypes = cudaMemHandleTypeNone;
+        props.location.type = cudaMemLocationTypeDevice;
+        props.location.id = dev;
+        cudaMemPool_t pool = nullptr;
+        if (cudaMemPoolCreate(&pool, &props) != cudaSuccess) {
+            cudaGetLastError();
+            return nullptr;
+        }
+        uint64_t keep = UINT64_MAX;
+        cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+        pools[dev] = pool;
+    }
+    return pools[dev];
+}
+
 template <typename T>
 int forward(const void *q, const void *k, const void *v, const float *beta, const float *M0,
             const float *z0, void *out, float *M_out, float *z_out, int64_t B, int64_t H,
@@ -333,9 +471,11 @@ int forward(const void *q, const void *k, const void *v, const float *beta, cons
 
     const int64_t nM = p.B * p.Hkv * p.S * p.d * p.d, nZ = p.B * p.Hkv * p.S * p.d;
     const bool tc_path = use_tc<T>(p);
-    const size_t bytes = (size_t)(nM + nZ) * sizeof(float) + (tc_path ? (size_t)nM * 2 : 0);
+    const size_t bytes = (size_t)workspace_bytes(p.B, p.Hkv, p.S, p.N, p.d);
     void *ws = nullptr;
-    if (cudaMallocAsync(&ws, bytes, st) != cudaSuccess) {
+    cudaMemPool_t pool = workspace_pool();
+    if (!pool) return INFINI_ERR_CUDA;
+    if (cudaMallocFromPoolAsync(&ws, bytes, pool, st) != cudaSuccess) {
         cudaGetLastError();
         return INFINI_ERR_OOM;
     }
@@ -389,7 +529,7 @@ int forward_noalloc(const void *q, const void *k, const void *v, const float *be
     if (rc != INFINI_OK) return rc;
     const int64_t nM = p.B * p.Hkv * p.S * p.d * p.d, nZ = p.B * p.Hkv * p.S * p.d;
     const bool tc_path = use_tc<T>(p);
-    const size_t bytes = (size_t)(nM + nZ) * sizeof(float) + (tc_path ? (size_t)nM * 2 : 0);
+    const size_t bytes = (size_t)workspace_bytes(p.B, p.Hkv, p.S, p.N, p.d);
     if (bytes > kNoAllocScratchBytes) return INFINI_ERR_UNSUPPORTED;
     void *ws = noalloc_scratch_address();
     if (!ws) return INFINI_ERR_CUDA;
@@ -444,10 +584,7 @@ int infini_attn_fwd_f32(const void *q, const void *k, const void *v, const float
 int64_t infini_attn_workspace_bytes(int64_t B, int64_t Hkv, int64_t L, int64_t N, int64_t d)
 {
     if (B <= 0 || Hkv <= 0 || L <= 0 || N <= 0 || d <= 0 || L % N != 0) return 0;
-    const int64_t S = L / N;
-    int64_t bytes = B * Hkv * S * (d * d + d) * (int64_t)sizeof(float);
-    if ((d == 64 || d == 128) && N % 128 == 0) bytes += B * Hkv * S * d * d * 2;   // bf16 copies
-    return bytes;
+    return infini::workspace_bytes(B, Hkv, L / N, N, d);
 }
 
 const char *infini_attn_status_string(int status)
@@ -484,8 +621,9 @@ int infini_attn_trace_enable(int on)
     std::lock_guard<std::mutex> g(mu);
     if (on) {   // a new trace: drop pending records and the accumulated table
         for (const Rec &r : recs) {
-            cudaEventDestroy(r.a);
-            cudaEventDestroy(r.b);
+            cudaEventSynchronize(r.b);
+            give_event(r.a);
+            give_event(r.b);
         }
         recs.clear();
         names.clear();
@@ -505,8 +643,8 @@ int64_t infini_attn_trace_report(char *buf, int64_t len)
         float t = 0.f;
         if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&t, r.a, r.b) != cudaSuccess)
             failed = true;
-        cudaEventDestroy(r.a);
-        cudaEventDestroy(r.b);
+        give_event(r.a);
+        give_event(r.b);
         size_t i = 0;
         while (i < names.size() && names[i] != r.name) ++i;
         if (i == names.size()) {

@@ -7,21 +7,23 @@
 //   M_s   = M_{s-1} + sigma(K_s)^T U_s,      z_s = z_{s-1} + sum_t sigma(k_t)
 // The update of value column e needs only column e of M_{s-1}, column e of V_s and the shared
 // z, so each CTA owns CB = 16 value columns of one chain and walks all segments; the chain's
-// D/16 CTAs run side by side.  Per 128-token chunk:
-//   1. TMA brings K (128 x d, 128-byte swizzle) and V[:, cols] (128 x 16) into a stage.
-//   2. The compute warpgroup (thread t = token t) overwrites its K row with sigma(K) in bf16.
-//   3. One thread issues R = sigma(K) [M_{s-1}^T | z_{s-1}]^T with M and z split into bf16
-//      hi + lo parts (two accumulating MMAs, N = 32): columns 0..15 are the prediction
-//      numerators, column 16 is den_t.
-//   4. Thread t forms U_t and writes U^T split into bf16 hi + lo parts (the residual is a
-//      small difference of large terms, so one bf16 rounding of it would cost ~1e-2 of M),
-//      next to a constant row of ones (hi part) / zeros (lo part).
-//   5. One thread issues Macc += sigma(K)^T [U_hi | 1] + sigma(K)^T [U_lo | 0] (sigma(K) read
-//      as the MN-major operand): columns 0..15 of the TMEM accumulator carry M[:, cols] in
-//      fp32, column 16 carries z.
-// At each segment end thread c (TMEM lane c = key feature c) reads its row of Macc, publishes
-// the bf16 snapshot M_s[c, cols] (and z_s from the chain's first CTA) for the segment kernel,
-// and refreshes the hi/lo operand copies.  d = 64 runs as d = 128 with zero columns.
+// d/16 CTAs run side by side.  sigma(K) is computed once per token beforehand
+// (k_sigma_bf16) and read here through TMA.  Per 128-token chunk g:
+//   1. TMA brings sigma(K) (128 x d, 128-byte swizzle) and V[:, cols] (128 x 16).
+//   2. One thread issues R = sigma(K) B^T with B = [M^T | z | 0 | M_lo^T | z_lo | 0] (64 rows,
+//      bf16: M and z split into hi + lo parts, side by side so one N = 64 MMA reads the
+//      sigma(K) tile once): R[0..15] + R[32..47] are the prediction numerators, R[16] + R[48]
+//      is den_t.
+//   3. Thread t forms U_t and writes [U_hi | 1 | 0 | U_lo | 0]^T (the residual is a small
+//      difference of large terms: one bf16 rounding of it would cost ~1e-2 of M).
+//   4. One thread issues Macc += sigma(K)^T [U_hi | 1 | 0 | U_lo | 0] (sigma(K) read as the
+//      MN-major operand): M[:, cols] = Macc[0..15] + Macc[32..47], z = Macc[16], in fp32.
+// Within a segment every R reads the same M_{s-1}, so R(g+1) is issued before the update of
+// chunk g (R accumulators and U tiles double-buffered); only the first chunk of a segment
+// waits for B (the initial state, or the boundary where thread c -- TMEM lane c = key
+// feature c -- reads its row of Macc,
+// publishes the bf16 snapshot M_s[c, cols] (and z_s from the chain's first CTA) for the
+// segment kernel, and rewrites the B operand).  d = 64 runs as d = 128 with zero features.
 // All waits are bounded (tc_common.cuh).
 #pragma once
 
@@ -30,28 +32,48 @@
 namespace infini {
 namespace tc {
 
+// sigma(x) = ELU(x) + 1 of every element, bf16 in and out, 8 elements per thread and step.
+__global__ void __launch_bounds__(256)
+k_sigma_bf16(const __nv_bfloat16 *__restrict__ x, __nv_bfloat16 *__restrict__ y, int64_t n8)
+{
+    const uint4 *src = reinterpret_cast<const uint4 *>(x);
+    uint4 *dst = reinterpret_cast<uint4 *>(y);
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n8;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        uint4 v = src[i];
+        uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            __nv_bfloat162 t = *reinterpret_cast<__nv_bfloat162 *>(&w[e]);
+            float a = __low2float(t), b = __high2float(t);
+            a = a > 0.f ? a + 1.f : __expf(a);
+            b = b > 0.f ? b + 1.f : __expf(b);
+            w[e] = pack_bf16x2(a, b);
+        }
+        dst[i] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+}
+
 struct ChainCfg {
     static constexpr int CB = 16;                 // value columns per CTA
-    static constexpr int NB = 32;                 // rows of the B operands: 16 + z/ones + pad
-    static constexpr int ST = 2;                  // K/V stages
+    static constexpr int NB = 64;                 // rows of the B operands (hi half, lo half)
+    static constexpr int LO = 32;                 // first row of the lo half
+    static constexpr int ST = 4;                  // sigma(K)/V stages
     static constexpr int KBOX = 128 * 128;        // 128 rows x 64 bf16
     static constexpr int KTILE = 2 * KBOX;        // 128 tokens x 128 features (padded)
     static constexpr int VTILE = 128 * CB * 2;    // 128 tokens x 16 bf16, unswizzled
-    static constexpr int BBOX = NB * 128;         // 32 rows x 64 bf16
-    static constexpr int BTILE = 2 * BBOX;        // 32 rows x 128 (features or tokens)
+    static constexpr int BBOX = NB * 128;         // 64 rows x 64 bf16
+    static constexpr int BTILE = 2 * BBOX;        // 64 rows x 128 (features or tokens)
     static constexpr int OFF_K = 0;
     static constexpr int OFF_V = OFF_K + ST * KTILE;
-    static constexpr int OFF_BH = OFF_V + ST * VTILE;   // [M | z]^T hi   (32 x 128 features)
-    static constexpr int OFF_BL = OFF_BH + BTILE;       // [M | z]^T lo
-    static constexpr int OFF_U = OFF_BL + BTILE;        // [U_hi | 1]^T   (32 x 128 tokens)
-    static constexpr int OFF_UL = OFF_U + BTILE;        // [U_lo | 0]^T
-    static constexpr int OFF_BAR = OFF_UL + BTILE;
-    static constexpr int NBAR = 2 * ST + 5;
+    static constexpr int OFF_B = OFF_V + ST * VTILE;    // [M | z]^T, hi and lo halves
+    static constexpr int OFF_U = OFF_B + BTILE;         // 2 x [U | 1]^T, hi and lo halves
+    static constexpr int OFF_BAR = OFF_U + 2 * BTILE;
+    static constexpr int NBAR = 2 * ST + 8;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int BYTES = OFF_MISC + 16;
     static constexpr int ALLOC = BYTES + 1024;
-    static_assert(OFF_BH % 1024 == 0 && OFF_U % 1024 == 0 && OFF_UL % 1024 == 0,
-                  "operand tiles must be 1024-aligned");
+    static_assert(OFF_B % 1024 == 0 && OFF_U % 1024 == 0, "operand tiles must be 1024-aligned");
 };
 
 struct ChainArgs {
@@ -63,7 +85,7 @@ struct ChainArgs {
     int N, S;
 };
 
-enum : int { WC_KV_EMPTY = 201, WC_A = 202, WC_U = 203, WC_KV_FULL = 204, WC_R = 205,
+enum : int { WC_KV_EMPTY = 201, WC_B = 202, WC_U = 203, WC_KV_FULL = 204, WC_R = 205,
              WC_UPD = 206, WC_DRAIN = 207 };
 
 __device__ __forceinline__ void chain_drain(uint64_t *bar, uint32_t parity)
@@ -77,11 +99,9 @@ __device__ __forceinline__ void chain_drain(uint64_t *bar, uint32_t parity)
     }
 }
 
-__device__ __forceinline__ float sigma_f(float x) { return x > 0.f ? x + 1.f : __expf(x); }
-
 template <int D>
 __global__ void __launch_bounds__(256, 1)
-k_delta_chain_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+k_delta_chain_tc(const __grid_constant__ CUtensorMap tmSK, const __grid_constant__ CUtensorMap tmV,
                  const ChainArgs a)
 {
     static_assert(D == 64 || D == 128, "tensor-core delta chain: d = 64 or 128");
@@ -100,14 +120,12 @@ k_delta_chain_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
 
     uint8_t *sK = smem + C::OFF_K;
     uint8_t *sV = smem + C::OFF_V;
-    uint8_t *sBH = smem + C::OFF_BH;
-    uint8_t *sBL = smem + C::OFF_BL;
+    uint8_t *sB = smem + C::OFF_B;
     uint8_t *sU = smem + C::OFF_U;
-    uint8_t *sUL = smem + C::OFF_UL;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
     uint64_t *kv_full = bars, *kv_empty = bars + ST;
-    uint64_t *a_ready = bars + 2 * ST, *r_full = a_ready + 1, *u_ready = r_full + 1;
-    uint64_t *upd_done = u_ready + 1, *mma_done = upd_done + 1;
+    uint64_t *r_full = bars + 2 * ST, *u_ready = r_full + 2, *upd_done = u_ready + 2;
+    uint64_t *b_ready = upd_done + 2, *mma_done = b_ready + 1;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
     volatile int *abort = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
 
@@ -116,25 +134,28 @@ k_delta_chain_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
             mbar_init(kv_full + i, 1);
             mbar_init(kv_empty + i, 1);
         }
-        mbar_init(a_ready, 128);
-        mbar_init(r_full, 1);
-        mbar_init(u_ready, 128);
-        mbar_init(upd_done, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(r_full + i, 1);
+            mbar_init(u_ready + i, 128);
+            mbar_init(upd_done + i, 1);
+        }
+        mbar_init(b_ready, 128);
         mbar_init(mma_done, 1);
         *abort = 0;
         fence_barrier_init();
     }
-    if (warp == 1) tmem_alloc(tmem_holder, 64);
+    if (warp == 1) tmem_alloc(tmem_holder, 256);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
-    const uint32_t T_M = tmem, T_R = tmem + 32;
+    const uint32_t T_M = tmem;
+    const uint32_t T_R[2] = {tmem + 64, tmem + 128};
 
     if (warp == 0) {
         if (lane == 0) {
             // ------------------------------------------------------------ producer
-            prefetch_tmap(&tmK);
+            prefetch_tmap(&tmSK);
             prefetch_tmap(&tmV);
             int issued = 0;
             for (int g = 0; g < total; ++g) {
@@ -144,7 +165,7 @@ k_delta_chain_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
                 const int row = s * a.N + i * 128;
                 mbar_arrive_expect_tx(kv_full + st, (uint32_t)(D * 128 * 2 + C::VTILE));
                 for (int kb = 0; kb < D / 64; ++kb)
-                    tma_load_3d(sK + st * C::KTILE + kb * C::KBOX, &tmK, kv_full + st, kb * 64, row,
+                    tma_load_3d(sK + st * C::KTILE + kb * C::KBOX, &tmSK, kv_full + st, kb * 64, row,
                                 (int)chain);
                 tma_load_3d(sV + st * C::VTILE, &tmV, kv_full + st, cb, row, (int)chain);
                 issued = g + 1;
@@ -157,45 +178,48 @@ k_delta_chain_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
         if (lane == 0) {
             // ------------------------------------------------------------ MMA issuer
             constexpr uint32_t idR = idesc_bf16(128, C::NB, 0, 0);   // sigma(K) . B^T
-            constexpr uint32_t idU = idesc_bf16(128, C::NB, 1, 0);   // sigma(K)^T . [U|1]
-            const uint32_t aK = smem_u32(sK), aBH = smem_u32(sBH), aBL = smem_u32(sBL);
-            const uint32_t aU = smem_u32(sU), aUL = smem_u32(sUL);
-            for (int g = 0; g < total; ++g) {
-                const int st = g % ST;
-                if (!mbar_wait(a_ready, g & 1, abort, WC_A)) break;
+            constexpr uint32_t idU = idesc_bf16(128, C::NB, 1, 0);   // sigma(K)^T . [U | 1]
+            const uint32_t aK = smem_u32(sK), aB = smem_u32(sB), aU = smem_u32(sU);
+            auto issue_r = [&](int g) -> bool {
+                // the first chunk of segment s waits for B holding M_{s-1}: phase 0 is the
+                // initial state written in the prologue, phase s the boundary after segment s-1
+                if (g % nch == 0 && !mbar_wait(b_ready, (g / nch) & 1, abort, WC_B))
+                    return false;
+                if (!mbar_wait(kv_full + g % ST, (g / ST) & 1, abort, WC_KV_FULL)) return false;
                 tc_fence_after();
-                const uint32_t kbase = aK + st * C::KTILE;
+                const uint32_t kbase = aK + (g % ST) * C::KTILE;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {        // K = 128 features in steps of 16
                     const uint32_t off = (kk >> 2) * C::KBOX + (kk & 3) * 32;
                     const uint32_t boff = (kk >> 2) * C::BBOX + (kk & 3) * 32;
-                    mma_ss(T_R, sdesc_sw128(kbase + off, 16, 1024), sdesc_sw128(aBH + boff, 16, 1024),
-                           idR, kk > 0 ? 1u : 0u);
+                    mma_ss(T_R[g & 1], sdesc_sw128(kbase + off, 16, 1024),
+                           sdesc_sw128(aB + boff, 16, 1024), idR, kk > 0 ? 1u : 0u);
                 }
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t off = (kk >> 2) * C::KBOX + (kk & 3) * 32;
-                    const uint32_t boff = (kk >> 2) * C::BBOX + (kk & 3) * 32;
-                    mma_ss(T_R, sdesc_sw128(kbase + off, 16, 1024), sdesc_sw128(aBL + boff, 16, 1024),
-                           idR, 1u);
-                }
-                mma_commit(r_full);
-                if (!mbar_wait(u_ready, g & 1, abort, WC_U)) break;
+                mma_commit(r_full + (g & 1));
+                return true;
+            };
+            auto issue_update = [&](int g) -> bool {
+                const int bb = g & 1;
+                if (!mbar_wait(u_ready + bb, (g >> 1) & 1, abort, WC_U)) return false;
                 tc_fence_after();
+                const uint32_t kbase = aK + (g % ST) * C::KTILE;
+                const uint32_t ub = aU + bb * C::BTILE;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {        // K = 128 tokens in steps of 16
                     const uint64_t ad = sdesc_sw128(kbase + kk * 2048, C::KBOX, 1024);
                     const uint32_t boff = (kk >> 2) * C::BBOX + (kk & 3) * 32;
-                    mma_ss(T_M, ad, sdesc_sw128(aU + boff, 16, 1024), idU, 1u);
+                    mma_ss(T_M, ad, sdesc_sw128(ub + boff, 16, 1024), idU, 1u);
                 }
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint64_t ad = sdesc_sw128(kbase + kk * 2048, C::KBOX, 1024);
-                    const uint32_t boff = (kk >> 2) * C::BBOX + (kk & 3) * 32;
-                    mma_ss(T_M, ad, sdesc_sw128(aUL + boff, 16, 1024), idU, 1u);
-                }
-                mma_commit(kv_empty + st);
-                mma_commit(upd_done);
+                mma_commit(kv_empty + g % ST);
+                mma_commit(upd_done + bb);
+                return true;
+            };
+            bool ok = issue_r(0);
+            for (int g = 0; ok && g < total; ++g) {
+                const bool next_starts_segment = (g + 1) % nch == 0;
+                if (g + 1 < total && !next_starts_segment) ok = issue_r(g + 1);
+                if (ok) ok = issue_update(g);
+                if (ok && g + 1 < total && next_starts_segment) ok = issue_r(g + 1);
             }
             mma_commit(mma_done);
             chain_drain(mma_done, 0);
@@ -205,30 +229,31 @@ k_delta_chain_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
         const int r = threadIdx.x - 128;           // token row of a chunk / key feature row
         const uint32_t lane_base = (uint32_t)((warp - 4) * 32) << 16;
         const __nv_bfloat16 one = __float2bfloat16_rn(1.f), zero = __float2bfloat16_rn(0.f);
-        // constant rows: [U_hi | 1]^T row 16 = ones, rows 17..31 = zeros; [U_lo | 0]^T rows
-        // 16..31 = zeros (both token boxes)
-        for (int i = r; i < 2 * 16 * 64; i += 128) {
-            const int box = i / (16 * 64), rr = 16 + (i / 64) % 16, t = i % 64;
-            const int o = box * C::BBOX + rr * 128 + ((((t >> 3) ^ (rr & 7))) << 4) + (t & 7) * 2;
-            *reinterpret_cast<__nv_bfloat16 *>(sU + o) = rr == 16 ? one : zero;
-            *reinterpret_cast<__nv_bfloat16 *>(sUL + o) = zero;
+        // constant rows of both [U | 1]^T tiles: 16 = ones, 17..31 and 48..63 = zeros
+        for (int i = r; i < 2 * 2 * 32 * 64; i += 128) {
+            const int buf = i / (2 * 32 * 64), box = (i / (32 * 64)) % 2, k32 = (i / 64) % 32;
+            const int rr = k32 < 16 ? 16 + k32 : 32 + k32;          // 16..31, 48..63
+            const int t = i % 64;
+            *reinterpret_cast<__nv_bfloat16 *>(sU + buf * C::BTILE + box * C::BBOX + rr * 128 +
+                                               ((((t >> 3) ^ (rr & 7))) << 4) + (t & 7) * 2) =
+                rr == 16 ? one : zero;
         }
-        if (D == 64)   // the padded feature box of every K stage stays zero
+        if (D == 64)   // the padded feature box of every stage stays zero
             for (int i = r; i < ST * C::KBOX / 16; i += 128) {
                 const int st = i / (C::KBOX / 16), o = i % (C::KBOX / 16);
                 reinterpret_cast<uint4 *>(sK + st * C::KTILE + C::KBOX)[o] = make_uint4(0, 0, 0, 0);
             }
-        // initial state: lane/row c = r holds [M0[c, cols] | z0[c] | 0 ...]
+        // column c of B: rows 0..15 = M[c, cols] hi, 16 = z[c] hi, 32..47 / 48 = lo parts
         auto write_b_col = [&](int c, const float *m16, float zc) {
-            // column c of the 32 x 128 hi / lo operands, rows 0..15 = M, 16 = z, 17.. = 0
             const int box = c >> 6, cc = c & 63;
-            for (int e = 0; e < C::NB; ++e) {
+#pragma unroll 1
+            for (int e = 0; e < C::LO; ++e) {
                 const float x = e < CB ? m16[e] : (e == CB ? zc : 0.f);
                 const __nv_bfloat16 hi = __float2bfloat16_rn(x);
                 const __nv_bfloat16 lo = __float2bfloat16_rn(x - __bfloat162float(hi));
-                const int o = box * C::BBOX + e * 128 + ((((cc >> 3) ^ (e & 7))) << 4) + (cc & 7) * 2;
-                *reinterpret_cast<__nv_bfloat16 *>(sBH + o) = hi;
-                *reinterpret_cast<__nv_bfloat16 *>(sBL + o) = lo;
+                const int o = box * C::BBOX + ((((cc >> 3) ^ (e & 7))) << 4) + (cc & 7) * 2;
+                *reinterpret_cast<__nv_bfloat16 *>(sB + o + e * 128) = hi;
+                *reinterpret_cast<__nv_bfloat16 *>(sB + o + (C::LO + e) * 128) = lo;
             }
         };
         {
@@ -247,38 +272,21 @@ k_delta_chain_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
             for (int e = 0; e < 32; ++e)
                 acc[e] = __float_as_uint(e < CB ? m16[e] : (e == CB ? zc : 0.f));
             tmem_st32(lane_base + T_M, acc);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) acc[e] = 0u;
+            tmem_st32(lane_base + T_M + 32, acc);
             tmem_st_wait();
             write_b_col(r, m16, zc);
         }
         fence_proxy_async_smem();
         tc_fence_before();
-        asm volatile("bar.sync 1, 128;" ::: "memory");
+        mbar_arrive(b_ready);                       // B holds the initial state
 
         bool ok = true;
         for (int g = 0; ok && g < total; ++g) {
-            const int st = g % ST, s = g / nch, i = g % nch;
+            const int st = g % ST, s = g / nch, i = g % nch, bb = g & 1;
             if (!(ok = mbar_wait(kv_full + st, (g / ST) & 1, abort, WC_KV_FULL))) break;
-            // sigma(K) in place, row r
-            uint8_t *krow = sK + st * C::KTILE;
-#pragma unroll
-            for (int kb = 0; kb < D / 64; ++kb) {
-#pragma unroll
-                for (int ch = 0; ch < 8; ++ch) {
-                    uint4 *p = reinterpret_cast<uint4 *>(krow + kb * C::KBOX + r * 128 +
-                                                         ((ch ^ (r & 7)) << 4));
-                    uint4 v = *p;
-                    uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        __nv_bfloat162 t2 = *reinterpret_cast<__nv_bfloat162 *>(&w[e]);
-                        w[e] = pack_bf16x2(sigma_f(__low2float(t2)), sigma_f(__high2float(t2)));
-                    }
-                    *p = make_uint4(w[0], w[1], w[2], w[3]);
-                }
-            }
-            fence_proxy_async_smem();
-            mbar_arrive(a_ready);
-            // this token's 16 values of V
+            // this token's 16 values of V in chunk g
             float vv[CB];
             {
                 const uint4 *vp = reinterpret_cast<const uint4 *>(sV + st * C::VTILE + r * CB * 2);
@@ -291,41 +299,44 @@ k_delta_chain_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
                     vv[2 * e + 1] = __high2float(t2);
                 }
             }
-            if (!(ok = mbar_wait(r_full, g & 1, abort, WC_R))) break;
+            if (!(ok = mbar_wait(r_full + bb, (g >> 1) & 1, abort, WC_R))) break;
             tc_fence_after();
-            uint32_t rr[32];
-            tmem_ld32(lane_base + T_R, rr);
+            uint32_t rh[32], rl[32];
+            tmem_ld32(lane_base + T_R[bb], rh);
+            tmem_ld32(lane_base + T_R[bb] + C::LO, rl);
             tmem_ld_wait();
-            const float den = __uint_as_float(rr[CB]);
+            const float den = __uint_as_float(rh[CB]) + __uint_as_float(rl[CB]);
             const float inv = den == 0.f ? 0.f : 1.f / den;
-            // sU is free once the previous chunk's update has completed
-            if (g > 0 && !(ok = mbar_wait(upd_done, (g - 1) & 1, abort, WC_UPD))) break;
+            // U tile bb is free once the update of chunk g-2 has completed
+            if (g >= 2 && !(ok = mbar_wait(upd_done + bb, ((g >> 1) - 1) & 1, abort, WC_UPD))) break;
             {
                 const int box = r >> 6, tt = r & 63;
+                uint8_t *ub = sU + bb * C::BTILE + box * C::BBOX + (tt & 7) * 2;
 #pragma unroll
                 for (int e = 0; e < CB; ++e) {
-                    const float u = vv[e] - __uint_as_float(rr[e]) * inv;
+                    const float u = vv[e] - (__uint_as_float(rh[e]) + __uint_as_float(rl[e])) * inv;
                     const __nv_bfloat16 hi = __float2bfloat16_rn(u);
-                    const int o = box * C::BBOX + e * 128 + ((((tt >> 3) ^ (e & 7))) << 4) + (tt & 7) * 2;
-                    *reinterpret_cast<__nv_bfloat16 *>(sU + o) = hi;
-                    *reinterpret_cast<__nv_bfloat16 *>(sUL + o) =
+                    const int o = ((((tt >> 3) ^ (e & 7))) << 4);
+                    *reinterpret_cast<__nv_bfloat16 *>(ub + o + e * 128) = hi;
+                    *reinterpret_cast<__nv_bfloat16 *>(ub + o + (C::LO + e) * 128) =
                         __float2bfloat16_rn(u - __bfloat162float(hi));
                 }
             }
             fence_proxy_async_smem();
             tc_fence_before();
-            mbar_arrive(u_ready);
+            mbar_arrive(u_ready + bb);
 
             if (i == nch - 1) {
                 // segment end: M_s, z_s from the accumulator (lane r = key feature r)
-                if (!(ok = mbar_wait(upd_done, g & 1, abort, WC_UPD))) break;
+                if (!(ok = mbar_wait(upd_done + bb, (g >> 1) & 1, abort, WC_UPD))) break;
                 tc_fence_after();
-                uint32_t acc[32];
+                uint32_t acc[32], acl[32];
                 tmem_ld32(lane_base + T_M, acc);
+                tmem_ld32(lane_base + T_M + C::LO, acl);
                 tmem_ld_wait();
                 float m16[CB];
 #pragma unroll
-                for (int e = 0; e < CB; ++e) m16[e] = __uint_as_float(acc[e]);
+                for (int e = 0; e < CB; ++e) m16[e] = __uint_as_float(acc[e]) + __uint_as_float(acl[e]);
                 const float zc = __uint_as_float(acc[CB]);
                 if (r < D) {
                     if (s + 1 < a.S) {
@@ -345,8 +356,12 @@ k_delta_chain_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
                         if (cb == 0) a.z_out[chain * D + r] = zc;
                     }
                 }
-                write_b_col(r, m16, zc);
-                fence_proxy_async_smem();
+                if (g + 1 < total) {
+                    write_b_col(r, m16, zc);
+                    fence_proxy_async_smem();
+                    tc_fence_before();
+                    mbar_arrive(b_ready);           // R of the next segment may read M_s
+                }
             }
         }
     }
@@ -355,7 +370,7 @@ k_delta_chain_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, 64);
+        tmem_dealloc(tmem, 256);
     }
 }
 

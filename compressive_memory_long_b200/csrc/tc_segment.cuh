@@ -258,14 +258,18 @@ k_segment_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
             tmem_ld32(tS + 64, raw[2]);
             tmem_ld32(tS + 96, raw[3]);
             tmem_ld_wait();
-            float mt = -INFINITY;
+            if (j == qt) {                                  // causal mask on the diagonal tile
 #pragma unroll
-            for (int c = 0; c < 128; ++c) {
-                float x = __uint_as_float(raw[c >> 5][c & 31]);
-                if (j == qt && c > r) x = -INFINITY;        // causal mask on the diagonal tile
-                raw[c >> 5][c & 31] = __float_as_uint(x);
-                mt = fmaxf(mt, x);
+                for (int c = 0; c < 128; ++c)
+                    if (c > r) raw[c >> 5][c & 31] = __float_as_uint(-INFINITY);
             }
+            float pm[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) pm[u] = __uint_as_float(raw[0][u]);
+#pragma unroll
+            for (int c = 8; c < 128; ++c) pm[c & 7] = fmaxf(pm[c & 7], __uint_as_float(raw[c >> 5][c & 31]));
+            const float mt = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                                   fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
             // PV_{j-1} must be complete before O is rescaled or P is rewritten
             if (j > 0 && !(ok = mbar_wait(pv_done, (j - 1) & 1, abort, W_PV))) break;
             tc_fence_after();
@@ -288,16 +292,16 @@ k_segment_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
                 }
             }
             const float mk = m_used * kscale;
-            float rs = 0.f;
+            float ps[4] = {0.f, 0.f, 0.f, 0.f};
             uint32_t pk[2][32];
 #pragma unroll
             for (int c = 0; c < 128; c += 2) {
                 const float p0 = ex2(fmaf(__uint_as_float(raw[c >> 5][c & 31]), kscale, -mk));
                 const float p1 = ex2(fmaf(__uint_as_float(raw[(c + 1) >> 5][(c + 1) & 31]), kscale, -mk));
-                rs += p0 + p1;
+                ps[(c >> 1) & 3] += p0 + p1;
                 pk[c >> 6][(c >> 1) & 31] = pack_bf16x2(p0, p1);
             }
-            l += rs;
+            l += (ps[0] + ps[1]) + (ps[2] + ps[3]);
             const uint32_t tP = lane_base + ((j & 1) ? T_P1 : T_P0);
             tmem_st32(tP, pk[0]);
             tmem_st32(tP + 32, pk[1]);

@@ -8,7 +8,9 @@
 // both read the same K/V tiles, which are loaded once.  Tile B needs key tiles 0..2p+1,
 // tile A 0..2p.  Two softmax warpgroups (A: warps 0-3, B: warps 4-7) work in ping-pong
 // with the tensor core: while one warpgroup turns its S tile into P, the MMA thread
-// (warp 9) runs the other tile's P V and Q K^T.  TMA producer: warp 8.
+// (warp 9) runs the other tile's P V and Q K^T.  TMA producer: warp 8; warps 10-11 idle.
+// The third warpgroup hands registers to the two softmax warpgroups (setmaxnreg), which
+// hold a full 128-score row each.
 //
 // TMEM (512 columns): S_A [0,128), S_B [128,256), O_A [256,256+d), O_B [256+d, 256+2d).
 // P (bf16) is written over the first 64 columns of its own S tile; S_X(j) is issued after
@@ -26,7 +28,12 @@ namespace tc {
 template <int D>
 struct Seg2Cfg {
     static_assert(D == 64 || D == 128, "tensor-core segment kernel: d = 64 or 128");
-    static constexpr int THREADS = 320;
+    static constexpr int THREADS = 384;
+    // register split (setmaxnreg): launched at REGS per thread; the producer / MMA warpgroup
+    // gives back to REGS_LOW, each softmax warpgroup grows to REGS_HIGH.  The three shares add
+    // up exactly to the launch's THREADS * REGS.
+    static constexpr int REGS = 168, REGS_LOW = 56, REGS_HIGH = 224;
+    static_assert(128 * (2 * REGS_HIGH + REGS_LOW) == THREADS * REGS, "register split");
     static constexpr int STAGES = (D == 128) ? 2 : 3;
     static constexpr int TILE = 128 * D * 2;
     static constexpr int BOX = 128 * 128;
@@ -71,7 +78,7 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
 }
 
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(384, 1)
 k_segment_tc2(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmM,
               const SegArgs a)
@@ -135,7 +142,9 @@ k_segment_tc2(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     const uint32_t T_S[2] = {tmem, tmem + 128};
     const uint32_t T_O[2] = {tmem + 256, tmem + 256 + D};
 
-    if (warp == 8) {
+    if (warp >= 8) {
+      asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::REGS_LOW));
+      if (warp == 8) {
         if (lane == 0) {
             // ------------------------------------------------------------ producer
             prefetch_tmap(&tmQ);
@@ -248,7 +257,9 @@ k_segment_tc2(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             mma_commit(mma_done);
             seg2_drain(mma_done, 0);
         }
-    } else if (warp < 8) {
+      }
+    } else {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::REGS_HIGH));
         // ---------------------------------------------------------------- softmax / epilogue
         const int x = warp >> 2;                          // 0: tile A, 1: tile B
         const int r = threadIdx.x & 127;                  // query row within the tile
@@ -266,21 +277,26 @@ k_segment_tc2(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             if (!(ok = mbar_wait(s_full + x, i & 1, abort, W2_S))) break;
             tc_fence_after();
             const bool diag = (i == qt);
-            // pass 1: row maximum
-            float mt = -INFINITY;
+            // the whole row of S in registers (one wait for four loads)
+            uint32_t v[4][32];
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                uint32_t c0[32], c1[32];
-                tmem_ld32(lane_base + T_S[x] + half * 64, c0);
-                tmem_ld32(lane_base + T_S[x] + half * 64 + 32, c1);
-                tmem_ld_wait();
+            for (int c = 0; c < 4; ++c) tmem_ld32(lane_base + T_S[x] + c * 32, v[c]);
+            tmem_ld_wait();
+            if (diag) {
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int col0 = half * 64 + e, col1 = col0 + 32;
-                    if (!(diag && col0 > r)) mt = fmaxf(mt, __uint_as_float(c0[e]));
-                    if (!(diag && col1 > r)) mt = fmaxf(mt, __uint_as_float(c1[e]));
-                }
+                for (int c = 0; c < 4; ++c)
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        if (c * 32 + e > r) v[c][e] = __float_as_uint(-INFINITY);
             }
+            // row maximum with eight independent partial maxima (no long dependency chain)
+            float pm[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) pm[u] = __uint_as_float(v[0][u]);
+#pragma unroll
+            for (int u = 8; u < 128; ++u) pm[u & 7] = fmaxf(pm[u & 7], __uint_as_float(v[u >> 5][u & 31]));
+            const float mt = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                                   fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
             const bool resc = (mt - m_used) * kscale > 8.f;
             float alpha = 1.f;
             if (resc) {
@@ -300,27 +316,22 @@ k_segment_tc2(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     tmem_st32(lane_base + T_O[x] + c, o);
                 }
             }
-            // pass 2: P = exp2((S - m) * scale) in bf16, written over the S tile's first columns
+            // P = exp2((S - m) * scale) in bf16, written over the S tile's first 64 columns
             const float mk = m_used * kscale;
-            float rs = 0.f;
-#pragma unroll 1
+            float ps[4] = {0.f, 0.f, 0.f, 0.f};     // independent partial row sums
+#pragma unroll
             for (int c = 0; c < 4; ++c) {
-                uint32_t v[32];
-                tmem_ld32(lane_base + T_S[x] + c * 32, v);
-                tmem_ld_wait();
                 uint32_t pk[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
-                    const int col = c * 32 + 2 * e;
-                    float p0 = ex2(fmaf(__uint_as_float(v[2 * e]), kscale, -mk));
-                    float p1 = ex2(fmaf(__uint_as_float(v[2 * e + 1]), kscale, -mk));
-                    if (diag && col > r) p0 = 0.f;
-                    if (diag && col + 1 > r) p1 = 0.f;
-                    rs += p0 + p1;
+                    const float p0 = ex2(fmaf(__uint_as_float(v[c][2 * e]), kscale, -mk));
+                    const float p1 = ex2(fmaf(__uint_as_float(v[c][2 * e + 1]), kscale, -mk));
+                    ps[e & 3] += p0 + p1;
                     pk[e] = pack_bf16x2(p0, p1);
                 }
                 tmem_st16(lane_base + T_S[x] + c * 16, pk);
             }
+            const float rs = (ps[0] + ps[1]) + (ps[2] + ps[3]);
             l += rs;
             tmem_st_wait();
             tc_fence_before();

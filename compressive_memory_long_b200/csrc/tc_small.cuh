@@ -1,0 +1,462 @@
+// Fused Infini-attention forward for 64-token segments and the additive memory rule, one
+// launch for the whole problem (sm_100a).
+//
+// The additive update (AI Wiki "Infini-Attention", "How does the compressive memory
+// work?") makes M_{s-1} = M0 + sum_{j<s} sigma(K_j)^T V_j a prefix sum ("What is linear
+// attention and the delta rule?"), so segments can be processed in parallel once each
+// knows the sum of its predecessors.  One CTA owns a unit of two consecutive segments
+// (128 tokens) of one head and:
+//   1. loads Q, K, V of the unit with TMA and forms sigma(K), sigma(Q) in shared memory;
+//   2. on the tensor cores: S = Q K^T over the unit (a 128 x 128 tile whose block-diagonal
+//      causal mask keeps each segment to its own keys, "What happens inside the
+//      Infini-attention block?"), and the per-segment increments
+//      [dM_s | dz_s] = sigma(K_s)^T [V_s | 1];
+//   3. publishes its aggregate dM_0 + dM_1 and finds the exclusive prefix M_start with a
+//      single-pass decoupled look-back over earlier units of the same head (Merrill and
+//      Garland, "Single-pass Parallel Prefix Scan with Decoupled Look-back", 2016): a
+//      predecessor's inclusive prefix ends the walk, its aggregate continues it;
+//   4. softmax and O = P V, then R_0 = sigma(Q) M_start and R_1 = sigma(Q) (M_start + dM_0)
+//      (rows of the first segment read R_0, rows of the second R_1), and the gated output.
+// Units take tickets in start order, so a CTA only waits for units that started before it
+// (running or finished): no unit waits on one that cannot run.  Every wait is bounded.
+// Layout limits: bf16, d = 64, N = 64, L % 128 == 0, one query head per key/value head.
+#pragma once
+
+#include "tc_common.cuh"
+
+namespace infini {
+namespace tc {
+
+struct SmallCfg {
+    static constexpr int D = 64, TOK = 128, SEG = 64;
+    static constexpr int BOX = 128 * 128;          // 128 rows x 64 bf16
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_K = OFF_Q + BOX;
+    static constexpr int OFF_V = OFF_K + BOX;      // V box, then a constant box (col 0 = 1)
+    static constexpr int OFF_SK = OFF_V + 2 * BOX; // sigma(K): features padded to 128
+    static constexpr int OFF_SQ = OFF_SK + 2 * BOX;
+    static constexpr int MB = 64 * 128;            // 64 key rows x 64 bf16 values
+    static constexpr int OFF_M0 = OFF_SQ + BOX;
+    static constexpr int OFF_M1 = OFF_M0 + MB;
+    static constexpr int OFF_Z = OFF_M1 + MB;      // z_start[64], z_mid[64] (fp32)
+    static constexpr int OFF_BAR = OFF_Z + 2 * 64 * 4;
+    static constexpr int NBAR = 10;
+    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+    static constexpr int BYTES = OFF_MISC + 32;
+    static constexpr int ALLOC = BYTES + 1024;
+    static constexpr int ROW = D + 1;              // floats per published state row
+};
+
+struct SmallArgs {
+    const float *beta;
+    const float *M0, *z0;          // may be NULL
+    __nv_bfloat16 *out;
+    float *M_out, *z_out;
+    int *ticket;                   // zeroed before the launch
+    int *flags;                    // [chains * U], zeroed before the launch
+    float *agg, *incl;             // [chains * U, D, D + 1]
+    int64_t L;
+    int U, H;
+};
+
+enum : int { FLAG_AGG = 1, FLAG_INCL = 2 };
+enum : int { WS_FULL = 501, WS_S = 502, WS_SIG = 503, WS_D = 504, WS_P = 505, WS_O = 506,
+             WS_M = 507, WS_R = 508, WS_LOOK = 509, WS_DRAIN = 510 };
+
+__device__ __forceinline__ void small_drain(uint64_t *bar, uint32_t parity)
+{
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity)) {
+        if (clock64() - t0 > kSpinLimitCycles) {
+            atomicCAS(&g_wait_status, 0, WS_DRAIN);
+            return;
+        }
+    }
+}
+
+__device__ __forceinline__ int ld_acquire_gpu(const int *p)
+{
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void st_release_gpu(int *p, int v)
+{
+    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ float sigma_s(float x) { return x > 0.f ? x + 1.f : __expf(x); }
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16])
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
+
+__global__ void __launch_bounds__(256, 1)
+k_small_linear_fused(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                     const __grid_constant__ CUtensorMap tmV, const SmallArgs a)
+{
+    using C = SmallCfg;
+    constexpr int D = C::D;
+    if (__syncthreads_or(threadIdx.x == 0 && wait_status_set())) return;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+    uint8_t *sQ = smem + C::OFF_Q, *sK = smem + C::OFF_K, *sV = smem + C::OFF_V;
+    uint8_t *sSK = smem + C::OFF_SK, *sSQ = smem + C::OFF_SQ;
+    uint8_t *sM0 = smem + C::OFF_M0, *sM1 = smem + C::OFF_M1;
+    float *sZ0 = reinterpret_cast<float *>(smem + C::OFF_Z), *sZ1 = sZ0 + 64;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
+    uint64_t *full = bars, *s_done = bars + 1, *sig_ready = bars + 2, *d_done = bars + 3;
+    uint64_t *p_ready = bars + 4, *o_done = bars + 5, *m_ready = bars + 6, *r_done = bars + 7;
+    uint64_t *mma_done = bars + 8;
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
+    volatile int *abort = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
+    volatile int *s_ticket = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 8);
+    volatile int *s_state = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 12);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        *s_ticket = atomicAdd(a.ticket, 1);
+        mbar_init(full, 1);
+        mbar_init(s_done, 1);
+        mbar_init(sig_ready, 128);
+        mbar_init(d_done, 1);
+        mbar_init(p_ready, 128);
+        mbar_init(o_done, 1);
+        mbar_init(m_ready, 128);
+        mbar_init(r_done, 1);
+        mbar_init(mma_done, 1);
+        *abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) tmem_alloc(tmem_holder, 512);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+    const uint32_t T_S = tmem, T_O = tmem + 128, T_R0 = tmem + 192, T_R1 = tmem + 256;
+    const uint32_t T_D0 = tmem + 320, T_D1 = tmem + 400;
+    const int t = *s_ticket;
+    const int64_t chain = t / a.U;          // = b * H + h (one query head per kv head)
+    const int unit = t % a.U;
+    const int64_t idx = chain * a.U + unit;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            prefetch_tmap(&tmQ);
+            prefetch_tmap(&tmK);
+            prefetch_tmap(&tmV);
+            mbar_arrive_expect_tx(full, 3 * C::BOX);
+            tma_load_3d(sQ, &tmQ, full, 0, unit * C::TOK, (int)chain);
+            tma_load_3d(sK, &tmK, full, 0, unit * C::TOK, (int)chain);
+            tma_load_3d(sV, &tmV, full, 0, unit * C::TOK, (int)chain);
+            if (*abort) small_drain(full, 0);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t idS = idesc_bf16(128, 128, 0, 0);
+            constexpr uint32_t idD = idesc_bf16(128, D + 16, 1, 1);
+            constexpr uint32_t idO = idesc_bf16(128, D, 0, 1);
+            const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
+            const uint32_t aSK = smem_u32(sSK), aSQ = smem_u32(sSQ);
+            const uint32_t aM0 = smem_u32(sM0), aM1 = smem_u32(sM1);
+            bool ok = mbar_wait(full, 0, abort, WS_FULL);
+            if (ok) {   // S = Q K^T over the unit
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk)
+                    mma_ss(T_S, sdesc_sw128(aQ + kk * 32, 16, 1024), sdesc_sw128(aK + kk * 32, 16, 1024),
+                           idS, kk > 0 ? 1u : 0u);
+                mma_commit(s_done);
+            }
+            if (ok) ok = mbar_wait(sig_ready, 0, abort, WS_SIG);
+            if (ok) {   // [dM_s | dz_s] = sigma(K_s)^T [V_s | 1], s = first and second segment
+                tc_fence_after();
+#pragma unroll
+                for (int seg = 0; seg < 2; ++seg)
+#pragma unroll
+                    for (int kk = 0; kk < C::SEG / 16; ++kk) {
+                        const uint32_t off = (seg * C::SEG + kk * 16) * 128;
+                        mma_ss(seg ? T_D1 : T_D0, sdesc_sw128(aSK + off, C::BOX, 1024),
+                               sdesc_sw128(aV + off, C::BOX, 1024), idD, kk > 0 ? 1u : 0u);
+                    }
+                mma_commit(d_done);
+            }
+            if (ok) ok = mbar_wait(p_ready, 0, abort, WS_P);
+            if (ok) {   // O = P V
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < C::TOK / 16; ++kk)
+                    mma_ts(T_O, T_S + kk * 8, sdesc_sw128(aV + kk * 2048, C::BOX, 1024), idO,
+                           kk > 0 ? 1u : 0u);
+                mma_commit(o_done);
+            }
+            if (ok) ok = mbar_wait(m_ready, 0, abort, WS_M);
+            if (ok) {   // R_0 = sigma(Q) M_start, R_1 = sigma(Q) M_mid
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    mma_ss(T_R0, sdesc_sw128(aSQ + kk * 32, 16, 1024),
+                           sdesc_sw128(aM0 + kk * 2048, C::MB, 1024), idO, kk > 0 ? 1u : 0u);
+                    mma_ss(T_R1, sdesc_sw128(aSQ + kk * 32, 16, 1024),
+                           sdesc_sw128(aM1 + kk * 2048, C::MB, 1024), idO, kk > 0 ? 1u : 0u);
+                }
+                mma_commit(r_done);
+            }
+            mma_commit(mma_done);
+            small_drain(mma_done, 0);
+        }
+    } else if (warp >= 4) {
+        const int r = threadIdx.x - 128;                 // row: token of the unit / feature
+        const uint32_t lane_base = (uint32_t)((warp - 4) * 32) << 16;
+        // constants: the box after V has column 0 = 1; the padded half of sigma(K) is 0
+        for (int i = r; i < 128 * 8; i += 128) {
+            const int row = i / 8, ch = i % 8;
+            *reinterpret_cast<uint4 *>(sV + C::BOX + row * 128 + ((ch ^ (row & 7)) << 4)) =
+                make_uint4(ch == 0 ? 0x3F80u : 0u, 0, 0, 0);
+            *reinterpret_cast<uint4 *>(sSK + C::BOX + row * 128 + ch * 16) = make_uint4(0, 0, 0, 0);
+        }
+        bool ok = mbar_wait(full, 0, abort, WS_FULL);
+        if (ok) {
+            // sigma(K) and sigma(Q) of row r (bf16, same swizzled position)
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch) {
+                const int o = r * 128 + ((ch ^ (r & 7)) << 4);
+                uint4 kq[2] = {*reinterpret_cast<const uint4 *>(sK + o), *reinterpret_cast<const uint4 *>(sQ + o)};
+                uint8_t *dst[2] = {sSK + o, sSQ + o};
+#pragma unroll
+                for (int w2 = 0; w2 < 2; ++w2) {
+                    uint32_t w[4] = {kq[w2].x, kq[w2].y, kq[w2].z, kq[w2].w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        __nv_bfloat162 t2 = *reinterpret_cast<__nv_bfloat162 *>(&w[e]);
+                        w[e] = pack_bf16x2(sigma_s(__low2float(t2)), sigma_s(__high2float(t2)));
+                    }
+                    *reinterpret_cast<uint4 *>(dst[w2]) = make_uint4(w[0], w[1], w[2], w[3]);
+                }
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(sig_ready);
+        }
+        // ---- local softmax over the unit's 128 x 128 scores (block-diagonal causal mask)
+        float l = 0.f;
+        if (ok) ok = mbar_wait(s_done, 0, abort, WS_S);
+        if (ok) {
+            tc_fence_after();
+            uint32_t v[4][32];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tmem_ld32(lane_base + T_S + c * 32, v[c]);
+            tmem_ld_wait();
+            const int lo = (r >> 6) << 6;                // first key of this row's segment
+            float mt = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const int col = c * 32 + e;
+                    if (col < lo || col > r) v[c][e] = __float_as_uint(-INFINITY);
+                    mt = fmaxf(mt, __uint_as_float(v[c][e]));
+                }
+            const float kscale = rsqrtf((float)D) * 1.4426950408889634f;
+            const float mk = mt * kscale;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const float p0 = ex2(fmaf(__uint_as_float(v[c][2 * e]), kscale, -mk));
+                    const float p1 = ex2(fmaf(__uint_as_float(v[c][2 * e + 1]), kscale, -mk));
+                    l += p0 + p1;
+                    pk[e] = pack_bf16x2(p0, p1);
+                }
+                asm volatile(
+                    "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+                    "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(lane_base + T_S + c * 16),
+                    "r"(pk[0]), "r"(pk[1]), "r"(pk[2]), "r"(pk[3]), "r"(pk[4]), "r"(pk[5]), "r"(pk[6]),
+                    "r"(pk[7]), "r"(pk[8]), "r"(pk[9]), "r"(pk[10]), "r"(pk[11]), "r"(pk[12]),
+                    "r"(pk[13]), "r"(pk[14]), "r"(pk[15])
+                    : "memory");
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(p_ready);
+        }
+        // ---- the memory: aggregate, look-back, the two states this unit reads
+        if (ok) ok = mbar_wait(d_done, 0, abort, WS_D);
+        float d0[C::ROW], agg[C::ROW];
+        if (ok) {
+            tc_fence_after();
+            uint32_t x0[32], x1[32], y0[32], y1[32];
+            uint32_t x2[16], y2[16];
+            tmem_ld32(lane_base + T_D0, x0);
+            tmem_ld32(lane_base + T_D0 + 32, x1);
+            tmem_ld16(lane_base + T_D0 + 64, x2);
+            tmem_ld32(lane_base + T_D1, y0);
+            tmem_ld32(lane_base + T_D1 + 32, y1);
+            tmem_ld16(lane_base + T_D1 + 64, y2);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                d0[j] = __uint_as_float(x0[j]);
+                d0[32 + j] = __uint_as_float(x1[j]);
+                agg[j] = d0[j] + __uint_as_float(y0[j]);
+                agg[32 + j] = d0[32 + j] + __uint_as_float(y1[j]);
+            }
+            d0[64] = __uint_as_float(x2[0]);
+            agg[64] = d0[64] + __uint_as_float(y2[0]);
+            if (r < D) {
+                float *dst = a.agg + (idx * D + r) * C::ROW;
+#pragma unroll
+                for (int j = 0; j < C::ROW; ++j) dst[j] = agg[j];
+            }
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        // Unit 0 publishes no aggregate, only its inclusive prefix: every other walk then ends
+        // at an inclusive prefix, and only unit 0 reads M0 / z0 -- which M_out / z_out (written
+        // by the last unit, after its walk) may alias.
+        if (ok && r == 0 && unit > 0) {
+            __threadfence();
+            st_release_gpu(a.flags + idx, FLAG_AGG);
+        }
+        // exclusive prefix: walk back over earlier units of this head
+        float ex[C::ROW];
+#pragma unroll
+        for (int j = 0; j < C::ROW; ++j) ex[j] = 0.f;
+        for (int j = unit - 1; ok && j >= 0; --j) {
+            if (r == 0) {
+                const int *fp = a.flags + chain * a.U + j;
+                int f = ld_acquire_gpu(fp);
+                const long long t0 = clock64();
+                while (f == 0) {
+                    if (clock64() - t0 > kSpinLimitCycles || wait_status_set()) {
+                        atomicCAS(&g_wait_status, 0, WS_LOOK);
+                        f = -1;
+                        break;
+                    }
+                    __nanosleep(64);
+                    f = ld_acquire_gpu(fp);
+                }
+                *s_state = f;
+            }
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            const int f = *s_state;
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            if (f < 0) {
+                ok = false;
+                *abort = 1;
+                break;
+            }
+            if (r < D) {
+                const float *src = (f == FLAG_INCL ? a.incl : a.agg) + ((chain * a.U + j) * D + r) * C::ROW;
+#pragma unroll
+                for (int q = 0; q < C::ROW; ++q) ex[q] += __ldcg(src + q);
+            }
+            if (f == FLAG_INCL) break;
+        }
+        if (ok && unit == 0 && r < D) {
+            if (a.M0)
+#pragma unroll 8
+                for (int q = 0; q < D; ++q) ex[q] += a.M0[(chain * D + r) * D + q];
+            if (a.z0) ex[D] += a.z0[chain * D + r];
+        }
+        if (ok) {
+            if (r < D) {
+                if (unit + 1 < a.U) {
+                    float *dst = a.incl + (idx * D + r) * C::ROW;
+#pragma unroll
+                    for (int q = 0; q < C::ROW; ++q) dst[q] = ex[q] + agg[q];
+                } else {
+                    float *mo = a.M_out + (chain * D + r) * D;
+#pragma unroll
+                    for (int q = 0; q < D; ++q) mo[q] = ex[q] + agg[q];
+                    a.z_out[chain * D + r] = ex[D] + agg[D];
+                }
+                // M_start and M_mid rows (key r) as bf16 B operands, z as fp32
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch) {
+                    uint32_t w0[4], w1[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int q = ch * 8 + 2 * e;
+                        w0[e] = pack_bf16x2(ex[q], ex[q + 1]);
+                        w1[e] = pack_bf16x2(ex[q] + d0[q], ex[q + 1] + d0[q + 1]);
+                    }
+                    const int o = r * 128 + ((ch ^ (r & 7)) << 4);
+                    *reinterpret_cast<uint4 *>(sM0 + o) = make_uint4(w0[0], w0[1], w0[2], w0[3]);
+                    *reinterpret_cast<uint4 *>(sM1 + o) = make_uint4(w1[0], w1[1], w1[2], w1[3]);
+                }
+                sZ0[r] = ex[D];
+                sZ1[r] = ex[D] + d0[D];
+            }
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            if (r == 0 && unit + 1 < a.U) {
+                __threadfence();
+                st_release_gpu(a.flags + idx, FLAG_INCL);
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(m_ready);
+        }
+        // ---- epilogue: gate the local and memory reads of row r
+        if (ok) ok = mbar_wait(o_done, 0, abort, WS_O);
+        if (ok) ok = mbar_wait(r_done, 0, abort, WS_R);
+        if (ok) {
+            tc_fence_after();
+            const float *zz = (r < C::SEG) ? sZ0 : sZ1;
+            float den = 0.f;
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch) {
+                const uint4 qv = *reinterpret_cast<const uint4 *>(sQ + r * 128 + ((ch ^ (r & 7)) << 4));
+                uint32_t w[4] = {qv.x, qv.y, qv.z, qv.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    __nv_bfloat162 t2 = *reinterpret_cast<__nv_bfloat162 *>(&w[e]);
+                    den = fmaf(sigma_s(__low2float(t2)), zz[ch * 8 + 2 * e], den);
+                    den = fmaf(sigma_s(__high2float(t2)), zz[ch * 8 + 2 * e + 1], den);
+                }
+            }
+            const int h = (int)(chain % a.H);
+            const float g = 1.f / (1.f + __expf(-a.beta[h]));
+            const float wl = (1.f - g) / l;
+            const float wm = den == 0.f ? 0.f : g / den;
+            const uint32_t tR = (r < C::SEG) ? T_R0 : T_R1;
+            __nv_bfloat16 *orow = a.out + (chain * a.L + (int64_t)unit * C::TOK + r) * D;
+#pragma unroll 1
+            for (int c = 0; c < D; c += 32) {
+                uint32_t o[32], rr0[32], rr1[32];
+                tmem_ld32(lane_base + T_O + c, o);
+                tmem_ld32(lane_base + T_R0 + c, rr0);
+                tmem_ld32(lane_base + T_R1 + c, rr1);
+                tmem_ld_wait();
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const float ra = __uint_as_float(tR == T_R0 ? rr0[2 * e] : rr1[2 * e]);
+                    const float rb = __uint_as_float(tR == T_R0 ? rr0[2 * e + 1] : rr1[2 * e + 1]);
+                    pk[e] = pack_bf16x2(fmaf(ra, wm, __uint_as_float(o[2 * e]) * wl),
+                                        fmaf(rb, wm, __uint_as_float(o[2 * e + 1]) * wl));
+                }
+                uint4 *dst = reinterpret_cast<uint4 *>(orow + c);
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+}  // namespace tc
+}  // namespace infini

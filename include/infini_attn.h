@@ -36,8 +36,9 @@
  *   - On an argument error nothing is launched and nothing is written.  Nothing aborts,
  *     throws or traps; every failure is an int status below.
  *   - Scratch: the call allocates its workspace (per-segment memory snapshots; the size
- *     is infini_attn_workspace_bytes) with cudaMallocAsync on `stream` and frees it with
- *     cudaFreeAsync on the same stream.
+ *     is infini_attn_workspace_bytes) stream-ordered on `stream` from a memory pool the
+ *     library owns on each device, and frees it on the same stream.  The pool keeps freed
+ *     memory for the next call (up to the largest workspace used so far).
  */
 #ifndef INFINI_ATTN_H
 #define INFINI_ATTN_H
@@ -123,7 +124,8 @@ INFINI_API int infini_attn_fwd_noalloc(const void *q, const void *k, const void 
                                        int64_t H, int64_t Hkv, int64_t L, int64_t N, int64_t d,
                                        int update_rule, infini_stream_t stream);
 
-/* Bytes of workspace one call allocates for these sizes (0 on invalid sizes). */
+/* Bytes of workspace one call allocates for these sizes (an upper bound over the kernels
+ * the call may choose; 0 on invalid sizes). */
 INFINI_API int64_t infini_attn_workspace_bytes(int64_t B, int64_t Hkv, int64_t L, int64_t N, int64_t d);
 
 /*

@@ -190,3 +190,45 @@ def test_tensor_core_first_segment_empty_memory():
     assert torch.count_nonzero(out[:, :, :256]) == 0
     assert torch.count_nonzero(out[:, :, 256:]) > 0
     assert binding.infini_attn_device_status() == 0
+
+
+# ---- the fused single-launch path (bf16, linear rule, N = 64, d = 64, MHA) -------------
+
+@pytest.mark.parametrize("S", [2, 4, 6, 16])
+def test_small_fused_shapes(S):
+    """One launch with the decoupled look-back: several units per head, nonzero state."""
+    from compressive_memory_long_b200 import binding
+    w = wl.Workload("small", B=2, H=3, Hkv=3, d=64, N=64, S=S, dtype="bf16", rule="linear",
+                    seed=23, beta_dist=("normal", 0.0, 1.5), M0_dist=("uniform", 0.0, 0.1),
+                    z0_dist=("uniform", 1.0, 2.0))
+    binding.infini_attn_trace_enable(True)
+    check_full(w)
+    binding.infini_attn_trace_enable(False)
+    assert list(binding.infini_attn_trace_report()) == ["small_fused"]
+    assert binding.infini_attn_device_status() == 0
+
+
+def test_small_fused_in_place_split():
+    from compressive_memory_long_b200 import binding
+    w = wl.Workload("small_split", B=1, H=2, Hkv=2, d=64, N=64, S=8, dtype="bf16",
+                    rule="linear", seed=24, beta_dist=("normal", 0.0, 1.0),
+                    M0_dist=("uniform", 0.0, 0.1), z0_dist=("uniform", 1.0, 2.0))
+    t = to_dev(wl.torch_inputs(w))
+    full, Mf, zf = binding.forward(t["q"], t["k"], t["v"], t["beta"], t["M0"], t["z0"], N=w.N,
+                                   rule=w.rule)
+    M, z = t["M0"].clone(), t["z0"].clone()
+    outs = []
+    for sl in (slice(0, 256), slice(256, 512)):
+        qs, ks, vs = (t[n][:, :, sl].contiguous() for n in ("q", "k", "v"))
+        o, _, _ = binding.forward(qs, ks, vs, t["beta"], M, z, N=w.N, rule=w.rule, M_out=M,
+                                  z_out=z)
+        outs.append(o)
+    torch.cuda.synchronize()
+    got = torch.cat(outs, dim=2).float()
+    assert rel_err(got.cpu(), full.float().cpu()) <= 1e-2
+    assert torch.allclose(M, Mf, rtol=1e-4, atol=1e-4) and torch.allclose(z, zf, rtol=1e-5)
+
+
+def test_n64_bandwidth_sampled():
+    w = wl.WORKLOADS["n64_bandwidth"]
+    check_sampled(w, chains=[(1, 5)], segs=[0, 1, 8191, 16383])
