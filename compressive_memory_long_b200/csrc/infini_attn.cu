@@ -279,7 +279,8 @@ bool use_small_fused(const Problem &p)
 int64_t workspace_bytes(int64_t B, int64_t Hkv, int64_t S, int64_t N, int64_t d)
 {
     const int64_t units = B * Hkv * S;
-    return units * (d * d + d) * 4 + units * d * d * 2 + units * N * d * 2 + units * 4 + 256;
+    return units * (d * d + d) * 4 + units * d * d * 2 + units * N * d * 2 + units * 4 +
+           B * Hkv * 4 + units * 16 + 512;
 }
 
 // The two-tile kernel redistributes registers with setmaxnreg; its split assumes the
@@ -334,20 +335,26 @@ int launch_small_fused(const Problem &p, const __nv_bfloat16 *q, const __nv_bflo
 {
     using C = tc::SmallCfg;
     const int64_t chains = p.B * p.Hkv, U = p.L / 128, units = chains * U;
-    // workspace: ticket + flags (zeroed here), then the published aggregates / prefixes
+    // workspace: ticket, per-head M0 reader counts, flags (all zeroed here), then the
+    // published aggregates / prefixes
     int *ticket = static_cast<int *>(ws);
-    int *flags = ticket + 64;
-    const size_t head = ((size_t)(64 + units) * 4 + 255) / 256 * 256;
+    int *m0_done = ticket + 64;
+    int *flags = m0_done + chains;
+    const size_t ints = 64 + chains + units;
+    const size_t head = (ints * 4 + 255) / 256 * 256;
     float *agg = reinterpret_cast<float *>(static_cast<char *>(ws) + head);
-    float *incl = agg + units * C::D * C::ROW;
-    if (cudaMemsetAsync(ws, 0, (size_t)(64 + units) * 4, st) != cudaSuccess) return INFINI_ERR_CUDA;
+    float *incl = agg + units * C::STATE;
+    if (cudaMemsetAsync(ws, 0, ints * 4, st) != cudaSuccess) return INFINI_ERR_CUDA;
     CUtensorMap mq, mk, mv;
     if (!make_map_bf16_3d(&mq, q, C::D, p.L, p.B * p.H, 128) ||
         !make_map_bf16_3d(&mk, k, C::D, p.L, chains, 128) ||
         !make_map_bf16_3d(&mv, v, C::D, p.L, chains, 128))
         return INFINI_ERR_CUDA;
     if (!opt_in_smem<tc::k_small_linear_fused>(C::ALLOC)) return INFINI_ERR_CUDA;
-    tc::SmallArgs a{beta, M0, z0, out, M_out, z_out, ticket, flags, agg, incl, p.L, (int)U, (int)p.H};
+    // few units per head: each sums its predecessors' aggregates directly
+    const int direct = U <= 64 ? 1 : 0;
+    tc::SmallArgs a{beta, M0, z0, out, M_out, z_out, ticket, m0_done, flags, agg, incl,
+                    p.L, (int)U, (int)p.H, (int)chains, direct};
     TRACED("small_fused", st);
     tc::k_small_linear_fused<<<(unsigned)units, 256, C::ALLOC, st>>>(mq, mk, mv, a);
     return INFINI_OK;

@@ -11,9 +11,10 @@
 //      causal mask keeps each segment to its own keys, "What happens inside the
 //      Infini-attention block?"), and the per-segment increments
 //      [dM_s | dz_s] = sigma(K_s)^T [V_s | 1];
-//   3. publishes its aggregate dM_0 + dM_1 and finds the exclusive prefix M_start with a
-//      single-pass decoupled look-back over earlier units of the same head (Merrill and
-//      Garland, "Single-pass Parallel Prefix Scan with Decoupled Look-back", 2016): a
+//   3. publishes its aggregate dM_0 + dM_1 and finds the exclusive prefix M_start: with few
+//      units per head ("direct" mode) by summing M0 and every earlier aggregate itself, else
+//      with a single-pass decoupled look-back over earlier units of the same head (Merrill
+//      and Garland, "Single-pass Parallel Prefix Scan with Decoupled Look-back", 2016): a
 //      predecessor's inclusive prefix ends the walk, its aggregate continues it;
 //   4. softmax and O = P V, then R_0 = sigma(Q) M_start and R_1 = sigma(Q) (M_start + dM_0)
 //      (rows of the first segment read R_0, rows of the second R_1), and the gated output.
@@ -39,12 +40,17 @@ struct SmallCfg {
     static constexpr int OFF_M0 = OFF_SQ + BOX;
     static constexpr int OFF_M1 = OFF_M0 + MB;
     static constexpr int OFF_Z = OFF_M1 + MB;      // z_start[64], z_mid[64] (fp32)
-    static constexpr int OFF_BAR = OFF_Z + 2 * 64 * 4;
+    static constexpr int ROW = 68;                 // floats per state row: 64 M, z, 3 pad
+    static constexpr int STATE = 64 * ROW;         // floats of one [64][ROW] state
+    static constexpr int STATE4 = STATE / 4;       // float4s of one state (1088)
+    static constexpr int OFF_AGG = OFF_Z + 2 * 64 * 4;   // this unit's aggregate [64][ROW]
+    static constexpr int OFF_D0 = OFF_AGG + STATE * 4;   // first segment's increment
+    static constexpr int OFF_EX = OFF_D0 + STATE * 4;    // exclusive prefix
+    static constexpr int OFF_BAR = OFF_EX + STATE * 4;
     static constexpr int NBAR = 10;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int BYTES = OFF_MISC + 32;
     static constexpr int ALLOC = BYTES + 1024;
-    static constexpr int ROW = D + 1;              // floats per published state row
 };
 
 struct SmallArgs {
@@ -53,10 +59,13 @@ struct SmallArgs {
     __nv_bfloat16 *out;
     float *M_out, *z_out;
     int *ticket;                   // zeroed before the launch
+    int *m0_done;                  // [chains] units that have read M0 (direct mode), zeroed
     int *flags;                    // [chains * U], zeroed before the launch
-    float *agg, *incl;             // [chains * U, D, D + 1]
+    float *agg, *incl;             // [chains * U, 64, ROW]
     int64_t L;
     int U, H;
+    int chains;
+    int direct;                    // 1: every unit sums M0 and all earlier aggregates itself
 };
 
 enum : int { FLAG_AGG = 1, FLAG_INCL = 2 };
@@ -97,6 +106,17 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16])
           "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
           "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
         : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_st16_s(uint32_t taddr, const uint32_t (&r)[16])
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+        "r"(r[15])
+        : "memory");
 }
 
 __global__ void __launch_bounds__(256, 1)
@@ -143,9 +163,10 @@ k_small_linear_fused(const __grid_constant__ CUtensorMap tmQ, const __grid_const
     const uint32_t tmem = *tmem_holder;
     const uint32_t T_S = tmem, T_O = tmem + 128, T_R0 = tmem + 192, T_R1 = tmem + 256;
     const uint32_t T_D0 = tmem + 320, T_D1 = tmem + 400;
+    // tickets interleave heads (unit-major), so every head advances side by side
     const int t = *s_ticket;
-    const int64_t chain = t / a.U;          // = b * H + h (one query head per kv head)
-    const int unit = t % a.U;
+    const int64_t chain = t % a.chains;     // = b * H + h (one query head per kv head)
+    const int unit = t / a.chains;
     const int64_t idx = chain * a.U + unit;
 
     if (warp == 0) {
@@ -223,160 +244,252 @@ k_small_linear_fused(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                 make_uint4(ch == 0 ? 0x3F80u : 0u, 0, 0, 0);
             *reinterpret_cast<uint4 *>(sSK + C::BOX + row * 128 + ch * 16) = make_uint4(0, 0, 0, 0);
         }
-        bool ok = mbar_wait(full, 0, abort, WS_FULL);
-        if (ok) {
-            // sigma(K) and sigma(Q) of row r (bf16, same swizzled position)
+        float *sAgg = reinterpret_cast<float *>(smem + C::OFF_AGG);
+        float *sD0 = reinterpret_cast<float *>(smem + C::OFF_D0);
+        float *sEx = reinterpret_cast<float *>(smem + C::OFF_EX);
+        auto sigma_row = [&](const uint8_t *src, uint8_t *dst) {   // bf16 row r, same swizzle
 #pragma unroll
             for (int ch = 0; ch < 8; ++ch) {
                 const int o = r * 128 + ((ch ^ (r & 7)) << 4);
-                uint4 kq[2] = {*reinterpret_cast<const uint4 *>(sK + o), *reinterpret_cast<const uint4 *>(sQ + o)};
-                uint8_t *dst[2] = {sSK + o, sSQ + o};
+                const uint4 x = *reinterpret_cast<const uint4 *>(src + o);
+                uint32_t w[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
-                for (int w2 = 0; w2 < 2; ++w2) {
-                    uint32_t w[4] = {kq[w2].x, kq[w2].y, kq[w2].z, kq[w2].w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        __nv_bfloat162 t2 = *reinterpret_cast<__nv_bfloat162 *>(&w[e]);
-                        w[e] = pack_bf16x2(sigma_s(__low2float(t2)), sigma_s(__high2float(t2)));
-                    }
-                    *reinterpret_cast<uint4 *>(dst[w2]) = make_uint4(w[0], w[1], w[2], w[3]);
+                for (int e = 0; e < 4; ++e) {
+                    __nv_bfloat162 t2 = *reinterpret_cast<__nv_bfloat162 *>(&w[e]);
+                    w[e] = pack_bf16x2(sigma_s(__low2float(t2)), sigma_s(__high2float(t2)));
                 }
+                *reinterpret_cast<uint4 *>(dst + o) = make_uint4(w[0], w[1], w[2], w[3]);
             }
+        };
+        bool ok = mbar_wait(full, 0, abort, WS_FULL);
+        if (ok) {                       // sigma(K) first: the increment MMAs need only it
+            sigma_row(sK, sSK);
             fence_proxy_async_smem();
             mbar_arrive(sig_ready);
         }
-        // ---- local softmax over the unit's 128 x 128 scores (block-diagonal causal mask)
+        // ---- local softmax: row r sees the 64 keys of its own segment, up to itself
         float l = 0.f;
         if (ok) ok = mbar_wait(s_done, 0, abort, WS_S);
         if (ok) {
             tc_fence_after();
-            uint32_t v[4][32];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) tmem_ld32(lane_base + T_S + c * 32, v[c]);
-            tmem_ld_wait();
             const int lo = (r >> 6) << 6;                // first key of this row's segment
-            float mt = -INFINITY;
+            uint32_t v[2][32];
+            tmem_ld32(lane_base + T_S + lo, v[0]);
+            tmem_ld32(lane_base + T_S + lo + 32, v[1]);
+            tmem_ld_wait();
+            float pm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-            for (int c = 0; c < 4; ++c)
+            for (int c = 0; c < 2; ++c)
 #pragma unroll
                 for (int e = 0; e < 32; ++e) {
-                    const int col = c * 32 + e;
-                    if (col < lo || col > r) v[c][e] = __float_as_uint(-INFINITY);
-                    mt = fmaxf(mt, __uint_as_float(v[c][e]));
+                    if (lo + c * 32 + e > r) v[c][e] = __float_as_uint(-INFINITY);
+                    pm[e & 3] = fmaxf(pm[e & 3], __uint_as_float(v[c][e]));
                 }
+            const float mt = fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3]));
             const float kscale = rsqrtf((float)D) * 1.4426950408889634f;
             const float mk = mt * kscale;
+            float ps[4] = {0.f, 0.f, 0.f, 0.f};
+            uint32_t zero16[16];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
+            for (int e = 0; e < 16; ++e) zero16[e] = 0u;
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
                 uint32_t pk[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
                     const float p0 = ex2(fmaf(__uint_as_float(v[c][2 * e]), kscale, -mk));
                     const float p1 = ex2(fmaf(__uint_as_float(v[c][2 * e + 1]), kscale, -mk));
-                    l += p0 + p1;
+                    ps[e & 3] += p0 + p1;
                     pk[e] = pack_bf16x2(p0, p1);
                 }
-                asm volatile(
-                    "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-                    "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(lane_base + T_S + c * 16),
-                    "r"(pk[0]), "r"(pk[1]), "r"(pk[2]), "r"(pk[3]), "r"(pk[4]), "r"(pk[5]), "r"(pk[6]),
-                    "r"(pk[7]), "r"(pk[8]), "r"(pk[9]), "r"(pk[10]), "r"(pk[11]), "r"(pk[12]),
-                    "r"(pk[13]), "r"(pk[14]), "r"(pk[15])
-                    : "memory");
+                // P over the S columns: this segment's keys, and zeros for the other segment
+                tmem_st16_s(lane_base + T_S + (lo >> 1) + c * 16, pk);
+                tmem_st16_s(lane_base + T_S + ((64 - lo) >> 1) + c * 16, zero16);
             }
+            l = (ps[0] + ps[1]) + (ps[2] + ps[3]);
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive(p_ready);
         }
-        // ---- the memory: aggregate, look-back, the two states this unit reads
+        if (ok) sigma_row(sQ, sSQ);    // sigma(Q) for the retrieval, off the critical path
+        // ---- this unit's increments into shared memory: D0 (first segment), D0 + D1
         if (ok) ok = mbar_wait(d_done, 0, abort, WS_D);
-        float d0[C::ROW], agg[C::ROW];
         if (ok) {
             tc_fence_after();
-            uint32_t x0[32], x1[32], y0[32], y1[32];
-            uint32_t x2[16], y2[16];
-            tmem_ld32(lane_base + T_D0, x0);
-            tmem_ld32(lane_base + T_D0 + 32, x1);
-            tmem_ld16(lane_base + T_D0 + 64, x2);
-            tmem_ld32(lane_base + T_D1, y0);
-            tmem_ld32(lane_base + T_D1 + 32, y1);
-            tmem_ld16(lane_base + T_D1 + 64, y2);
-            tmem_ld_wait();
+#pragma unroll 1
+            for (int c0 = 0; c0 < 80; c0 += 16) {
+                uint32_t x[16], y[16];
+                tmem_ld16(lane_base + T_D0 + c0, x);
+                tmem_ld16(lane_base + T_D1 + c0, y);
+                tmem_ld_wait();
+                if (r < D) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                d0[j] = __uint_as_float(x0[j]);
-                d0[32 + j] = __uint_as_float(x1[j]);
-                agg[j] = d0[j] + __uint_as_float(y0[j]);
-                agg[32 + j] = d0[32 + j] + __uint_as_float(y1[j]);
-            }
-            d0[64] = __uint_as_float(x2[0]);
-            agg[64] = d0[64] + __uint_as_float(y2[0]);
-            if (r < D) {
-                float *dst = a.agg + (idx * D + r) * C::ROW;
-#pragma unroll
-                for (int j = 0; j < C::ROW; ++j) dst[j] = agg[j];
+                    for (int e = 0; e < 16; ++e) {
+                        const int col = c0 + e;
+                        if (col < C::ROW) {
+                            const float x0 = __uint_as_float(x[e]);
+                            sD0[r * C::ROW + col] = x0;
+                            sAgg[r * C::ROW + col] = x0 + __uint_as_float(y[e]);
+                        }
+                    }
+                }
             }
         }
         asm volatile("bar.sync 1, 128;" ::: "memory");
-        // Unit 0 publishes no aggregate, only its inclusive prefix: every other walk then ends
-        // at an inclusive prefix, and only unit 0 reads M0 / z0 -- which M_out / z_out (written
-        // by the last unit, after its walk) may alias.
-        if (ok && r == 0 && unit > 0) {
+        // publish the aggregate (coalesced 16-byte stores by all 128 threads)
+        if (ok && (unit > 0 || a.direct)) {
+            float4 *dst = reinterpret_cast<float4 *>(a.agg + idx * C::STATE);
+            const float4 *src = reinterpret_cast<const float4 *>(sAgg);
+            for (int i = r; i < C::STATE4; i += 128) dst[i] = src[i];
             __threadfence();
-            st_release_gpu(a.flags + idx, FLAG_AGG);
         }
-        // exclusive prefix: walk back over earlier units of this head
-        float ex[C::ROW];
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        // Unit 0 of a long head publishes no aggregate, only its inclusive prefix: every other
+        // walk then ends at an inclusive prefix, and only unit 0 reads M0 / z0 -- which M_out /
+        // z_out (written by the last unit, after its walk) may alias.
+        if (ok && r == 0 && (unit > 0 || a.direct)) st_release_gpu(a.flags + idx, FLAG_AGG);
+
+        // ---- exclusive prefix of this unit, kept as float4 per thread (i = r + 128 k)
+        constexpr int KQ = (C::STATE4 + 127) / 128;
+        float4 ex[KQ];
 #pragma unroll
-        for (int j = 0; j < C::ROW; ++j) ex[j] = 0.f;
-        for (int j = unit - 1; ok && j >= 0; --j) {
-            if (r == 0) {
-                const int *fp = a.flags + chain * a.U + j;
-                int f = ld_acquire_gpu(fp);
-                const long long t0 = clock64();
-                while (f == 0) {
-                    if (clock64() - t0 > kSpinLimitCycles || wait_status_set()) {
-                        atomicCAS(&g_wait_status, 0, WS_LOOK);
-                        f = -1;
-                        break;
+        for (int k = 0; k < KQ; ++k) ex[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+        auto add_state = [&](const float *base) {
+            const float4 *src = reinterpret_cast<const float4 *>(base);
+#pragma unroll
+            for (int k = 0; k < KQ; ++k) {
+                const int i = r + 128 * k;
+                if (i < C::STATE4) {
+                    const float4 x = __ldcg(src + i);
+                    ex[k].x += x.x; ex[k].y += x.y; ex[k].z += x.z; ex[k].w += x.w;
+                }
+            }
+        };
+        auto add_initial = [&]() {      // M0 and z0 into the [64][ROW] layout
+#pragma unroll
+            for (int k = 0; k < KQ; ++k) {
+                const int i = r + 128 * k;
+                if (i < C::STATE4) {
+                    const int row = i / (C::ROW / 4), c4 = i % (C::ROW / 4);
+                    if (c4 < D / 4) {
+                        if (a.M0) {
+                            const float4 m = *reinterpret_cast<const float4 *>(a.M0 + (chain * D + row) * D + 4 * c4);
+                            ex[k].x += m.x; ex[k].y += m.y; ex[k].z += m.z; ex[k].w += m.w;
+                        }
+                    } else if (a.z0) {
+                        ex[k].x += a.z0[chain * D + row];
                     }
-                    __nanosleep(64);
-                    f = ld_acquire_gpu(fp);
+                }
+            }
+        };
+        if (a.direct) {
+            // wait until every earlier unit of the head has published its aggregate
+            if (ok && r == 0) {
+                int f = 0;
+                for (int j = 0; j < unit && f >= 0; ++j) {
+                    const int *fp = a.flags + chain * a.U + j;
+                    const long long t0 = clock64();
+                    while ((f = ld_acquire_gpu(fp)) == 0) {
+                        if (clock64() - t0 > kSpinLimitCycles || wait_status_set()) {
+                            atomicCAS(&g_wait_status, 0, WS_LOOK);
+                            f = -1;
+                            break;
+                        }
+                        __nanosleep(32);
+                    }
                 }
                 *s_state = f;
             }
             asm volatile("bar.sync 1, 128;" ::: "memory");
-            const int f = *s_state;
-            asm volatile("bar.sync 1, 128;" ::: "memory");
-            if (f < 0) {
+            if (ok && unit > 0 && *s_state < 0) {
                 ok = false;
                 *abort = 1;
-                break;
             }
-            if (r < D) {
-                const float *src = (f == FLAG_INCL ? a.incl : a.agg) + ((chain * a.U + j) * D + r) * C::ROW;
-#pragma unroll
-                for (int q = 0; q < C::ROW; ++q) ex[q] += __ldcg(src + q);
+            if (ok) {
+                for (int j = 0; j < unit; ++j) add_state(a.agg + (chain * a.U + j) * C::STATE);
+                add_initial();
             }
-            if (f == FLAG_INCL) break;
-        }
-        if (ok && unit == 0 && r < D) {
-            if (a.M0)
-#pragma unroll 8
-                for (int q = 0; q < D; ++q) ex[q] += a.M0[(chain * D + r) * D + q];
-            if (a.z0) ex[D] += a.z0[chain * D + r];
+            // the last unit may overwrite M0 / z0 (they may alias M_out / z_out) only after
+            // every other unit of the head has read them
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            if (ok && r == 0) {
+                __threadfence();
+                if (unit + 1 < a.U) {
+                    atomicAdd(a.m0_done + chain, 1);
+                } else {
+                    const long long t0 = clock64();
+                    while (ld_acquire_gpu(a.m0_done + chain) < a.U - 1) {
+                        if (clock64() - t0 > kSpinLimitCycles || wait_status_set()) {
+                            atomicCAS(&g_wait_status, 0, WS_LOOK);
+                            *s_state = -1;
+                            break;
+                        }
+                        __nanosleep(32);
+                    }
+                }
+            }
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            if (ok && unit + 1 == a.U && *s_state < 0) {
+                ok = false;
+                *abort = 1;
+            }
+        } else {
+            for (int j = unit - 1; ok && j >= 0; --j) {
+                if (r == 0) {
+                    const int *fp = a.flags + chain * a.U + j;
+                    int f = ld_acquire_gpu(fp);
+                    const long long t0 = clock64();
+                    while (f == 0) {
+                        if (clock64() - t0 > kSpinLimitCycles || wait_status_set()) {
+                            atomicCAS(&g_wait_status, 0, WS_LOOK);
+                            f = -1;
+                            break;
+                        }
+                        __nanosleep(32);
+                        f = ld_acquire_gpu(fp);
+                    }
+                    *s_state = f;
+                }
+                asm volatile("bar.sync 1, 128;" ::: "memory");
+                const int f = *s_state;
+                asm volatile("bar.sync 1, 128;" ::: "memory");
+                if (f < 0) {
+                    ok = false;
+                    *abort = 1;
+                    break;
+                }
+                add_state((f == FLAG_INCL ? a.incl : a.agg) + (chain * a.U + j) * C::STATE);
+                if (f == FLAG_INCL) break;
+            }
+            if (ok && unit == 0) add_initial();
         }
         if (ok) {
+            float4 *sEx4 = reinterpret_cast<float4 *>(sEx);
+            const float4 *sAgg4 = reinterpret_cast<const float4 *>(sAgg);
+#pragma unroll
+            for (int k = 0; k < KQ; ++k) {
+                const int i = r + 128 * k;
+                if (i < C::STATE4) {
+                    sEx4[i] = ex[k];
+                    if (!a.direct && unit + 1 < a.U) {      // inclusive prefix for successors
+                        const float4 g = sAgg4[i];
+                        reinterpret_cast<float4 *>(a.incl + idx * C::STATE)[i] =
+                            make_float4(ex[k].x + g.x, ex[k].y + g.y, ex[k].z + g.z, ex[k].w + g.w);
+                    }
+                }
+            }
+            if (!a.direct && unit + 1 < a.U) __threadfence();
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (ok) {
+            if (r == 0 && !a.direct && unit + 1 < a.U) st_release_gpu(a.flags + idx, FLAG_INCL);
             if (r < D) {
-                if (unit + 1 < a.U) {
-                    float *dst = a.incl + (idx * D + r) * C::ROW;
-#pragma unroll
-                    for (int q = 0; q < C::ROW; ++q) dst[q] = ex[q] + agg[q];
-                } else {
+                const float *exr = sEx + r * C::ROW, *d0r = sD0 + r * C::ROW, *agr = sAgg + r * C::ROW;
+                if (unit + 1 == a.U) {                 // the head's final state
                     float *mo = a.M_out + (chain * D + r) * D;
-#pragma unroll
-                    for (int q = 0; q < D; ++q) mo[q] = ex[q] + agg[q];
-                    a.z_out[chain * D + r] = ex[D] + agg[D];
+#pragma unroll 8
+                    for (int q = 0; q < D; ++q) mo[q] = exr[q] + agr[q];
+                    a.z_out[chain * D + r] = exr[D] + agr[D];
                 }
                 // M_start and M_mid rows (key r) as bf16 B operands, z as fp32
 #pragma unroll
@@ -385,20 +498,15 @@ k_small_linear_fused(const __grid_constant__ CUtensorMap tmQ, const __grid_const
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const int q = ch * 8 + 2 * e;
-                        w0[e] = pack_bf16x2(ex[q], ex[q + 1]);
-                        w1[e] = pack_bf16x2(ex[q] + d0[q], ex[q + 1] + d0[q + 1]);
+                        w0[e] = pack_bf16x2(exr[q], exr[q + 1]);
+                        w1[e] = pack_bf16x2(exr[q] + d0r[q], exr[q + 1] + d0r[q + 1]);
                     }
                     const int o = r * 128 + ((ch ^ (r & 7)) << 4);
                     *reinterpret_cast<uint4 *>(sM0 + o) = make_uint4(w0[0], w0[1], w0[2], w0[3]);
                     *reinterpret_cast<uint4 *>(sM1 + o) = make_uint4(w1[0], w1[1], w1[2], w1[3]);
                 }
-                sZ0[r] = ex[D];
-                sZ1[r] = ex[D] + d0[D];
-            }
-            asm volatile("bar.sync 1, 128;" ::: "memory");
-            if (r == 0 && unit + 1 < a.U) {
-                __threadfence();
-                st_release_gpu(a.flags + idx, FLAG_INCL);
+                sZ0[r] = exr[D];
+                sZ1[r] = exr[D] + d0r[D];
             }
             fence_proxy_async_smem();
             mbar_arrive(m_ready);
@@ -408,40 +516,37 @@ k_small_linear_fused(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         if (ok) ok = mbar_wait(r_done, 0, abort, WS_R);
         if (ok) {
             tc_fence_after();
+            asm volatile("bar.sync 1, 128;" ::: "memory");   // every row's z is in place
             const float *zz = (r < C::SEG) ? sZ0 : sZ1;
             float den = 0.f;
 #pragma unroll
-            for (int ch = 0; ch < 8; ++ch) {
-                const uint4 qv = *reinterpret_cast<const uint4 *>(sQ + r * 128 + ((ch ^ (r & 7)) << 4));
+            for (int ch = 0; ch < 8; ++ch) {    // sigma(q) . z from the bf16 sigma(Q) row
+                const uint4 qv = *reinterpret_cast<const uint4 *>(sSQ + r * 128 + ((ch ^ (r & 7)) << 4));
                 uint32_t w[4] = {qv.x, qv.y, qv.z, qv.w};
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     __nv_bfloat162 t2 = *reinterpret_cast<__nv_bfloat162 *>(&w[e]);
-                    den = fmaf(sigma_s(__low2float(t2)), zz[ch * 8 + 2 * e], den);
-                    den = fmaf(sigma_s(__high2float(t2)), zz[ch * 8 + 2 * e + 1], den);
+                    den = fmaf(__low2float(t2), zz[ch * 8 + 2 * e], den);
+                    den = fmaf(__high2float(t2), zz[ch * 8 + 2 * e + 1], den);
                 }
             }
             const int h = (int)(chain % a.H);
             const float g = 1.f / (1.f + __expf(-a.beta[h]));
             const float wl = (1.f - g) / l;
             const float wm = den == 0.f ? 0.f : g / den;
-            const uint32_t tR = (r < C::SEG) ? T_R0 : T_R1;
+            const uint32_t tR = (r < C::SEG) ? T_R0 : T_R1;   // uniform per warp
             __nv_bfloat16 *orow = a.out + (chain * a.L + (int64_t)unit * C::TOK + r) * D;
 #pragma unroll 1
             for (int c = 0; c < D; c += 32) {
-                uint32_t o[32], rr0[32], rr1[32];
+                uint32_t o[32], rr[32];
                 tmem_ld32(lane_base + T_O + c, o);
-                tmem_ld32(lane_base + T_R0 + c, rr0);
-                tmem_ld32(lane_base + T_R1 + c, rr1);
+                tmem_ld32(lane_base + tR + c, rr);
                 tmem_ld_wait();
                 uint32_t pk[16];
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const float ra = __uint_as_float(tR == T_R0 ? rr0[2 * e] : rr1[2 * e]);
-                    const float rb = __uint_as_float(tR == T_R0 ? rr0[2 * e + 1] : rr1[2 * e + 1]);
-                    pk[e] = pack_bf16x2(fmaf(ra, wm, __uint_as_float(o[2 * e]) * wl),
-                                        fmaf(rb, wm, __uint_as_float(o[2 * e + 1]) * wl));
-                }
+                for (int e = 0; e < 16; ++e)
+                    pk[e] = pack_bf16x2(fmaf(__uint_as_float(rr[2 * e]), wm, __uint_as_float(o[2 * e]) * wl),
+                                        fmaf(__uint_as_float(rr[2 * e + 1]), wm, __uint_as_float(o[2 * e + 1]) * wl));
                 uint4 *dst = reinterpret_cast<uint4 *>(orow + c);
 #pragma unroll
                 for (int e = 0; e < 4; ++e)

@@ -40,7 +40,8 @@ def test_status_strings_and_version():
 def test_workspace_bytes():
     units = 2 * 8 * 16
     assert binding.infini_attn_workspace_bytes(2, 8, 1024, 64, 64) == \
-        units * (64 * 64 + 64) * 4 + units * 64 * 64 * 2 + units * 64 * 64 * 2 + units * 4 + 256
+        units * (64 * 64 + 64) * 4 + units * 64 * 64 * 2 + units * 64 * 64 * 2 + units * 4 + \
+        2 * 8 * 4 + units * 16 + 512
     assert binding.infini_attn_workspace_bytes(1, 1, 100, 64, 64) == 0
     assert binding.infini_attn_workspace_bytes(0, 1, 64, 64, 64) == 0
 
