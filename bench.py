@@ -69,7 +69,7 @@ def algorithmic(w: wl.Workload, kernel: str):
     e = w.elem_bytes
     B, H, Hkv, L, N, d, S = w.B, w.H, w.Hkv, w.L, w.N, w.d, w.S
     state_bytes = 2 * B * Hkv * (d * d + d) * 4
-    if kernel == "small_fused":     # the whole forward in one launch
+    if kernel in ("small_fused", "small_pieces"):     # the whole forward in one launch
         f1, b1 = algorithmic(w, "segment")
         f2, b2 = algorithmic(w, "linear_state")
         return f1 + f2, b1 + state_bytes

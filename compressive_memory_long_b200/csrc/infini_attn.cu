@@ -19,6 +19,7 @@
 #include "tc_delta.cuh"
 #include "tc_linear.cuh"
 #include "tc_small.cuh"
+#include "tc_pieces.cuh"
 
 #include <cudaTypedefs.h>
 
@@ -68,7 +69,7 @@ int check_args(const void *q, const void *k, const void *v, const float *beta, c
     if (rule != INFINI_UPDATE_LINEAR && rule != INFINI_UPDATE_DELTA) return INFINI_ERR_INVALID_ARG;
     // keep every element count far inside int64 and every grid inside 2^31 CTAs
     if (B > (1 << 20) || H > (1 << 16) || L > ((int64_t)1 << 34) ||
-        B * H * L > ((int64_t)1 << 40))
+        B * H * L > ((int64_t)1 << 40) || B * H * (L / 128) > ((int64_t)1 << 30))
         return INFINI_ERR_INVALID_ARG;
     const void *ptrs[] = {q, k, v, beta, M0, z0, out, M_out, z_out};
     for (const void *p : ptrs)
@@ -273,6 +274,9 @@ bool use_small_fused(const Problem &p)
            p.H == p.Hkv && p.L % 128 == 0;
 }
 
+// Long heads (16 units of 128 tokens or more) go to the persistent piece kernel.
+bool use_pieces(const Problem &p) { return p.L / 128 >= 16; }
+
 // Workspace of one call: fp32 snapshots (M, z) for every segment, bf16 copies of M for the
 // tensor-core kernels, and room for the fused path's flags; an upper bound for every path.
 // Layout: [fp32 snapshots M | z][bf16 copies of M][sigma(K) in bf16][flags of the fused path].
@@ -328,6 +332,13 @@ int launch_segment_tc(const Problem &p, const __nv_bfloat16 *q, const __nv_bfloa
     return INFINI_OK;
 }
 
+int64_t small_workspace_bytes(const Problem &p)
+{
+    const int64_t chains = p.B * p.Hkv, units = chains * (p.L / 128);
+    const int64_t head = ((64 + chains + units) * 4 + 255) / 256 * 256;
+    return head + 2 * units * tc::SmallCfg::STATE * 4;
+}
+
 int launch_small_fused(const Problem &p, const __nv_bfloat16 *q, const __nv_bfloat16 *k,
                        const __nv_bfloat16 *v, const float *beta, const float *M0,
                        const float *z0, __nv_bfloat16 *out, float *M_out, float *z_out,
@@ -360,6 +371,74 @@ int launch_small_fused(const Problem &p, const __nv_bfloat16 *q, const __nv_bflo
     return INFINI_OK;
 }
 
+int sm_count()
+{
+    int sms = 148, dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+        cudaGetLastError();
+        sms = 148;
+    }
+    return sms;
+}
+
+// Long heads of 64-token segments: the persistent piece kernel.  Units per piece: about four
+// pieces per CTA across the grid, at most PieceCfg::MAX_UNITS.
+struct PiecePlan {
+    int64_t chains, U, UP, P, total;
+};
+
+PiecePlan piece_plan(const Problem &p)
+{
+    PiecePlan pl;
+    pl.chains = p.B * p.H;
+    pl.U = p.L / 128;
+    const int64_t target = 4 * (int64_t)sm_count();
+    int64_t up = (pl.chains * pl.U) / target;
+    up = up < 1 ? 1 : (up > tc::PieceCfg::MAX_UNITS ? tc::PieceCfg::MAX_UNITS : up);
+    pl.UP = up;
+    pl.P = (pl.U + up - 1) / up;
+    pl.total = pl.chains * pl.P;
+    return pl;
+}
+
+// workspace of the piece kernel: ticket and flags (zeroed per call), then the published
+// aggregate and inclusive prefix of every piece
+int64_t pieces_workspace_bytes(const Problem &p)
+{
+    const PiecePlan pl = piece_plan(p);
+    const int64_t head = ((64 + pl.total) * 4 + 255) / 256 * 256;
+    return head + 2 * pl.total * tc::PieceCfg::STATE * 4;
+}
+
+int launch_pieces(const Problem &p, const __nv_bfloat16 *q, const __nv_bfloat16 *k,
+                  const __nv_bfloat16 *v, const float *beta, const float *M0, const float *z0,
+                  __nv_bfloat16 *out, float *M_out, float *z_out, void *ws, cudaStream_t st)
+{
+    using C = tc::PieceCfg;
+    const PiecePlan pl = piece_plan(p);
+    int *ticket = static_cast<int *>(ws);
+    int *flags = ticket + 64;
+    const size_t ints = 64 + pl.total;
+    const size_t head = (ints * 4 + 255) / 256 * 256;
+    float *agg = reinterpret_cast<float *>(static_cast<char *>(ws) + head);
+    float *incl = agg + pl.total * C::STATE;
+    if (cudaMemsetAsync(ws, 0, ints * 4, st) != cudaSuccess) return INFINI_ERR_CUDA;
+    CUtensorMap mq, mk, mv;
+    if (!make_map_bf16_3d(&mq, q, C::D, p.L, p.B * p.H, 128) ||
+        !make_map_bf16_3d(&mk, k, C::D, p.L, pl.chains, 128) ||
+        !make_map_bf16_3d(&mv, v, C::D, p.L, pl.chains, 128))
+        return INFINI_ERR_CUDA;
+    if (!opt_in_smem<tc::k_small_pieces>(C::ALLOC)) return INFINI_ERR_CUDA;
+    tc::PieceArgs a{beta, M0, z0, out, M_out, z_out, ticket, flags, agg, incl, p.L,
+                    (int)pl.U, (int)pl.UP, (int)pl.P, (int)p.H, (int)pl.chains, (int)pl.total};
+    const int64_t sms = sm_count();
+    const int64_t grid = pl.total < sms ? pl.total : sms;
+    TRACED("small_pieces", st);
+    tc::k_small_pieces<<<(unsigned)grid, C::THREADS, C::ALLOC, st>>>(mq, mk, mv, a);
+    return INFINI_OK;
+}
+
 template <typename T, int D>
 int launch_all(const Problem &p, const T *q, const T *k, const T *v, const float *beta,
                const float *M0, const float *z0, T *out, float *M_out, float *z_out,
@@ -367,7 +446,9 @@ int launch_all(const Problem &p, const T *q, const T *k, const T *v, const float
 {
     if constexpr (sizeof(T) == 2 && D == 64) {
         if (use_small_fused<T>(p)) {
-            const int rc = launch_small_fused(p, q, k, v, beta, M0, z0, out, M_out, z_out, snapM, st);
+            const int rc = use_pieces(p)
+                ? launch_pieces(p, q, k, v, beta, M0, z0, out, M_out, z_out, snapM, st)
+                : launch_small_fused(p, q, k, v, beta, M0, z0, out, M_out, z_out, snapM, st);
             if (rc != INFINI_OK) return rc;
             return cudaGetLastError() == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
         }
@@ -478,7 +559,10 @@ int forward(const void *q, const void *k, const void *v, const float *beta, cons
 
     const int64_t nM = p.B * p.Hkv * p.S * p.d * p.d, nZ = p.B * p.Hkv * p.S * p.d;
     const bool tc_path = use_tc<T>(p);
-    const size_t bytes = (size_t)workspace_bytes(p.B, p.Hkv, p.S, p.N, p.d);
+    // the fused 64-token paths need far less than the general upper bound
+    const size_t bytes = (size_t)(!use_small_fused<T>(p) ? workspace_bytes(p.B, p.Hkv, p.S, p.N, p.d)
+                                  : use_pieces(p)        ? pieces_workspace_bytes(p)
+                                                         : small_workspace_bytes(p));
     void *ws = nullptr;
     cudaMemPool_t pool = workspace_pool();
     if (!pool) return INFINI_ERR_CUDA;

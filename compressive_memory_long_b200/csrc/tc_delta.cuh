@@ -160,7 +160,7 @@ k_delta_chain_tc(const __grid_constant__ CUtensorMap tmSK, const __grid_constant
             int issued = 0;
             for (int g = 0; g < total; ++g) {
                 const int st = g % ST, s = g / nch, i = g % nch;
-                if (g >= ST && !mbar_wait(kv_empty + st, ((g / ST) - 1) & 1, abort, WC_KV_EMPTY))
+                if (g >= ST && !mbar_wait_short(kv_empty + st, ((g / ST) - 1) & 1, abort, WC_KV_EMPTY))
                     break;
                 const int row = s * a.N + i * 128;
                 mbar_arrive_expect_tx(kv_full + st, (uint32_t)(D * 128 * 2 + C::VTILE));
@@ -183,9 +183,9 @@ k_delta_chain_tc(const __grid_constant__ CUtensorMap tmSK, const __grid_constant
             auto issue_r = [&](int g) -> bool {
                 // the first chunk of segment s waits for B holding M_{s-1}: phase 0 is the
                 // initial state written in the prologue, phase s the boundary after segment s-1
-                if (g % nch == 0 && !mbar_wait(b_ready, (g / nch) & 1, abort, WC_B))
+                if (g % nch == 0 && !mbar_wait_short(b_ready, (g / nch) & 1, abort, WC_B))
                     return false;
-                if (!mbar_wait(kv_full + g % ST, (g / ST) & 1, abort, WC_KV_FULL)) return false;
+                if (!mbar_wait_short(kv_full + g % ST, (g / ST) & 1, abort, WC_KV_FULL)) return false;
                 tc_fence_after();
                 const uint32_t kbase = aK + (g % ST) * C::KTILE;
 #pragma unroll
@@ -200,7 +200,7 @@ k_delta_chain_tc(const __grid_constant__ CUtensorMap tmSK, const __grid_constant
             };
             auto issue_update = [&](int g) -> bool {
                 const int bb = g & 1;
-                if (!mbar_wait(u_ready + bb, (g >> 1) & 1, abort, WC_U)) return false;
+                if (!mbar_wait_short(u_ready + bb, (g >> 1) & 1, abort, WC_U)) return false;
                 tc_fence_after();
                 const uint32_t kbase = aK + (g % ST) * C::KTILE;
                 const uint32_t ub = aU + bb * C::BTILE;
@@ -285,7 +285,7 @@ k_delta_chain_tc(const __grid_constant__ CUtensorMap tmSK, const __grid_constant
         bool ok = true;
         for (int g = 0; ok && g < total; ++g) {
             const int st = g % ST, s = g / nch, i = g % nch, bb = g & 1;
-            if (!(ok = mbar_wait(kv_full + st, (g / ST) & 1, abort, WC_KV_FULL))) break;
+            if (!(ok = mbar_wait_short(kv_full + st, (g / ST) & 1, abort, WC_KV_FULL))) break;
             // this token's 16 values of V in chunk g
             float vv[CB];
             {
@@ -299,7 +299,7 @@ k_delta_chain_tc(const __grid_constant__ CUtensorMap tmSK, const __grid_constant
                     vv[2 * e + 1] = __high2float(t2);
                 }
             }
-            if (!(ok = mbar_wait(r_full + bb, (g >> 1) & 1, abort, WC_R))) break;
+            if (!(ok = mbar_wait_short(r_full + bb, (g >> 1) & 1, abort, WC_R))) break;
             tc_fence_after();
             uint32_t rh[32], rl[32];
             tmem_ld32(lane_base + T_R[bb], rh);
@@ -308,7 +308,7 @@ k_delta_chain_tc(const __grid_constant__ CUtensorMap tmSK, const __grid_constant
             const float den = __uint_as_float(rh[CB]) + __uint_as_float(rl[CB]);
             const float inv = den == 0.f ? 0.f : 1.f / den;
             // U tile bb is free once the update of chunk g-2 has completed
-            if (g >= 2 && !(ok = mbar_wait(upd_done + bb, ((g >> 1) - 1) & 1, abort, WC_UPD))) break;
+            if (g >= 2 && !(ok = mbar_wait_short(upd_done + bb, ((g >> 1) - 1) & 1, abort, WC_UPD))) break;
             {
                 const int box = r >> 6, tt = r & 63;
                 uint8_t *ub = sU + bb * C::BTILE + box * C::BBOX + (tt & 7) * 2;
@@ -328,7 +328,7 @@ k_delta_chain_tc(const __grid_constant__ CUtensorMap tmSK, const __grid_constant
 
             if (i == nch - 1) {
                 // segment end: M_s, z_s from the accumulator (lane r = key feature r)
-                if (!(ok = mbar_wait(upd_done + bb, (g >> 1) & 1, abort, WC_UPD))) break;
+                if (!(ok = mbar_wait_short(upd_done + bb, (g >> 1) & 1, abort, WC_UPD))) break;
                 tc_fence_after();
                 uint32_t acc[32], acl[32];
                 tmem_ld32(lane_base + T_M, acc);

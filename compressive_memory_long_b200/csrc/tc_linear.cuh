@@ -102,7 +102,7 @@ k_linear_state_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant
             int issued = 0;
             for (int g = 0; g < total; ++g) {
                 const int st = g % ST, s = g / nch, i = g % nch;
-                if (g >= ST && !mbar_wait(kv_empty + st, ((g / ST) - 1) & 1, abort, WL_KV_EMPTY))
+                if (g >= ST && !mbar_wait_short(kv_empty + st, ((g / ST) - 1) & 1, abort, WL_KV_EMPTY))
                     break;
                 const int row = s * a.N + i * 128;
                 mbar_arrive_expect_tx(kv_full + st, (uint32_t)(2 * D * 128 * 2));
@@ -130,7 +130,7 @@ k_linear_state_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant
             const uint32_t aK = smem_u32(sK), aV = smem_u32(sV);
             for (int g = 0; g < total; ++g) {
                 const int st = g % ST, i = g % nch;
-                if (!mbar_wait(a_ready, g & 1, abort, WL_A)) break;
+                if (!mbar_wait_short(a_ready, g & 1, abort, WL_A)) break;
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {        // 128 tokens in steps of 16
@@ -200,7 +200,7 @@ k_linear_state_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant
 
         for (int g = 0; g < total; ++g) {
             const int st = g % ST, s = g / nch, i = g % nch;
-            if (!mbar_wait(kv_full + st, (g / ST) & 1, abort, WL_KV_FULL)) break;
+            if (!mbar_wait_short(kv_full + st, (g / ST) & 1, abort, WL_KV_FULL)) break;
             uint8_t *krow = sK + st * C::KTILE;
 #pragma unroll
             for (int kb = 0; kb < D / 64; ++kb) {
@@ -221,7 +221,7 @@ k_linear_state_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant
             fence_proxy_async_smem();
             mbar_arrive(a_ready);
             if (i == nch - 1) {
-                if (!mbar_wait(seg_done, s & 1, abort, WL_SEG)) break;
+                if (!mbar_wait_short(seg_done, s & 1, abort, WL_SEG)) break;
                 tc_fence_after();
                 if (r < D) {
                     // row r of [M_s | z_s]

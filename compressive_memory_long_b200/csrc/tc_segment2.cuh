@@ -289,14 +289,15 @@ k_segment_tc2(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     for (int e = 0; e < 32; ++e)
                         if (c * 32 + e > r) v[c][e] = __float_as_uint(-INFINITY);
             }
-            // row maximum with eight independent partial maxima (no long dependency chain)
-            float pm[8];
+            // row maximum: three-input max, four independent partial maxima
+            float pm[4];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) pm[u] = __uint_as_float(v[0][u]);
+            for (int u = 0; u < 4; ++u) pm[u] = __uint_as_float(v[0][u]);
 #pragma unroll
-            for (int u = 8; u < 128; ++u) pm[u & 7] = fmaxf(pm[u & 7], __uint_as_float(v[u >> 5][u & 31]));
-            const float mt = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
-                                   fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+            for (int u = 4; u < 128; u += 2)
+                pm[(u >> 1) & 3] = max3f(pm[(u >> 1) & 3], __uint_as_float(v[u >> 5][u & 31]),
+                                         __uint_as_float(v[u >> 5][(u & 31) + 1]));
+            const float mt = fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3]));
             const bool resc = (mt - m_used) * kscale > 8.f;
             float alpha = 1.f;
             if (resc) {
@@ -318,20 +319,27 @@ k_segment_tc2(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             }
             // P = exp2((S - m) * scale) in bf16, written over the S tile's first 64 columns
             const float mk = m_used * kscale;
-            float ps[4] = {0.f, 0.f, 0.f, 0.f};     // independent partial row sums
+            // scale-and-shift and the partial row sums on packed fp32 pairs
+            const uint64_t ks2 = f2_pack(kscale, kscale), nm2 = f2_pack(-mk, -mk);
+            uint64_t ps2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 uint32_t pk[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
-                    const float p0 = ex2(fmaf(__uint_as_float(v[c][2 * e]), kscale, -mk));
-                    const float p1 = ex2(fmaf(__uint_as_float(v[c][2 * e + 1]), kscale, -mk));
-                    ps[e & 3] += p0 + p1;
+                    float y0, y1;
+                    f2_unpack(f2_fma(f2_pack(__uint_as_float(v[c][2 * e]), __uint_as_float(v[c][2 * e + 1])),
+                                     ks2, nm2), y0, y1);
+                    const float p0 = ex2(y0), p1 = ex2(y1);
+                    ps2[e & 3] = f2_add(ps2[e & 3], f2_pack(p0, p1));
                     pk[e] = pack_bf16x2(p0, p1);
                 }
                 tmem_st16(lane_base + T_S[x] + c * 16, pk);
             }
-            const float rs = (ps[0] + ps[1]) + (ps[2] + ps[3]);
+            float rsum[8];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) f2_unpack(ps2[u], rsum[2 * u], rsum[2 * u + 1]);
+            const float rs = ((rsum[0] + rsum[1]) + (rsum[2] + rsum[3])) + ((rsum[4] + rsum[5]) + (rsum[6] + rsum[7]));
             l += rs;
             tmem_st_wait();
             tc_fence_before();

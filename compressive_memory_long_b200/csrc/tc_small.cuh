@@ -188,7 +188,7 @@ k_small_linear_fused(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
             const uint32_t aSK = smem_u32(sSK), aSQ = smem_u32(sSQ);
             const uint32_t aM0 = smem_u32(sM0), aM1 = smem_u32(sM1);
-            bool ok = mbar_wait(full, 0, abort, WS_FULL);
+            bool ok = mbar_wait_short(full, 0, abort, WS_FULL);
             if (ok) {   // S = Q K^T over the unit
                 tc_fence_after();
 #pragma unroll
@@ -197,7 +197,7 @@ k_small_linear_fused(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                            idS, kk > 0 ? 1u : 0u);
                 mma_commit(s_done);
             }
-            if (ok) ok = mbar_wait(sig_ready, 0, abort, WS_SIG);
+            if (ok) ok = mbar_wait_short(sig_ready, 0, abort, WS_SIG);
             if (ok) {   // [dM_s | dz_s] = sigma(K_s)^T [V_s | 1], s = first and second segment
                 tc_fence_after();
 #pragma unroll
@@ -210,7 +210,7 @@ k_small_linear_fused(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                     }
                 mma_commit(d_done);
             }
-            if (ok) ok = mbar_wait(p_ready, 0, abort, WS_P);
+            if (ok) ok = mbar_wait_short(p_ready, 0, abort, WS_P);
             if (ok) {   // O = P V
                 tc_fence_after();
 #pragma unroll
@@ -219,7 +219,7 @@ k_small_linear_fused(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                            kk > 0 ? 1u : 0u);
                 mma_commit(o_done);
             }
-            if (ok) ok = mbar_wait(m_ready, 0, abort, WS_M);
+            if (ok) ok = mbar_wait_short(m_ready, 0, abort, WS_M);
             if (ok) {   // R_0 = sigma(Q) M_start, R_1 = sigma(Q) M_mid
                 tc_fence_after();
 #pragma unroll
@@ -261,7 +261,7 @@ k_small_linear_fused(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                 *reinterpret_cast<uint4 *>(dst + o) = make_uint4(w[0], w[1], w[2], w[3]);
             }
         };
-        bool ok = mbar_wait(full, 0, abort, WS_FULL);
+        bool ok = mbar_wait_short(full, 0, abort, WS_FULL);
         if (ok) {                       // sigma(K) first: the increment MMAs need only it
             sigma_row(sK, sSK);
             fence_proxy_async_smem();
@@ -269,7 +269,7 @@ k_small_linear_fused(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         }
         // ---- local softmax: row r sees the 64 keys of its own segment, up to itself
         float l = 0.f;
-        if (ok) ok = mbar_wait(s_done, 0, abort, WS_S);
+        if (ok) ok = mbar_wait_short(s_done, 0, abort, WS_S);
         if (ok) {
             tc_fence_after();
             const int lo = (r >> 6) << 6;                // first key of this row's segment
@@ -313,7 +313,7 @@ k_small_linear_fused(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         }
         if (ok) sigma_row(sQ, sSQ);    // sigma(Q) for the retrieval, off the critical path
         // ---- this unit's increments into shared memory: D0 (first segment), D0 + D1
-        if (ok) ok = mbar_wait(d_done, 0, abort, WS_D);
+        if (ok) ok = mbar_wait_short(d_done, 0, abort, WS_D);
         if (ok) {
             tc_fence_after();
 #pragma unroll 1
@@ -512,8 +512,8 @@ k_small_linear_fused(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             mbar_arrive(m_ready);
         }
         // ---- epilogue: gate the local and memory reads of row r
-        if (ok) ok = mbar_wait(o_done, 0, abort, WS_O);
-        if (ok) ok = mbar_wait(r_done, 0, abort, WS_R);
+        if (ok) ok = mbar_wait_short(o_done, 0, abort, WS_O);
+        if (ok) ok = mbar_wait_short(r_done, 0, abort, WS_R);
         if (ok) {
             tc_fence_after();
             asm volatile("bar.sync 1, 128;" ::: "memory");   // every row's z is in place

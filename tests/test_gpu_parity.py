@@ -229,6 +229,46 @@ def test_small_fused_in_place_split():
     assert torch.allclose(M, Mf, rtol=1e-4, atol=1e-4) and torch.allclose(z, zf, rtol=1e-5)
 
 
+# ---- the persistent piece kernel (same layouts, heads of 16 or more 128-token units) -----
+
+@pytest.mark.parametrize("B,H,S", [(2, 3, 32), (1, 2, 66), (2, 8, 150), (1, 16, 600)])
+def test_small_pieces_shapes(B, H, S):
+    """Pieces of one or several units, a shorter last piece, look-back over many pieces."""
+    from compressive_memory_long_b200 import binding
+    w = wl.Workload("pieces", B=B, H=H, Hkv=H, d=64, N=64, S=S, dtype="bf16", rule="linear",
+                    seed=31 + S, beta_dist=("normal", 0.0, 1.5), M0_dist=("uniform", 0.0, 0.1),
+                    z0_dist=("uniform", 1.0, 2.0))
+    binding.infini_attn_trace_enable(True)
+    check_full(w)
+    binding.infini_attn_trace_enable(False)
+    assert list(binding.infini_attn_trace_report()) == ["small_pieces"]
+    assert binding.infini_attn_device_status() == 0
+
+
+def test_small_pieces_zero_state_and_split():
+    """No initial state (the first segment has no memory term), then the same sequence in
+    two calls with the memory carried in place."""
+    from compressive_memory_long_b200 import binding
+    w = wl.Workload("pieces_split", B=1, H=4, Hkv=4, d=64, N=64, S=96, dtype="bf16",
+                    rule="linear", seed=41, beta_dist=("normal", 0.0, 1.0))
+    check_full(w)
+    t = to_dev(wl.torch_inputs(w))
+    full, Mf, zf = binding.forward(t["q"], t["k"], t["v"], t["beta"], None, None, N=w.N,
+                                   rule=w.rule)
+    M = torch.zeros_like(Mf)
+    z = torch.zeros_like(zf)
+    outs = []
+    for sl in (slice(0, 2048), slice(2048, 6144)):
+        qs, ks, vs = (t[n][:, :, sl].contiguous() for n in ("q", "k", "v"))
+        o, _, _ = binding.forward(qs, ks, vs, t["beta"], M, z, N=w.N, rule=w.rule, M_out=M,
+                                  z_out=z)
+        outs.append(o)
+    torch.cuda.synchronize()
+    got = torch.cat(outs, dim=2).float()
+    assert rel_err(got.cpu(), full.float().cpu()) <= 1e-2
+    assert torch.allclose(M, Mf, rtol=1e-4, atol=1e-3) and torch.allclose(z, zf, rtol=1e-5)
+
+
 def test_n64_bandwidth_sampled():
     w = wl.WORKLOADS["n64_bandwidth"]
     check_sampled(w, chains=[(1, 5)], segs=[0, 1, 8191, 16383])
