@@ -277,6 +277,14 @@ __device__ __forceinline__ float ex2(float x)
     return y;
 }
 
+// The feature map sigma(x) = ELU(x) + 1 (x + 1 for x > 0, e^x otherwise) without a branch:
+// for x > 0, e^min(x,0) = 1 < x + 1; for x <= 0, e^x >= x + 1.  So the larger of x + 1 and
+// e^min(x,0) is sigma(x) everywhere, and a warp never diverges on the sign of x.
+__device__ __forceinline__ float elu1(float x)
+{
+    return fmaxf(x + 1.f, ex2(fminf(x, 0.f) * 1.4426950408889634f));
+}
+
 // Packed fp32 pairs (sm_100 f32x2 arithmetic: one instruction for two lanes of work).
 __device__ __forceinline__ uint64_t f2_pack(float lo, float hi)
 {

@@ -46,8 +46,8 @@ k_sigma_bf16(const __nv_bfloat16 *__restrict__ x, __nv_bfloat16 *__restrict__ y,
         for (int e = 0; e < 4; ++e) {
             __nv_bfloat162 t = *reinterpret_cast<__nv_bfloat162 *>(&w[e]);
             float a = __low2float(t), b = __high2float(t);
-            a = a > 0.f ? a + 1.f : __expf(a);
-            b = b > 0.f ? b + 1.f : __expf(b);
+            a = elu1(a);
+            b = elu1(b);
             w[e] = pack_bf16x2(a, b);
         }
         dst[i] = make_uint4(w[0], w[1], w[2], w[3]);

@@ -51,7 +51,7 @@ struct LinArgs {
 
 enum : int { WL_KV_EMPTY = 301, WL_A = 302, WL_KV_FULL = 303, WL_SEG = 304, WL_DRAIN = 305 };
 
-__device__ __forceinline__ float sigma_lin(float x) { return x > 0.f ? x + 1.f : __expf(x); }
+__device__ __forceinline__ float sigma_lin(float x) { return elu1(x); }
 
 template <int D>
 __global__ void __launch_bounds__(256, 1)

@@ -38,6 +38,7 @@ struct PieceCfg {
     static constexpr int D = 64, TOK = 128, SEG = 64, ST = 2;
     static constexpr int THREADS = 416;
     static constexpr int MAX_UNITS = 16;              // units per piece
+    static constexpr int PREFETCH = 6;                // steps the L2 prefetch runs ahead
     static constexpr int BOX = 128 * 128;             // 128 rows x 64 bf16
     static constexpr int STAGE = 3 * BOX;             // Q, K, V of one unit
     static constexpr int OFF_SK = ST * STAGE;         // sigma(K), one per work group
@@ -237,9 +238,8 @@ k_small_pieces(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             prefetch_tmap(&tmQ);
             prefetch_tmap(&tmK);
             prefetch_tmap(&tmV);
-            uint32_t g = 0, cA[2] = {0, 0}, cB[2] = {0, 0};
-            uint64_t *lastbar[2] = {nullptr, nullptr};
-            uint32_t lastpar[2] = {0, 0};
+            // per stage: A- and B-loads issued so far, and the barrier / parity of the last one
+            uint32_t g = 0, cA0 = 0, cA1 = 0, cB0 = 0, cB1 = 0, last0 = 0, last1 = 0;
             bool ok = true;
             for (int k = 0; ok; ++k) {
                 if (k >= 2 && !(ok = mbar_wait_short(info_empty + (k & 1), ((k >> 1) - 1) & 1, abort, WP_INFO)))
@@ -251,15 +251,27 @@ k_small_pieces(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                 if (t < 0) break;
                 int chain, pc, u0, n;
                 piece_units(t, chain, pc, u0, n);
+                // L2 prefetch of the piece's tiles a few steps ahead of the loads (the loads
+                // are limited to two stages in flight, too few to cover HBM latency alone)
+                auto prefetch = [&](int x) {
+                    if (x >= 2 * n) return;
+                    const int row = (u0 + (x < n ? x : x - n)) * C::TOK;
+                    if (x >= n) tma_prefetch_l2_3d(&tmQ, 0, row, chain);
+                    tma_prefetch_l2_3d(&tmK, 0, row, chain);
+                    tma_prefetch_l2_3d(&tmV, 0, row, chain);
+                };
+                for (int x = 0; x < C::PREFETCH; ++x) prefetch(x);
                 for (int phase = 0; ok && phase < 2; ++phase)
                     for (int i = 0; i < n; ++i, ++g) {
                         const int w = g & 1;
+                        prefetch(phase * n + i + C::PREFETCH);
                         if (g >= 2 && !(ok = mbar_wait_short(kv_empty + w, ((g >> 1) - 1) & 1, abort, WP_KVE)))
                             break;
                         const int row = (u0 + i) * C::TOK;
                         uint64_t *bar = phase ? fullB + w : fullA + w;
-                        lastbar[w] = bar;
-                        lastpar[w] = (phase ? cB[w]++ : cA[w]++) & 1;
+                        const uint32_t use = phase ? (w ? cB1++ : cB0++) : (w ? cA1++ : cA0++);
+                        // bits: parity, B (1) or A (0), valid
+                        (w ? last1 : last0) = (use & 1) | (phase << 1) | 4;
                         mbar_arrive_expect_tx(bar, (phase ? 3 : 2) * C::BOX);
                         if (phase) tma_load_3d(stage_q(w), &tmQ, bar, 0, row, chain);
                         tma_load_3d(stage_k(w), &tmK, bar, 0, row, chain);
@@ -267,8 +279,8 @@ k_small_pieces(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                     }
             }
             // nothing may still be landing in shared memory when the CTA exits
-            for (int w = 0; w < 2; ++w)
-                if (lastbar[w]) piece_drain(lastbar[w], lastpar[w]);
+            if (last0) piece_drain(((last0 >> 1) & 1) ? fullB : fullA, last0 & 1);
+            if (last1) piece_drain(((last1 >> 1) & 1) ? fullB + 1 : fullA + 1, last1 & 1);
         }
     } else if (warp == 3) {
         if (lane == 0) {
@@ -276,7 +288,7 @@ k_small_pieces(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             constexpr uint32_t idV = idesc_bf16(128, 64, 1, 1);     // sigma(K)^T V
             constexpr uint32_t idZ = idesc_bf16(128, 16, 1, 0);     // sigma(K)^T 1
             const uint32_t aOnes = smem_u32(smem + C::OFF_ONES);
-            uint32_t g = 0, cA[2] = {0, 0}, cB[2] = {0, 0}, nfree = 0;
+            uint32_t g = 0, cA0 = 0, cA1 = 0, cB0 = 0, cB1 = 0, nfree = 0;
             bool ok = true, first = true;
             // rows 64-127 of the A operand (features 64-127 do not exist) read whatever
             // follows sigma(K) in shared memory; those TMEM lanes are never read
@@ -301,7 +313,7 @@ k_small_pieces(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                 piece_units(t, chain, pc, u0, n);
                 for (int i = 0; ok && i < n; ++i, ++g) {                 // A-steps
                     const int w = g & 1;
-                    if (!(ok = mbar_wait_short(fullA + w, cA[w]++ & 1, abort, WP_FULL))) break;
+                    if (!(ok = mbar_wait_short(fullA + w, (w ? cA1++ : cA0++) & 1, abort, WP_FULL))) break;
                     if (!(ok = mbar_wait_short(sig_full + w, (g >> 1) & 1, abort, WP_SIG))) break;
                     if (i == 0 && !first && !(ok = wait_free())) break;
                     first = false;
@@ -314,7 +326,7 @@ k_small_pieces(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                 }
                 for (int i = 0; ok && i < n; ++i, ++g) {                 // B-steps
                     const int w = g & 1;
-                    if (!(ok = mbar_wait_short(fullB + w, cB[w]++ & 1, abort, WP_FULL))) break;
+                    if (!(ok = mbar_wait_short(fullB + w, (w ? cB1++ : cB0++) & 1, abort, WP_FULL))) break;
                     if (!(ok = mbar_wait_short(sig_full + w, (g >> 1) & 1, abort, WP_SIG))) break;
                     if (!(ok = wait_free())) break;                          // memory before the unit
                     tc_fence_after();
@@ -336,7 +348,7 @@ k_small_pieces(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             // ------------------------------------------------ attention MMAs
             constexpr uint32_t idS = idesc_bf16(128, 128, 0, 0);
             constexpr uint32_t idO = idesc_bf16(128, 64, 0, 1);
-            uint32_t g = 0, cB[2] = {0, 0};
+            uint32_t g = 0, cB0 = 0, cB1 = 0;
             bool ok = true, have_prev = false;
             int pw = 0, pj = 0;
             // P V of a unit, then its retrieval added to the same accumulator
@@ -375,7 +387,7 @@ k_small_pieces(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                 have_prev = false;
                 g += n;                                                     // A-steps
                 for (int i = 0; ok && i < n; ++i, ++g) {                   // B-steps
-                    const int w = g & 1, j = cB[w]++;
+                    const int w = g & 1, j = w ? cB1++ : cB0++;
                     if (!(ok = mbar_wait_short(fullB + w, j & 1, abort, WP_FULL))) break;
                     if (j >= 1 && !(ok = mbar_wait_short(pv_done + w, (j - 1) & 1, abort, WP_PV))) break;
                     tc_fence_after();
@@ -402,9 +414,11 @@ k_small_pieces(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         const int rr = r < 64 ? r : r + 64;                      // row in the sigma(Q) buffer
         uint32_t g = 0, cA = 0, cB = 0;                          // this group's A- / B-steps
         bool ok = true;
-        // sigma of row r of a 128 x 64 tile into row dr of dst (same swizzle: dr % 8 == r % 8)
+        // sigma of row r of a 128 x 64 tile into row dr of dst (same swizzle: dr % 8 == r % 8).
+        // Not unrolled: with five roles on each SM sub-partition, instruction-cache misses
+        // cost more than the loop overhead.
         auto sigma_row_to = [&](const uint8_t *src, uint8_t *dst, int dr) {
-#pragma unroll
+#pragma unroll 1
             for (int ch = 0; ch < 8; ++ch) {
                 const int c = (ch ^ (r & 7)) << 4;
                 const uint4 x = *reinterpret_cast<const uint4 *>(src + r * 128 + c);
@@ -412,7 +426,7 @@ k_small_pieces(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     __nv_bfloat162 t2 = *reinterpret_cast<__nv_bfloat162 *>(&w4[e]);
-                    w4[e] = pack_bf16x2(sigma_s(__low2float(t2)), sigma_s(__high2float(t2)));
+                    w4[e] = pack_bf16x2(elu1(__low2float(t2)), elu1(__high2float(t2)));
                 }
                 *reinterpret_cast<uint4 *>(dst + dr * 128 + c) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
             }
@@ -550,7 +564,7 @@ k_small_pieces(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         // ---------------------------------------------------- memory rows (warps 0-1)
         const int r = threadIdx.x;                               // key feature 0..63
         const uint32_t tACC = tmem + C::T_ACC + ((uint32_t)(warp * 32) << 16);
-        uint32_t g = 0, cB[2] = {0, 0}, nfull = 0;              // steps; B-steps per slot
+        uint32_t g = 0, cB0 = 0, cB1 = 0, nfull = 0;            // steps; B-steps per slot
         bool ok = true;
         float ex[D + 1];                                         // memory before the piece
         auto wait_full = [&]() -> bool {
@@ -585,7 +599,8 @@ k_small_pieces(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         };
         // a slot's memory buffers are free once its previous unit's retrieval has run
         auto wait_slot = [&](int w) -> bool {
-            return cB[w] == 0 || mbar_wait(o_full + w, (cB[w] - 1) & 1, abort, WP_O);
+            const uint32_t c = w ? cB1 : cB0;
+            return c == 0 || mbar_wait(o_full + w, (c - 1) & 1, abort, WP_O);
         };
         for (int k = 0; ok; ++k) {
             int t;
@@ -743,7 +758,7 @@ k_small_pieces(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                 mbar_arrive(acc_free);
                 fence_proxy_async_smem();
                 mbar_arrive(m_ready + w);
-                ++cB[w];
+                if (w) ++cB1; else ++cB0;
                 // the next unit's buffers must be free before its memory is written
                 if (i + 1 < n && !(ok = wait_slot(w ^ 1))) break;
                 if (!(ok = wait_full())) break;                       // after the unit

@@ -326,8 +326,8 @@ k_segment_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
                     for (int e = 0; e < 4; ++e) {
                         __nv_bfloat162 t = *reinterpret_cast<__nv_bfloat162 *>(&w[e]);
                         float x0 = __low2float(t), x1 = __high2float(t);
-                        x0 = x0 > 0.f ? x0 + 1.f : __expf(x0);
-                        x1 = x1 > 0.f ? x1 + 1.f : __expf(x1);
+                        x0 = elu1(x0);
+                        x1 = elu1(x1);
                         const int c = cb * 64 + ch * 8 + 2 * e;
                         den = fmaf(x0, sZ[c], den);
                         den = fmaf(x1, sZ[c + 1], den);

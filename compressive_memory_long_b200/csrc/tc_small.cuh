@@ -95,7 +95,7 @@ __device__ __forceinline__ void st_release_gpu(int *p, int v)
     asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-__device__ __forceinline__ float sigma_s(float x) { return x > 0.f ? x + 1.f : __expf(x); }
+__device__ __forceinline__ float sigma_s(float x) { return elu1(x); }
 
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16])
 {
@@ -247,18 +247,23 @@ k_small_linear_fused(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         float *sAgg = reinterpret_cast<float *>(smem + C::OFF_AGG);
         float *sD0 = reinterpret_cast<float *>(smem + C::OFF_D0);
         float *sEx = reinterpret_cast<float *>(smem + C::OFF_EX);
-        auto sigma_row = [&](const uint8_t *src, uint8_t *dst) {   // bf16 row r, same swizzle
+        // bf16 row r, same swizzle; the whole row is loaded before the first store so the
+        // loads are not serialised behind stores that might alias them
+        auto sigma_row = [&](const uint8_t *src, uint8_t *dst) {
+            uint4 x[8];
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch)
+                x[ch] = *reinterpret_cast<const uint4 *>(src + r * 128 + ((ch ^ (r & 7)) << 4));
 #pragma unroll
             for (int ch = 0; ch < 8; ++ch) {
-                const int o = r * 128 + ((ch ^ (r & 7)) << 4);
-                const uint4 x = *reinterpret_cast<const uint4 *>(src + o);
-                uint32_t w[4] = {x.x, x.y, x.z, x.w};
+                uint32_t w[4] = {x[ch].x, x[ch].y, x[ch].z, x[ch].w};
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     __nv_bfloat162 t2 = *reinterpret_cast<__nv_bfloat162 *>(&w[e]);
                     w[e] = pack_bf16x2(sigma_s(__low2float(t2)), sigma_s(__high2float(t2)));
                 }
-                *reinterpret_cast<uint4 *>(dst + o) = make_uint4(w[0], w[1], w[2], w[3]);
+                *reinterpret_cast<uint4 *>(dst + r * 128 + ((ch ^ (r & 7)) << 4)) =
+                    make_uint4(w[0], w[1], w[2], w[3]);
             }
         };
         bool ok = mbar_wait_short(full, 0, abort, WS_FULL);
