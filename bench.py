@@ -20,6 +20,7 @@ instead, on bounded samples of the same workload.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import os
 import statistics
@@ -44,8 +45,14 @@ FLUSH_BYTES = 256 << 20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from an ncu
-# capture, keyed by (workload, kernel).  Absent: no capture of the current kernel.
-NCU_TRAFFIC_BYTES: dict = {}
+# capture, keyed by (workload, kernel).  Absent: no capture of the current kernel.  The
+# summaries with the commands are under profiles/.  The N = 64 bandwidth figure is the
+# 2048-segment capture scaled to 16384 segments (traffic grows with the units processed).
+NCU_TRAFFIC_BYTES: dict = {
+    ("hf_repro_n64", "small_fused"): 6359552,
+    ("gqa8b_n2048_delta", "segment_tc"): 408132608 + 236034560,
+    ("n64_bandwidth", "small_pieces"): (1445475000 + 280086016) * 8,
+}
 
 
 def load_peaks():
@@ -273,8 +280,13 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="CPU-oracle sample size for cpu_baseline (0 disables)")
+    ap.add_argument("--segments", type=int, default=0,
+                    help="run the workload with this many segments instead (small profiling "
+                         "captures of a large workload's kernels); 0 keeps the workload's own")
     args = ap.parse_args()
     w = wl.WORKLOADS[args.workload]
+    if args.segments > 0:
+        w = dataclasses.replace(w, name=f"{w.name}@S{args.segments}", S=args.segments)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
 

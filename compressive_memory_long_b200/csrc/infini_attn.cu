@@ -364,8 +364,9 @@ int launch_small_fused(const Problem &p, const __nv_bfloat16 *q, const __nv_bflo
     if (!opt_in_smem<tc::k_small_linear_fused>(C::ALLOC)) return INFINI_ERR_CUDA;
     // few units per head: each sums its predecessors' aggregates directly
     const int direct = U <= 64 ? 1 : 0;
+    const int in_place = ((M0 && M0 == M_out) || (z0 && z0 == z_out)) ? 1 : 0;
     tc::SmallArgs a{beta, M0, z0, out, M_out, z_out, ticket, m0_done, flags, agg, incl,
-                    p.L, (int)U, (int)p.H, (int)chains, direct};
+                    p.L, (int)U, (int)p.H, (int)chains, direct, in_place};
     TRACED("small_fused", st);
     tc::k_small_linear_fused<<<(unsigned)units, 256, C::ALLOC, st>>>(mq, mk, mv, a);
     return INFINI_OK;

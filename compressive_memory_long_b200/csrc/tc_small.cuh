@@ -66,6 +66,7 @@ struct SmallArgs {
     int U, H;
     int chains;
     int direct;                    // 1: every unit sums M0 and all earlier aggregates itself
+    int in_place;                  // 1: M_out / z_out are the very buffers M0 / z0
 };
 
 enum : int { FLAG_AGG = 1, FLAG_INCL = 2 };
@@ -247,23 +248,20 @@ k_small_linear_fused(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         float *sAgg = reinterpret_cast<float *>(smem + C::OFF_AGG);
         float *sD0 = reinterpret_cast<float *>(smem + C::OFF_D0);
         float *sEx = reinterpret_cast<float *>(smem + C::OFF_EX);
-        // bf16 row r, same swizzle; the whole row is loaded before the first store so the
-        // loads are not serialised behind stores that might alias them
+        // bf16 row r, same swizzle.  Not unrolled: the kernel runs its code once per CTA, so
+        // fewer distinct instructions (instruction-cache misses) matter more than loop overhead.
         auto sigma_row = [&](const uint8_t *src, uint8_t *dst) {
-            uint4 x[8];
-#pragma unroll
-            for (int ch = 0; ch < 8; ++ch)
-                x[ch] = *reinterpret_cast<const uint4 *>(src + r * 128 + ((ch ^ (r & 7)) << 4));
-#pragma unroll
+#pragma unroll 1
             for (int ch = 0; ch < 8; ++ch) {
-                uint32_t w[4] = {x[ch].x, x[ch].y, x[ch].z, x[ch].w};
+                const int o = r * 128 + ((ch ^ (r & 7)) << 4);
+                const uint4 x = *reinterpret_cast<const uint4 *>(src + o);
+                uint32_t w[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     __nv_bfloat162 t2 = *reinterpret_cast<__nv_bfloat162 *>(&w[e]);
                     w[e] = pack_bf16x2(sigma_s(__low2float(t2)), sigma_s(__high2float(t2)));
                 }
-                *reinterpret_cast<uint4 *>(dst + r * 128 + ((ch ^ (r & 7)) << 4)) =
-                    make_uint4(w[0], w[1], w[2], w[3]);
+                *reinterpret_cast<uint4 *>(dst + o) = make_uint4(w[0], w[1], w[2], w[3]);
             }
         };
         bool ok = mbar_wait_short(full, 0, abort, WS_FULL);
@@ -414,10 +412,10 @@ k_small_linear_fused(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                 for (int j = 0; j < unit; ++j) add_state(a.agg + (chain * a.U + j) * C::STATE);
                 add_initial();
             }
-            // the last unit may overwrite M0 / z0 (they may alias M_out / z_out) only after
-            // every other unit of the head has read them
+            // in place, the last unit may overwrite M0 / z0 only after every other unit of
+            // the head has read them
             asm volatile("bar.sync 1, 128;" ::: "memory");
-            if (ok && r == 0) {
+            if (ok && r == 0 && a.in_place) {
                 __threadfence();
                 if (unit + 1 < a.U) {
                     atomicAdd(a.m0_done + chain, 1);
