@@ -238,6 +238,7 @@ k_small_pieces(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             prefetch_tmap(&tmQ);
             prefetch_tmap(&tmK);
             prefetch_tmap(&tmV);
+            const uint64_t pol_last = l2_policy_evict_last(), pol_first = l2_policy_evict_first();
             // per stage: A- and B-loads issued so far, and the barrier / parity of the last one
             uint32_t g = 0, cA0 = 0, cA1 = 0, cB0 = 0, cB1 = 0, last0 = 0, last1 = 0;
             bool ok = true;
@@ -273,9 +274,12 @@ k_small_pieces(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                         // bits: parity, B (1) or A (0), valid
                         (w ? last1 : last0) = (use & 1) | (phase << 1) | 4;
                         mbar_arrive_expect_tx(bar, (phase ? 3 : 2) * C::BOX);
-                        if (phase) tma_load_3d(stage_q(w), &tmQ, bar, 0, row, chain);
-                        tma_load_3d(stage_k(w), &tmK, bar, 0, row, chain);
-                        tma_load_3d(stage_v(w), &tmV, bar, 0, row, chain);
+                        // keys and values stay in L2 from the A-step to the B-step of their
+                        // unit; queries and the B-step's second read are last uses
+                        const uint64_t pol = phase ? pol_first : pol_last;
+                        if (phase) tma_load_3d_hint(stage_q(w), &tmQ, bar, 0, row, chain, pol);
+                        tma_load_3d_hint(stage_k(w), &tmK, bar, 0, row, chain, pol);
+                        tma_load_3d_hint(stage_v(w), &tmV, bar, 0, row, chain, pol);
                     }
             }
             // nothing may still be landing in shared memory when the CTA exits
@@ -552,8 +556,8 @@ k_small_pieces(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                             pk[e] = pack_bf16x2(__uint_as_float(o[2 * e]), __uint_as_float(o[2 * e + 1]));
                         uint4 *dst = reinterpret_cast<uint4 *>(orow + c);
 #pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+                        for (int e = 0; e < 4; ++e)   // streaming: the output is not read again
+                            __stcs(dst + e, make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]));
                     }
                     tc_fence_before();
                     mbar_arrive(epi_done + wg);

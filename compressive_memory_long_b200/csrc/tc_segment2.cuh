@@ -32,7 +32,7 @@ struct Seg2Cfg {
     // register split (setmaxnreg): launched at REGS per thread; the producer / MMA warpgroup
     // gives back to REGS_LOW, each softmax warpgroup grows to REGS_HIGH.  The three shares add
     // up exactly to the launch's THREADS * REGS.
-    static constexpr int REGS = 168, REGS_LOW = 56, REGS_HIGH = 224;
+    static constexpr int REGS = 168, REGS_LOW = 88, REGS_HIGH = 208;
     static_assert(128 * (2 * REGS_HIGH + REGS_LOW) == THREADS * REGS, "register split");
     static constexpr int STAGES = (D == 128) ? 2 : 3;
     static constexpr int TILE = 128 * D * 2;

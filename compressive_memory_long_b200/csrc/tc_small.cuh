@@ -264,14 +264,53 @@ k_small_linear_fused(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                 *reinterpret_cast<uint4 *>(dst + o) = make_uint4(w[0], w[1], w[2], w[3]);
             }
         };
+        float l = 0.f;                  // softmax row sum
         bool ok = mbar_wait_short(full, 0, abort, WS_FULL);
         if (ok) {                       // sigma(K) first: the increment MMAs need only it
             sigma_row(sK, sSK);
             fence_proxy_async_smem();
             mbar_arrive(sig_ready);
         }
+        // ---- this unit's increments into shared memory: D0 (first segment), D0 + D1
+        if (ok) ok = mbar_wait_short(d_done, 0, abort, WS_D);
+        if (ok) {
+            tc_fence_after();
+#pragma unroll 1
+            for (int c0 = 0; c0 < 80; c0 += 16) {
+                uint32_t x[16], y[16];
+                tmem_ld16(lane_base + T_D0 + c0, x);
+                tmem_ld16(lane_base + T_D1 + c0, y);
+                tmem_ld_wait();
+                if (r < D) {
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const int col = c0 + e;
+                        if (col < C::ROW) {
+                            const float x0 = __uint_as_float(x[e]);
+                            sD0[r * C::ROW + col] = x0;
+                            sAgg[r * C::ROW + col] = x0 + __uint_as_float(y[e]);
+                        }
+                    }
+                }
+            }
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        // publish the aggregate (coalesced 16-byte stores by all 128 threads)
+        if (ok && (unit > 0 || a.direct)) {
+            float4 *dst = reinterpret_cast<float4 *>(a.agg + idx * C::STATE);
+            const float4 *src = reinterpret_cast<const float4 *>(sAgg);
+            for (int i = r; i < C::STATE4; i += 128) dst[i] = src[i];
+            __threadfence();
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        // Unit 0 of a long head publishes no aggregate, only its inclusive prefix: every other
+        // walk then ends at an inclusive prefix, and only unit 0 reads M0 / z0 -- which M_out /
+        // z_out (written by the last unit, after its walk) may alias.
+        if (ok && r == 0 && (unit > 0 || a.direct)) st_release_gpu(a.flags + idx, FLAG_AGG);
+
+        // the local softmax and sigma(Q) come after the aggregate is published: later units
+        // of the head wait for it, while this unit's own softmax is not on their path
         // ---- local softmax: row r sees the 64 keys of its own segment, up to itself
-        float l = 0.f;
         if (ok) ok = mbar_wait_short(s_done, 0, abort, WS_S);
         if (ok) {
             tc_fence_after();
@@ -315,42 +354,6 @@ k_small_linear_fused(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             mbar_arrive(p_ready);
         }
         if (ok) sigma_row(sQ, sSQ);    // sigma(Q) for the retrieval, off the critical path
-        // ---- this unit's increments into shared memory: D0 (first segment), D0 + D1
-        if (ok) ok = mbar_wait_short(d_done, 0, abort, WS_D);
-        if (ok) {
-            tc_fence_after();
-#pragma unroll 1
-            for (int c0 = 0; c0 < 80; c0 += 16) {
-                uint32_t x[16], y[16];
-                tmem_ld16(lane_base + T_D0 + c0, x);
-                tmem_ld16(lane_base + T_D1 + c0, y);
-                tmem_ld_wait();
-                if (r < D) {
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const int col = c0 + e;
-                        if (col < C::ROW) {
-                            const float x0 = __uint_as_float(x[e]);
-                            sD0[r * C::ROW + col] = x0;
-                            sAgg[r * C::ROW + col] = x0 + __uint_as_float(y[e]);
-                        }
-                    }
-                }
-            }
-        }
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        // publish the aggregate (coalesced 16-byte stores by all 128 threads)
-        if (ok && (unit > 0 || a.direct)) {
-            float4 *dst = reinterpret_cast<float4 *>(a.agg + idx * C::STATE);
-            const float4 *src = reinterpret_cast<const float4 *>(sAgg);
-            for (int i = r; i < C::STATE4; i += 128) dst[i] = src[i];
-            __threadfence();
-        }
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        // Unit 0 of a long head publishes no aggregate, only its inclusive prefix: every other
-        // walk then ends at an inclusive prefix, and only unit 0 reads M0 / z0 -- which M_out /
-        // z_out (written by the last unit, after its walk) may alias.
-        if (ok && r == 0 && (unit > 0 || a.direct)) st_release_gpu(a.flags + idx, FLAG_AGG);
 
         // ---- exclusive prefix of this unit, kept as float4 per thread (i = r + 128 k)
         constexpr int KQ = (C::STATE4 + 127) / 128;
