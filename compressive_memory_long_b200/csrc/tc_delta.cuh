@@ -10,14 +10,14 @@
 // d/16 CTAs run side by side.  sigma(K) is computed once per token beforehand
 // (k_sigma_bf16) and read here through TMA.  Per 128-token chunk g:
 //   1. TMA brings sigma(K) (128 x d, 128-byte swizzle) and V[:, cols] (128 x 16).
-//   2. One thread issues R = sigma(K) B^T with B = [M^T | z | 0 | M_lo^T | z_lo | 0] (64 rows,
-//      bf16: M and z split into hi + lo parts, side by side so one N = 64 MMA reads the
-//      sigma(K) tile once): R[0..15] + R[32..47] are the prediction numerators, R[16] + R[48]
-//      is den_t.
+//   2. One thread issues R = sigma(K) B^T with B = [M^T | z | 0 | M_lo^T | z_lo | 0] (48 rows,
+//      bf16: M and z split into hi + lo parts, side by side so one N = 48 MMA reads the
+//      sigma(K) tile once; the lo half starts at row 24): R[0..15] + R[24..39] are the
+//      prediction numerators, R[16] + R[40] is den_t.
 //   3. Thread t forms U_t and writes [U_hi | 1 | 0 | U_lo | 0]^T (the residual is a small
 //      difference of large terms: one bf16 rounding of it would cost ~1e-2 of M).
 //   4. One thread issues Macc += sigma(K)^T [U_hi | 1 | 0 | U_lo | 0] (sigma(K) read as the
-//      MN-major operand): M[:, cols] = Macc[0..15] + Macc[32..47], z = Macc[16], in fp32.
+//      MN-major operand): M[:, cols] = Macc[0..15] + Macc[24..39], z = Macc[16], in fp32.
 // Within a segment every R reads the same M_{s-1}, so R(g+1) is issued before the update of
 // chunk g (R accumulators and U tiles double-buffered); only the first chunk of a segment
 // waits for B (the initial state, or the boundary where thread c -- TMEM lane c = key
@@ -56,14 +56,14 @@ k_sigma_bf16(const __nv_bfloat16 *__restrict__ x, __nv_bfloat16 *__restrict__ y,
 
 struct ChainCfg {
     static constexpr int CB = 16;                 // value columns per CTA
-    static constexpr int NB = 64;                 // rows of the B operands (hi half, lo half)
-    static constexpr int LO = 32;                 // first row of the lo half
+    static constexpr int NB = 48;                 // rows of the B operands (hi half, lo half)
+    static constexpr int LO = 24;                 // first row of the lo half (a multiple of 8)
     static constexpr int ST = 4;                  // sigma(K)/V stages
     static constexpr int KBOX = 128 * 128;        // 128 rows x 64 bf16
     static constexpr int KTILE = 2 * KBOX;        // 128 tokens x 128 features (padded)
     static constexpr int VTILE = 128 * CB * 2;    // 128 tokens x 16 bf16, unswizzled
-    static constexpr int BBOX = NB * 128;         // 64 rows x 64 bf16
-    static constexpr int BTILE = 2 * BBOX;        // 64 rows x 128 (features or tokens)
+    static constexpr int BBOX = NB * 128;         // 48 rows x 64 bf16
+    static constexpr int BTILE = 2 * BBOX;        // 48 rows x 128 (features or tokens)
     static constexpr int OFF_K = 0;
     static constexpr int OFF_V = OFF_K + ST * KTILE;
     static constexpr int OFF_B = OFF_V + ST * VTILE;    // [M | z]^T, hi and lo halves
@@ -229,10 +229,10 @@ k_delta_chain_tc(const __grid_constant__ CUtensorMap tmSK, const __grid_constant
         const int r = threadIdx.x - 128;           // token row of a chunk / key feature row
         const uint32_t lane_base = (uint32_t)((warp - 4) * 32) << 16;
         const __nv_bfloat16 one = __float2bfloat16_rn(1.f), zero = __float2bfloat16_rn(0.f);
-        // constant rows of both [U | 1]^T tiles: 16 = ones, 17..31 and 48..63 = zeros
-        for (int i = r; i < 2 * 2 * 32 * 64; i += 128) {
-            const int buf = i / (2 * 32 * 64), box = (i / (32 * 64)) % 2, k32 = (i / 64) % 32;
-            const int rr = k32 < 16 ? 16 + k32 : 32 + k32;          // 16..31, 48..63
+        // constant rows of both [U | 1]^T tiles: 16 = ones, 17..23 and 40..47 = zeros
+        for (int i = r; i < 2 * 2 * 16 * 64; i += 128) {
+            const int buf = i / (2 * 16 * 64), box = (i / (16 * 64)) % 2, k16 = (i / 64) % 16;
+            const int rr = k16 < 8 ? 16 + k16 : 32 + k16;           // 16..23, 40..47
             const int t = i % 64;
             *reinterpret_cast<__nv_bfloat16 *>(sU + buf * C::BTILE + box * C::BBOX + rr * 128 +
                                                ((((t >> 3) ^ (rr & 7))) << 4) + (t & 7) * 2) =
