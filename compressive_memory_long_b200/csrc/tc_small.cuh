@@ -98,6 +98,21 @@ __device__ __forceinline__ void st_release_gpu(int *p, int v)
 
 __device__ __forceinline__ float sigma_s(float x) { return elu1(x); }
 
+// Named barrier 1 over the 128 work threads that also ORs a predicate across them.
+__device__ __forceinline__ bool bar_or_128(bool v)
+{
+    uint32_t out;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, 1, 128, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(out)
+        : "r"((uint32_t)v)
+        : "memory");
+    return out != 0;
+}
+
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16])
 {
     asm volatile(
@@ -155,6 +170,7 @@ k_small_linear_fused(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         mbar_init(r_done, 1);
         mbar_init(mma_done, 1);
         *abort = 0;
+        *s_state = 0;
         fence_barrier_init();
     }
     if (warp == 1) tmem_alloc(tmem_holder, 512);
@@ -389,25 +405,22 @@ k_small_linear_fused(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             }
         };
         if (a.direct) {
-            // wait until every earlier unit of the head has published its aggregate
-            if (ok && r == 0) {
-                int f = 0;
-                for (int j = 0; j < unit && f >= 0; ++j) {
-                    const int *fp = a.flags + chain * a.U + j;
-                    const long long t0 = clock64();
-                    while ((f = ld_acquire_gpu(fp)) == 0) {
-                        if (clock64() - t0 > kSpinLimitCycles || wait_status_set()) {
-                            atomicCAS(&g_wait_status, 0, WS_LOOK);
-                            f = -1;
-                            break;
-                        }
-                        __nanosleep(32);
+            // wait until every earlier unit of the head has published its aggregate: thread j
+            // watches unit j, so the flags are polled side by side (unit < 64 <= 128 here)
+            bool bad = false;
+            if (ok && r < unit) {
+                const int *fp = a.flags + chain * a.U + r;
+                const long long t0 = clock64();
+                while (ld_acquire_gpu(fp) == 0) {
+                    if (clock64() - t0 > kSpinLimitCycles || wait_status_set()) {
+                        atomicCAS(&g_wait_status, 0, WS_LOOK);
+                        bad = true;
+                        break;
                     }
+                    __nanosleep(32);
                 }
-                *s_state = f;
             }
-            asm volatile("bar.sync 1, 128;" ::: "memory");
-            if (ok && unit > 0 && *s_state < 0) {
+            if (bar_or_128(bad) && ok) {
                 ok = false;
                 *abort = 1;
             }
@@ -477,6 +490,15 @@ k_small_linear_fused(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                 const int i = r + 128 * k;
                 if (i < C::STATE4) {
                     sEx4[i] = ex[k];
+                    if (unit + 1 == a.U) {                  // the head's final state
+                        const float4 g = sAgg4[i];
+                        const int row = i / (C::ROW / 4), c4 = i % (C::ROW / 4);
+                        if (c4 < D / 4)
+                            reinterpret_cast<float4 *>(a.M_out + (chain * D + row) * D)[c4] =
+                                make_float4(ex[k].x + g.x, ex[k].y + g.y, ex[k].z + g.z, ex[k].w + g.w);
+                        else
+                            a.z_out[chain * D + row] = ex[k].x + g.x;
+                    }
                     if (!a.direct && unit + 1 < a.U) {      // inclusive prefix for successors
                         const float4 g = sAgg4[i];
                         reinterpret_cast<float4 *>(a.incl + idx * C::STATE)[i] =
@@ -490,13 +512,7 @@ k_small_linear_fused(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         if (ok) {
             if (r == 0 && !a.direct && unit + 1 < a.U) st_release_gpu(a.flags + idx, FLAG_INCL);
             if (r < D) {
-                const float *exr = sEx + r * C::ROW, *d0r = sD0 + r * C::ROW, *agr = sAgg + r * C::ROW;
-                if (unit + 1 == a.U) {                 // the head's final state
-                    float *mo = a.M_out + (chain * D + r) * D;
-#pragma unroll 8
-                    for (int q = 0; q < D; ++q) mo[q] = exr[q] + agr[q];
-                    a.z_out[chain * D + r] = exr[D] + agr[D];
-                }
+                const float *exr = sEx + r * C::ROW, *d0r = sD0 + r * C::ROW;
                 // M_start and M_mid rows (key r) as bf16 B operands, z as fp32
 #pragma unroll
                 for (int ch = 0; ch < 8; ++ch) {
