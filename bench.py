@@ -5,6 +5,12 @@ One step = one full forward (every segment's local attention, memory retrieval, 
 memory update) over one batch of the workload's synthetic inputs, through the C ABI.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+                  [--tail T] [--decode]
+
+``--tail T`` appends a final segment of T < N tokens to every head of the workload.
+``--decode`` times the token-by-token decode step instead of the forward: one step is one
+segment of N tokens fed one at a time (every batch row and head per call), the fold of
+the segment into the memory included; tokens/s counts B * N tokens per step.
 
 Prints ONE JSON line on rank 0.  Under torchrun (N > 1) every rank runs its own batch of
 the workload on its own GPU (independent problems: no data-path collective, weak
@@ -37,6 +43,7 @@ if ROOT not in sys.path:
 from compressive_memory_long_b200 import workloads as wl  # noqa: E402
 
 METRIC = "Infini-attention fwd tokens/s at 1 B200; % of bf16 TC peak or HBM roofline"
+DECODE_METRIC = "Infini-attention decode tokens/s at 1 B200 (one token per call, per sequence)"
 DEFAULT_WORKLOAD = "hf_repro_n64"
 FLUSH_BYTES = 256 << 20
 
@@ -76,6 +83,12 @@ def algorithmic(w: wl.Workload, kernel: str):
     e = w.elem_bytes
     B, H, Hkv, L, N, d, S = w.B, w.H, w.Hkv, w.L, w.N, w.d, w.S
     state_bytes = 2 * B * Hkv * (d * d + d) * 4
+    if kernel == "decode_attn":     # one token per (b, h): the cached rows once, M and z once
+        rows = (N - 2) / 2.0            # average cached rows over offsets 0 .. N - 2
+        byts = (B * Hkv * (2 * rows * d * e + (d * d + d) * 4) + 2 * B * H * d * e
+                + 2 * B * Hkv * d * e)
+        flops = B * H * (4 * d * (rows + 1) + 2 * d * d)
+        return flops, byts
     if kernel in ("small_fused", "small_pieces"):     # the whole forward in one launch
         f1, b1 = algorithmic(w, "segment")
         f2, b2 = algorithmic(w, "linear_state")
@@ -233,7 +246,7 @@ def oracle_sample(w: wl.Workload, seconds: float):
     return tok / dt, dt, desc
 
 
-def run_reference(args, w: wl.Workload):
+def run_reference(args, w: wl.Workload, metric: str = METRIC):
     world, rank, _ = dist_env()
     if rank != 0:
         return 0
@@ -248,7 +261,7 @@ def run_reference(args, w: wl.Workload):
         secs += dt
     value = float(statistics.mean(vals))
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "impl": "reference", "metric": metric, "value": value, "unit": "tokens/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1000.0 * secs / max(1, args.steps), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
@@ -264,9 +277,149 @@ def run_reference(args, w: wl.Workload):
 
 def config_of(w: wl.Workload):
     return {"workload": w.name, "B": w.B, "H": w.H, "Hkv": w.Hkv, "d": w.d, "N": w.N,
-            "S": w.S, "L": w.L, "rule": w.rule, "activations": w.dtype,
+            "S": w.S, "tail": w.tail, "L": w.L, "rule": w.rule, "activations": w.dtype,
             "l2": "256 MiB write before every step (L2 flushed)",
             "description": w.description}
+
+
+# ---- the decode step (our arm, --decode) ----
+
+def run_decode(args, w: wl.Workload, world: int, rank: int, local: int, dev):
+    """One step = the N tokens of one segment through infini_attn_decode_step, one call per
+    token (all batch rows and heads at once); the call at offset N - 1 folds the segment.
+
+    The N calls of a step are captured once in a CUDA graph (the calls allocate nothing),
+    and the timed region replays it: device time without the host's per-call overhead.
+    The decode kernel's own time comes from a second graph of the calls at offsets
+    0 .. N - 2 (no fold).  ``e2e`` makes the same calls eagerly from Python, each token's
+    inputs copied from pinned host memory and its output copied back.
+    """
+    from compressive_memory_long_b200 import binding
+    host = wl.torch_inputs(w, pin_memory=True)
+    # per-token slabs [N, B, heads, d], contiguous per token
+    tok = {n: host[n].permute(2, 0, 1, 3).contiguous().pin_memory() for n in ("q", "k", "v")}
+    t = {n: x.to(dev, non_blocking=True) for n, x in tok.items()}
+    beta = host["beta"].to(dev)
+    dt = w.torch_dtype
+    kc = torch.zeros((w.B, w.Hkv, w.N, w.d), dtype=dt, device=dev)
+    vc = torch.zeros_like(kc)
+    M = torch.zeros((w.B, w.Hkv, w.d, w.d), dtype=torch.float32, device=dev)
+    z = torch.zeros((w.B, w.Hkv, w.d), dtype=torch.float32, device=dev)
+    outs = torch.empty((w.N, w.B, w.H, w.d), dtype=dt, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def calls(n_pos):
+        for p in range(n_pos):
+            binding.decode_step(t["q"][p], t["k"][p], t["v"][p], beta, kc, vc, p, M, z,
+                                rule=w.rule, out=outs[p])
+
+    for _ in range(2):
+        calls(w.N)
+    torch.cuda.synchronize(dev)
+    g_step, g_attn = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_step):
+        calls(w.N)
+    with torch.cuda.graph(g_attn):
+        calls(w.N - 1)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        flush.zero_()
+        g_step.replay()
+    torch.cuda.synchronize(dev)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clocks:
+        for i in range(args.steps):
+            flush.zero_()
+            starts[i].record(stream)
+            g_step.replay()
+            ends[i].record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(world)
+    total_ms = max_over_ranks(float(sum(s.elapsed_time(e) for s, e in zip(starts, ends))),
+                              world, dev)
+    per_step = w.N + (1 if w.rule == "linear" else 2)     # decode calls + fold kernels
+    launches = int(per_step * args.steps * world)
+    tokens = w.B * w.N * args.steps * world
+    value = tokens / (total_ms / 1000.0)
+
+    # the decode kernel alone: graph of the calls at offsets 0 .. N - 2
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = max(1, args.steps)
+    flush.zero_()
+    a0.record(stream)
+    for _ in range(reps):
+        g_attn.replay()
+    a1.record(stream)
+    torch.cuda.synchronize(dev)
+    n_attn = (w.N - 1) * reps
+    dom_ms = max_over_ranks(a0.elapsed_time(a1) / n_attn, world, dev)
+    peaks, peak_src = load_peaks()
+    flops, byts = algorithmic(w, "decode_attn")
+    achieved = byts / (dom_ms / 1e3) / 1e9
+    roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": achieved / peaks["hbm_gbs"], "traffic": None, "kernel": "decode_attn",
+            "kernel_ms": dom_ms, "peak_source": f"{peak_src} (burst)",
+            "algorithmic_flops": flops, "algorithmic_bytes": byts,
+            "kernel_share": dom_ms * w.N / (total_ms / args.steps)}
+    kernels = {"decode_attn": {"launches": n_attn, "ms": a0.elapsed_time(a1)}}
+    del g_step, g_attn
+
+    out_h = torch.empty(outs.shape, dtype=dt, pin_memory=True)
+    e_starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    e_ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+
+    def e2e_step(i=None):
+        if i is not None:
+            e_starts[i].record(stream)
+        for p in range(w.N):
+            for n in ("q", "k", "v"):
+                t[n][p].copy_(tok[n][p], non_blocking=True)
+            binding.decode_step(t["q"][p], t["k"][p], t["v"][p], beta, kc, vc, p, M, z,
+                                rule=w.rule, out=outs[p])
+            out_h[p].copy_(outs[p], non_blocking=True)
+        if i is not None:
+            e_ends[i].record(stream)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    for i in range(args.steps):
+        flush.zero_()
+        e2e_step(i)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    e2e_ms = max_over_ranks(float(sum(s.elapsed_time(e) for s, e in zip(e_starts, e_ends))),
+                            world, dev)
+    h2d = sum(x.numel() * x.element_size() for x in tok.values())
+    d2h = out_h.numel() * out_h.element_size()
+
+    cpu = None
+    if rank == 0 and world == 1 and args.cpu_seconds > 0:
+        v, sec, desc = oracle_sample(w, args.cpu_seconds)
+        cpu = {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+               "sample": "oracle forward over the same segment (the outputs the decode "
+                         f"reproduces): {desc}; {sec:.1f} s on 1 host core"}
+    if rank == 0:
+        line = {
+            "metric": DECODE_METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
+            "config": dict(config_of(w), timing="CUDA graph of one segment's calls"),
+            "roofline": roof, "cpu_baseline": cpu,
+            "e2e": {"value": w.B * w.N * args.steps * world / (e2e_ms / 1000.0),
+                    "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches, "kernels": kernels, "clocks": clocks.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
 
 
 # ---- our arm ----
@@ -280,6 +433,10 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="CPU-oracle sample size for cpu_baseline (0 disables)")
+    ap.add_argument("--tail", type=int, default=0,
+                    help="append a final segment of this many (< N) tokens to every head")
+    ap.add_argument("--decode", action="store_true",
+                    help="time the token-by-token decode step over one segment instead")
     ap.add_argument("--segments", type=int, default=0,
                     help="run the workload with this many segments instead (small profiling "
                          "captures of a large workload's kernels); 0 keeps the workload's own")
@@ -287,11 +444,17 @@ def main():
     w = wl.WORKLOADS[args.workload]
     if args.segments > 0:
         w = dataclasses.replace(w, name=f"{w.name}@S{args.segments}", S=args.segments)
+    if args.tail:
+        if not 0 < args.tail < w.N:
+            ap.error("--tail must be in (0, N)")
+        w = dataclasses.replace(w, name=f"{w.name}+T{args.tail}", tail=args.tail)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.decode:
+        w = dataclasses.replace(w, name=f"{w.name}:decode", S=1, tail=0)
 
     if args.impl == "reference":
-        return run_reference(args, w)
+        return run_reference(args, w, DECODE_METRIC if args.decode else METRIC)
 
     world, rank, local = dist_env()
     if world != args.gpus:
@@ -305,6 +468,9 @@ def main():
                                 device_id=dev)
 
     from compressive_memory_long_b200 import binding
+
+    if args.decode:
+        return run_decode(args, w, world, rank, local, dev)
 
     host = wl.torch_inputs(w, pin_memory=True)
     t = {k: (None if x is None else x.to(dev, non_blocking=True)) for k, x in host.items()}

@@ -6,8 +6,9 @@ fails to load, importing this module raises.
 
 Names mirror the C ABI in ``include/infini_attn.h``:
 ``infini_attn_fwd`` (bf16), ``infini_attn_fwd_f32``, ``infini_attn_workspace_bytes``,
-``infini_attn_status_string``, ``infini_attn_version``; ``forward`` allocates the outputs
-and picks the entry point from q's dtype.
+``infini_attn_status_string``, ``infini_attn_version``, ``infini_attn_decode_step`` (+
+``_f32``), ``infini_attn_fold`` (+ ``_f32``); ``forward``, ``decode_step`` and ``fold``
+allocate what is missing and pick the entry point from the activation dtype.
 """
 from __future__ import annotations
 
@@ -28,10 +29,16 @@ STATUS = {0: "INFINI_OK", 1: "INFINI_ERR_INVALID_ARG", 2: "INFINI_ERR_UNSUPPORTE
 #: C functions and their (argtypes, restype), exactly as include/infini_attn.h declares them
 _P, _I64, _I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
 _FWD_ARGS = [_P] * 9 + [_I64] * 6 + [_I, _P]
+_DEC_ARGS = [_P] * 6 + [_I64] + [_P] * 3 + [_I64] * 5 + [_I, _P]
+_FOLD_ARGS = [_P, _P, _I64, _P, _P] + [_I64] * 4 + [_I, _P]
 SIGNATURES = {
     "infini_attn_fwd": (_FWD_ARGS, _I),
     "infini_attn_fwd_f32": (_FWD_ARGS, _I),
     "infini_attn_fwd_noalloc": (_FWD_ARGS, _I),
+    "infini_attn_decode_step": (_DEC_ARGS, _I),
+    "infini_attn_decode_step_f32": (_DEC_ARGS, _I),
+    "infini_attn_fold": (_FOLD_ARGS, _I),
+    "infini_attn_fold_f32": (_FOLD_ARGS, _I),
     "infini_attn_workspace_bytes": ([_I64] * 5, _I64),
     "infini_attn_status_string": ([_I], ctypes.c_char_p),
     "infini_attn_version": ([], _I),
@@ -170,3 +177,56 @@ def forward(q, k, v, beta, M0=None, z0=None, *, N: int, rule="linear", out=None,
     else:
         raise ValueError(f"unsupported activation dtype {q.dtype}")
     return out, M_out, z_out
+
+
+def decode_step(q, k, v, beta, k_cache, v_cache, pos: int, M, z, *, rule="linear", out=None,
+                stream=None):
+    """One token of every (batch, head) at offset ``pos`` of its current segment.
+
+    q [B,H,d], k/v [B,Hkv,d] (bf16 or fp32), beta [H] fp32, k_cache/v_cache [B,Hkv,N,d]
+    (the activation dtype; row ``pos`` is written), M [B,Hkv,d,d] / z [B,Hkv,d] fp32 (folded
+    in place when pos == N - 1).  Returns out [B,H,d].
+    """
+    B, H, d = q.shape
+    Hkv, N = k_cache.shape[1], k_cache.shape[2]
+    dev = q.device
+    _check(q, "q", q.dtype, (B, H, d), dev)
+    _check(k, "k", q.dtype, (B, Hkv, d), dev)
+    _check(v, "v", q.dtype, (B, Hkv, d), dev)
+    _check(beta, "beta", torch.float32, (H,), dev)
+    _check(k_cache, "k_cache", q.dtype, (B, Hkv, N, d), dev)
+    _check(v_cache, "v_cache", q.dtype, (B, Hkv, N, d), dev)
+    _check(M, "M", torch.float32, (B, Hkv, d, d), dev)
+    _check(z, "z", torch.float32, (B, Hkv, d), dev)
+    if out is None:
+        out = torch.empty_like(q)
+    if q.dtype == torch.bfloat16:
+        fn = LIB.infini_attn_decode_step
+    elif q.dtype == torch.float32:
+        fn = LIB.infini_attn_decode_step_f32
+    else:
+        raise ValueError(f"unsupported activation dtype {q.dtype}")
+    rc = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(k_cache), _ptr(v_cache), int(pos),
+            _ptr(M), _ptr(z), _ptr(out), B, H, Hkv, N, d, RULES[rule], _stream_handle(stream))
+    if rc != 0:
+        raise InfiniError(rc, infini_attn_status_string(rc))
+    return out
+
+
+def fold(k_cache, v_cache, n: int, M, z, *, rule="linear", stream=None):
+    """Fold the first ``n`` cached rows of every chain into (M, z), in place."""
+    B, Hkv, N, d = k_cache.shape
+    dev = k_cache.device
+    _check(v_cache, "v_cache", k_cache.dtype, (B, Hkv, N, d), dev)
+    _check(M, "M", torch.float32, (B, Hkv, d, d), dev)
+    _check(z, "z", torch.float32, (B, Hkv, d), dev)
+    if k_cache.dtype == torch.bfloat16:
+        fn = LIB.infini_attn_fold
+    elif k_cache.dtype == torch.float32:
+        fn = LIB.infini_attn_fold_f32
+    else:
+        raise ValueError(f"unsupported activation dtype {k_cache.dtype}")
+    rc = fn(_ptr(k_cache), _ptr(v_cache), int(n), _ptr(M), _ptr(z), B, Hkv, N, d, RULES[rule],
+            _stream_handle(stream))
+    if rc != 0:
+        raise InfiniError(rc, infini_attn_status_string(rc))

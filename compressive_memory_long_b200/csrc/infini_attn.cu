@@ -20,6 +20,7 @@
 #include "tc_linear.cuh"
 #include "tc_small.cuh"
 #include "tc_pieces.cuh"
+#include "decode.cuh"
 
 #include <cudaTypedefs.h>
 
@@ -33,8 +34,11 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[INFINI_NOALLOC_
 namespace infini {
 namespace {
 
+// L is the row count of every head (the row stride of q, k, v, out); S = floor(L / N) full
+// segments cover the first Lf = S * N rows and T = L - Lf rows (0 <= T < N) form a final,
+// shorter segment.
 struct Problem {
-    int64_t B, H, Hkv, L, N, d, S;
+    int64_t B, H, Hkv, L, N, d, S, Lf, T;
     int rule;
 };
 
@@ -65,7 +69,7 @@ int check_args(const void *q, const void *k, const void *v, const float *beta, c
 {
     if (!q || !k || !v || !beta || !out || !M_out || !z_out) return INFINI_ERR_INVALID_ARG;
     if (B <= 0 || H <= 0 || Hkv <= 0 || L <= 0 || N <= 0 || d <= 0) return INFINI_ERR_INVALID_ARG;
-    if (H % Hkv != 0 || L % N != 0) return INFINI_ERR_INVALID_ARG;
+    if (H % Hkv != 0) return INFINI_ERR_INVALID_ARG;
     if (rule != INFINI_UPDATE_LINEAR && rule != INFINI_UPDATE_DELTA) return INFINI_ERR_INVALID_ARG;
     // keep every element count far inside int64 and every grid inside 2^31 CTAs
     if (B > (1 << 20) || H > (1 << 16) || L > ((int64_t)1 << 34) ||
@@ -85,6 +89,7 @@ int check_args(const void *q, const void *k, const void *v, const float *beta, c
     if (d != 32 && d != 64 && d != 128) return INFINI_ERR_UNSUPPORTED;
     if (N % 64 != 0) return INFINI_ERR_UNSUPPORTED;
     pb->B = B; pb->H = H; pb->Hkv = Hkv; pb->L = L; pb->N = N; pb->d = d; pb->S = L / N;
+    pb->Lf = pb->S * N; pb->T = L - pb->Lf;
     pb->rule = rule;
     return INFINI_OK;
 }
@@ -236,7 +241,7 @@ int launch_delta_chain_tc(const Problem &p, const __nv_bfloat16 *k, const __nv_b
     using C = tc::ChainCfg;
     // sigma(K) once per token, into the workspace after the bf16 snapshots
     __nv_bfloat16 *sk = snapMb + p.B * p.Hkv * p.S * (int64_t)D * D;
-    const int64_t n8 = p.B * p.Hkv * p.L * (int64_t)D / 8;
+    const int64_t n8 = p.B * p.Hkv * p.L * (int64_t)D / 8;   // every row, the tail's too
     {
         int sms = 148;
         int dev = 0;
@@ -271,21 +276,24 @@ template <typename T>
 bool use_small_fused(const Problem &p)
 {
     return sizeof(T) == 2 && p.d == 64 && p.N == 64 && p.rule == INFINI_UPDATE_LINEAR &&
-           p.H == p.Hkv && p.L % 128 == 0;
+           p.H == p.Hkv && p.Lf % 128 == 0;
 }
 
 // Long heads (16 units of 128 tokens or more) go to the persistent piece kernel.
-bool use_pieces(const Problem &p) { return p.L / 128 >= 16; }
+bool use_pieces(const Problem &p) { return p.Lf / 128 >= 16; }
 
 // Workspace of one call: fp32 snapshots (M, z) for every segment, bf16 copies of M for the
 // tensor-core kernels, and room for the fused path's flags; an upper bound for every path.
 // Layout: [fp32 snapshots M | z][bf16 copies of M][sigma(K) in bf16][flags of the fused path].
-int64_t workspace_bytes(int64_t B, int64_t Hkv, int64_t S, int64_t N, int64_t d)
+// The sigma(K) copy spans every row, a final short segment's too; that segment needs no
+// workspace of its own.
+int64_t workspace_bytes(int64_t B, int64_t Hkv, int64_t L, int64_t N, int64_t d)
 {
-    const int64_t units = B * Hkv * S;
-    return units * (d * d + d) * 4 + units * d * d * 2 + units * N * d * 2 + units * 4 +
+    const int64_t S = L / N, units = B * Hkv * S;
+    return units * (d * d + d) * 4 + units * d * d * 2 + B * Hkv * L * d * 2 + units * 4 +
            B * Hkv * 4 + units * 16 + 512;
 }
+
 
 // The two-tile kernel redistributes registers with setmaxnreg; its split assumes the
 // register count per thread it was compiled with.  Checked once per kernel: a mismatch
@@ -334,7 +342,7 @@ int launch_segment_tc(const Problem &p, const __nv_bfloat16 *q, const __nv_bfloa
 
 int64_t small_workspace_bytes(const Problem &p)
 {
-    const int64_t chains = p.B * p.Hkv, units = chains * (p.L / 128);
+    const int64_t chains = p.B * p.Hkv, units = chains * (p.Lf / 128);
     const int64_t head = ((64 + chains + units) * 4 + 255) / 256 * 256;
     return head + 2 * units * tc::SmallCfg::STATE * 4;
 }
@@ -345,7 +353,7 @@ int launch_small_fused(const Problem &p, const __nv_bfloat16 *q, const __nv_bflo
                        void *ws, cudaStream_t st)
 {
     using C = tc::SmallCfg;
-    const int64_t chains = p.B * p.Hkv, U = p.L / 128, units = chains * U;
+    const int64_t chains = p.B * p.Hkv, U = p.Lf / 128, units = chains * U;
     // workspace: ticket, per-head M0 reader counts, flags (all zeroed here), then the
     // published aggregates / prefixes
     int *ticket = static_cast<int *>(ws);
@@ -393,7 +401,7 @@ PiecePlan piece_plan(const Problem &p)
 {
     PiecePlan pl;
     pl.chains = p.B * p.H;
-    pl.U = p.L / 128;
+    pl.U = p.Lf / 128;
     const int64_t target = 4 * (int64_t)sm_count();
     int64_t up = (pl.chains * pl.U) / target;
     up = up < 1 ? 1 : (up > tc::PieceCfg::MAX_UNITS ? tc::PieceCfg::MAX_UNITS : up);
@@ -471,7 +479,7 @@ int launch_all(const Problem &p, const T *q, const T *k, const T *v, const float
         {
             TRACED("linear_increments", st);
             k_linear_increments<T, D><<<(unsigned)(chains * S), 256, 0, st>>>(k, v, snapM, snapZ,
-                                                                             p.L, N, S);
+                                                                             p.L, N, S, N);
         }
         {
             TRACED("linear_scan", st);
@@ -496,7 +504,7 @@ int launch_all(const Problem &p, const T *q, const T *k, const T *v, const float
         if (!done) {
             TRACED("delta_chain", st);
             k_delta_chain<T, D, CB><<<(unsigned)(chains * (D / CB)), 256, 0, st>>>(
-                k, v, snapM, snapZ, snapMb, M_out, z_out, p.L, N, S);
+                k, v, snapM, snapZ, snapMb, M_out, z_out, p.L, N, S, N);
         }
     }
     if constexpr (sizeof(T) == 2 && (D == 64 || D == 128)) {
@@ -512,9 +520,83 @@ int launch_all(const Problem &p, const T *q, const T *k, const T *v, const float
     {
         TRACED("segment_simt", st);
         k_segment_simt<T, D><<<(unsigned)ctas, 256, smem, st>>>(q, k, v, beta, snapM, snapZ, out,
-                                                               p.L, N, S, (int)p.H, (int)p.Hkv);
+                                                               p.L, N, S, (int)p.H, (int)p.Hkv, N);
     }
     return cudaGetLastError() == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
+}
+
+// Fold the first n rows (stride L rows per chain) of k, v into (M, z), in place, with the
+// CUDA-core state kernels run as one segment of n tokens (N rounded up to 64; rows past n
+// are never read).  Linear: the increments are added into M and z by their owners.
+// Delta: each CTA reads its column block of M and all of z, and writes back only its
+// columns; z advances in a second kernel once every block has read it.  No workspace.
+template <typename T, int D>
+void launch_fold_inplace(const T *k, const T *v, int64_t L, int64_t n, float *M, float *z,
+                         int64_t chains, int rule, cudaStream_t st)
+{
+    if (n <= 0) return;
+    const int Np = (int)((n + 63) / 64 * 64);
+    if (rule == INFINI_UPDATE_LINEAR) {
+        TRACED("fold_linear", st);
+        k_linear_increments<T, D><<<(unsigned)chains, 256, 0, st>>>(k, v, M, z, L, Np, 1, (int)n, 1);
+        return;
+    }
+    {
+        TRACED("fold_delta_chain", st);
+        k_delta_chain<T, D, 16><<<(unsigned)(chains * (D / 16)), 256, 0, st>>>(
+            k, v, M, z, nullptr, M, nullptr, L, Np, 1, (int)n);
+    }
+    TRACED("fold_z", st);
+    k_z_fold<T, D><<<(unsigned)chains, 256, 0, st>>>(k, z, L, (int)n);
+}
+
+// The final short segment (T rows after the S full segments, 0 < T < N).  The state
+// before it is in (M_out, z_out): the full segments left it there, or, without full
+// segments, it is copied from (M0, z0) (zeros when NULL).  The CUDA-core segment kernel
+// computes its outputs from that state (N rounded up to 64, valid = T); then the tail is
+// folded into (M_out, z_out) in place.
+template <typename T, int D>
+int launch_tail(const Problem &p, const T *q, const T *k, const T *v, const float *beta,
+                const float *M0, const float *z0, T *out, float *M_out, float *z_out,
+                cudaStream_t st)
+{
+    const int64_t chains = p.B * p.Hkv, off = p.Lf * D;
+    const int Tn = (int)p.T, Np = (Tn + 63) / 64 * 64;
+    if (p.S == 0) {
+        const size_t mb = (size_t)chains * D * D * 4, zb = (size_t)chains * D * 4;
+        if (M0 != M_out &&
+            (M0 ? cudaMemcpyAsync(M_out, M0, mb, cudaMemcpyDeviceToDevice, st)
+                : cudaMemsetAsync(M_out, 0, mb, st)) != cudaSuccess)
+            return INFINI_ERR_CUDA;
+        if (z0 != z_out &&
+            (z0 ? cudaMemcpyAsync(z_out, z0, zb, cudaMemcpyDeviceToDevice, st)
+                : cudaMemsetAsync(z_out, 0, zb, st)) != cudaSuccess)
+            return INFINI_ERR_CUDA;
+    }
+    const size_t smem = SimtSegSmem<D>::bytes;
+    if (!opt_in_smem<k_segment_simt<T, D>>(smem)) return INFINI_ERR_CUDA;
+    {
+        TRACED("tail_segment", st);
+        k_segment_simt<T, D><<<(unsigned)(p.B * p.H * (Np / 64)), 256, smem, st>>>(
+            q + off, k + off, v + off, beta, M_out, z_out, out + off, p.L, Np, 1, (int)p.H,
+            (int)p.Hkv, Tn);
+    }
+    launch_fold_inplace<T, D>(k + off, v + off, p.L, Tn, M_out, z_out, chains, p.rule, st);
+    return cudaGetLastError() == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
+}
+
+// The full segments, then the final short one (if any).
+template <typename T, int D>
+int launch_forward(const Problem &p, const T *q, const T *k, const T *v, const float *beta,
+                   const float *M0, const float *z0, T *out, float *M_out, float *z_out,
+                   float *snapM, float *snapZ, __nv_bfloat16 *snapMb, cudaStream_t st)
+{
+    if (p.S > 0) {
+        const int rc = launch_all<T, D>(p, q, k, v, beta, M0, z0, out, M_out, z_out, snapM, snapZ,
+                                        snapMb, st);
+        if (rc != INFINI_OK || p.T == 0) return rc;
+    }
+    return launch_tail<T, D>(p, q, k, v, beta, M0, z0, out, M_out, z_out, st);
 }
 
 // The library's own stream-ordered pool on the current device.  Its release threshold keeps
@@ -561,15 +643,18 @@ int forward(const void *q, const void *k, const void *v, const float *beta, cons
     const int64_t nM = p.B * p.Hkv * p.S * p.d * p.d, nZ = p.B * p.Hkv * p.S * p.d;
     const bool tc_path = use_tc<T>(p);
     // the fused 64-token paths need far less than the general upper bound
-    const size_t bytes = (size_t)(!use_small_fused<T>(p) ? workspace_bytes(p.B, p.Hkv, p.S, p.N, p.d)
-                                  : use_pieces(p)        ? pieces_workspace_bytes(p)
-                                                         : small_workspace_bytes(p));
+    const int64_t bytes = p.S == 0                ? 0
+                          : !use_small_fused<T>(p) ? workspace_bytes(p.B, p.Hkv, p.L, p.N, p.d)
+                          : use_pieces(p)          ? pieces_workspace_bytes(p)
+                                                   : small_workspace_bytes(p);
     void *ws = nullptr;
-    cudaMemPool_t pool = workspace_pool();
-    if (!pool) return INFINI_ERR_CUDA;
-    if (cudaMallocFromPoolAsync(&ws, bytes, pool, st) != cudaSuccess) {
-        cudaGetLastError();
-        return INFINI_ERR_OOM;
+    if (bytes > 0) {
+        cudaMemPool_t pool = workspace_pool();
+        if (!pool) return INFINI_ERR_CUDA;
+        if (cudaMallocFromPoolAsync(&ws, (size_t)bytes, pool, st) != cudaSuccess) {
+            cudaGetLastError();
+            return INFINI_ERR_OOM;
+        }
     }
     float *snapM = static_cast<float *>(ws), *snapZ = snapM + nM;
     __nv_bfloat16 *snapMb = tc_path ? reinterpret_cast<__nv_bfloat16 *>(snapZ + nZ) : nullptr;
@@ -577,11 +662,11 @@ int forward(const void *q, const void *k, const void *v, const float *beta, cons
             *tv = static_cast<const T *>(v);
     T *to = static_cast<T *>(out);
     switch (p.d) {
-    case 32: rc = launch_all<T, 32>(p, tq, tk, tv, beta, M0, z0, to, M_out, z_out, snapM, snapZ, snapMb, st); break;
-    case 64: rc = launch_all<T, 64>(p, tq, tk, tv, beta, M0, z0, to, M_out, z_out, snapM, snapZ, snapMb, st); break;
-    default: rc = launch_all<T, 128>(p, tq, tk, tv, beta, M0, z0, to, M_out, z_out, snapM, snapZ, snapMb, st); break;
+    case 32: rc = launch_forward<T, 32>(p, tq, tk, tv, beta, M0, z0, to, M_out, z_out, snapM, snapZ, snapMb, st); break;
+    case 64: rc = launch_forward<T, 64>(p, tq, tk, tv, beta, M0, z0, to, M_out, z_out, snapM, snapZ, snapMb, st); break;
+    default: rc = launch_forward<T, 128>(p, tq, tk, tv, beta, M0, z0, to, M_out, z_out, snapM, snapZ, snapMb, st); break;
     }
-    if (cudaFreeAsync(ws, st) != cudaSuccess && rc == INFINI_OK) rc = INFINI_ERR_CUDA;
+    if (ws && cudaFreeAsync(ws, st) != cudaSuccess && rc == INFINI_OK) rc = INFINI_ERR_CUDA;
     return rc;
 }
 
@@ -621,7 +706,7 @@ int forward_noalloc(const void *q, const void *k, const void *v, const float *be
     if (rc != INFINI_OK) return rc;
     const int64_t nM = p.B * p.Hkv * p.S * p.d * p.d, nZ = p.B * p.Hkv * p.S * p.d;
     const bool tc_path = use_tc<T>(p);
-    const size_t bytes = (size_t)workspace_bytes(p.B, p.Hkv, p.S, p.N, p.d);
+    const size_t bytes = (size_t)workspace_bytes(p.B, p.Hkv, p.L, p.N, p.d);
     if (bytes > kNoAllocScratchBytes) return INFINI_ERR_UNSUPPORTED;
     void *ws = noalloc_scratch_address();
     if (!ws) return INFINI_ERR_CUDA;
@@ -635,10 +720,103 @@ int forward_noalloc(const void *q, const void *k, const void *v, const float *be
             *tv = static_cast<const T *>(v);
     T *to = static_cast<T *>(out);
     switch (p.d) {
-    case 32: return launch_all<T, 32>(p, tq, tk, tv, beta, M0, z0, to, M_out, z_out, snapM, snapZ, snapMb, st);
-    case 64: return launch_all<T, 64>(p, tq, tk, tv, beta, M0, z0, to, M_out, z_out, snapM, snapZ, snapMb, st);
-    default: return launch_all<T, 128>(p, tq, tk, tv, beta, M0, z0, to, M_out, z_out, snapM, snapZ, snapMb, st);
+    case 32: return launch_forward<T, 32>(p, tq, tk, tv, beta, M0, z0, to, M_out, z_out, snapM, snapZ, snapMb, st);
+    case 64: return launch_forward<T, 64>(p, tq, tk, tv, beta, M0, z0, to, M_out, z_out, snapM, snapZ, snapMb, st);
+    default: return launch_forward<T, 128>(p, tq, tk, tv, beta, M0, z0, to, M_out, z_out, snapM, snapZ, snapMb, st);
     }
+}
+
+// ---- token-by-token decode and the fold of a cached segment -------------------------------
+
+int check_cache_state(const void *k_cache, const void *v_cache, const float *M, const float *z,
+                      int64_t B, int64_t Hkv, int64_t N, int64_t d, int rule, int64_t esize)
+{
+    if (!k_cache || !v_cache || !M || !z) return INFINI_ERR_INVALID_ARG;
+    if (B <= 0 || Hkv <= 0 || N <= 0 || d <= 0) return INFINI_ERR_INVALID_ARG;
+    if (rule != INFINI_UPDATE_LINEAR && rule != INFINI_UPDATE_DELTA) return INFINI_ERR_INVALID_ARG;
+    if (B > (1 << 20) || Hkv > (1 << 16) || N > ((int64_t)1 << 30) || B * Hkv * N > ((int64_t)1 << 40))
+        return INFINI_ERR_INVALID_ARG;
+    const void *ptrs[] = {k_cache, v_cache, M, z};
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return INFINI_ERR_INVALID_ARG;
+    const int64_t cbytes = B * Hkv * N * d * esize, mbytes = B * Hkv * d * d * 4,
+                  zbytes = B * Hkv * d * 4;
+    if (ranges_overlap(k_cache, cbytes, v_cache, cbytes) || ranges_overlap(k_cache, cbytes, M, mbytes) ||
+        ranges_overlap(k_cache, cbytes, z, zbytes) || ranges_overlap(v_cache, cbytes, M, mbytes) ||
+        ranges_overlap(v_cache, cbytes, z, zbytes) || ranges_overlap(M, mbytes, z, zbytes))
+        return INFINI_ERR_INVALID_ARG;
+    if (d != 32 && d != 64 && d != 128) return INFINI_ERR_UNSUPPORTED;
+    return INFINI_OK;
+}
+
+template <typename T>
+int fold_launch(const void *k_cache, const void *v_cache, int64_t n, float *M, float *z,
+                int64_t B, int64_t Hkv, int64_t N, int64_t d, int rule, cudaStream_t st)
+{
+    const T *kc = static_cast<const T *>(k_cache), *vc = static_cast<const T *>(v_cache);
+    const int64_t chains = B * Hkv;
+    switch (d) {
+    case 32: launch_fold_inplace<T, 32>(kc, vc, N, n, M, z, chains, rule, st); break;
+    case 64: launch_fold_inplace<T, 64>(kc, vc, N, n, M, z, chains, rule, st); break;
+    default: launch_fold_inplace<T, 128>(kc, vc, N, n, M, z, chains, rule, st); break;
+    }
+    return cudaGetLastError() == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
+}
+
+template <typename T>
+int fold(const void *k_cache, const void *v_cache, int64_t n, float *M, float *z, int64_t B,
+         int64_t Hkv, int64_t N, int64_t d, int rule, infini_stream_t stream)
+{
+    int rc = check_cache_state(k_cache, v_cache, M, z, B, Hkv, N, d, rule, (int64_t)sizeof(T));
+    if (rc != INFINI_OK) return rc;
+    if (n < 0 || n > N) return INFINI_ERR_INVALID_ARG;
+    if (n == 0) return INFINI_OK;
+    cudaGetLastError();
+    return fold_launch<T>(k_cache, v_cache, n, M, z, B, Hkv, N, d, rule,
+                          reinterpret_cast<cudaStream_t>(stream));
+}
+
+template <typename T>
+int decode_step(const void *q, const void *k, const void *v, const float *beta, void *k_cache,
+                void *v_cache, int64_t pos, float *M, float *z, void *out, int64_t B, int64_t H,
+                int64_t Hkv, int64_t N, int64_t d, int rule, infini_stream_t stream)
+{
+    int rc = check_cache_state(k_cache, v_cache, M, z, B, Hkv, N, d, rule, (int64_t)sizeof(T));
+    if (rc != INFINI_OK && rc != INFINI_ERR_UNSUPPORTED) return rc;
+    const int rc_shape = rc;
+    if (!q || !k || !v || !beta || !out) return INFINI_ERR_INVALID_ARG;
+    if (H <= 0 || H % Hkv != 0 || H > (1 << 16) || B * H > ((int64_t)1 << 31) - 1)
+        return INFINI_ERR_INVALID_ARG;
+    if (pos < 0 || pos >= N) return INFINI_ERR_INVALID_ARG;
+    const void *ptrs[] = {q, k, v, beta, out};
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return INFINI_ERR_INVALID_ARG;
+    const int64_t es = (int64_t)sizeof(T), obytes = B * H * d * es, kvbytes = B * Hkv * d * es,
+                  cbytes = B * Hkv * N * d * es;
+    if (ranges_overlap(out, obytes, q, obytes) || ranges_overlap(out, obytes, k, kvbytes) ||
+        ranges_overlap(out, obytes, v, kvbytes) || ranges_overlap(out, obytes, k_cache, cbytes) ||
+        ranges_overlap(out, obytes, v_cache, cbytes) ||
+        ranges_overlap(out, obytes, M, B * Hkv * d * d * 4) ||
+        ranges_overlap(out, obytes, z, B * Hkv * d * 4))
+        return INFINI_ERR_INVALID_ARG;
+    if (rc_shape != INFINI_OK) return rc_shape;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaGetLastError();
+    const T *tq = static_cast<const T *>(q), *tk = static_cast<const T *>(k),
+            *tv = static_cast<const T *>(v);
+    T *kc = static_cast<T *>(k_cache), *vc = static_cast<T *>(v_cache), *to = static_cast<T *>(out);
+    {
+        TRACED("decode_attn", st);
+        const unsigned grid = (unsigned)(B * H);
+        switch (d) {
+        case 32: k_decode_attn<T, 32><<<grid, 256, 0, st>>>(tq, tk, tv, beta, kc, vc, (int)pos, (int)N, M, z, to, (int)H, (int)Hkv); break;
+        case 64: k_decode_attn<T, 64><<<grid, 256, 0, st>>>(tq, tk, tv, beta, kc, vc, (int)pos, (int)N, M, z, to, (int)H, (int)Hkv); break;
+        default: k_decode_attn<T, 128><<<grid, 256, 0, st>>>(tq, tk, tv, beta, kc, vc, (int)pos, (int)N, M, z, to, (int)H, (int)Hkv); break;
+        }
+    }
+    if (cudaGetLastError() != cudaSuccess) return INFINI_ERR_CUDA;
+    if (pos + 1 < N) return INFINI_OK;
+    return fold_launch<T>(kc, vc, N, M, z, B, Hkv, N, d, rule, st);   // the segment is complete
 }
 
 }  // namespace
@@ -673,10 +851,43 @@ int infini_attn_fwd_f32(const void *q, const void *k, const void *v, const float
                                   update_rule, stream);
 }
 
+int infini_attn_decode_step(const void *q, const void *k, const void *v, const float *beta,
+                            void *k_cache, void *v_cache, int64_t pos, float *M, float *z,
+                            void *out, int64_t B, int64_t H, int64_t Hkv, int64_t N, int64_t d,
+                            int update_rule, infini_stream_t stream)
+{
+    return infini::decode_step<__nv_bfloat16>(q, k, v, beta, k_cache, v_cache, pos, M, z, out, B,
+                                              H, Hkv, N, d, update_rule, stream);
+}
+
+int infini_attn_decode_step_f32(const void *q, const void *k, const void *v, const float *beta,
+                                void *k_cache, void *v_cache, int64_t pos, float *M, float *z,
+                                void *out, int64_t B, int64_t H, int64_t Hkv, int64_t N,
+                                int64_t d, int update_rule, infini_stream_t stream)
+{
+    return infini::decode_step<float>(q, k, v, beta, k_cache, v_cache, pos, M, z, out, B, H, Hkv,
+                                      N, d, update_rule, stream);
+}
+
+int infini_attn_fold(const void *k_cache, const void *v_cache, int64_t n, float *M, float *z,
+                     int64_t B, int64_t Hkv, int64_t N, int64_t d, int update_rule,
+                     infini_stream_t stream)
+{
+    return infini::fold<__nv_bfloat16>(k_cache, v_cache, n, M, z, B, Hkv, N, d, update_rule,
+                                       stream);
+}
+
+int infini_attn_fold_f32(const void *k_cache, const void *v_cache, int64_t n, float *M, float *z,
+                         int64_t B, int64_t Hkv, int64_t N, int64_t d, int update_rule,
+                         infini_stream_t stream)
+{
+    return infini::fold<float>(k_cache, v_cache, n, M, z, B, Hkv, N, d, update_rule, stream);
+}
+
 int64_t infini_attn_workspace_bytes(int64_t B, int64_t Hkv, int64_t L, int64_t N, int64_t d)
 {
-    if (B <= 0 || Hkv <= 0 || L <= 0 || N <= 0 || d <= 0 || L % N != 0) return 0;
-    return infini::workspace_bytes(B, Hkv, L / N, N, d);
+    if (B <= 0 || Hkv <= 0 || L <= 0 || N <= 0 || d <= 0) return 0;
+    return infini::workspace_bytes(B, Hkv, L, N, d);
 }
 
 const char *infini_attn_status_string(int status)

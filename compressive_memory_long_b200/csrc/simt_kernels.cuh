@@ -11,6 +11,11 @@
 // Workspace convention shared with the host code: for chain c = b * Hkv + kvh and segment
 // s, snapM[(c * S + s) * d * d ...] and snapZ[(c * S + s) * d ...] hold (M_{s-1}, z_{s-1}),
 // the memory the segment reads.
+//
+// `valid` is the number of tokens a segment really has (N for every full segment).  A
+// final segment shorter than N runs with N rounded up to 64 and valid = its length: the
+// rows past `valid` are never read (they count as a zero key / value whose feature map is
+// 0, not sigma(0)) and never written.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -30,11 +35,14 @@ __device__ __forceinline__ float feature_map(float x) { return x > 0.f ? x + 1.f
 // Linear rule, step 1: per (chain, segment) the increments dM_s = sigma(K_s)^T V_s and
 // dz_s = sum_t sigma(K_s,t), written into the snapshot slot of that segment (the scan
 // below turns the slots into exclusive prefix sums).  One CTA per (chain, segment).
+// With `accumulate` set the increments are added to the slot instead (S = 1 and the slot
+// is the memory itself: the in-place fold of one segment; each element has one owner).
 // ---------------------------------------------------------------------------------------
 template <typename T, int D>
 __global__ void __launch_bounds__(256)
 k_linear_increments(const T *__restrict__ k, const T *__restrict__ v, float *__restrict__ snapM,
-                    float *__restrict__ snapZ, int64_t L, int N, int S)
+                    float *__restrict__ snapZ, int64_t L, int N, int S, int valid,
+                    int accumulate = 0)
 {
     constexpr int TK = 32, R = D / 16;
     __shared__ float sK[TK][D + 1];
@@ -55,8 +63,9 @@ k_linear_increments(const T *__restrict__ k, const T *__restrict__ v, float *__r
     for (int t0 = 0; t0 < N; t0 += TK) {
         for (int i = tid; i < TK * D; i += 256) {
             const int t = i / D, c = i % D;
-            sK[t][c] = feature_map(ld_f(K + (int64_t)(t0 + t) * D + c));
-            sV[t][c] = ld_f(V + (int64_t)(t0 + t) * D + c);
+            const bool in = t0 + t < valid;
+            sK[t][c] = in ? feature_map(ld_f(K + (int64_t)(t0 + t) * D + c)) : 0.f;
+            sV[t][c] = in ? ld_f(V + (int64_t)(t0 + t) * D + c) : 0.f;
         }
         __syncthreads();
 #pragma unroll 4
@@ -79,8 +88,40 @@ k_linear_increments(const T *__restrict__ k, const T *__restrict__ v, float *__r
 #pragma unroll
     for (int i = 0; i < R; ++i)
 #pragma unroll
-        for (int j = 0; j < R; ++j) dst[(ty + 16 * i) * D + tx + 16 * j] = acc[i][j];
-    if (tid < D) snapZ[(chain * S + s) * D + tid] = zacc;
+        for (int j = 0; j < R; ++j) {
+            float *e = dst + (ty + 16 * i) * D + tx + 16 * j;
+            *e = accumulate ? *e + acc[i][j] : acc[i][j];
+        }
+    if (tid < D) {
+        float *e = snapZ + (chain * S + s) * D + tid;
+        *e = accumulate ? *e + zacc : zacc;
+    }
+}
+
+// ---------------------------------------------------------------------------------------
+// z += sum_{t < valid} sigma(k_t) for every chain, in place (the delta rule's in-place fold
+// writes M by column blocks and leaves z to this kernel, so that no CTA of the chain reads
+// a z another CTA has already advanced).  One CTA per chain.
+// ---------------------------------------------------------------------------------------
+template <typename T, int D>
+__global__ void __launch_bounds__(256)
+k_z_fold(const T *__restrict__ k, float *z, int64_t L, int valid)
+{
+    constexpr int PARTS = 256 / D;
+    __shared__ float part[PARTS][D];
+    const int64_t chain = blockIdx.x;
+    const int f = threadIdx.x % D, p = threadIdx.x / D;
+    const T *K = k + chain * L * D;
+    float acc = 0.f;
+    for (int t = p; t < valid; t += PARTS) acc += feature_map(ld_f(K + (int64_t)t * D + f));
+    part[p][f] = acc;
+    __syncthreads();
+    if (threadIdx.x < D) {
+        float sum = 0.f;
+#pragma unroll
+        for (int i = 0; i < PARTS; ++i) sum += part[i][f];
+        z[chain * D + f] += sum;
+    }
 }
 
 // ---------------------------------------------------------------------------------------
@@ -162,16 +203,16 @@ k_state_init(const float *M0, const float *z0, float *__restrict__ snapM,
 // Delta rule, step 2: the sequential chain.  The update of value column e needs only
 // column e of M_{s-1}, column e of V_s and the shared z_{s-1}, so each CTA owns CB columns
 // of one chain's M (in shared memory, fp32) and walks all S segments; z is recomputed by
-// every CTA of the chain.  Before segment s >= 1 the CTA publishes its columns of M_{s-1}
+// every CTA of the chain (z_out NULL: z is not written).  Before segment s >= 1 the CTA publishes its columns of M_{s-1}
 // into snapshot slot s (CTA 0 of the chain also publishes z).  Within a segment every
 // token's prediction reads M_{s-1}: the increments are accumulated in registers and added
 // after the whole segment.
 // ---------------------------------------------------------------------------------------
 template <typename T, int D, int CB>
 __global__ void __launch_bounds__(256)
-k_delta_chain(const T *__restrict__ k, const T *__restrict__ v, float *__restrict__ snapM,
-              float *__restrict__ snapZ, __nv_bfloat16 *__restrict__ snapMb, float *M_out,
-              float *z_out, int64_t L, int N, int S)
+k_delta_chain(const T *__restrict__ k, const T *__restrict__ v, float *snapM,
+              float *snapZ, __nv_bfloat16 *__restrict__ snapMb, float *M_out,
+              float *z_out, int64_t L, int N, int S, int valid)
 {
     constexpr int TK = 32, NBLK = D / CB, PER = D * CB / 256;
     static_assert(PER >= 1 && (D * CB) % 256 == 0, "column block too small");
@@ -215,11 +256,11 @@ k_delta_chain(const T *__restrict__ k, const T *__restrict__ v, float *__restric
         for (int t0 = 0; t0 < N; t0 += TK) {
             for (int i = tid; i < TK * D; i += 256) {
                 const int t = i / D, c = i % D;
-                sK[t][c] = feature_map(ld_f(K + (int64_t)(t0 + t) * D + c));
+                sK[t][c] = t0 + t < valid ? feature_map(ld_f(K + (int64_t)(t0 + t) * D + c)) : 0.f;
             }
             for (int i = tid; i < TK * CB; i += 256) {
                 const int t = i / CB, e = i % CB;
-                sV[t][e] = ld_f(V + (int64_t)(t0 + t) * D + cb + e);
+                sV[t][e] = t0 + t < valid ? ld_f(V + (int64_t)(t0 + t) * D + cb + e) : 0.f;
             }
             __syncthreads();
             // den_t = sigma(k_t) . z_{s-1}: one warp per token
@@ -262,7 +303,7 @@ k_delta_chain(const T *__restrict__ k, const T *__restrict__ v, float *__restric
         __syncthreads();
     }
     for (int i = tid; i < D * CB; i += 256) M_out[chain * D * D + (i / CB) * D + cb + i % CB] = sM[i / CB][i % CB];
-    if (cb == 0)
+    if (cb == 0 && z_out)
         for (int i = tid; i < D; i += 256) z_out[chain * D + i] = sz[i];
 }
 
@@ -284,7 +325,7 @@ __global__ void __launch_bounds__(256)
 k_segment_simt(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
                const float *__restrict__ beta, const float *__restrict__ snapM,
                const float *__restrict__ snapZ, T *__restrict__ out, int64_t L, int N, int S,
-               int H, int Hkv)
+               int H, int Hkv, int valid)
 {
     constexpr int BQ = 64, BK = 64, RJ = D / 16;
     extern __shared__ float smem[];
@@ -308,7 +349,9 @@ k_segment_simt(const T *__restrict__ q, const T *__restrict__ k, const T *__rest
     const T *Vseg = v + (chain * L + (int64_t)s * N) * D;
 
     const int tid = threadIdx.x, tx = tid % 16, ty = tid / 16;
-    for (int i = tid; i < BQ * D; i += 256) sQ[(i / D) * (D + 1) + i % D] = ld_f(Q + i);
+    const int q0 = qt * BQ;                 // first query row within the segment
+    for (int i = tid; i < BQ * D; i += 256)
+        sQ[(i / D) * (D + 1) + i % D] = q0 + i / D < valid ? ld_f(Q + i) : 0.f;
 
     const float sl2 = rsqrtf((float)D) * 1.4426950408889634f;   // softmax scale * log2(e)
     float m[4], l[4], o[4][RJ];
@@ -325,8 +368,9 @@ k_segment_simt(const T *__restrict__ q, const T *__restrict__ k, const T *__rest
         const T *Kt = Kseg + (int64_t)kt * BK * D;
         const T *Vt = Vseg + (int64_t)kt * BK * D;
         for (int i = tid; i < BK * D; i += 256) {
-            sK[(i / D) * (D + 1) + i % D] = ld_f(Kt + i);
-            sV[i] = ld_f(Vt + i);
+            const bool in = kt * BK + i / D < valid;
+            sK[(i / D) * (D + 1) + i % D] = in ? ld_f(Kt + i) : 0.f;
+            sV[i] = in ? ld_f(Vt + i) : 0.f;
         }
         __syncthreads();
         float sc[4][4];
@@ -434,6 +478,7 @@ k_segment_simt(const T *__restrict__ q, const T *__restrict__ k, const T *__rest
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const int r = ty + 16 * i;
+        if (q0 + r >= valid) continue;
         const float inv_l = 1.f / l[i];
 #pragma unroll
         for (int j = 0; j < RJ; ++j) {

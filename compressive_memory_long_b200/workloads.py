@@ -49,10 +49,11 @@ class Workload:
     k_boost_frac: float = 0.0         # fraction of K rows (per (b, kv head)) scaled ...
     k_boost: float = 1.0              # ... by this factor before rounding
     description: str = ""
+    tail: int = 0                     # tokens of a final segment shorter than N (0 <= tail < N)
 
     @property
     def L(self) -> int:
-        return self.N * self.S
+        return self.N * self.S + self.tail
 
     @property
     def G(self) -> int:

@@ -5,8 +5,10 @@
  * block?" and "How does the compressive memory work?"; the Hugging Face reproduction
  * analysis, "Infini-Attention Mechanism", steps 1-6):
  *
- *   The length-L sequence of every (batch b, query head h) is cut into S = L / N segments of
- *   N tokens, processed in order.  For segment s and query row q_t:
+ *   The length-L sequence of every (batch b, query head h) is cut into segments of N
+ *   tokens, processed in order; when N does not divide L the last segment is shorter
+ *   (L mod N tokens) and is processed the same way, its update included.  For segment s
+ *   and query row q_t:
  *     A_dot = causal softmax(q_t K_s^T / sqrt(d)) V_s     keys of segment s only, j <= t
  *     A_mem = sigma(q_t) M_{s-1} / (sigma(q_t) . z_{s-1}) sigma(x) = ELU(x) + 1; 0 while the
  *                                                          denominator is exactly 0
@@ -65,7 +67,7 @@ enum {
 
 enum {
     INFINI_OK = 0,
-    INFINI_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size, L % N != 0, bad rule,
+    INFINI_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size or position, bad rule,
                                    partial overlap of a state output with its input        */
     INFINI_ERR_UNSUPPORTED = 2, /* valid but not built: d not in {32, 64, 128}, N % 64 != 0 */
     INFINI_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed                      */
@@ -78,7 +80,8 @@ enum {
  * in fp32, memory M / z in fp32, out rounded to nearest-even).
  *
  *   B, H, Hkv : batch, query heads, key/value heads (H % Hkv == 0)
- *   L, N, d   : sequence length, segment length (L % N == 0), head dimension
+ *   L, N, d   : sequence length, segment length, head dimension (L need not be a
+ *               multiple of N: the final L mod N tokens form a shorter last segment)
  *   update_rule : INFINI_UPDATE_LINEAR or INFINI_UPDATE_DELTA
  * Returns INFINI_OK or an error status.
  */
@@ -92,6 +95,53 @@ INFINI_API int infini_attn_fwd_f32(const void *q, const void *k, const void *v, 
                         const float *M0, const float *z0, void *out, float *M_out,
                         float *z_out, int64_t B, int64_t H, int64_t Hkv, int64_t L, int64_t N,
                         int64_t d, int update_rule, infini_stream_t stream);
+
+/*
+ * Token-by-token decode (bf16 activations; the _f32 variant takes fp32 ones).  One call
+ * processes one new token of every (batch, head) at offset `pos` of its current segment
+ * and gives the output the forward would give that token:
+ *   - local attention over the current segment's keys at offsets 0..pos: rows 0..pos-1 of
+ *     the cache, then this token's own key and value, which the call writes into row pos;
+ *   - retrieval from (M, z), the memory from before the current segment;
+ *   - the gate, as in the forward.
+ * When pos == N - 1 the segment is complete: after the output, the call folds all N cached
+ * rows into (M, z) in place (the linear or delta update of the forward), and the next
+ * token starts a new segment at pos = 0.  At the end of a stream whose last segment is
+ * shorter, infini_attn_fold folds the rows cached so far; feeding a whole sequence this way
+ * then leaves the forward's M_out / z_out in (M, z).
+ *
+ *   q [B, H, d], k / v [B, Hkv, d]: this token;  out [B, H, d]
+ *   k_cache / v_cache [B, Hkv, N, d]: the current segment's keys and values (caller-owned;
+ *     rows >= pos are not read)
+ *   M [B, Hkv, d, d], z [B, Hkv, d] fp32: read, and updated in place when pos == N - 1
+ *     (start a stream with zeros, or with a forward's M_out / z_out)
+ *   0 <= pos < N; N any positive length; d in {32, 64, 128}
+ * Everything runs on `stream`, and neither call allocates memory (both may be captured in
+ * a CUDA graph).  out must not overlap any other buffer; caches, M and z must not overlap
+ * one another.
+ */
+INFINI_API int infini_attn_decode_step(const void *q, const void *k, const void *v,
+                                       const float *beta, void *k_cache, void *v_cache,
+                                       int64_t pos, float *M, float *z, void *out, int64_t B,
+                                       int64_t H, int64_t Hkv, int64_t N, int64_t d,
+                                       int update_rule, infini_stream_t stream);
+INFINI_API int infini_attn_decode_step_f32(const void *q, const void *k, const void *v,
+                                           const float *beta, void *k_cache, void *v_cache,
+                                           int64_t pos, float *M, float *z, void *out,
+                                           int64_t B, int64_t H, int64_t Hkv, int64_t N,
+                                           int64_t d, int update_rule, infini_stream_t stream);
+
+/*
+ * Fold the first n rows (0 <= n <= N; 0 does nothing) of every chain's cache into (M, z),
+ * in place, with the update rule of the forward: the end of a stream whose last segment is
+ * shorter than N.  Layouts as for infini_attn_decode_step; no allocation.
+ */
+INFINI_API int infini_attn_fold(const void *k_cache, const void *v_cache, int64_t n, float *M,
+                                float *z, int64_t B, int64_t Hkv, int64_t N, int64_t d,
+                                int update_rule, infini_stream_t stream);
+INFINI_API int infini_attn_fold_f32(const void *k_cache, const void *v_cache, int64_t n,
+                                    float *M, float *z, int64_t B, int64_t Hkv, int64_t N,
+                                    int64_t d, int update_rule, infini_stream_t stream);
 
 /*
  * Allocation-free variant of infini_attn_fwd (bf16 activations); same parameters, same

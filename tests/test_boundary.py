@@ -42,7 +42,10 @@ def test_workspace_bytes():
     assert binding.infini_attn_workspace_bytes(2, 8, 1024, 64, 64) == \
         units * (64 * 64 + 64) * 4 + units * 64 * 64 * 2 + units * 64 * 64 * 2 + units * 4 + \
         2 * 8 * 4 + units * 16 + 512
-    assert binding.infini_attn_workspace_bytes(1, 1, 100, 64, 64) == 0
+    # a final short segment needs no slot of its own; the sigma(K) copy spans every row
+    assert binding.infini_attn_workspace_bytes(1, 1, 100, 64, 64) == \
+        (64 * 64 + 64) * 4 + 64 * 64 * 2 + 100 * 64 * 2 + 4 + 4 + 16 + 512
+    assert binding.infini_attn_workspace_bytes(1, 1, 40, 64, 64) == 40 * 64 * 2 + 4 + 512
     assert binding.infini_attn_workspace_bytes(0, 1, 64, 64, 64) == 0
 
 
@@ -70,7 +73,7 @@ INVALID, UNSUPPORTED = 1, 2
     (dict(beta=None), INVALID), (dict(out=None), INVALID), (dict(M_out=None), INVALID),
     (dict(z_out=None), INVALID),
     (dict(B=0), INVALID), (dict(H=0), INVALID), (dict(L=-64), INVALID), (dict(N=0), INVALID),
-    (dict(d=0), INVALID), (dict(H=3, Hkv=2), INVALID), (dict(L=100, N=64), INVALID),
+    (dict(d=0), INVALID), (dict(H=3, Hkv=2), INVALID),
     (dict(rule=2), INVALID), (dict(rule=-1), INVALID),
     (dict(q=BASE + 8), INVALID), (dict(M_out=BASE + (7 << 32) + 4), INVALID),
     (dict(M_out=(1 << 40) + (4 << 32) + 64), INVALID),     # partial overlap with M0
@@ -87,3 +90,55 @@ def test_python_binding_checks_shapes():
     q = torch.zeros(1, 2, 64, 32)
     with pytest.raises(ValueError):
         binding.forward(q, q, q, torch.zeros(2), N=64)     # CPU tensors are refused
+
+
+DEC_PTRS = ["q", "k", "v", "beta", "k_cache", "v_cache", "M", "z", "out"]
+
+
+def call_decode(entry="infini_attn_decode_step", B=1, H=2, Hkv=2, N=64, d=64, pos=0, rule=0,
+                **ptr):
+    gap = 1 << 32
+    p = {name: BASE + i * gap for i, name in enumerate(DEC_PTRS)}
+    p.update(ptr)
+    a = [None if p[n] is None else ctypes.c_void_p(p[n]) for n in DEC_PTRS]
+    f = getattr(binding.LIB, entry)
+    return f(a[0], a[1], a[2], a[3], a[4], a[5], pos, a[6], a[7], a[8], B, H, Hkv, N, d, rule,
+             None)
+
+
+@pytest.mark.parametrize("entry", ["infini_attn_decode_step", "infini_attn_decode_step_f32"])
+@pytest.mark.parametrize("kw,status", [
+    *[(dict({n: None}), INVALID) for n in DEC_PTRS],
+    (dict(pos=-1), INVALID), (dict(pos=64), INVALID), (dict(N=0), INVALID),
+    (dict(H=3, Hkv=2), INVALID), (dict(Hkv=0), INVALID), (dict(rule=2), INVALID),
+    (dict(q=BASE + 8), INVALID), (dict(k_cache=BASE + (4 << 32) + 4), INVALID),
+    (dict(v_cache=BASE + (4 << 32)), INVALID),                 # both caches at one address
+    (dict(out=BASE + (6 << 32)), INVALID),                     # out on top of M
+    (dict(z=BASE + (6 << 32) + 64), INVALID),                  # z inside M
+    (dict(d=48), UNSUPPORTED), (dict(d=256), UNSUPPORTED),
+])
+def test_decode_argument_errors(entry, kw, status):
+    assert call_decode(entry, **kw) == status
+
+
+FOLD_PTRS = ["k_cache", "v_cache", "M", "z"]
+
+
+def call_fold(entry="infini_attn_fold", n=1, B=1, Hkv=2, N=64, d=64, rule=0, **ptr):
+    gap = 1 << 32
+    p = {name: BASE + i * gap for i, name in enumerate(FOLD_PTRS)}
+    p.update(ptr)
+    a = [None if p[x] is None else ctypes.c_void_p(p[x]) for x in FOLD_PTRS]
+    return getattr(binding.LIB, entry)(a[0], a[1], n, a[2], a[3], B, Hkv, N, d, rule, None)
+
+
+@pytest.mark.parametrize("entry", ["infini_attn_fold", "infini_attn_fold_f32"])
+@pytest.mark.parametrize("kw,status", [
+    *[(dict({n: None}), INVALID) for n in FOLD_PTRS],
+    (dict(n=-1), INVALID), (dict(n=65), INVALID), (dict(B=0), INVALID), (dict(rule=-1), INVALID),
+    (dict(M=BASE + (2 << 32) + 4), INVALID), (dict(z=BASE + (2 << 32)), INVALID),
+    (dict(d=16), UNSUPPORTED),
+    (dict(n=0), 0),                     # nothing to fold: returns before any CUDA call
+])
+def test_fold_argument_errors(entry, kw, status):
+    assert call_fold(entry, **kw) == status

@@ -148,10 +148,11 @@ def test_in_place_state_and_streaming_split(rule):
 
 def test_device_argument_errors():
     from compressive_memory_long_b200 import binding
-    q = torch.zeros(1, 2, 100, 64, dtype=torch.bfloat16, device="cuda")
+    q = torch.zeros(1, 2, 128, 64, dtype=torch.bfloat16, device="cuda")
+    k = torch.zeros(1, 3, 128, 64, dtype=torch.bfloat16, device="cuda")
     beta = torch.zeros(2, device="cuda")
-    with pytest.raises(binding.InfiniError) as e:
-        binding.forward(q, q, q, beta, N=64)
+    with pytest.raises(binding.InfiniError) as e:      # H % Hkv != 0
+        binding.forward(q, k, k, beta, N=64)
     assert e.value.status == 1
     q = torch.zeros(1, 2, 128, 48, dtype=torch.bfloat16, device="cuda")
     with pytest.raises(binding.InfiniError) as e:
