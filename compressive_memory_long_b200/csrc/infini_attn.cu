@@ -7,6 +7,7 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <algorithm>
 #include <atomic>
 #include <mutex>
 #include <string>
@@ -227,7 +228,7 @@ int launch_linear_state_tc(const Problem &p, const __nv_bfloat16 *k, const __nv_
         !make_map_bf16_3d(&mv, v, D, p.L, p.B * p.Hkv, 128))
         return INFINI_ERR_CUDA;
     if (!opt_in_smem<tc::k_linear_state_tc<D>>(C::ALLOC)) return INFINI_ERR_CUDA;
-    tc::LinArgs a{M0, z0, snapZ, snapMb, M_out, z_out, (int)p.N, (int)p.S};
+    tc::LinArgs a{M0, z0, snapZ, snapMb, M_out, z_out, (int)p.N, (int)p.S, p.L};
     TRACED("linear_state_tc", st);
     tc::k_linear_state_tc<D><<<(unsigned)(p.B * p.Hkv), 256, C::ALLOC, st>>>(mk, mv, a);
     return INFINI_OK;
@@ -285,11 +286,11 @@ bool use_pieces(const Problem &p) { return p.Lf / 128 >= 16; }
 // Workspace of one call: fp32 snapshots (M, z) for every segment, bf16 copies of M for the
 // tensor-core kernels, and room for the fused path's flags; an upper bound for every path.
 // Layout: [fp32 snapshots M | z][bf16 copies of M][sigma(K) in bf16][flags of the fused path].
-// The sigma(K) copy spans every row, a final short segment's too; that segment needs no
-// workspace of its own.
+// A final short segment counts as a segment here (the tensor-core path gives it a snapshot
+// slot); the sigma(K) copy spans every row.
 int64_t workspace_bytes(int64_t B, int64_t Hkv, int64_t L, int64_t N, int64_t d)
 {
-    const int64_t S = L / N, units = B * Hkv * S;
+    const int64_t S = (L + N - 1) / N, units = B * Hkv * S;
     return units * (d * d + d) * 4 + units * d * d * 2 + B * Hkv * L * d * 2 + units * 4 +
            B * Hkv * 4 + units * 16 + 512;
 }
@@ -585,6 +586,23 @@ int launch_tail(const Problem &p, const T *q, const T *k, const T *v, const floa
     return cudaGetLastError() == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
 }
 
+// The problem the kernels run.  On the tensor-core path a final short segment is simply
+// one more segment: TMA fills its rows past L with zeros, the memory kernels leave those
+// rows out of the update (zero sigma(K)), and the segment kernel neither computes tiles
+// that start past L nor stores rows past L.  Elsewhere the CUDA-core tail follows the
+// full segments.
+template <typename T>
+Problem effective(const Problem &p)
+{
+    Problem e = p;
+    if (p.T > 0 && use_tc<T>(p)) {
+        e.S = p.S + 1;
+        e.Lf = e.S * p.N;
+        e.T = 0;
+    }
+    return e;
+}
+
 // The full segments, then the final short one (if any).
 template <typename T, int D>
 int launch_forward(const Problem &p, const T *q, const T *k, const T *v, const float *beta,
@@ -637,6 +655,7 @@ int forward(const void *q, const void *k, const void *v, const float *beta, cons
     int rc = check_args(q, k, v, beta, M0, z0, out, M_out, z_out, B, H, Hkv, L, N, d, rule,
                         (int64_t)sizeof(T), &p);
     if (rc != INFINI_OK) return rc;
+    p = effective<T>(p);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     cudaGetLastError();   // clear a stale error left by someone else's launch
 
@@ -704,6 +723,7 @@ int forward_noalloc(const void *q, const void *k, const void *v, const float *be
     int rc = check_args(q, k, v, beta, M0, z0, out, M_out, z_out, B, H, Hkv, L, N, d, rule,
                         (int64_t)sizeof(T), &p);
     if (rc != INFINI_OK) return rc;
+    p = effective<T>(p);
     const int64_t nM = p.B * p.Hkv * p.S * p.d * p.d, nZ = p.B * p.Hkv * p.S * p.d;
     const bool tc_path = use_tc<T>(p);
     const size_t bytes = (size_t)workspace_bytes(p.B, p.Hkv, p.L, p.N, p.d);
@@ -805,7 +825,44 @@ int decode_step(const void *q, const void *k, const void *v, const float *beta, 
     const T *tq = static_cast<const T *>(q), *tk = static_cast<const T *>(k),
             *tv = static_cast<const T *>(v);
     T *kc = static_cast<T *>(k_cache), *vc = static_cast<T *>(v_cache), *to = static_cast<T *>(out);
-    {
+    if (H / Hkv <= kDecodeGMax) {
+        // one cluster per (batch, kv head) with its whole query group; a tile of keys per
+        // CTA, at most 8 CTAs (the portable cluster size)
+        const int KT = sizeof(T) == 2 ? DecCfg<T, 128>::KT : DecCfg<float, 128>::KT;
+        const int CL = (int)std::min<int64_t>(8, (pos + KT) / KT);
+        size_t smem = 0;
+        bool ok = false;
+        switch (d) {
+        case 32: smem = DecCfg<T, 32>::BYTES; ok = opt_in_smem<k_decode_split<T, 32>>(smem); break;
+        case 64: smem = DecCfg<T, 64>::BYTES; ok = opt_in_smem<k_decode_split<T, 64>>(smem); break;
+        default: smem = DecCfg<T, 128>::BYTES; ok = opt_in_smem<k_decode_split<T, 128>>(smem); break;
+        }
+        if (!ok) return INFINI_ERR_CUDA;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)(B * Hkv * CL));
+        cfg.blockDim = dim3(256);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = st;
+        cudaLaunchAttribute at[1];
+        at[0].id = cudaLaunchAttributeClusterDimension;
+        at[0].val.clusterDim.x = (unsigned)CL;
+        at[0].val.clusterDim.y = 1;
+        at[0].val.clusterDim.z = 1;
+        cfg.attrs = at;
+        cfg.numAttrs = 1;
+        const int ip = (int)pos, iN = (int)N, iH = (int)H, iHkv = (int)Hkv;
+        cudaError_t e;
+        TRACED("decode_attn", st);
+        switch (d) {
+        case 32: e = cudaLaunchKernelEx(&cfg, k_decode_split<T, 32>, tq, tk, tv, beta, kc, vc, ip, iN, (const float *)M, (const float *)z, to, iH, iHkv); break;
+        case 64: e = cudaLaunchKernelEx(&cfg, k_decode_split<T, 64>, tq, tk, tv, beta, kc, vc, ip, iN, (const float *)M, (const float *)z, to, iH, iHkv); break;
+        default: e = cudaLaunchKernelEx(&cfg, k_decode_split<T, 128>, tq, tk, tv, beta, kc, vc, ip, iN, (const float *)M, (const float *)z, to, iH, iHkv); break;
+        }
+        if (e != cudaSuccess) {
+            cudaGetLastError();
+            return INFINI_ERR_CUDA;
+        }
+    } else {   // groups of more than 8 query heads: one CTA per (batch, query head)
         TRACED("decode_attn", st);
         const unsigned grid = (unsigned)(B * H);
         switch (d) {

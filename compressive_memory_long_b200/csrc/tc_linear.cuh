@@ -34,7 +34,7 @@ struct LinCfg {
     static constexpr int OFF_K = 0;
     static constexpr int OFF_V = OFF_K + ST * KTILE;
     static constexpr int OFF_BAR = OFF_V + ST * VTILE;
-    static constexpr int NBAR = 2 * ST + 3;
+    static constexpr int NBAR = 3 * ST + 2;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int BYTES = OFF_MISC + 16;
     static constexpr int ALLOC = BYTES + 1024;
@@ -47,6 +47,7 @@ struct LinArgs {
     __nv_bfloat16 *snapMb;     // [chains, S, D, D]
     float *M_out, *z_out;
     int N, S;
+    int64_t L;                 // rows per chain: rows of the last segment past L count as absent
 };
 
 enum : int { WL_KV_EMPTY = 301, WL_A = 302, WL_KV_FULL = 303, WL_SEG = 304, WL_DRAIN = 305 };
@@ -74,7 +75,9 @@ k_linear_state_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant
     uint8_t *sV = smem + C::OFF_V;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
     uint64_t *kv_full = bars, *kv_empty = bars + ST;
-    uint64_t *a_ready = bars + 2 * ST, *seg_done = a_ready + 1, *mma_done = seg_done + 1;
+    // one a_ready per stage: the sigma pass may finish a chunk before the MMA thread has seen
+    // the previous one, and a barrier waited by parity must not complete twice unobserved
+    uint64_t *a_ready = bars + 2 * ST, *seg_done = a_ready + ST, *mma_done = seg_done + 1;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
     volatile int *abort = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
 
@@ -82,8 +85,8 @@ k_linear_state_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant
         for (int i = 0; i < ST; ++i) {
             mbar_init(kv_full + i, 1);
             mbar_init(kv_empty + i, 1);
+            mbar_init(a_ready + i, 128);
         }
-        mbar_init(a_ready, 128);
         mbar_init(seg_done, 1);
         mbar_init(mma_done, 1);
         *abort = 0;
@@ -130,7 +133,7 @@ k_linear_state_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant
             const uint32_t aK = smem_u32(sK), aV = smem_u32(sV);
             for (int g = 0; g < total; ++g) {
                 const int st = g % ST, i = g % nch;
-                if (!mbar_wait_short(a_ready, g & 1, abort, WL_A)) break;
+                if (!mbar_wait_short(a_ready + st, (g / ST) & 1, abort, WL_A)) break;
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {        // 128 tokens in steps of 16
@@ -202,6 +205,8 @@ k_linear_state_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant
             const int st = g % ST, s = g / nch, i = g % nch;
             if (!mbar_wait_short(kv_full + st, (g / ST) & 1, abort, WL_KV_FULL)) break;
             uint8_t *krow = sK + st * C::KTILE;
+            // a row past L (the zero fill of a short last segment) gets sigma = 0, not sigma(0)
+            const bool live = (int64_t)s * a.N + i * 128 + r < a.L;
 #pragma unroll
             for (int kb = 0; kb < D / 64; ++kb) {
 #pragma unroll
@@ -213,13 +218,14 @@ k_linear_state_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         __nv_bfloat162 t2 = *reinterpret_cast<__nv_bfloat162 *>(&w[e]);
-                        w[e] = pack_bf16x2(sigma_lin(__low2float(t2)), sigma_lin(__high2float(t2)));
+                        w[e] = live ? pack_bf16x2(sigma_lin(__low2float(t2)), sigma_lin(__high2float(t2)))
+                                    : 0u;
                     }
                     *p = make_uint4(w[0], w[1], w[2], w[3]);
                 }
             }
             fence_proxy_async_smem();
-            mbar_arrive(a_ready);
+            mbar_arrive(a_ready + st);
             if (i == nch - 1) {
                 if (!mbar_wait_short(seg_done, s & 1, abort, WL_SEG)) break;
                 tc_fence_after();

@@ -52,7 +52,7 @@ struct SegArgs {
     const float *beta;
     const float *snapZ;    // [chains * S, D] fp32 z_{s-1}
     __nv_bfloat16 *out;    // [B, H, L, D]
-    int64_t L;
+    int64_t L;             // rows per head; the last of the S segments may end before N rows
     int N, S, H, Hkv;
 };
 
@@ -92,6 +92,8 @@ k_segment_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
     bid /= qtiles;
     const int s = (int)(bid % a.S);
     bid /= a.S;
+    // a last segment shorter than N: tiles past the head's L rows have nothing to do
+    if ((int64_t)s * a.N + qt * C::BQ >= a.L) return;
     const int64_t bh = bid;
     const int h = (int)(bh % a.H);
     const int64_t b = bh / a.H;
@@ -343,8 +345,9 @@ k_segment_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
                 const float g = 1.f / (1.f + __expf(-a.beta[h]));
                 const float wl = (1.f - g) / l;
                 const float wm = den == 0.f ? 0.f : g / den;
-                __nv_bfloat16 *orow =
-                    a.out + ((bh * a.L) + (int64_t)s * a.N + (int64_t)qt * C::BQ + r) * D;
+                const int64_t row = (int64_t)s * a.N + (int64_t)qt * C::BQ + r;
+                const bool live = row < a.L;                     // rows past L: not stored
+                __nv_bfloat16 *orow = a.out + (bh * a.L + row) * D;
 #pragma unroll 1
                 for (int c = 0; c < D; c += 32) {
                     uint32_t o[32], rr[32];
@@ -359,9 +362,10 @@ k_segment_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
                         pk[e] = pack_bf16x2(y0, y1);
                     }
                     uint4 *dst = reinterpret_cast<uint4 *>(orow + c);
+                    if (live)
 #pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+                        for (int e = 0; e < 4; ++e)
+                            dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
                 }
             }
         }

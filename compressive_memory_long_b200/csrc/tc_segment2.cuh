@@ -95,6 +95,8 @@ k_segment_tc2(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     bid /= npairs;
     const int s = (int)(bid % a.S);
     bid /= a.S;
+    // a last segment shorter than N: tiles past the head's L rows have nothing to do
+    if ((int64_t)s * a.N + p * 256 >= a.L) return;
     const int64_t bh = bid;
     const int h = (int)(bh % a.H);
     const int64_t b = bh / a.H;
@@ -379,7 +381,9 @@ k_segment_tc2(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 const float g = 1.f / (1.f + __expf(-a.beta[h]));
                 const float wl = (1.f - g) / l;
                 const float wm = den == 0.f ? 0.f : g / den;
-                __nv_bfloat16 *orow = a.out + ((bh * a.L) + (int64_t)s * a.N + (int64_t)qt * 128 + r) * D;
+                const int64_t row = (int64_t)s * a.N + (int64_t)qt * 128 + r;
+                const bool live = row < a.L;                     // rows past L: not stored
+                __nv_bfloat16 *orow = a.out + (bh * a.L + row) * D;
 #pragma unroll 1
                 for (int c = 0; c < D; c += 32) {
                     uint32_t o[32], rr[32];
@@ -394,9 +398,10 @@ k_segment_tc2(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                         pk[e] = pack_bf16x2(y0, y1);
                     }
                     uint4 *dst = reinterpret_cast<uint4 *>(orow + c);
+                    if (live)
 #pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+                        for (int e = 0; e < 4; ++e)
+                            dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
                 }
             }
         }

@@ -42,10 +42,11 @@ def test_workspace_bytes():
     assert binding.infini_attn_workspace_bytes(2, 8, 1024, 64, 64) == \
         units * (64 * 64 + 64) * 4 + units * 64 * 64 * 2 + units * 64 * 64 * 2 + units * 4 + \
         2 * 8 * 4 + units * 16 + 512
-    # a final short segment needs no slot of its own; the sigma(K) copy spans every row
+    # a final short segment counts as a segment; the sigma(K) copy spans every row
     assert binding.infini_attn_workspace_bytes(1, 1, 100, 64, 64) == \
-        (64 * 64 + 64) * 4 + 64 * 64 * 2 + 100 * 64 * 2 + 4 + 4 + 16 + 512
-    assert binding.infini_attn_workspace_bytes(1, 1, 40, 64, 64) == 40 * 64 * 2 + 4 + 512
+        2 * (64 * 64 + 64) * 4 + 2 * 64 * 64 * 2 + 100 * 64 * 2 + 2 * 4 + 4 + 2 * 16 + 512
+    assert binding.infini_attn_workspace_bytes(1, 1, 40, 64, 64) == \
+        (64 * 64 + 64) * 4 + 64 * 64 * 2 + 40 * 64 * 2 + 4 + 4 + 16 + 512
     assert binding.infini_attn_workspace_bytes(0, 1, 64, 64, 64) == 0
 
 
