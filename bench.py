@@ -20,7 +20,11 @@ Timing: W untimed warm-up steps, then K steps each bracketed by CUDA events on t
 stream, with a 256 MiB write (larger than the 126 MB L2) before every step, outside the
 events, so each step starts with a cold L2.  The library's launch trace (CUDA events
 around each of its kernels, on the same stream) gives the dominant kernel's device time
-for the roofline and the launch count.  ``--impl reference`` times the fp64 CPU oracle
+for the roofline and the launch count.  A launch-bound workload (one whose workspace fits
+the allocation-free entry point's fixed array) is timed as replays of a CUDA graph of that
+call, and its per-kernel times come from the same steps run eagerly with the trace on.
+``e2e`` pipelines the steps as a serving loop would: step i + 1's inputs are copied in
+while step i computes and step i - 1's results are copied out.  ``--impl reference`` times the fp64 CPU oracle
 instead, on bounded samples of the same workload.
 """
 from __future__ import annotations
@@ -485,26 +489,55 @@ def main():
         fwd(t["q"], t["k"], t["v"], t["beta"], t["M0"], t["z0"], out, M_out, z_out, w.N,
             w.rule, stream)
 
+    # Launch-bound workloads (a workspace that fits the allocation-free entry point's fixed
+    # array): the timed step replays a CUDA graph of that call, as a serving loop would; the
+    # per-kernel times for the roofline come from an eager traced pass of the same steps.
+    graph = None
+    if w.dtype == "bf16" and binding.infini_attn_workspace_bytes(
+            w.B, w.Hkv, w.L, w.N, w.d) <= binding.NOALLOC_SCRATCH_BYTES:
+        def call_noalloc():
+            binding.infini_attn_fwd_noalloc(t["q"], t["k"], t["v"], t["beta"], t["M0"], t["z0"],
+                                            out, M_out, z_out, w.N, w.rule)
+        call_noalloc()
+        torch.cuda.synchronize(dev)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            call_noalloc()
+        torch.cuda.synchronize(dev)
+
+    def timed_step():
+        if graph is not None:
+            graph.replay()
+        else:
+            step()
+
     for _ in range(args.warmup):
         flush.zero_()
-        step()
+        timed_step()
     torch.cuda.synchronize(dev)
 
-    # ---- timed region (device time; trace on for per-kernel events) ----
+    # ---- timed region (device time; trace on for per-kernel events unless graphed) ----
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     barrier(world)
     torch.cuda.synchronize(dev)
-    binding.infini_attn_trace_enable(True)
+    binding.infini_attn_trace_enable(graph is None)
     with ClockSampler(local) as clocks:
         for i in range(args.steps):
             flush.zero_()
             starts[i].record(stream)
-            step()
+            timed_step()
             ends[i].record(stream)
         torch.cuda.synchronize(dev)
     binding.infini_attn_trace_enable(False)
     barrier(world)
+    if graph is not None:       # the same steps eagerly, traced, for the per-kernel times
+        binding.infini_attn_trace_enable(True)
+        for i in range(args.steps):
+            flush.zero_()
+            step()
+        torch.cuda.synchronize(dev)
+        binding.infini_attn_trace_enable(False)
     trace = binding.infini_attn_trace_report()
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     total_ms = max_over_ranks(float(sum(step_ms)), world, dev)
@@ -535,39 +568,58 @@ def main():
                  "kernel_share": kernels[dom]["ms"] / sum(v["ms"] for v in kernels.values())})
 
     # ---- end to end through the public call with host buffers ----
+    # The steps run as a serving loop would run them: two device buffer sets, step i + 1's
+    # inputs copied in from pinned host memory (copy-in stream) while step i computes and
+    # step i - 1's out / M / z are copied back (copy-out stream).  Every step's copies are
+    # inside the timed region, which runs from before the first copy-in to after the last
+    # copy-out.  No L2 flush here: each step's inputs arrive through the copy itself.
     out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
     M_h = torch.empty(M_out.shape, dtype=torch.float32, pin_memory=True)
     z_h = torch.empty(z_out.shape, dtype=torch.float32, pin_memory=True)
     h2d = sum(x.numel() * x.element_size() for x in host.values() if x is not None)
     d2h = sum(x.numel() * x.element_size() for x in (out_h, M_h, z_h))
-    e_starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    e_ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    t2 = {k: (None if x is None else torch.empty_like(x)) for k, x in t.items()}
+    sets = [(t, out, M_out, z_out),
+            (t2, torch.empty_like(out), torch.empty_like(M_out), torch.empty_like(z_out))]
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_c = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
 
-    def e2e_step(i=None):
-        if i is not None:
-            e_starts[i].record(stream)
-        for kname, x in host.items():
-            if x is not None:
-                t[kname].copy_(x, non_blocking=True)
-        step()
-        out_h.copy_(out, non_blocking=True)
-        M_h.copy_(M_out, non_blocking=True)
-        z_h.copy_(z_out, non_blocking=True)
-        if i is not None:
-            e_ends[i].record(stream)
+    def e2e_run(n):
+        for i in range(n):
+            b = i % 2
+            ti, oi, Mi, zi = sets[b]
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(ev_c[b])          # step i - 2 has read this input set
+                for kname, x in host.items():
+                    if x is not None:
+                        ti[kname].copy_(x, non_blocking=True)
+                ev_in[b].record(s_in)
+            stream.wait_event(ev_in[b])
+            if i >= 2:
+                stream.wait_event(ev_out[b])          # step i - 2's results are copied out
+            fwd(ti["q"], ti["k"], ti["v"], ti["beta"], ti["M0"], ti["z0"], oi, Mi, zi, w.N,
+                w.rule, stream)
+            ev_c[b].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_c[b])
+                out_h.copy_(oi, non_blocking=True)
+                M_h.copy_(Mi, non_blocking=True)
+                z_h.copy_(zi, non_blocking=True)
+                ev_out[b].record(s_out)
 
-    for _ in range(args.warmup):
-        flush.zero_()
-        e2e_step()
+    e2e_run(args.warmup)
     barrier(world)
     torch.cuda.synchronize(dev)
-    for i in range(args.steps):
-        flush.zero_()
-        e2e_step(i)
+    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e_start.record(s_in)
+    e2e_run(args.steps)
+    e_end.record(s_out)
     torch.cuda.synchronize(dev)
     barrier(world)
-    e2e_ms = max_over_ranks(float(sum(s.elapsed_time(e) for s, e in zip(e_starts, e_ends))),
-                            world, dev)
+    e2e_ms = max_over_ranks(float(e_start.elapsed_time(e_end)), world, dev)
 
     # ---- CPU oracle baseline (rank 0, single GPU only) ----
     cpu = None
@@ -582,10 +634,13 @@ def main():
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": total_ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
-            "data": "synthetic", "config": config_of(w),
+            "data": "synthetic",
+            "config": dict(config_of(w), launch="CUDA graph of infini_attn_fwd_noalloc"
+                           if graph is not None else "eager infini_attn_fwd calls"),
             "roofline": roof, "cpu_baseline": cpu,
             "e2e": {"value": w.tokens * args.steps * world / (e2e_ms / 1000.0),
-                    "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                    "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "pipelined": "copy-in, compute and copy-out streams overlap across steps"},
             "gpu_launches": launches, "kernels": kernels,
             "clocks": clocks.summary(),
         }

@@ -205,8 +205,9 @@ k_linear_state_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant
             const int st = g % ST, s = g / nch, i = g % nch;
             if (!mbar_wait_short(kv_full + st, (g / ST) & 1, abort, WL_KV_FULL)) break;
             uint8_t *krow = sK + st * C::KTILE;
-            // a row past L (the zero fill of a short last segment) gets sigma = 0, not sigma(0)
-            const bool live = (int64_t)s * a.N + i * 128 + r < a.L;
+            // a row past L (the zero fill of a short last segment) gets sigma = 0, not sigma(0):
+            // a mask, not a select, so the element loop stays free of branches
+            const uint32_t keep = (int64_t)s * a.N + i * 128 + r < a.L ? 0xFFFFFFFFu : 0u;
 #pragma unroll
             for (int kb = 0; kb < D / 64; ++kb) {
 #pragma unroll
@@ -218,8 +219,7 @@ k_linear_state_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         __nv_bfloat162 t2 = *reinterpret_cast<__nv_bfloat162 *>(&w[e]);
-                        w[e] = live ? pack_bf16x2(sigma_lin(__low2float(t2)), sigma_lin(__high2float(t2)))
-                                    : 0u;
+                        w[e] = pack_bf16x2(sigma_lin(__low2float(t2)), sigma_lin(__high2float(t2))) & keep;
                     }
                     *p = make_uint4(w[0], w[1], w[2], w[3]);
                 }

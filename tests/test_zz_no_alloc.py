@@ -63,3 +63,28 @@ def test_noalloc_rejects_problems_beyond_its_array():
     ptrs = [ctypes.c_void_p(base + i * gap) for i in range(9)]
     rc = binding.LIB.infini_attn_fwd_noalloc(*ptrs, w.B, w.H, w.Hkv, w.L, w.N, w.d, 1, None)
     assert rc == 2          # INFINI_ERR_UNSUPPORTED
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("name", ["hf_repro_n64"])
+def test_noalloc_call_replays_as_cuda_graph(name):
+    """The call captured once in a CUDA graph (as the benchmark times launch-bound
+    workloads) and replayed gives the eager call's results, bit for bit."""
+    w = wl.WORKLOADS[name]
+    t = {k: (None if x is None else x.cuda()) for k, x in wl.torch_inputs(w).items()}
+    ref = run(binding.infini_attn_fwd_noalloc, t, w)
+    out = torch.empty_like(t["q"])
+    M = torch.empty((w.B, w.Hkv, w.d, w.d), dtype=torch.float32, device="cuda")
+    z = torch.empty((w.B, w.Hkv, w.d), dtype=torch.float32, device="cuda")
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        binding.infini_attn_fwd_noalloc(t["q"], t["k"], t["v"], t["beta"], t["M0"], t["z0"],
+                                        out, M, z, w.N, w.rule)
+    for _ in range(3):
+        out.zero_()
+        M.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(out, ref[0]) and torch.equal(M, ref[1]) and torch.equal(z, ref[2])
+    del g
+    assert binding.infini_attn_device_status() == 0
