@@ -7,8 +7,9 @@ fails to load, importing this module raises.
 Names mirror the C ABI in ``include/infini_attn.h``:
 ``infini_attn_fwd`` (bf16), ``infini_attn_fwd_f32``, ``infini_attn_workspace_bytes``,
 ``infini_attn_status_string``, ``infini_attn_version``, ``infini_attn_decode_step`` (+
-``_f32``), ``infini_attn_fold`` (+ ``_f32``); ``forward``, ``decode_step`` and ``fold``
-allocate what is missing and pick the entry point from the activation dtype.
+``_f32``), ``infini_attn_fold`` (+ ``_f32``), ``infini_attn_state`` (+ ``_f32``);
+``forward``, ``decode_step``, ``fold`` and ``state`` allocate what is missing and pick the
+entry point from the activation dtype.
 """
 from __future__ import annotations
 
@@ -31,6 +32,7 @@ _P, _I64, _I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
 _FWD_ARGS = [_P] * 9 + [_I64] * 6 + [_I, _P]
 _DEC_ARGS = [_P] * 6 + [_I64] + [_P] * 3 + [_I64] * 5 + [_I, _P]
 _FOLD_ARGS = [_P, _P, _I64, _P, _P] + [_I64] * 4 + [_I, _P]
+_STATE_ARGS = [_P] * 6 + [_I64] * 5 + [_I, _P]
 SIGNATURES = {
     "infini_attn_fwd": (_FWD_ARGS, _I),
     "infini_attn_fwd_f32": (_FWD_ARGS, _I),
@@ -39,6 +41,8 @@ SIGNATURES = {
     "infini_attn_decode_step_f32": (_DEC_ARGS, _I),
     "infini_attn_fold": (_FOLD_ARGS, _I),
     "infini_attn_fold_f32": (_FOLD_ARGS, _I),
+    "infini_attn_state": (_STATE_ARGS, _I),
+    "infini_attn_state_f32": (_STATE_ARGS, _I),
     "infini_attn_workspace_bytes": ([_I64] * 5, _I64),
     "infini_attn_status_string": ([_I], ctypes.c_char_p),
     "infini_attn_version": ([], _I),
@@ -230,3 +234,30 @@ def fold(k_cache, v_cache, n: int, M, z, *, rule="linear", stream=None):
             _stream_handle(stream))
     if rc != 0:
         raise InfiniError(rc, infini_attn_status_string(rc))
+
+
+def state(k, v, M0=None, z0=None, *, N: int, rule="linear", M_out=None, z_out=None,
+          stream=None):
+    """The memory after the whole sequence without the outputs: k/v [B,Hkv,L,d] (bf16 or
+    fp32), M0 [B,Hkv,d,d] / z0 [B,Hkv,d] fp32 or None.  Returns (M_out, z_out)."""
+    B, Hkv, L, d = k.shape
+    dev = k.device
+    _check(k, "k", k.dtype, (B, Hkv, L, d), dev)
+    _check(v, "v", k.dtype, (B, Hkv, L, d), dev)
+    _check(M0, "M0", torch.float32, (B, Hkv, d, d), dev)
+    _check(z0, "z0", torch.float32, (B, Hkv, d), dev)
+    if M_out is None:
+        M_out = torch.empty((B, Hkv, d, d), dtype=torch.float32, device=dev)
+    if z_out is None:
+        z_out = torch.empty((B, Hkv, d), dtype=torch.float32, device=dev)
+    if k.dtype == torch.bfloat16:
+        fn = LIB.infini_attn_state
+    elif k.dtype == torch.float32:
+        fn = LIB.infini_attn_state_f32
+    else:
+        raise ValueError(f"unsupported activation dtype {k.dtype}")
+    rc = fn(_ptr(k), _ptr(v), _ptr(M0), _ptr(z0), _ptr(M_out), _ptr(z_out), B, Hkv, L, int(N),
+            d, RULES[rule], _stream_handle(stream))
+    if rc != 0:
+        raise InfiniError(rc, infini_attn_status_string(rc))
+    return M_out, z_out

@@ -66,7 +66,7 @@ bool ranges_overlap(const void *a, int64_t na, const void *b, int64_t nb)
 int check_args(const void *q, const void *k, const void *v, const float *beta, const float *M0,
                const float *z0, const void *out, const float *M_out, const float *z_out,
                int64_t B, int64_t H, int64_t Hkv, int64_t L, int64_t N, int64_t d, int rule,
-               int64_t esize, Problem *pb)
+               int64_t esize, Problem *pb, bool out_checked = true)
 {
     if (!q || !k || !v || !beta || !out || !M_out || !z_out) return INFINI_ERR_INVALID_ARG;
     if (B <= 0 || H <= 0 || Hkv <= 0 || L <= 0 || N <= 0 || d <= 0) return INFINI_ERR_INVALID_ARG;
@@ -83,10 +83,12 @@ int check_args(const void *q, const void *k, const void *v, const float *beta, c
     if (partial_overlap(M0, mbytes, M_out, mbytes) || partial_overlap(z0, zbytes, z_out, zbytes))
         return INFINI_ERR_INVALID_ARG;
     const int64_t obytes = B * H * L * d * esize, kvbytes = B * Hkv * L * d * esize;
-    if (ranges_overlap(out, obytes, q, obytes) || ranges_overlap(out, obytes, k, kvbytes) ||
-        ranges_overlap(out, obytes, v, kvbytes) || ranges_overlap(out, obytes, M_out, mbytes) ||
-        ranges_overlap(out, obytes, z_out, zbytes) || ranges_overlap(M_out, mbytes, z_out, zbytes))
+    if (out_checked &&
+        (ranges_overlap(out, obytes, q, obytes) || ranges_overlap(out, obytes, k, kvbytes) ||
+         ranges_overlap(out, obytes, v, kvbytes) || ranges_overlap(out, obytes, M_out, mbytes) ||
+         ranges_overlap(out, obytes, z_out, zbytes)))
         return INFINI_ERR_INVALID_ARG;
+    if (ranges_overlap(M_out, mbytes, z_out, zbytes)) return INFINI_ERR_INVALID_ARG;
     if (d != 32 && d != 64 && d != 128) return INFINI_ERR_UNSUPPORTED;
     if (N % 64 != 0) return INFINI_ERR_UNSUPPORTED;
     pb->B = B; pb->H = H; pb->Hkv = Hkv; pb->L = L; pb->N = N; pb->d = d; pb->S = L / N;
@@ -449,13 +451,15 @@ int launch_pieces(const Problem &p, const __nv_bfloat16 *q, const __nv_bfloat16 
     return INFINI_OK;
 }
 
+// outputs = false: the memory chain only (M_out, z_out), no segment kernel.
 template <typename T, int D>
 int launch_all(const Problem &p, const T *q, const T *k, const T *v, const float *beta,
                const float *M0, const float *z0, T *out, float *M_out, float *z_out,
-               float *snapM, float *snapZ, __nv_bfloat16 *snapMb, cudaStream_t st)
+               float *snapM, float *snapZ, __nv_bfloat16 *snapMb, cudaStream_t st,
+               bool outputs = true)
 {
     if constexpr (sizeof(T) == 2 && D == 64) {
-        if (use_small_fused<T>(p)) {
+        if (outputs && use_small_fused<T>(p)) {
             const int rc = use_pieces(p)
                 ? launch_pieces(p, q, k, v, beta, M0, z0, out, M_out, z_out, snapM, st)
                 : launch_small_fused(p, q, k, v, beta, M0, z0, out, M_out, z_out, snapM, st);
@@ -508,6 +512,7 @@ int launch_all(const Problem &p, const T *q, const T *k, const T *v, const float
                 k, v, snapM, snapZ, snapMb, M_out, z_out, p.L, N, S, N);
         }
     }
+    if (!outputs) return cudaGetLastError() == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
     if constexpr (sizeof(T) == 2 && (D == 64 || D == 128)) {
         if (snapMb) {
             const int rc = launch_segment_tc<D>(p, q, k, v, beta, snapMb, snapZ, out, st);
@@ -559,7 +564,7 @@ void launch_fold_inplace(const T *k, const T *v, int64_t L, int64_t n, float *M,
 template <typename T, int D>
 int launch_tail(const Problem &p, const T *q, const T *k, const T *v, const float *beta,
                 const float *M0, const float *z0, T *out, float *M_out, float *z_out,
-                cudaStream_t st)
+                cudaStream_t st, bool outputs = true)
 {
     const int64_t chains = p.B * p.Hkv, off = p.Lf * D;
     const int Tn = (int)p.T, Np = (Tn + 63) / 64 * 64;
@@ -575,8 +580,8 @@ int launch_tail(const Problem &p, const T *q, const T *k, const T *v, const floa
             return INFINI_ERR_CUDA;
     }
     const size_t smem = SimtSegSmem<D>::bytes;
-    if (!opt_in_smem<k_segment_simt<T, D>>(smem)) return INFINI_ERR_CUDA;
-    {
+    if (outputs && !opt_in_smem<k_segment_simt<T, D>>(smem)) return INFINI_ERR_CUDA;
+    if (outputs) {
         TRACED("tail_segment", st);
         k_segment_simt<T, D><<<(unsigned)(p.B * p.H * (Np / 64)), 256, smem, st>>>(
             q + off, k + off, v + off, beta, M_out, z_out, out + off, p.L, Np, 1, (int)p.H,
@@ -607,14 +612,15 @@ Problem effective(const Problem &p)
 template <typename T, int D>
 int launch_forward(const Problem &p, const T *q, const T *k, const T *v, const float *beta,
                    const float *M0, const float *z0, T *out, float *M_out, float *z_out,
-                   float *snapM, float *snapZ, __nv_bfloat16 *snapMb, cudaStream_t st)
+                   float *snapM, float *snapZ, __nv_bfloat16 *snapMb, cudaStream_t st,
+                   bool outputs = true)
 {
     if (p.S > 0) {
         const int rc = launch_all<T, D>(p, q, k, v, beta, M0, z0, out, M_out, z_out, snapM, snapZ,
-                                        snapMb, st);
+                                        snapMb, st, outputs);
         if (rc != INFINI_OK || p.T == 0) return rc;
     }
-    return launch_tail<T, D>(p, q, k, v, beta, M0, z0, out, M_out, z_out, st);
+    return launch_tail<T, D>(p, q, k, v, beta, M0, z0, out, M_out, z_out, st, outputs);
 }
 
 // The library's own stream-ordered pool on the current device.  Its release threshold keeps
@@ -744,6 +750,57 @@ int forward_noalloc(const void *q, const void *k, const void *v, const float *be
     case 64: return launch_forward<T, 64>(p, tq, tk, tv, beta, M0, z0, to, M_out, z_out, snapM, snapZ, snapMb, st);
     default: return launch_forward<T, 128>(p, tq, tk, tv, beta, M0, z0, to, M_out, z_out, snapM, snapZ, snapMb, st);
     }
+}
+
+// ---- the memory chain alone -----------------------------------------------------------------
+
+// The state after the whole sequence, without the outputs: the forward's memory kernels on
+// the same workspace, the segment kernels left out.  Arguments as the forward's, less q,
+// beta and out (H is taken as Hkv).
+template <typename T>
+int state_only(const void *k, const void *v, const float *M0, const float *z0, float *M_out,
+               float *z_out, int64_t B, int64_t Hkv, int64_t L, int64_t N, int64_t d, int rule,
+               infini_stream_t stream)
+{
+    if (!k || !v || !M_out || !z_out) return INFINI_ERR_INVALID_ARG;
+    // the forward's checks with k standing in for q and out (never written: no outputs) and
+    // M_out for beta (never read)
+    const int64_t es = (int64_t)sizeof(T), kvbytes = B * Hkv * L * d * es;
+    if (B > 0 && Hkv > 0 && L > 0 && d > 0 &&
+        (ranges_overlap(M_out, B * Hkv * d * d * 4, k, kvbytes) ||
+         ranges_overlap(M_out, B * Hkv * d * d * 4, v, kvbytes) ||
+         ranges_overlap(z_out, B * Hkv * d * 4, k, kvbytes) ||
+         ranges_overlap(z_out, B * Hkv * d * 4, v, kvbytes)))
+        return INFINI_ERR_INVALID_ARG;
+    Problem p;
+    int rc = check_args(k, k, v, M_out, M0, z0, k, M_out, z_out, B, Hkv, Hkv, L, N, d, rule, es,
+                        &p, /*out_checked=*/false);
+    if (rc != INFINI_OK) return rc;
+    p = effective<T>(p);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaGetLastError();
+    const int64_t nM = p.B * p.Hkv * p.S * p.d * p.d, nZ = p.B * p.Hkv * p.S * p.d;
+    const bool tc_path = use_tc<T>(p);
+    const int64_t bytes = p.S == 0 ? 0 : workspace_bytes(p.B, p.Hkv, p.L, p.N, p.d);
+    void *ws = nullptr;
+    if (bytes > 0) {
+        cudaMemPool_t pool = workspace_pool();
+        if (!pool) return INFINI_ERR_CUDA;
+        if (cudaMallocFromPoolAsync(&ws, (size_t)bytes, pool, st) != cudaSuccess) {
+            cudaGetLastError();
+            return INFINI_ERR_OOM;
+        }
+    }
+    float *snapM = static_cast<float *>(ws), *snapZ = snapM + nM;
+    __nv_bfloat16 *snapMb = tc_path ? reinterpret_cast<__nv_bfloat16 *>(snapZ + nZ) : nullptr;
+    const T *tk = static_cast<const T *>(k), *tv = static_cast<const T *>(v);
+    switch (p.d) {
+    case 32: rc = launch_forward<T, 32>(p, tk, tk, tv, nullptr, M0, z0, nullptr, M_out, z_out, snapM, snapZ, snapMb, st, false); break;
+    case 64: rc = launch_forward<T, 64>(p, tk, tk, tv, nullptr, M0, z0, nullptr, M_out, z_out, snapM, snapZ, snapMb, st, false); break;
+    default: rc = launch_forward<T, 128>(p, tk, tk, tv, nullptr, M0, z0, nullptr, M_out, z_out, snapM, snapZ, snapMb, st, false); break;
+    }
+    if (ws && cudaFreeAsync(ws, st) != cudaSuccess && rc == INFINI_OK) rc = INFINI_ERR_CUDA;
+    return rc;
 }
 
 // ---- token-by-token decode and the fold of a cached segment -------------------------------
@@ -906,6 +963,22 @@ int infini_attn_fwd_f32(const void *q, const void *k, const void *v, const float
 {
     return infini::forward<float>(q, k, v, beta, M0, z0, out, M_out, z_out, B, H, Hkv, L, N, d,
                                   update_rule, stream);
+}
+
+int infini_attn_state(const void *k, const void *v, const float *M0, const float *z0,
+                      float *M_out, float *z_out, int64_t B, int64_t Hkv, int64_t L, int64_t N,
+                      int64_t d, int update_rule, infini_stream_t stream)
+{
+    return infini::state_only<__nv_bfloat16>(k, v, M0, z0, M_out, z_out, B, Hkv, L, N, d,
+                                             update_rule, stream);
+}
+
+int infini_attn_state_f32(const void *k, const void *v, const float *M0, const float *z0,
+                          float *M_out, float *z_out, int64_t B, int64_t Hkv, int64_t L,
+                          int64_t N, int64_t d, int update_rule, infini_stream_t stream)
+{
+    return infini::state_only<float>(k, v, M0, z0, M_out, z_out, B, Hkv, L, N, d, update_rule,
+                                     stream);
 }
 
 int infini_attn_decode_step(const void *q, const void *k, const void *v, const float *beta,

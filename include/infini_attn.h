@@ -97,6 +97,23 @@ INFINI_API int infini_attn_fwd_f32(const void *q, const void *k, const void *v, 
                         int64_t d, int update_rule, infini_stream_t stream);
 
 /*
+ * The memory after the whole sequence, without the outputs (bf16 keys / values; the _f32
+ * variant takes fp32 ones): M_out / z_out exactly as infini_attn_fwd would leave them, from
+ * the forward's memory kernels alone.  With M0 = z0 = NULL this is the increment of a
+ * sequence chunk under the additive rule, the quantity ranks exchange when one sequence is
+ * cut across devices (the memory before a chunk is M0 plus the increments of the chunks
+ * before it).  Arguments, layouts, aliasing and errors as for infini_attn_fwd, without q,
+ * beta and out.
+ */
+INFINI_API int infini_attn_state(const void *k, const void *v, const float *M0, const float *z0,
+                                 float *M_out, float *z_out, int64_t B, int64_t Hkv, int64_t L,
+                                 int64_t N, int64_t d, int update_rule, infini_stream_t stream);
+INFINI_API int infini_attn_state_f32(const void *k, const void *v, const float *M0,
+                                     const float *z0, float *M_out, float *z_out, int64_t B,
+                                     int64_t Hkv, int64_t L, int64_t N, int64_t d,
+                                     int update_rule, infini_stream_t stream);
+
+/*
  * Token-by-token decode (bf16 activations; the _f32 variant takes fp32 ones).  One call
  * processes one new token of every (batch, head) at offset `pos` of its current segment
  * and gives the output the forward would give that token:

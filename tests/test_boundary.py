@@ -143,3 +143,28 @@ def call_fold(entry="infini_attn_fold", n=1, B=1, Hkv=2, N=64, d=64, rule=0, **p
 ])
 def test_fold_argument_errors(entry, kw, status):
     assert call_fold(entry, **kw) == status
+
+
+STATE_PTRS = ["k", "v", "M0", "z0", "M_out", "z_out"]
+
+
+def call_state(entry="infini_attn_state", B=1, Hkv=2, L=128, N=64, d=64, rule=0, **ptr):
+    gap = 1 << 32
+    p = {name: BASE + i * gap for i, name in enumerate(STATE_PTRS)}
+    p.update(ptr)
+    a = [None if p[x] is None else ctypes.c_void_p(p[x]) for x in STATE_PTRS]
+    return getattr(binding.LIB, entry)(*a, B, Hkv, L, N, d, rule, None)
+
+
+@pytest.mark.parametrize("entry", ["infini_attn_state", "infini_attn_state_f32"])
+@pytest.mark.parametrize("kw,status", [
+    (dict(k=None), INVALID), (dict(v=None), INVALID), (dict(M_out=None), INVALID),
+    (dict(z_out=None), INVALID), (dict(B=0), INVALID), (dict(L=0), INVALID),
+    (dict(rule=5), INVALID), (dict(k=BASE + 4), INVALID),
+    (dict(M_out=BASE + (2 << 32) + 64), INVALID),            # partial overlap with M0
+    (dict(M_out=BASE), INVALID),                             # on top of k
+    (dict(z_out=BASE + (1 << 32) + 16), INVALID),            # inside v
+    (dict(d=48), UNSUPPORTED), (dict(N=100), UNSUPPORTED),
+])
+def test_state_argument_errors(entry, kw, status):
+    assert call_state(entry, **kw) == status
