@@ -61,7 +61,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # 2048-segment capture scaled to 16384 segments (traffic grows with the units processed).
 NCU_TRAFFIC_BYTES: dict = {
     ("hf_repro_n64", "small_fused"): 6362112,
-    ("gqa8b_n2048_delta", "segment_tc"): 407551488 + 236756224,
+    ("gqa8b_n2048_delta", "segment_tc"): 407576576 + 234468608,
     ("n64_bandwidth", "small_pieces"): (1028091000 + 268262400) * 8,
 }
 

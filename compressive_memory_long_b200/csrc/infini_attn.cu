@@ -811,7 +811,9 @@ int check_cache_state(const void *k_cache, const void *v_cache, const float *M, 
     if (!k_cache || !v_cache || !M || !z) return INFINI_ERR_INVALID_ARG;
     if (B <= 0 || Hkv <= 0 || N <= 0 || d <= 0) return INFINI_ERR_INVALID_ARG;
     if (rule != INFINI_UPDATE_LINEAR && rule != INFINI_UPDATE_DELTA) return INFINI_ERR_INVALID_ARG;
-    if (B > (1 << 20) || Hkv > (1 << 16) || N > ((int64_t)1 << 30) || B * Hkv * N > ((int64_t)1 << 40))
+    // grids of up to 8 CTAs per chain stay below 2^31 CTAs
+    if (B > (1 << 20) || Hkv > (1 << 16) || B * Hkv > ((int64_t)1 << 27) ||
+        N > ((int64_t)1 << 30) || B * Hkv * N > ((int64_t)1 << 40))
         return INFINI_ERR_INVALID_ARG;
     const void *ptrs[] = {k_cache, v_cache, M, z};
     for (const void *p : ptrs)

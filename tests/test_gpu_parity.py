@@ -98,6 +98,13 @@ def test_gqa8b_sampled(rule):
     check_sampled(w, chains=[(0, 3)], segs=[0, 1, 15])
 
 
+def test_gqa8b_short_last_segment_sampled():
+    """The 8B-class layout with a 1000-token seventeenth segment (run on the tensor-core
+    kernels as one more segment): the first and the short segment of two chains."""
+    w = wl.WORKLOADS["gqa8b_n2048_delta"].replace(name="gqa8b_tail1000", tail=1000)
+    check_sampled(w, chains=[(0, 0), (0, 7)], segs=[0, 16])
+
+
 def test_stream1m_sampled():
     w = wl.WORKLOADS["stream1m_n2048_delta"]
     check_sampled(w, chains=[(0, 7)], segs=[0, 1, 511])
