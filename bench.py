@@ -295,8 +295,8 @@ def run_decode(args, w: wl.Workload, world: int, rank: int, local: int, dev):
     The N calls of a step are captured once in a CUDA graph (the calls allocate nothing),
     and the timed region replays it: device time without the host's per-call overhead.
     The decode kernel's own time comes from a second graph of the calls at offsets
-    0 .. N - 2 (no fold).  ``e2e`` makes the same calls eagerly from Python, each token's
-    inputs copied from pinned host memory and its output copied back.
+    0 .. N - 2 (no fold).  ``e2e`` adds each token's copies to the graph: its q, k, v from
+    pinned host memory before its call and its output back after it.
     """
     from compressive_memory_long_b200 import binding
     host = wl.torch_inputs(w, pin_memory=True)
@@ -372,32 +372,30 @@ def run_decode(args, w: wl.Workload, world: int, rank: int, local: int, dev):
     del g_step, g_attn
 
     out_h = torch.empty(outs.shape, dtype=dt, pin_memory=True)
-    e_starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    e_ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-
-    def e2e_step(i=None):
-        if i is not None:
-            e_starts[i].record(stream)
+    g_e2e = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_e2e):
         for p in range(w.N):
             for n in ("q", "k", "v"):
                 t[n][p].copy_(tok[n][p], non_blocking=True)
             binding.decode_step(t["q"][p], t["k"][p], t["v"][p], beta, kc, vc, p, M, z,
                                 rule=w.rule, out=outs[p])
             out_h[p].copy_(outs[p], non_blocking=True)
-        if i is not None:
-            e_ends[i].record(stream)
-
     for _ in range(args.warmup):
-        e2e_step()
+        g_e2e.replay()
     barrier(world)
     torch.cuda.synchronize(dev)
+    e_starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    e_ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     for i in range(args.steps):
         flush.zero_()
-        e2e_step(i)
+        e_starts[i].record(stream)
+        g_e2e.replay()
+        e_ends[i].record(stream)
     torch.cuda.synchronize(dev)
     barrier(world)
     e2e_ms = max_over_ranks(float(sum(s.elapsed_time(e) for s, e in zip(e_starts, e_ends))),
                             world, dev)
+    del g_e2e
     h2d = sum(x.numel() * x.element_size() for x in tok.values())
     d2h = out_h.numel() * out_h.element_size()
 
