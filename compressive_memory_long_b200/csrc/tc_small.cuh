@@ -172,6 +172,18 @@ k_small_linear_fused(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         *abort = 0;
         *s_state = 0;
         fence_barrier_init();
+        // this thread knows its unit already: start the loads before the TMEM allocation
+        // and the block barrier, so they overlap both
+        const int t0 = *s_ticket;
+        const int64_t ch = t0 % a.chains;
+        const int un = t0 / a.chains;
+        prefetch_tmap(&tmQ);
+        prefetch_tmap(&tmK);
+        prefetch_tmap(&tmV);
+        mbar_arrive_expect_tx(full, 3 * C::BOX);
+        tma_load_3d(sQ, &tmQ, full, 0, un * C::TOK, (int)ch);
+        tma_load_3d(sK, &tmK, full, 0, un * C::TOK, (int)ch);
+        tma_load_3d(sV, &tmV, full, 0, un * C::TOK, (int)ch);
     }
     if (warp == 1) tmem_alloc(tmem_holder, 512);
     tc_fence_before();
@@ -187,16 +199,7 @@ k_small_linear_fused(const __grid_constant__ CUtensorMap tmQ, const __grid_const
     const int64_t idx = chain * a.U + unit;
 
     if (warp == 0) {
-        if (lane == 0) {
-            prefetch_tmap(&tmQ);
-            prefetch_tmap(&tmK);
-            prefetch_tmap(&tmV);
-            mbar_arrive_expect_tx(full, 3 * C::BOX);
-            tma_load_3d(sQ, &tmQ, full, 0, unit * C::TOK, (int)chain);
-            tma_load_3d(sK, &tmK, full, 0, unit * C::TOK, (int)chain);
-            tma_load_3d(sV, &tmV, full, 0, unit * C::TOK, (int)chain);
-            if (*abort) small_drain(full, 0);
-        }
+        if (lane == 0 && *abort) small_drain(full, 0);   // the loads were issued above
     } else if (warp == 1) {
         if (lane == 0) {
             constexpr uint32_t idS = idesc_bf16(128, 128, 0, 0);
