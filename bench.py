@@ -435,6 +435,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="CPU-oracle sample size for cpu_baseline (0 disables)")
+    ap.add_argument("--segment-len", type=int, default=0,
+                    help="run the workload's tokens in segments of this length instead (other "
+                         "kernels' profiles: N = 128 selects the one-tile segment kernel)")
     ap.add_argument("--tail", type=int, default=0,
                     help="append a final segment of this many (< N) tokens to every head")
     ap.add_argument("--decode", action="store_true",
@@ -446,6 +449,11 @@ def main():
     w = wl.WORKLOADS[args.workload]
     if args.segments > 0:
         w = dataclasses.replace(w, name=f"{w.name}@S{args.segments}", S=args.segments)
+    if args.segment_len:
+        if args.segment_len <= 0 or args.segment_len % 64 or w.L % args.segment_len:
+            ap.error("--segment-len must be a positive multiple of 64 dividing L")
+        w = dataclasses.replace(w, name=f"{w.name}@N{args.segment_len}", N=args.segment_len,
+                                S=w.L // args.segment_len)
     if args.tail:
         if not 0 < args.tail < w.N:
             ap.error("--tail must be in (0, N)")

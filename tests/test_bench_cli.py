@@ -13,6 +13,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
     (["--tail", "-3"], "--tail must be in (0, N)"),
     (["--warmup", "2"], "--warmup must be >= 3"),
     (["--workload", "no_such_workload"], "invalid choice"),
+    (["--segment-len", "100"], "--segment-len must be"),
 ])
 def test_bench_rejects_bad_flags(args, needle):
     r = subprocess.run([sys.executable, "bench.py", *args], cwd=ROOT, capture_output=True,
