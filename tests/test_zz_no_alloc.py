@@ -40,6 +40,12 @@ def run(entry, t, w):
     wl.Workload("noalloc_tc", B=1, H=4, Hkv=2, d=128, N=256, S=3, dtype="bf16", rule="delta",
                 seed=31, beta_dist=("normal", 0.0, 1.0), M0_dist=("uniform", 0.0, 0.1),
                 z0_dist=("uniform", 1.0, 2.0)),
+    # short last segments: one more tensor-core segment; the CUDA-core tail after fused units
+    wl.Workload("noalloc_tc_tail", B=1, H=4, Hkv=2, d=128, N=256, S=2, tail=100,
+                dtype="bf16", rule="delta", seed=32, beta_dist=("normal", 0.0, 1.0)),
+    wl.Workload("noalloc_fused_tail", B=2, H=4, Hkv=4, d=64, N=64, S=6, tail=21,
+                dtype="bf16", rule="linear", seed=33, beta_dist=("normal", 0.0, 1.0),
+                M0_dist=("uniform", 0.0, 0.1), z0_dist=("uniform", 1.0, 2.0)),
 ], ids=lambda w: w.name)
 def test_noalloc_matches_allocating_entry_point(w):
     assert binding.infini_attn_workspace_bytes(w.B, w.Hkv, w.L, w.N, w.d) <= \
