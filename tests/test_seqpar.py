@@ -45,10 +45,11 @@ def _oracle_fns():
 W = wl.Workload("seqpar", B=2, H=4, Hkv=2, d=16, N=8, S=5, tail=3, dtype="f32", rule="linear",
                 seed=51, beta_dist=("normal", 0.0, 1.0), M0_dist=("uniform", 0.0, 0.1),
                 z0_dist=("uniform", 1.0, 2.0))
-CUTS = [0, 16, 43]          # rank 0: tokens 0-15 (two segments), rank 1: 16-42 (ragged end)
+CUTS2 = [0, 16, 43]         # rank 0: tokens 0-15 (two segments), rank 1: 16-42 (ragged end)
+CUTS3 = [0, 8, 32, 43]      # one, three and 1 3/8 segments
 
 
-def _rank_main(rank, world, port, results):
+def _rank_main(rank, world, port, results, CUTS=CUTS2):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
@@ -77,13 +78,15 @@ def _rank_main(rank, world, port, results):
         dist.destroy_process_group()
 
 
-def test_two_rank_sequence_split_equals_one_run():
+@pytest.mark.parametrize("cuts", [CUTS2, CUTS3], ids=["2ranks", "3ranks"])
+def test_sequence_split_equals_one_run(cuts):
     import oracle
-    world, port = 2, _free_port()
+    world, port = len(cuts) - 1, _free_port()
     ctx = mp.get_context("spawn")
     mgr = ctx.Manager()
     results = mgr.dict()
-    procs = [ctx.Process(target=_rank_main, args=(r, world, port, results)) for r in range(world)]
+    procs = [ctx.Process(target=_rank_main, args=(r, world, port, results, cuts))
+             for r in range(world)]
     for p in procs:
         p.start()
     for p in procs:
@@ -92,10 +95,10 @@ def test_two_rank_sequence_split_equals_one_run():
     q, k, v, beta, M0, z0 = wl.host_inputs(W)
     ro, rM, rz = oracle.infini_attn_fwd(q, k, v, beta, M0, z0, N=W.N, rule="linear")
     # the oracle takes its initial memory in fp32, so rank 1's prefix is rounded to fp32 once
-    got = np.concatenate([results[0][0], results[1][0]], axis=2)
+    got = np.concatenate([results[r][0] for r in range(world)], axis=2)
     np.testing.assert_allclose(got, ro, rtol=1e-6, atol=1e-9)
     for r in range(world):          # every rank ends with the memory after the whole sequence
         np.testing.assert_allclose(results[r][1], rM, rtol=1e-6, atol=1e-9)
         np.testing.assert_allclose(results[r][2], rz, rtol=1e-6, atol=1e-9)
     assert results["boundary"] == "rejected"
-    assert results["delta0"] == results["delta1"] == "rejected"
+    assert all(results[f"delta{r}"] == "rejected" for r in range(world))
