@@ -8,7 +8,8 @@ The arithmetic lives in ``infini_oracle.c`` (plain loops, one thread, double
 precision), written from AI Wiki "Infini-Attention", sections "What happens inside the
 Infini-attention block?" and "How does the compressive memory work?".  Its pins (the
 checks that tie it to the pages and to mathematics rather than to itself) are in
-``tests/test_oracle_pins.py``.
+``tests/test_oracle_pins.py``.  ``backward.py`` holds fp64 reference gradients of the same
+forward (for a backward pass not built yet), pinned in ``tests/test_backward_oracle_pins.py``.
 """
 from __future__ import annotations
 
