@@ -48,7 +48,7 @@ from compressive_memory_long_b200 import workloads as wl  # noqa: E402
 
 METRIC = "Infini-attention fwd tokens/s at 1 B200; % of bf16 TC peak or HBM roofline"
 DECODE_METRIC = "Infini-attention decode tokens/s at 1 B200 (one token per call, per sequence)"
-DEFAULT_WORKLOAD = "hf_repro_n64"
+DEFAULT_WORKLOAD = "stream1m_n2048_delta"
 FLUSH_BYTES = 256 << 20
 
 # Measured roofline denominators of this GPU pool (measured copy bandwidth and
@@ -85,8 +85,9 @@ def algorithmic(w: wl.Workload, kernel: str):
 
     segment kernel: local causal attention 2 d N (N + 1) + retrieval 2 N d^2 flops per
     (b, h, segment); bytes = q, k, v read once and out written once.
-    state kernels: update 2 N d^2 (linear) or 4 N d^2 (delta) flops per (b, kv head,
-    segment); bytes = k, v read once plus M/z read and written once.
+    memory increments (and the CUDA-core state kernels): update 2 N d^2 (linear) or 4 N d^2
+    (delta) flops per (b, kv head, segment); bytes = k, v read once plus M/z read and written
+    once.  The z sums, the prefix and the recurrence over the increments: state bytes only.
     """
     e = w.elem_bytes
     B, H, Hkv, L, N, d, S = w.B, w.H, w.Hkv, w.L, w.N, w.d, w.S
@@ -104,7 +105,7 @@ def algorithmic(w: wl.Workload, kernel: str):
     if kernel.startswith("segment"):
         flops = B * H * S * (2 * d * N * (N + 1) + 2 * N * d * d)
         byts = (2 * H + 2 * Hkv) * B * L * d * e
-    elif kernel.startswith(("linear_increments", "linear_state", "delta_chain")):
+    elif kernel.startswith(("linear_increments", "linear_state", "delta_chain", "mem_increments")):
         per = 2 if w.rule == "linear" else 4
         flops = B * Hkv * S * per * N * d * d
         byts = 2 * B * Hkv * L * d * e + state_bytes

@@ -48,6 +48,9 @@ SIGNATURES = {
     "infini_attn_version": ([], _I),
     "infini_attn_device_status": ([_P], _I),
     "infini_attn_trace_enable": ([_I], _I),
+    "infini_attn_test_fail_allocations": ([_I], _I),
+    "infini_attn_test_wait_limit": ([_I64], _I),
+    "infini_attn_test_withhold_publish": ([_I], _I),
     "infini_attn_trace_report": ([ctypes.c_char_p, _I64], _I64),
 }
 
@@ -88,6 +91,21 @@ def infini_attn_workspace_bytes(B, Hkv, L, N, d) -> int:
 def infini_attn_device_status(stream=None) -> int:
     """Synchronise the stream; INFINI_ERR_TIMEOUT (5) if a bounded device wait gave up."""
     return LIB.infini_attn_device_status(_stream_handle(stream))
+
+
+def infini_attn_test_fail_allocations(n: int) -> int:
+    """Test hook: the next ``n`` workspace allocations fail (INFINI_ERR_OOM)."""
+    return LIB.infini_attn_test_fail_allocations(int(n))
+
+
+def infini_attn_test_wait_limit(cycles: int) -> int:
+    """Test hook: bound of every device wait in SM cycles (<= 0 restores the default)."""
+    return LIB.infini_attn_test_wait_limit(int(cycles))
+
+
+def infini_attn_test_withhold_publish(on: bool) -> int:
+    """Test hook: the fused 64-token kernel's first unit per head skips its publish."""
+    return LIB.infini_attn_test_withhold_publish(1 if on else 0)
 
 
 def infini_attn_trace_enable(on: bool) -> bool:

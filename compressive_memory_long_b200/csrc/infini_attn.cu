@@ -17,8 +17,7 @@
 #include "simt_kernels.cuh"
 #include "tc_segment.cuh"
 #include "tc_segment2.cuh"
-#include "tc_delta.cuh"
-#include "tc_linear.cuh"
+#include "tc_memory.cuh"
 #include "tc_small.cuh"
 #include "tc_pieces.cuh"
 #include "decode.cuh"
@@ -219,54 +218,6 @@ bool make_map_bf16_3d(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D>
-int launch_linear_state_tc(const Problem &p, const __nv_bfloat16 *k, const __nv_bfloat16 *v,
-                           const float *M0, const float *z0, float *snapZ, __nv_bfloat16 *snapMb,
-                           float *M_out, float *z_out, cudaStream_t st)
-{
-    using C = tc::LinCfg<D>;
-    CUtensorMap mk, mv;
-    if (!make_map_bf16_3d(&mk, k, D, p.L, p.B * p.Hkv, 128) ||
-        !make_map_bf16_3d(&mv, v, D, p.L, p.B * p.Hkv, 128))
-        return INFINI_ERR_CUDA;
-    if (!opt_in_smem<tc::k_linear_state_tc<D>>(C::ALLOC)) return INFINI_ERR_CUDA;
-    tc::LinArgs a{M0, z0, snapZ, snapMb, M_out, z_out, (int)p.N, (int)p.S, p.L};
-    TRACED("linear_state_tc", st);
-    tc::k_linear_state_tc<D><<<(unsigned)(p.B * p.Hkv), 256, C::ALLOC, st>>>(mk, mv, a);
-    return INFINI_OK;
-}
-
-template <int D>
-int launch_delta_chain_tc(const Problem &p, const __nv_bfloat16 *k, const __nv_bfloat16 *v,
-                          const float *snapM, float *snapZ, __nv_bfloat16 *snapMb, float *M_out,
-                          float *z_out, cudaStream_t st)
-{
-    using C = tc::ChainCfg;
-    // sigma(K) once per token, into the workspace after the bf16 snapshots
-    __nv_bfloat16 *sk = snapMb + p.B * p.Hkv * p.S * (int64_t)D * D;
-    const int64_t n8 = p.B * p.Hkv * p.L * (int64_t)D / 8;   // every row, the tail's too
-    {
-        int sms = 148;
-        int dev = 0;
-        if (cudaGetDevice(&dev) == cudaSuccess)
-            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        const int64_t want = (n8 + 255) / 256;
-        const unsigned grid = (unsigned)(want < (int64_t)sms * 16 ? want : (int64_t)sms * 16);
-        TRACED("sigma_keys", st);
-        tc::k_sigma_bf16<<<grid, 256, 0, st>>>(k, sk, n8);
-    }
-    CUtensorMap mk, mv;
-    if (!make_map_bf16_3d(&mk, sk, D, p.L, p.B * p.Hkv, 128) ||
-        !make_map_bf16_3d(&mv, v, D, p.L, p.B * p.Hkv, 128, C::CB, false))
-        return INFINI_ERR_CUDA;
-    if (!opt_in_smem<tc::k_delta_chain_tc<D>>(C::ALLOC)) return INFINI_ERR_CUDA;
-    tc::ChainArgs a{snapM, snapZ, snapZ, snapMb, M_out, z_out, (int)p.N, (int)p.S};
-    const int64_t ctas = p.B * p.Hkv * (D / C::CB);
-    TRACED("delta_chain_tc", st);
-    tc::k_delta_chain_tc<D><<<(unsigned)ctas, 256, C::ALLOC, st>>>(mk, mv, a);
-    return INFINI_OK;
-}
-
 // The tensor-core segment kernel covers bf16 activations, d in {64, 128}, N % 128 == 0.
 template <typename T>
 bool use_tc(const Problem &p)
@@ -285,18 +236,105 @@ bool use_small_fused(const Problem &p)
 // Long heads (16 units of 128 tokens or more) go to the persistent piece kernel.
 bool use_pieces(const Problem &p) { return p.Lf / 128 >= 16; }
 
-// Workspace of one call: fp32 snapshots (M, z) for every segment, bf16 copies of M for the
-// tensor-core kernels, and room for the fused path's flags; an upper bound for every path.
-// Layout: [fp32 snapshots M | z][bf16 copies of M][sigma(K) in bf16][flags of the fused path].
-// A final short segment counts as a segment here (the tensor-core path gives it a snapshot
-// slot); the sigma(K) copy spans every row.
-int64_t workspace_bytes(int64_t B, int64_t Hkv, int64_t L, int64_t N, int64_t d)
+// Workspace of one call.  CUDA-core path: fp32 snapshots (M_{s-1}, z_{s-1}) of every
+// segment.  Tensor-core path: z_{s-1} and dz_s (fp32), the bf16 snapshots M_{s-1} the
+// segment kernel reads, the increments B_s (fp32) and, for the delta rule, A_s in two bf16
+// parts.  A final short segment counts as a segment.  The fused 64-token paths size their
+// own (much smaller) workspace.
+int64_t simt_workspace_bytes(int64_t units, int64_t d) { return units * (d * d + d) * 4 + 256; }
+
+int64_t tc_workspace_bytes(int64_t units, int64_t d, bool delta)
 {
-    const int64_t S = (L + N - 1) / N, units = B * Hkv * S;
-    return units * (d * d + d) * 4 + units * d * d * 2 + B * Hkv * L * d * 2 + units * 4 +
-           B * Hkv * 4 + units * 16 + 512;
+    return units * (2 * d * 4 + d * d * 2 + d * d * 4 + (delta ? 2 * d * d * 2 : 0)) + 256;
 }
 
+// An upper bound over every path (the exported figure).
+int64_t workspace_bytes(int64_t B, int64_t Hkv, int64_t L, int64_t N, int64_t d)
+{
+    const int64_t units = B * Hkv * ((L + N - 1) / N);
+    return std::max(simt_workspace_bytes(units, d), tc_workspace_bytes(units, d, true));
+}
+
+// Pointers into one call's workspace.
+struct Workspace {
+    void *raw = nullptr;
+    float *snapM = nullptr, *snapZ = nullptr;          // CUDA-core path
+    float *dz = nullptr, *Bs = nullptr;                // tensor-core path (+ snapZ)
+    __nv_bfloat16 *snapMb = nullptr, *Ahi = nullptr, *Alo = nullptr;
+};
+
+Workspace carve_workspace(void *raw, int64_t units, int64_t d, bool tc_path)
+{
+    Workspace w;
+    w.raw = raw;
+    if (!raw) return w;
+    char *c = static_cast<char *>(raw);
+    if (!tc_path) {
+        w.snapM = reinterpret_cast<float *>(c);
+        w.snapZ = w.snapM + units * d * d;
+        return w;
+    }
+    w.snapZ = reinterpret_cast<float *>(c);
+    w.dz = w.snapZ + units * d;
+    w.Bs = w.dz + units * d;
+    w.snapMb = reinterpret_cast<__nv_bfloat16 *>(w.Bs + units * d * d);
+    w.Ahi = w.snapMb + units * d * d;
+    w.Alo = w.Ahi + units * d * d;
+    return w;
+}
+
+// The memory path of the tensor-core forward: z prefix, per-segment increments on the
+// tensor cores, then the recurrence (delta) or the running sum (linear).  Leaves the
+// snapshots (z_{s-1} fp32, M_{s-1} bf16) for the segment kernel, and M_out / z_out.
+template <int D>
+int launch_memory_tc(const Problem &p, const __nv_bfloat16 *k, const __nv_bfloat16 *v,
+                     const float *M0, const float *z0, const Workspace &ws, float *M_out,
+                     float *z_out, cudaStream_t st)
+{
+    const int64_t chains = p.B * p.Hkv, units = chains * p.S;
+    const int S = (int)p.S, N = (int)p.N;
+    const bool delta = p.rule == INFINI_UPDATE_DELTA;
+    {
+        TRACED("z_sum", st);
+        tc::k_zsum<D><<<(unsigned)units, 256, 0, st>>>(k, ws.dz, p.L, N, S);
+    }
+    {
+        TRACED("z_scan", st);
+        tc::k_zscan<D><<<(unsigned)chains, D * 8, 0, st>>>(ws.dz, z0, ws.snapZ, z_out, S);
+    }
+    CUtensorMap mk, mv;
+    if (!make_map_bf16_3d(&mk, k, D, p.L, chains, 64) || !make_map_bf16_3d(&mv, v, D, p.L, chains, 64))
+        return INFINI_ERR_CUDA;
+    tc::IncrArgs ia{ws.snapZ, ws.Bs, ws.Ahi, ws.Alo, p.L, N, S};
+    if (delta) {
+        using C = tc::IncrCfg<D, true>;
+        if (!opt_in_smem<tc::k_mem_incr<D, true>>(C::ALLOC)) return INFINI_ERR_CUDA;
+        TRACED("mem_increments", st);
+        tc::k_mem_incr<D, true><<<(unsigned)units, C::THREADS, C::ALLOC, st>>>(mk, mv, ia);
+    } else {
+        using C = tc::IncrCfg<D, false>;
+        if (!opt_in_smem<tc::k_mem_incr<D, false>>(C::ALLOC)) return INFINI_ERR_CUDA;
+        TRACED("mem_increments", st);
+        tc::k_mem_incr<D, false><<<(unsigned)units, C::THREADS, C::ALLOC, st>>>(mk, mv, ia);
+    }
+    if (!delta) {
+        const int64_t n4 = chains * D * D / 4;
+        TRACED("mem_prefix", st);
+        tc::k_mem_prefix<D><<<(unsigned)((n4 + 255) / 256), 256, 0, st>>>(ws.Bs, M0, ws.snapMb,
+                                                                          M_out, S, chains);
+        return INFINI_OK;
+    }
+    using MC = tc::MChainCfg<D>;
+    CUtensorMap mah, mal;
+    if (!make_map_bf16_3d(&mah, ws.Ahi, D, D, units, D) ||
+        !make_map_bf16_3d(&mal, ws.Alo, D, D, units, D))
+        return INFINI_ERR_CUDA;
+    if (!opt_in_smem<tc::k_mem_chain<D>>(MC::ALLOC)) return INFINI_ERR_CUDA;
+    tc::MChainArgs ca{M0, ws.Bs, ws.snapMb, M_out, S};
+    TRACED("mem_chain", st);
+    tc::k_mem_chain<D><<<(unsigned)(chains * (D / MC::CB)), 256, MC::ALLOC, st>>>(mah, mal, ca);
+    return INFINI_OK;
+}
 
 // The two-tile kernel redistributes registers with setmaxnreg; its split assumes the
 // register count per thread it was compiled with.  Checked once per kernel: a mismatch
@@ -455,15 +493,25 @@ int launch_pieces(const Problem &p, const __nv_bfloat16 *q, const __nv_bfloat16 
 template <typename T, int D>
 int launch_all(const Problem &p, const T *q, const T *k, const T *v, const float *beta,
                const float *M0, const float *z0, T *out, float *M_out, float *z_out,
-               float *snapM, float *snapZ, __nv_bfloat16 *snapMb, cudaStream_t st,
-               bool outputs = true)
+               const Workspace &ws, cudaStream_t st, bool outputs = true)
 {
     if constexpr (sizeof(T) == 2 && D == 64) {
         if (outputs && use_small_fused<T>(p)) {
             const int rc = use_pieces(p)
-                ? launch_pieces(p, q, k, v, beta, M0, z0, out, M_out, z_out, snapM, st)
-                : launch_small_fused(p, q, k, v, beta, M0, z0, out, M_out, z_out, snapM, st);
+                ? launch_pieces(p, q, k, v, beta, M0, z0, out, M_out, z_out, ws.raw, st)
+                : launch_small_fused(p, q, k, v, beta, M0, z0, out, M_out, z_out, ws.raw, st);
             if (rc != INFINI_OK) return rc;
+            return cudaGetLastError() == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
+        }
+    }
+    if constexpr (sizeof(T) == 2 && (D == 64 || D == 128)) {
+        if (ws.snapMb) {       // the tensor-core path
+            int rc = launch_memory_tc<D>(p, k, v, M0, z0, ws, M_out, z_out, st);
+            if (rc != INFINI_OK) return rc;
+            if (outputs) {
+                rc = launch_segment_tc<D>(p, q, k, v, beta, ws.snapMb, ws.snapZ, out, st);
+                if (rc != INFINI_OK) return rc;
+            }
             return cudaGetLastError() == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
         }
     }
@@ -471,16 +519,8 @@ int launch_all(const Problem &p, const T *q, const T *k, const T *v, const float
     const int S = (int)p.S, N = (int)p.N;
     const int64_t per = (int64_t)D * D + D;
     const unsigned state_grid = (unsigned)((chains * per + 255) / 256);
-    bool linear_tc = false;
-    if constexpr (sizeof(T) == 2 && (D == 64 || D == 128)) {
-        if (p.rule == INFINI_UPDATE_LINEAR && snapMb) {
-            const int rc = launch_linear_state_tc<D>(p, k, v, M0, z0, snapZ, snapMb, M_out, z_out, st);
-            if (rc != INFINI_OK) return rc;
-            linear_tc = true;
-        }
-    }
-    if (linear_tc) {
-    } else if (p.rule == INFINI_UPDATE_LINEAR) {
+    float *snapM = ws.snapM, *snapZ = ws.snapZ;
+    if (p.rule == INFINI_UPDATE_LINEAR) {
         {
             TRACED("linear_increments", st);
             k_linear_increments<T, D><<<(unsigned)(chains * S), 256, 0, st>>>(k, v, snapM, snapZ,
@@ -488,38 +528,20 @@ int launch_all(const Problem &p, const T *q, const T *k, const T *v, const float
         }
         {
             TRACED("linear_scan", st);
-            k_linear_scan<<<state_grid, 256, 0, st>>>(snapM, snapZ, snapMb, M0, z0, M_out, z_out,
+            k_linear_scan<<<state_grid, 256, 0, st>>>(snapM, snapZ, nullptr, M0, z0, M_out, z_out,
                                                       S, D, chains);
         }
     } else {
         constexpr int CB = 16;
         {
             TRACED("state_init", st);
-            k_state_init<<<state_grid, 256, 0, st>>>(M0, z0, snapM, snapZ, snapMb, S, D, chains);
+            k_state_init<<<state_grid, 256, 0, st>>>(M0, z0, snapM, snapZ, nullptr, S, D, chains);
         }
-        bool done = false;
-        if constexpr (sizeof(T) == 2 && (D == 64 || D == 128)) {
-            if (snapMb) {
-                const int rc = launch_delta_chain_tc<D>(p, k, v, snapM, snapZ, snapMb, M_out,
-                                                        z_out, st);
-                if (rc != INFINI_OK) return rc;
-                done = true;
-            }
-        }
-        if (!done) {
-            TRACED("delta_chain", st);
-            k_delta_chain<T, D, CB><<<(unsigned)(chains * (D / CB)), 256, 0, st>>>(
-                k, v, snapM, snapZ, snapMb, M_out, z_out, p.L, N, S, N);
-        }
+        TRACED("delta_chain", st);
+        k_delta_chain<T, D, CB><<<(unsigned)(chains * (D / CB)), 256, 0, st>>>(
+            k, v, snapM, snapZ, nullptr, M_out, z_out, p.L, N, S, N);
     }
     if (!outputs) return cudaGetLastError() == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
-    if constexpr (sizeof(T) == 2 && (D == 64 || D == 128)) {
-        if (snapMb) {
-            const int rc = launch_segment_tc<D>(p, q, k, v, beta, snapMb, snapZ, out, st);
-            if (rc != INFINI_OK) return rc;
-            return cudaGetLastError() == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
-        }
-    }
     const size_t smem = SimtSegSmem<D>::bytes;
     if (!opt_in_smem<k_segment_simt<T, D>>(smem)) return INFINI_ERR_CUDA;
     const int64_t ctas = p.B * p.H * p.S * (p.N / 64);
@@ -612,15 +634,55 @@ Problem effective(const Problem &p)
 template <typename T, int D>
 int launch_forward(const Problem &p, const T *q, const T *k, const T *v, const float *beta,
                    const float *M0, const float *z0, T *out, float *M_out, float *z_out,
-                   float *snapM, float *snapZ, __nv_bfloat16 *snapMb, cudaStream_t st,
-                   bool outputs = true)
+                   const Workspace &ws, cudaStream_t st, bool outputs = true)
 {
     if (p.S > 0) {
-        const int rc = launch_all<T, D>(p, q, k, v, beta, M0, z0, out, M_out, z_out, snapM, snapZ,
-                                        snapMb, st, outputs);
+        const int rc = launch_all<T, D>(p, q, k, v, beta, M0, z0, out, M_out, z_out, ws, st,
+                                        outputs);
         if (rc != INFINI_OK || p.T == 0) return rc;
     }
     return launch_tail<T, D>(p, q, k, v, beta, M0, z0, out, M_out, z_out, st, outputs);
+}
+
+// Workspace the chosen path of one forward call needs (p as returned by effective()): the
+// fused 64-token paths need far less than the general upper bound workspace_bytes().
+template <typename T>
+int64_t call_workspace_bytes(const Problem &p)
+{
+    if (p.S == 0) return 0;
+    if (use_small_fused<T>(p)) return use_pieces(p) ? pieces_workspace_bytes(p) : small_workspace_bytes(p);
+    const int64_t units = p.B * p.Hkv * p.S;
+    return use_tc<T>(p) ? tc_workspace_bytes(units, p.d, p.rule == INFINI_UPDATE_DELTA)
+                        : simt_workspace_bytes(units, p.d);
+}
+
+// Enqueue the forward (or, with outputs = false, the memory chain alone) on a workspace.
+template <typename T>
+int dispatch(const Problem &p, const void *q, const void *k, const void *v, const float *beta,
+             const float *M0, const float *z0, void *out, float *M_out, float *z_out, void *raw,
+             cudaStream_t st, bool outputs = true)
+{
+    const Workspace ws = carve_workspace(raw, p.B * p.Hkv * p.S, p.d, use_tc<T>(p));
+    const T *tq = static_cast<const T *>(q), *tk = static_cast<const T *>(k),
+            *tv = static_cast<const T *>(v);
+    T *to = static_cast<T *>(out);
+    switch (p.d) {
+    case 32: return launch_forward<T, 32>(p, tq, tk, tv, beta, M0, z0, to, M_out, z_out, ws, st, outputs);
+    case 64: return launch_forward<T, 64>(p, tq, tk, tv, beta, M0, z0, to, M_out, z_out, ws, st, outputs);
+    default: return launch_forward<T, 128>(p, tq, tk, tv, beta, M0, z0, to, M_out, z_out, ws, st, outputs);
+    }
+}
+
+// Test hook (infini_attn_test_fail_allocations): the next n workspace allocations fail as
+// if the device were out of memory.
+std::atomic<int> g_fail_allocs{0};
+
+bool take_failed_allocation()
+{
+    int n = g_fail_allocs.load();
+    while (n > 0)
+        if (g_fail_allocs.compare_exchange_weak(n, n - 1)) return true;
+    return false;
 }
 
 // The library's own stream-ordered pool on the current device.  Its release threshold keeps
@@ -665,15 +727,10 @@ int forward(const void *q, const void *k, const void *v, const float *beta, cons
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     cudaGetLastError();   // clear a stale error left by someone else's launch
 
-    const int64_t nM = p.B * p.Hkv * p.S * p.d * p.d, nZ = p.B * p.Hkv * p.S * p.d;
-    const bool tc_path = use_tc<T>(p);
-    // the fused 64-token paths need far less than the general upper bound
-    const int64_t bytes = p.S == 0                ? 0
-                          : !use_small_fused<T>(p) ? workspace_bytes(p.B, p.Hkv, p.L, p.N, p.d)
-                          : use_pieces(p)          ? pieces_workspace_bytes(p)
-                                                   : small_workspace_bytes(p);
+    const int64_t bytes = call_workspace_bytes<T>(p);
     void *ws = nullptr;
     if (bytes > 0) {
+        if (take_failed_allocation()) return INFINI_ERR_OOM;
         cudaMemPool_t pool = workspace_pool();
         if (!pool) return INFINI_ERR_CUDA;
         if (cudaMallocFromPoolAsync(&ws, (size_t)bytes, pool, st) != cudaSuccess) {
@@ -681,16 +738,7 @@ int forward(const void *q, const void *k, const void *v, const float *beta, cons
             return INFINI_ERR_OOM;
         }
     }
-    float *snapM = static_cast<float *>(ws), *snapZ = snapM + nM;
-    __nv_bfloat16 *snapMb = tc_path ? reinterpret_cast<__nv_bfloat16 *>(snapZ + nZ) : nullptr;
-    const T *tq = static_cast<const T *>(q), *tk = static_cast<const T *>(k),
-            *tv = static_cast<const T *>(v);
-    T *to = static_cast<T *>(out);
-    switch (p.d) {
-    case 32: rc = launch_forward<T, 32>(p, tq, tk, tv, beta, M0, z0, to, M_out, z_out, snapM, snapZ, snapMb, st); break;
-    case 64: rc = launch_forward<T, 64>(p, tq, tk, tv, beta, M0, z0, to, M_out, z_out, snapM, snapZ, snapMb, st); break;
-    default: rc = launch_forward<T, 128>(p, tq, tk, tv, beta, M0, z0, to, M_out, z_out, snapM, snapZ, snapMb, st); break;
-    }
+    rc = dispatch<T>(p, q, k, v, beta, M0, z0, out, M_out, z_out, ws, st);
     if (ws && cudaFreeAsync(ws, st) != cudaSuccess && rc == INFINI_OK) rc = INFINI_ERR_CUDA;
     return rc;
 }
@@ -730,26 +778,18 @@ int forward_noalloc(const void *q, const void *k, const void *v, const float *be
                         (int64_t)sizeof(T), &p);
     if (rc != INFINI_OK) return rc;
     p = effective<T>(p);
-    const int64_t nM = p.B * p.Hkv * p.S * p.d * p.d, nZ = p.B * p.Hkv * p.S * p.d;
-    const bool tc_path = use_tc<T>(p);
-    const size_t bytes = (size_t)workspace_bytes(p.B, p.Hkv, p.L, p.N, p.d);
+    // admitted by what the chosen path needs (the fused 64-token paths need far less than the
+    // general bound infini_attn_workspace_bytes reports)
+    const size_t bytes = (size_t)call_workspace_bytes<T>(p);
     if (bytes > kNoAllocScratchBytes) return INFINI_ERR_UNSUPPORTED;
     void *ws = noalloc_scratch_address();
     if (!ws) return INFINI_ERR_CUDA;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     cudaGetLastError();
-    // Nothing in the array needs to start at zero: every snapshot slot a kernel reads was
-    // written earlier in the same call (increments / initial state, then the scan or chain).
-    float *snapM = static_cast<float *>(ws), *snapZ = snapM + nM;
-    T *snapMb = tc_path ? reinterpret_cast<T *>(snapZ + nZ) : nullptr;
-    const T *tq = static_cast<const T *>(q), *tk = static_cast<const T *>(k),
-            *tv = static_cast<const T *>(v);
-    T *to = static_cast<T *>(out);
-    switch (p.d) {
-    case 32: return launch_forward<T, 32>(p, tq, tk, tv, beta, M0, z0, to, M_out, z_out, snapM, snapZ, snapMb, st);
-    case 64: return launch_forward<T, 64>(p, tq, tk, tv, beta, M0, z0, to, M_out, z_out, snapM, snapZ, snapMb, st);
-    default: return launch_forward<T, 128>(p, tq, tk, tv, beta, M0, z0, to, M_out, z_out, snapM, snapZ, snapMb, st);
-    }
+    // Nothing in the array has to hold anything on entry: every snapshot slot a kernel reads
+    // was written earlier in the same call (increments / initial state, then the scan or
+    // chain), and the fused 64-token paths clear their tickets and flags first.
+    return dispatch<T>(p, q, k, v, beta, M0, z0, out, M_out, z_out, ws, st);
 }
 
 // ---- the memory chain alone -----------------------------------------------------------------
@@ -779,11 +819,13 @@ int state_only(const void *k, const void *v, const float *M0, const float *z0, f
     p = effective<T>(p);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     cudaGetLastError();
-    const int64_t nM = p.B * p.Hkv * p.S * p.d * p.d, nZ = p.B * p.Hkv * p.S * p.d;
-    const bool tc_path = use_tc<T>(p);
-    const int64_t bytes = p.S == 0 ? 0 : workspace_bytes(p.B, p.Hkv, p.L, p.N, p.d);
+    const int64_t units = p.B * p.Hkv * p.S;
+    const int64_t bytes = p.S == 0 ? 0
+                          : use_tc<T>(p) ? tc_workspace_bytes(units, p.d, p.rule == INFINI_UPDATE_DELTA)
+                                         : simt_workspace_bytes(units, p.d);
     void *ws = nullptr;
     if (bytes > 0) {
+        if (take_failed_allocation()) return INFINI_ERR_OOM;
         cudaMemPool_t pool = workspace_pool();
         if (!pool) return INFINI_ERR_CUDA;
         if (cudaMallocFromPoolAsync(&ws, (size_t)bytes, pool, st) != cudaSuccess) {
@@ -791,14 +833,7 @@ int state_only(const void *k, const void *v, const float *M0, const float *z0, f
             return INFINI_ERR_OOM;
         }
     }
-    float *snapM = static_cast<float *>(ws), *snapZ = snapM + nM;
-    __nv_bfloat16 *snapMb = tc_path ? reinterpret_cast<__nv_bfloat16 *>(snapZ + nZ) : nullptr;
-    const T *tk = static_cast<const T *>(k), *tv = static_cast<const T *>(v);
-    switch (p.d) {
-    case 32: rc = launch_forward<T, 32>(p, tk, tk, tv, nullptr, M0, z0, nullptr, M_out, z_out, snapM, snapZ, snapMb, st, false); break;
-    case 64: rc = launch_forward<T, 64>(p, tk, tk, tv, nullptr, M0, z0, nullptr, M_out, z_out, snapM, snapZ, snapMb, st, false); break;
-    default: rc = launch_forward<T, 128>(p, tk, tk, tv, nullptr, M0, z0, nullptr, M_out, z_out, snapM, snapZ, snapMb, st, false); break;
-    }
+    rc = dispatch<T>(p, k, k, v, nullptr, M0, z0, nullptr, M_out, z_out, ws, st, false);
     if (ws && cudaFreeAsync(ws, st) != cudaSuccess && rc == INFINI_OK) rc = INFINI_ERR_CUDA;
     return rc;
 }
@@ -1048,6 +1083,27 @@ int infini_attn_device_status(infini_stream_t stream)
     const int zero = 0;
     cudaMemcpyToSymbol(infini::tc::g_wait_status, &zero, sizeof(int));
     return INFINI_ERR_TIMEOUT;
+}
+
+int infini_attn_test_fail_allocations(int n)
+{
+    if (n < 0) return INFINI_ERR_INVALID_ARG;
+    infini::g_fail_allocs.store(n);
+    return INFINI_OK;
+}
+
+int infini_attn_test_wait_limit(int64_t cycles)
+{
+    const long long v = cycles > 0 ? (long long)cycles : infini::tc::kSpinLimitCycles;
+    return cudaMemcpyToSymbol(infini::tc::g_spin_limit, &v, sizeof(v)) == cudaSuccess
+        ? INFINI_OK : INFINI_ERR_CUDA;
+}
+
+int infini_attn_test_withhold_publish(int on)
+{
+    const int v = on ? 1 : 0;
+    return cudaMemcpyToSymbol(infini::tc::g_test_withhold, &v, sizeof(v)) == cudaSuccess
+        ? INFINI_OK : INFINI_ERR_CUDA;
 }
 
 int infini_attn_trace_enable(int on)

@@ -29,6 +29,17 @@ __device__ int g_wait_status;
 // About 0.5 s at the B200's top SM clock: far above any legitimate wait in these kernels.
 constexpr long long kSpinLimitCycles = 1000000000LL;
 
+// The bound every wait applies, in SM clock cycles.  Only a test hook lowers it
+// (infini_attn_test_wait_limit), to make a withheld publish time out quickly.
+__device__ long long g_spin_limit = kSpinLimitCycles;
+
+__device__ __forceinline__ long long spin_limit() { return g_spin_limit; }
+
+// Test hook (infini_attn_test_withhold_publish): when nonzero, the first unit of every head
+// in the fused 64-token kernel publishes nothing, so the bounded waits of the units after it
+// run out and report INFINI_ERR_TIMEOUT.
+__device__ int g_test_withhold;
+
 // The status word is sticky: once a wait anywhere has given up, every other CTA stops
 // waiting and later launches return at once, until the host reads and clears it.
 __device__ __forceinline__ bool wait_status_set()
@@ -102,7 +113,7 @@ __device__ __forceinline__ bool mbar_wait_short(uint64_t *bar, uint32_t parity, 
     const long long t0 = clock64();
     uint32_t n = 0;
     while (!mbar_try_wait_short(bar, parity)) {
-        if (*abort || clock64() - t0 > kSpinLimitCycles || ((++n & 1023) == 0 && wait_status_set())) {
+        if (*abort || clock64() - t0 > spin_limit() || ((++n & 1023) == 0 && wait_status_set())) {
             atomicCAS(&g_wait_status, 0, where);
             *abort = 1;
             return false;
@@ -111,7 +122,7 @@ __device__ __forceinline__ bool mbar_wait_short(uint64_t *bar, uint32_t parity, 
     return true;
 }
 
-// Wait for the phase with the given parity to complete.  Gives up after kSpinLimitCycles
+// Wait for the phase with the given parity to complete.  Gives up after spin_limit() cycles
 // (or at once if *abort is already set), records `where` in g_wait_status, sets *abort so
 // every other role of the CTA stops waiting too, and returns false.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
@@ -121,7 +132,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
     const long long t0 = clock64();
     uint32_t n = 0;
     while (!mbar_try_wait(bar, parity)) {
-        if (*abort || clock64() - t0 > kSpinLimitCycles || ((++n & 1023) == 0 && wait_status_set())) {
+        if (*abort || clock64() - t0 > spin_limit() || ((++n & 1023) == 0 && wait_status_set())) {
             atomicCAS(&g_wait_status, 0, where);
             *abort = 1;
             return false;

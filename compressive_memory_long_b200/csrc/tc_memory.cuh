@@ -1,0 +1,638 @@
+// The memory chain of both update rules, split into a parallel part and a short serial
+// part (sm_100a).
+//
+// AI Wiki "Infini-Attention", "How does the compressive memory work?":
+//   linear: M_s = M_{s-1} + sigma(K_s)^T V_s
+//   delta : M_s = M_{s-1} + sigma(K_s)^T (V_s - sigma(K_s) M_{s-1} / den),
+//           den_t = sigma(k_t) . z_{s-1}   (a row whose den is 0 predicts 0)
+//   both  : z_s = z_{s-1} + sum_t sigma(k_t)
+// The delta update is linear in M_{s-1}, and den needs only z_{s-1}, which never depends
+// on M:
+//   M_s = M_{s-1} + B_s - A_s M_{s-1},
+//   B_s = sigma(K_s)^T V_s,   A_s = sigma(K_s)^T diag(1/den) sigma(K_s)   (d x d each).
+// So the contractions over a segment's N tokens leave the serial path:
+//   k_zsum      per (chain, segment): dz_s = sum_t sigma(k_t), fp32 on the CUDA cores
+//   k_zscan     per chain: z_{s-1} for every segment (what the segment kernel and den read)
+//   k_mem_incr  per (chain, segment), all at once, on the tensor cores: B_s and (delta) A_s
+//   k_mem_chain delta: per (chain, 32 value columns), the recurrence in segment order, one
+//               d x d x 32 product per segment on the tensor cores
+//   k_mem_prefix linear: the running sum M0 + sum_{j<s} B_j, elementwise
+// The last two write the bf16 snapshots M_{s-1} the segment kernel reads, and M_out.
+//
+// Precision: sigma(K) enters the contractions as two bf16 parts, sigma_hi = bf16(sigma) and
+// sigma_lo = bf16(sigma - sigma_hi); with sigma ~ 1 a single bf16 rounding (2^-9) would
+// cost about 5e-3 of M over 32 segments of 2048 tokens, the split about 3e-6.  The products
+// are sigma_hi [V | W_hi] + sigma_lo [V | W_hi] + sigma_hi W_lo with W = diag(1/den) sigma
+// split the same way (sigma_lo W_lo is below the fp32 rounding of the sums).  In the chain
+// A_s and M_{s-1} are split too (three products).  z is summed in fp32 from sigma itself.
+// Rows of a short last segment past L carry sigma = 0 (not sigma(0) = 1): they add nothing.
+// All waits are bounded (tc_common.cuh).
+#pragma once
+
+#include "tc_common.cuh"
+
+namespace infini {
+namespace tc {
+
+// ---------------------------------------------------------------- z: column sums and prefix
+
+// dz[chain * S + s][f] = sum over the rows t < L of segment s of sigma(k_t[f]).  One CTA per
+// (chain, segment); thread (row lane, 8-feature chunk) reads 16-byte pieces of rows.
+template <int D>
+__global__ void __launch_bounds__(256)
+k_zsum(const __nv_bfloat16 *__restrict__ k, float *__restrict__ dz, int64_t L, int N, int S)
+{
+    constexpr int CHK = D / 8;              // 16-byte chunks per row
+    constexpr int RL = 256 / CHK;           // rows read side by side
+    __shared__ float part[RL][D];
+    const int64_t cs = blockIdx.x;
+    const int64_t chain = cs / S;
+    const int s = (int)(cs % S);
+    const int ch = threadIdx.x % CHK, rl = threadIdx.x / CHK;
+    const int64_t row0 = (int64_t)s * N;
+    const int rows = (int)(L - row0 < N ? L - row0 : N);
+    const uint4 *src = reinterpret_cast<const uint4 *>(k + (chain * L + row0) * D) + ch;
+    float acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+#pragma unroll 4
+    for (int r = rl; r < rows; r += RL) {
+        const uint4 v = __ldg(src + (int64_t)r * CHK);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const __nv_bfloat162 t = *reinterpret_cast<const __nv_bfloat162 *>(&w[e]);
+            acc[2 * e] += elu1(__low2float(t));
+            acc[2 * e + 1] += elu1(__high2float(t));
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) part[rl][ch * 8 + e] = acc[e];
+    __syncthreads();
+    for (int f = threadIdx.x; f < D; f += 256) {
+        float t = 0.f;
+        for (int j = 0; j < RL; ++j) t += part[j][f];
+        dz[cs * D + f] = t;
+    }
+}
+
+// snapZ[chain * S + s] = z_{s-1} = z0 + sum_{j<s} dz_j for every segment, z_out = z_S.
+// One CTA of 8 x D threads per chain: 8 groups of consecutive segments are summed side by
+// side, then each group walks its segments again from the prefix of the groups before it.
+// z0 is read before the first barrier, so z_out may alias it.
+template <int D>
+__global__ void __launch_bounds__(D * 8)
+k_zscan(const float *__restrict__ dz, const float *z0, float *__restrict__ snapZ, float *z_out,
+        int S)
+{
+    __shared__ float tot[8][D];
+    const int f = threadIdx.x % D, g = threadIdx.x / D;
+    const int64_t chain = blockIdx.x;
+    const int per = (S + 7) / 8;
+    const int s0 = g * per < S ? g * per : S, s1 = s0 + per < S ? s0 + per : S;
+    const float *src = dz + chain * S * D + f;
+    float t = 0.f;
+#pragma unroll 8
+    for (int s = s0; s < s1; ++s) t += src[(int64_t)s * D];
+    float z = z0 ? z0[chain * D + f] : 0.f;
+    tot[g][f] = t;
+    __syncthreads();
+    for (int j = 0; j < g; ++j) z += tot[j][f];
+    float *dst = snapZ + chain * S * D + f;
+    for (int s = s0; s < s1; ++s) {
+        dst[(int64_t)s * D] = z;
+        z += src[(int64_t)s * D];
+    }
+    if (g == 7) z_out[chain * D + f] = z;
+}
+
+// ---------------------------------------------------------------- per-segment increments
+
+template <int D, bool DELTA>
+struct IncrCfg {
+    static_assert(D == 64 || D == 128, "tensor-core memory increments: d = 64 or 128");
+    static constexpr int CH = 64;                    // tokens per chunk
+    static constexpr int NB = D / 64;                // 64-column boxes of V and of W
+    static constexpr int BOX = CH * 128;             // 64 rows x 64 bf16 (128-byte rows)
+    static constexpr int ATILE = 2 * BOX;            // sigma: features padded to 128
+    static constexpr int NBB = DELTA ? 3 * NB : NB;  // B boxes: V | W_hi | W_lo
+    static constexpr int OFF_SH = 0;                 // sigma_hi, written over the K tile
+    static constexpr int OFF_SL = ATILE;             // sigma_lo
+    static constexpr int OFF_B = 2 * ATILE;
+    static constexpr int STAGE = 2 * ATILE + NBB * BOX;
+    static constexpr int ST = 2;
+    static constexpr int OFF_Z = ST * STAGE;         // z_{s-1} (delta)
+    static constexpr int OFF_BAR = OFF_Z + 128 * 4;
+    static constexpr int NBAR = 3 * ST + 1;
+    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+    static constexpr int BYTES = OFF_MISC + 16;
+    static constexpr int ALLOC = BYTES + 1024;
+    static constexpr int NVW = DELTA ? 2 * D : D;    // N of the [V | W_hi] products
+    static constexpr uint32_t TMEM_COLS = NVW <= 64 ? 64 : (NVW <= 128 ? 128 : 256);
+    static constexpr int THREADS = 384;
+    static constexpr int FPT = D / 4;                // features per worker thread
+    static_assert(STAGE % 1024 == 0 && BOX % 1024 == 0, "operand tiles must be 1024-aligned");
+};
+
+struct IncrArgs {
+    const float *snapZ;        // [chains * S, D]: z_{s-1} (delta)
+    float *Bs;                 // [chains * S, D, D] fp32: sigma(K_s)^T V_s
+    __nv_bfloat16 *Ahi, *Alo;  // [chains * S, D, D]: A_s split into two bf16 parts (delta)
+    int64_t L;
+    int N, S;
+};
+
+enum : int { WI_KV_EMPTY = 501, WI_KV_FULL = 502, WI_A = 503, WI_ACC = 504, WI_DRAIN = 505 };
+
+__device__ __forceinline__ void incr_drain(uint64_t *bar, uint32_t parity)
+{
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity)) {
+        if (clock64() - t0 > spin_limit()) {
+            atomicCAS(&g_wait_status, 0, WI_DRAIN);
+            return;
+        }
+    }
+}
+
+// One CTA per (chain, segment).  Warp 0: TMA producer of 64-token K / V chunks (two stages).
+// Warp 1: MMA issuer.  Warps 4-11: four threads per token row turn the K tile into
+// sigma_hi / sigma_lo (in place / beside it) and, for the delta rule, write W = sigma / den
+// (hi, lo) beside V; after the last chunk they read the accumulators (lane i = key feature i)
+// and store row i of B_s (warps 4-7) and of A_s (warps 8-11).
+// TMEM: columns [0, D) accumulate B_s, [D, 2D) A_s.
+template <int D, bool DELTA>
+__global__ void __launch_bounds__(384, 1)
+k_mem_incr(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+           const IncrArgs a)
+{
+    using C = IncrCfg<D, DELTA>;
+    constexpr int ST = C::ST;
+    if (__syncthreads_or(threadIdx.x == 0 && wait_status_set())) return;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+
+    const int64_t cs = blockIdx.x;                 // chain * S + s
+    const int64_t chain = cs / a.S;
+    const int s = (int)(cs % a.S);
+    const int64_t row0 = (int64_t)s * a.N;
+    const int rows = (int)(a.L - row0 < a.N ? a.L - row0 : a.N);
+    const int nch = (rows + C::CH - 1) / C::CH;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    float *sZ = reinterpret_cast<float *>(smem + C::OFF_Z);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
+    uint64_t *kv_full = bars, *kv_empty = bars + ST, *a_ready = bars + 2 * ST;
+    uint64_t *acc_full = bars + 3 * ST;
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
+    volatile int *abort = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < ST; ++i) {
+            mbar_init(kv_full + i, 1);
+            mbar_init(kv_empty + i, 1);
+            mbar_init(a_ready + i, 256);
+        }
+        mbar_init(acc_full, 1);
+        *abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) tmem_alloc(tmem_holder, C::TMEM_COLS);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t T = *tmem_holder;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ------------------------------------------------------------ producer
+            prefetch_tmap(&tmK);
+            prefetch_tmap(&tmV);
+            int issued = 0;
+            for (int g = 0; g < nch; ++g) {
+                const int st = g % ST;
+                if (g >= ST && !mbar_wait_short(kv_empty + st, ((g / ST) - 1) & 1, abort, WI_KV_EMPTY))
+                    break;
+                uint8_t *stage = smem + st * C::STAGE;
+                const int row = (int)row0 + g * C::CH;
+                mbar_arrive_expect_tx(kv_full + st, (uint32_t)(2 * C::NB * C::BOX));
+                for (int b = 0; b < C::NB; ++b) {
+                    tma_load_3d(stage + C::OFF_SH + b * C::BOX, &tmK, kv_full + st, b * 64, row,
+                                (int)chain);
+                    tma_load_3d(stage + C::OFF_B + b * C::BOX, &tmV, kv_full + st, b * 64, row,
+                                (int)chain);
+                }
+                issued = g + 1;
+            }
+            if (*abort)
+                for (int g = (issued > ST ? issued - ST : 0); g < issued; ++g)
+                    incr_drain(kv_full + g % ST, (g / ST) & 1);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ------------------------------------------------------------ MMA issuer
+            constexpr uint32_t idVW = idesc_bf16(128, C::NVW, 1, 1);   // sigma^T [V | W_hi]
+            constexpr uint32_t idWl = idesc_bf16(128, D, 1, 1);        // sigma_hi^T W_lo
+            const uint32_t base = smem_u32(smem);
+            for (int g = 0; g < nch; ++g) {
+                const int st = g % ST;
+                if (!mbar_wait_short(a_ready + st, (g / ST) & 1, abort, WI_A)) break;
+                tc_fence_after();
+                const uint32_t sb = base + st * C::STAGE;
+#pragma unroll
+                for (int kk = 0; kk < C::CH / 16; ++kk) {       // 16 tokens per step
+                    const uint64_t ah = sdesc_sw128(sb + C::OFF_SH + kk * 2048, C::BOX, 1024);
+                    const uint64_t al = sdesc_sw128(sb + C::OFF_SL + kk * 2048, C::BOX, 1024);
+                    const uint64_t bvw = sdesc_sw128(sb + C::OFF_B + kk * 2048, C::BOX, 1024);
+                    mma_ss(T, ah, bvw, idVW, (g > 0 || kk > 0) ? 1u : 0u);
+                    mma_ss(T, al, bvw, idVW, 1u);
+                    if constexpr (DELTA) {
+                        const uint64_t bwl =
+                            sdesc_sw128(sb + C::OFF_B + 2 * C::NB * C::BOX + kk * 2048, C::BOX, 1024);
+                        mma_ss(T + D, ah, bwl, idWl, 1u);
+                    }
+                }
+                mma_commit(kv_empty + st);
+            }
+            mma_commit(acc_full);
+            incr_drain(acc_full, 0);
+        }
+    } else if (warp >= 4) {
+        // ---------------------------------------------------------------- workers
+        const int w = threadIdx.x - 128;            // 0..255
+        const int t = w >> 2, q = w & 3;            // token row of the chunk, feature quarter
+        const int f0 = q * C::FPT;                  // first feature of this thread
+        const int box = f0 >> 6, cq = (f0 & 63) >> 3;
+        constexpr int CPT = C::FPT / 8;             // 16-byte chunks per thread
+        if constexpr (DELTA)
+            for (int i = w; i < D; i += 256) sZ[i] = a.snapZ[cs * D + i];
+        if (D == 64)    // the padded feature box of sigma_hi / sigma_lo stays zero
+            for (int i = w; i < ST * 2 * (C::BOX / 16); i += 256) {
+                const int st = i / (2 * (C::BOX / 16)), o = i % (2 * (C::BOX / 16));
+                const int which = o / (C::BOX / 16), oo = o % (C::BOX / 16);
+                reinterpret_cast<uint4 *>(smem + st * C::STAGE + which * C::ATILE + C::BOX)[oo] =
+                    make_uint4(0, 0, 0, 0);
+            }
+        asm volatile("bar.sync 1, 256;" ::: "memory");
+
+        bool ok = true;
+        for (int g = 0; g < nch; ++g) {
+            const int st = g % ST;
+            if (!(ok = mbar_wait(kv_full + st, (g / ST) & 1, abort, WI_KV_FULL))) break;
+            uint8_t *stage = smem + st * C::STAGE;
+            // rows past the head's L (zero-filled by TMA) carry sigma = 0
+            const uint32_t keep = g * C::CH + t < rows ? 0xFFFFFFFFu : 0u;
+            float sg[C::FPT];
+#pragma unroll
+            for (int i = 0; i < CPT; ++i) {
+                const int off = box * C::BOX + t * 128 + (((cq + i) ^ (t & 7)) << 4);
+                uint4 *ph = reinterpret_cast<uint4 *>(stage + C::OFF_SH + off);
+                const uint4 v = *ph;
+                const uint32_t in[4] = {v.x, v.y, v.z, v.w};
+                uint32_t hi[4], lo[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162 *>(&in[e]);
+                    const float s0 = __uint_as_float(__float_as_uint(elu1(__low2float(x))) & keep);
+                    const float s1 = __uint_as_float(__float_as_uint(elu1(__high2float(x))) & keep);
+                    sg[i * 8 + 2 * e] = s0;
+                    sg[i * 8 + 2 * e + 1] = s1;
+                    const __nv_bfloat162 h = __floats2bfloat162_rn(s0, s1);
+                    hi[e] = *reinterpret_cast<const uint32_t *>(&h);
+                    lo[e] = pack_bf16x2(s0 - __low2float(h), s1 - __high2float(h));
+                }
+                *ph = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                *reinterpret_cast<uint4 *>(stage + C::OFF_SL + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+            }
+            if constexpr (DELTA) {
+                float den = 0.f;
+#pragma unroll
+                for (int e = 0; e < C::FPT; ++e) den = fmaf(sg[e], sZ[f0 + e], den);
+                den += __shfl_xor_sync(0xffffffffu, den, 1);
+                den += __shfl_xor_sync(0xffffffffu, den, 2);
+                const float inv = den == 0.f ? 0.f : 1.f / den;
+#pragma unroll
+                for (int i = 0; i < CPT; ++i) {
+                    const int off = box * C::BOX + t * 128 + (((cq + i) ^ (t & 7)) << 4);
+                    uint32_t hi[4], lo[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float w0 = sg[i * 8 + 2 * e] * inv, w1 = sg[i * 8 + 2 * e + 1] * inv;
+                        const __nv_bfloat162 h = __floats2bfloat162_rn(w0, w1);
+                        hi[e] = *reinterpret_cast<const uint32_t *>(&h);
+                        lo[e] = pack_bf16x2(w0 - __low2float(h), w1 - __high2float(h));
+                    }
+                    *reinterpret_cast<uint4 *>(stage + C::OFF_B + C::NB * C::BOX + off) =
+                        make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                    *reinterpret_cast<uint4 *>(stage + C::OFF_B + 2 * C::NB * C::BOX + off) =
+                        make_uint4(lo[0], lo[1], lo[2], lo[3]);
+                }
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(a_ready + st);
+        }
+        // ---- epilogue: lane i of the accumulator is key feature i
+        if (ok) ok = mbar_wait(acc_full, 0, abort, WI_ACC);
+        if (ok) {
+            tc_fence_after();
+            const int i = (warp & 3) * 32 + lane;
+            const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+            const bool second = warp >= 8;              // warps 8-11: A_s (delta)
+            if (!second || DELTA) {
+                if (D == 128 || (warp & 3) < 2) {       // lanes past d hold nothing
+#pragma unroll 1
+                    for (int c0 = 0; c0 < D; c0 += 32) {
+                        uint32_t r[32];
+                        tmem_ld32(lane_base + T + (second ? D : 0) + c0, r);
+                        tmem_ld_wait();
+                        const int64_t o = (cs * D + i) * D + c0;
+                        if (!second) {
+                            float4 *dst = reinterpret_cast<float4 *>(a.Bs + o);
+#pragma unroll
+                            for (int e = 0; e < 8; ++e)
+                                dst[e] = make_float4(__uint_as_float(r[4 * e]), __uint_as_float(r[4 * e + 1]),
+                                                     __uint_as_float(r[4 * e + 2]), __uint_as_float(r[4 * e + 3]));
+                        } else {
+                            uint32_t hi[16], lo[16];
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) {
+                                const float x0 = __uint_as_float(r[2 * e]), x1 = __uint_as_float(r[2 * e + 1]);
+                                const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+                                hi[e] = *reinterpret_cast<const uint32_t *>(&h);
+                                lo[e] = pack_bf16x2(x0 - __low2float(h), x1 - __high2float(h));
+                            }
+                            uint4 *dh = reinterpret_cast<uint4 *>(a.Ahi + o);
+                            uint4 *dl = reinterpret_cast<uint4 *>(a.Alo + o);
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                dh[e] = make_uint4(hi[4 * e], hi[4 * e + 1], hi[4 * e + 2], hi[4 * e + 3]);
+                                dl[e] = make_uint4(lo[4 * e], lo[4 * e + 1], lo[4 * e + 2], lo[4 * e + 3]);
+                            }
+                        }
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(T, C::TMEM_COLS);
+    }
+}
+
+// ---------------------------------------------------------------- the serial parts
+
+// Additive rule: M_{s-1} = M0 + sum_{j<s} B_j.  One thread per 4 consecutive elements of a
+// chain's M walks the segments, writing the bf16 snapshot of every M_{s-1} and M_out.  Each
+// element is read from M0 and written to M_out by the same thread, so they may alias.
+template <int D>
+__global__ void __launch_bounds__(256)
+k_mem_prefix(const float *__restrict__ Bs, const float *M0, __nv_bfloat16 *__restrict__ snapMb,
+             float *M_out, int S, int64_t chains)
+{
+    constexpr int64_t E4 = (int64_t)D * D / 4;
+    const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    if (i >= chains * E4) return;
+    const int64_t chain = i / E4, e = i % E4;
+    float4 m = M0 ? reinterpret_cast<const float4 *>(M0)[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+    const float4 *b = reinterpret_cast<const float4 *>(Bs) + chain * S * E4 + e;
+    uint2 *snap = reinterpret_cast<uint2 *>(snapMb) + chain * S * E4 + e;
+#pragma unroll 4
+    for (int s = 0; s < S; ++s) {
+        snap[(int64_t)s * E4] = make_uint2(pack_bf16x2(m.x, m.y), pack_bf16x2(m.z, m.w));
+        const float4 x = b[(int64_t)s * E4];
+        m.x += x.x;
+        m.y += x.y;
+        m.z += x.z;
+        m.w += x.w;
+    }
+    reinterpret_cast<float4 *>(M_out)[i] = m;
+}
+
+template <int D>
+struct MChainCfg {
+    static_assert(D == 64 || D == 128, "tensor-core delta recurrence: d = 64 or 128");
+    static constexpr int CB = 32;                   // value columns per CTA
+    static constexpr int NK = D / 64;               // 64-wide boxes along the contraction
+    static constexpr int ABOX = 128 * 128;          // 128 rows x 64 bf16
+    static constexpr int ATILE = NK * ABOX;         // A_hi (or A_lo) of one segment
+    static constexpr int ST = 2;
+    static constexpr int BBOX = CB * 128;           // CB rows x 64 bf16 (K-major M^T)
+    static constexpr int BTILE = NK * BBOX;
+    static constexpr int OFF_A = 0;                 // per stage: A_hi | A_lo
+    static constexpr int OFF_B = ST * 2 * ATILE;    // M^T hi | M^T lo
+    static constexpr int OFF_BAR = OFF_B + 2 * BTILE;
+    static constexpr int NBAR = 2 * ST + 3;
+    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+    static constexpr int BYTES = OFF_MISC + 16;
+    static constexpr int ALLOC = BYTES + 1024;
+    static_assert(OFF_B % 1024 == 0 && BTILE % 1024 == 0, "operand tiles must be 1024-aligned");
+};
+
+struct MChainArgs {
+    const float *M0;           // may be NULL (zeros); may alias M_out exactly
+    const float *Bs;           // [chains * S, D, D]
+    __nv_bfloat16 *snapMb;     // [chains * S, D, D]: bf16 M_{s-1}
+    float *M_out;
+    int S;
+};
+
+enum : int { WM_A_EMPTY = 601, WM_B = 602, WM_A_FULL = 603, WM_D = 604, WM_DRAIN = 605 };
+
+__device__ __forceinline__ void mchain_drain(uint64_t *bar, uint32_t parity)
+{
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity)) {
+        if (clock64() - t0 > spin_limit()) {
+            atomicCAS(&g_wait_status, 0, WM_DRAIN);
+            return;
+        }
+    }
+}
+
+// Delta rule: M_s = M_{s-1} + B_s - A_s M_{s-1} in segment order.  One CTA per (chain, 32
+// value columns); column block j of M_s needs only column block j of M_{s-1}.  Warp 0: TMA
+// of A_s (hi and lo parts, K-major, two stages ahead).  Warp 1: MMA issuer, D = A_hi M_hi +
+// A_hi M_lo + A_lo M_hi into 32 TMEM columns.  Warps 4-7: thread i holds row i of the block
+// in fp32 registers, writes the snapshot and the M^T hi / lo operand, then applies
+// M += B_s - D.  d = 64 runs as 128 rows with zero rows 64..127 of A.
+template <int D>
+__global__ void __launch_bounds__(256, 1)
+k_mem_chain(const __grid_constant__ CUtensorMap tmAh, const __grid_constant__ CUtensorMap tmAl,
+            const MChainArgs a)
+{
+    using C = MChainCfg<D>;
+    constexpr int ST = C::ST, CB = C::CB;
+    constexpr int NBLK = D / CB;
+    if (__syncthreads_or(threadIdx.x == 0 && wait_status_set())) return;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+
+    const int64_t chain = blockIdx.x / NBLK;
+    const int cb = (blockIdx.x % NBLK) * CB;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
+    uint64_t *a_full = bars, *a_empty = bars + ST, *b_ready = bars + 2 * ST, *d_full = b_ready + 1;
+    uint64_t *mma_done = d_full + 1;
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
+    volatile int *abort = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < ST; ++i) {
+            mbar_init(a_full + i, 1);
+            mbar_init(a_empty + i, 1);
+        }
+        mbar_init(b_ready, 128);
+        mbar_init(d_full, 1);
+        mbar_init(mma_done, 1);
+        *abort = 0;
+        fence_barrier_init();
+    }
+    if (D == 64)   // rows 64..127 of every A tile stay zero (the loads fill rows 0..63)
+        for (int i = threadIdx.x; i < ST * 2 * (C::ABOX / 32); i += 256) {
+            const int t = i / (C::ABOX / 32), o = i % (C::ABOX / 32);
+            reinterpret_cast<uint4 *>(smem + C::OFF_A + t * C::ATILE + C::ABOX / 2)[o] =
+                make_uint4(0, 0, 0, 0);
+        }
+    if (warp == 1) tmem_alloc(tmem_holder, 32);
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t T = *tmem_holder;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            prefetch_tmap(&tmAh);
+            prefetch_tmap(&tmAl);
+            int issued = 0;
+            for (int s = 0; s < a.S; ++s) {
+                const int st = s % ST;
+                if (s >= ST && !mbar_wait_short(a_empty + st, ((s / ST) - 1) & 1, abort, WM_A_EMPTY))
+                    break;
+                uint8_t *dst = smem + C::OFF_A + st * 2 * C::ATILE;
+                const int slot = (int)(chain * a.S + s);
+                mbar_arrive_expect_tx(a_full + st, (uint32_t)(2 * C::NK * D * 128));
+                for (int b = 0; b < C::NK; ++b) {
+                    tma_load_3d(dst + b * C::ABOX, &tmAh, a_full + st, b * 64, 0, slot);
+                    tma_load_3d(dst + C::ATILE + b * C::ABOX, &tmAl, a_full + st, b * 64, 0, slot);
+                }
+                issued = s + 1;
+            }
+            if (*abort)
+                for (int s = (issued > ST ? issued - ST : 0); s < issued; ++s)
+                    mchain_drain(a_full + s % ST, (s / ST) & 1);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t id = idesc_bf16(128, CB, 0, 0);
+            const uint32_t aA = smem_u32(smem + C::OFF_A), aB = smem_u32(smem + C::OFF_B);
+            for (int s = 0; s < a.S; ++s) {
+                const int st = s % ST;
+                if (!mbar_wait_short(b_ready, s & 1, abort, WM_B)) break;
+                if (!mbar_wait_short(a_full + st, (s / ST) & 1, abort, WM_A_FULL)) break;
+                tc_fence_after();
+                const uint32_t ah = aA + st * 2 * C::ATILE, al = ah + C::ATILE;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t ao = (kk >> 2) * C::ABOX + (kk & 3) * 32;
+                    const uint32_t bo = (kk >> 2) * C::BBOX + (kk & 3) * 32;
+                    const uint64_t dah = sdesc_sw128(ah + ao, 16, 1024);
+                    const uint64_t dbh = sdesc_sw128(aB + bo, 16, 1024);
+                    mma_ss(T, dah, dbh, id, kk > 0 ? 1u : 0u);
+                    mma_ss(T, dah, sdesc_sw128(aB + C::BTILE + bo, 16, 1024), id, 1u);
+                    mma_ss(T, sdesc_sw128(al + ao, 16, 1024), dbh, id, 1u);
+                }
+                mma_commit(a_empty + st);
+                mma_commit(d_full);
+            }
+            mma_commit(mma_done);
+            mchain_drain(mma_done, 0);
+        }
+    } else if (warp >= 4) {
+        const int i = threadIdx.x - 128;            // row of M (key feature), TMEM lane
+        const bool live = i < D;
+        const uint32_t lane_base = (uint32_t)((warp - 4) * 32) << 16;
+        uint8_t *sB = smem + C::OFF_B;
+        float m[CB];
+#pragma unroll
+        for (int j = 0; j < CB; ++j) m[j] = 0.f;
+        if (live && a.M0) {
+            const float4 *src = reinterpret_cast<const float4 *>(a.M0 + (chain * D + i) * D + cb);
+#pragma unroll
+            for (int e = 0; e < CB / 4; ++e) {
+                const float4 x = src[e];
+                m[4 * e] = x.x;
+                m[4 * e + 1] = x.y;
+                m[4 * e + 2] = x.z;
+                m[4 * e + 3] = x.w;
+            }
+        }
+        // element (j, k = i) of a K-major [CB rows x D] tile
+        const int kb = i >> 6, kc = i & 63;
+        bool ok = true;
+        for (int s = 0; s < a.S; ++s) {
+            const int64_t slot = chain * a.S + s;
+            if (live) {
+                uint32_t pk[CB / 2];
+#pragma unroll
+                for (int e = 0; e < CB / 2; ++e) pk[e] = pack_bf16x2(m[2 * e], m[2 * e + 1]);
+                uint4 *dst = reinterpret_cast<uint4 *>(a.snapMb + (slot * D + i) * D + cb);
+#pragma unroll
+                for (int e = 0; e < CB / 8; ++e)
+                    dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+#pragma unroll
+                for (int j = 0; j < CB; ++j) {
+                    const __nv_bfloat16 hi = __float2bfloat16_rn(m[j]);
+                    const __nv_bfloat16 lo = __float2bfloat16_rn(m[j] - __bfloat162float(hi));
+                    const int o = kb * C::BBOX + j * 128 + ((((kc >> 3) ^ (j & 7))) << 4) + (kc & 7) * 2;
+                    *reinterpret_cast<__nv_bfloat16 *>(sB + o) = hi;
+                    *reinterpret_cast<__nv_bfloat16 *>(sB + C::BTILE + o) = lo;
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(b_ready);
+            float4 bs[CB / 4];
+            if (live) {
+                const float4 *src = reinterpret_cast<const float4 *>(a.Bs + (slot * D + i) * D + cb);
+#pragma unroll
+                for (int e = 0; e < CB / 4; ++e) bs[e] = src[e];
+            }
+            if (!(ok = mbar_wait(d_full, s & 1, abort, WM_D))) break;
+            tc_fence_after();
+            uint32_t r[32];
+            tmem_ld32(lane_base + T, r);
+            tmem_ld_wait();
+            if (live) {
+#pragma unroll
+                for (int e = 0; e < CB / 4; ++e) {
+                    m[4 * e] += bs[e].x - __uint_as_float(r[4 * e]);
+                    m[4 * e + 1] += bs[e].y - __uint_as_float(r[4 * e + 1]);
+                    m[4 * e + 2] += bs[e].z - __uint_as_float(r[4 * e + 2]);
+                    m[4 * e + 3] += bs[e].w - __uint_as_float(r[4 * e + 3]);
+                }
+            }
+            tc_fence_before();
+        }
+        if (ok && live) {
+            float4 *dst = reinterpret_cast<float4 *>(a.M_out + (chain * D + i) * D + cb);
+#pragma unroll
+            for (int e = 0; e < CB / 4; ++e)
+                dst[e] = make_float4(m[4 * e], m[4 * e + 1], m[4 * e + 2], m[4 * e + 3]);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(T, 32);
+    }
+}
+
+}  // namespace tc
+}  // namespace infini

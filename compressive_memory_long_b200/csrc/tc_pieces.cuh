@@ -94,7 +94,7 @@ __device__ __forceinline__ void piece_drain(uint64_t *bar, uint32_t parity)
 {
     const long long t0 = clock64();
     while (!mbar_try_wait(bar, parity)) {
-        if (clock64() - t0 > kSpinLimitCycles) {
+        if (clock64() - t0 > spin_limit()) {
             atomicCAS(&g_wait_status, 0, WP_DRAIN);
             return;
         }
@@ -659,7 +659,7 @@ k_small_pieces(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                     const int f = pred >= 0 ? ld_acquire_gpu(a.flags + chain + (int64_t)pred * a.chains) : 0;
                     const uint32_t inc = __ballot_sync(0xffffffffu, pred >= 0 && f == FLAG_INCL);
                     const uint32_t none = __ballot_sync(0xffffffffu, pred >= 0 && f == 0);
-                    const uint32_t quit = __ballot_sync(0xffffffffu, *abort != 0 || clock64() - t0 > kSpinLimitCycles);
+                    const uint32_t quit = __ballot_sync(0xffffffffu, *abort != 0 || clock64() - t0 > spin_limit());
                     if (lane == 0) {
                         look[warp * 3] = inc;
                         look[warp * 3 + 1] = none;

@@ -66,7 +66,7 @@ __device__ __forceinline__ void mbar_drain(uint64_t *bar, uint32_t parity)
 {
     const long long t0 = clock64();
     while (!mbar_try_wait(bar, parity)) {
-        if (clock64() - t0 > kSpinLimitCycles) {
+        if (clock64() - t0 > spin_limit()) {
             atomicCAS(&g_wait_status, 0, W_DRAIN);
             return;
         }

@@ -77,7 +77,7 @@ __device__ __forceinline__ void small_drain(uint64_t *bar, uint32_t parity)
 {
     const long long t0 = clock64();
     while (!mbar_try_wait(bar, parity)) {
-        if (clock64() - t0 > kSpinLimitCycles) {
+        if (clock64() - t0 > spin_limit()) {
             atomicCAS(&g_wait_status, 0, WS_DRAIN);
             return;
         }
@@ -325,7 +325,9 @@ k_small_linear_fused(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         // Unit 0 of a long head publishes no aggregate, only its inclusive prefix: every other
         // walk then ends at an inclusive prefix, and only unit 0 reads M0 / z0 -- which M_out /
         // z_out (written by the last unit, after its walk) may alias.
-        if (ok && r == 0 && (unit > 0 || a.direct)) st_release_gpu(a.flags + idx, FLAG_AGG);
+        // (a test hook can make unit 0 withhold its publishes: the later units' waits run out)
+        const bool withhold = unit == 0 && g_test_withhold != 0;
+        if (ok && r == 0 && (unit > 0 || a.direct) && !withhold) st_release_gpu(a.flags + idx, FLAG_AGG);
 
         // the local softmax and sigma(Q) come after the aggregate is published: later units
         // of the head wait for it, while this unit's own softmax is not on their path
@@ -415,7 +417,7 @@ k_small_linear_fused(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                 const int *fp = a.flags + chain * a.U + r;
                 const long long t0 = clock64();
                 while (ld_acquire_gpu(fp) == 0) {
-                    if (clock64() - t0 > kSpinLimitCycles || wait_status_set()) {
+                    if (clock64() - t0 > spin_limit() || wait_status_set()) {
                         atomicCAS(&g_wait_status, 0, WS_LOOK);
                         bad = true;
                         break;
@@ -441,7 +443,7 @@ k_small_linear_fused(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                 } else {
                     const long long t0 = clock64();
                     while (ld_acquire_gpu(a.m0_done + chain) < a.U - 1) {
-                        if (clock64() - t0 > kSpinLimitCycles || wait_status_set()) {
+                        if (clock64() - t0 > spin_limit() || wait_status_set()) {
                             atomicCAS(&g_wait_status, 0, WS_LOOK);
                             *s_state = -1;
                             break;
@@ -462,7 +464,7 @@ k_small_linear_fused(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                     int f = ld_acquire_gpu(fp);
                     const long long t0 = clock64();
                     while (f == 0) {
-                        if (clock64() - t0 > kSpinLimitCycles || wait_status_set()) {
+                        if (clock64() - t0 > spin_limit() || wait_status_set()) {
                             atomicCAS(&g_wait_status, 0, WS_LOOK);
                             f = -1;
                             break;
@@ -513,7 +515,7 @@ k_small_linear_fused(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         }
         asm volatile("bar.sync 1, 128;" ::: "memory");
         if (ok) {
-            if (r == 0 && !a.direct && unit + 1 < a.U) st_release_gpu(a.flags + idx, FLAG_INCL);
+            if (r == 0 && !a.direct && unit + 1 < a.U && !withhold) st_release_gpu(a.flags + idx, FLAG_INCL);
             if (r < D) {
                 const float *exr = sEx + r * C::ROW, *d0r = sD0 + r * C::ROW;
                 // M_start and M_mid rows (key r) as bf16 B operands, z as fp32

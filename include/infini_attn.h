@@ -172,8 +172,10 @@ INFINI_API int infini_attn_fold_f32(const void *k_cache, const void *v_cache, in
  *
  *   - Its workspace is a fixed device array of INFINI_NOALLOC_SCRATCH_BYTES inside the
  *     library; every GPU that loads the library holds that array until the process exits.
- *     A problem whose workspace (infini_attn_workspace_bytes) exceeds it is rejected with
- *     INFINI_ERR_UNSUPPORTED, before anything is launched.
+ *     A problem whose workspace exceeds it is rejected with INFINI_ERR_UNSUPPORTED, before
+ *     anything is launched.  The size that counts is what the kernels chosen for the
+ *     problem need: infini_attn_workspace_bytes is an upper bound over all of them, and the
+ *     fused 64-token paths need much less.
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call before any
  *     stream capture begins.
@@ -221,6 +223,29 @@ INFINI_API int infini_attn_version(void);
  */
 INFINI_API int infini_attn_trace_enable(int on);
 INFINI_API int64_t infini_attn_trace_report(char *buf, int64_t len);
+
+/*
+ * Test hooks: they let the library's failure paths be exercised without a real failure.
+ * None of them is needed for normal use, and all are off by default.
+ *
+ * infini_attn_test_fail_allocations(n): the next n workspace allocations of this process
+ *   fail as an exhausted device would make them fail: the calls return INFINI_ERR_OOM before
+ *   anything is launched or written.  n = 0 turns the hook off.  INFINI_ERR_INVALID_ARG if
+ *   n < 0.
+ * infini_attn_test_wait_limit(cycles): the bound every device wait of the current device
+ *   applies, in SM clock cycles (default about 0.5 s at the top clock; cycles <= 0 restores
+ *   it).  A wait that reaches it gives up as described for infini_attn_device_status.
+ * infini_attn_test_withhold_publish(on): on the current device, the first unit of every head
+ *   in the fused 64-token kernel (additive rule, d = 64, N = 64, H == Hkv, at most 64 units
+ *   of 128 tokens per head) skips publishing its memory aggregate, so the later units'
+ *   waits for it run out: the call's outputs are then incomplete and
+ *   infini_attn_device_status reports INFINI_ERR_TIMEOUT.  Nothing traps or hangs.
+ * The last two copy to device variables synchronously (INFINI_ERR_CUDA if that fails); use
+ * them while no call of this library is running on the device.
+ */
+INFINI_API int infini_attn_test_fail_allocations(int n);
+INFINI_API int infini_attn_test_wait_limit(int64_t cycles);
+INFINI_API int infini_attn_test_withhold_publish(int on);
 
 #ifdef __cplusplus
 }

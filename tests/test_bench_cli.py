@@ -9,7 +9,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
 @pytest.mark.parametrize("args,needle", [
-    (["--tail", "64"], "--tail must be in (0, N)"),         # hf_repro_n64 has N = 64
+    (["--workload", "hf_repro_n64", "--tail", "64"], "--tail must be in (0, N)"),   # N = 64
+    (["--tail", "2048"], "--tail must be in (0, N)"),       # the default workload has N = 2048
     (["--tail", "-3"], "--tail must be in (0, N)"),
     (["--warmup", "2"], "--warmup must be >= 3"),
     (["--workload", "no_such_workload"], "invalid choice"),

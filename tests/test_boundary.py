@@ -37,17 +37,28 @@ def test_status_strings_and_version():
     assert binding.infini_attn_version() >= 100
 
 
+def tc_bytes(units, d, delta=True):
+    """z_{s-1} and dz_s (fp32), bf16 M_{s-1}, fp32 B_s, bf16 hi / lo A_s, per segment."""
+    return units * (2 * d * 4 + d * d * 2 + d * d * 4 + (2 * d * d * 2 if delta else 0)) + 256
+
+
 def test_workspace_bytes():
+    """An upper bound over every path: the tensor-core memory path's per-segment state is
+    the larger one (the CUDA-core path keeps fp32 snapshots only)."""
     units = 2 * 8 * 16
-    assert binding.infini_attn_workspace_bytes(2, 8, 1024, 64, 64) == \
-        units * (64 * 64 + 64) * 4 + units * 64 * 64 * 2 + units * 64 * 64 * 2 + units * 4 + \
-        2 * 8 * 4 + units * 16 + 512
-    # a final short segment counts as a segment; the sigma(K) copy spans every row
-    assert binding.infini_attn_workspace_bytes(1, 1, 100, 64, 64) == \
-        2 * (64 * 64 + 64) * 4 + 2 * 64 * 64 * 2 + 100 * 64 * 2 + 2 * 4 + 4 + 2 * 16 + 512
-    assert binding.infini_attn_workspace_bytes(1, 1, 40, 64, 64) == \
-        (64 * 64 + 64) * 4 + 64 * 64 * 2 + 40 * 64 * 2 + 4 + 4 + 16 + 512
+    assert binding.infini_attn_workspace_bytes(2, 8, 1024, 64, 64) == tc_bytes(units, 64)
+    assert tc_bytes(units, 64) >= units * (64 * 64 + 64) * 4 + 256
+    # a final short segment counts as a segment
+    assert binding.infini_attn_workspace_bytes(1, 1, 100, 64, 64) == tc_bytes(2, 64)
+    assert binding.infini_attn_workspace_bytes(1, 1, 40, 64, 64) == tc_bytes(1, 64)
+    assert binding.infini_attn_workspace_bytes(1, 4, 8192, 2048, 128) == tc_bytes(16, 128)
     assert binding.infini_attn_workspace_bytes(0, 1, 64, 64, 64) == 0
+
+
+def test_allocation_failure_hook_arguments():
+    """The host-side hook only counts: a negative count is refused, 0 disarms it."""
+    assert binding.infini_attn_test_fail_allocations(-1) == 1
+    assert binding.infini_attn_test_fail_allocations(0) == 0
 
 
 BASE = 1 << 40      # fake, 16-byte aligned, never dereferenced

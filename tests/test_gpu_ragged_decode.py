@@ -61,19 +61,19 @@ RAGGED = [
     (make("one_token", B=1, H=1, Hkv=1, d=64, N=64, S=0, tail=1, state=True, seed=21),
      "tail_segment", True),
     (make("tc2_delta", B=1, H=4, Hkv=2, d=128, N=256, S=2, tail=100, rule="delta", seed=14),
-     "delta_chain_tc", False),
+     "mem_chain", False),
     (make("tc2_delta_long", B=1, H=2, Hkv=2, d=128, N=768, S=1, tail=520, rule="delta",
           seed=23), "segment_tc", False),
     (make("tc_linear", B=2, H=2, Hkv=2, d=128, N=128, S=3, tail=127, state=True, seed=15),
-     "linear_state_tc", False),
+     "mem_prefix", False),
     (make("tc_linear64", B=1, H=3, Hkv=3, d=64, N=256, S=1, tail=129, state=True, seed=24),
-     "linear_state_tc", False),
+     "mem_prefix", False),
     (make("tc_delta64", B=1, H=2, Hkv=1, d=64, N=128, S=2, tail=64, rule="delta", seed=16),
-     "delta_chain_tc", False),
+     "mem_chain", False),
     (make("only_tail", B=1, H=2, Hkv=1, d=128, N=256, S=0, tail=200, rule="delta", state=True,
           seed=19), "segment_tc", False),
     (make("only_tail_linear", B=1, H=2, Hkv=2, d=64, N=512, S=0, tail=3, seed=25),
-     "linear_state_tc", False),
+     "mem_prefix", False),
 ]
 
 
