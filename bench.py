@@ -48,6 +48,7 @@ from compressive_memory_long_b200 import workloads as wl  # noqa: E402
 
 METRIC = "Infini-attention fwd tokens/s at 1 B200; % of bf16 TC peak or HBM roofline"
 DECODE_METRIC = "Infini-attention decode tokens/s at 1 B200 (one token per call, per sequence)"
+BACKWARD_METRIC = "Infini-attention backward tokens/s at 1 B200 (all gradients of one forward)"
 DEFAULT_WORKLOAD = "stream1m_n2048_delta"
 FLUSH_BYTES = 256 << 20
 
@@ -68,6 +69,11 @@ NCU_TRAFFIC_BYTES: dict = {
     ("batched_n1024_linear", "segment_tc"): (1678875648 + 519356672) * 2,
     ("stream1m_n2048_delta", "segment_tc"): (411272448 + 114843136) * 32,
 }
+
+
+def fp32_fma_peak_tflops(sm_mhz=1965.0, sms=148):
+    """CUDA-core fp32 peak: SMs x 128 FP32 lanes x 2 flops (one FMA) x the SM clock."""
+    return sms * 128 * 2 * sm_mhz * 1e6 / 1e12
 
 
 def load_peaks():
@@ -429,6 +435,98 @@ def run_decode(args, w: wl.Workload, world: int, rank: int, local: int, dev):
     return 0
 
 
+# ---- the backward pass (our arm, --backward) ----
+
+def backward_flops(w: wl.Workload):
+    """Algorithmic flops of one backward: the local attention's five N x N x d products over
+    the causal half (recomputed scores, dP, dS K, dS^T Q, P^T dA) plus the retrieval's and
+    the memory's d x d contractions (forward recompute and gradients, about four times the
+    forward's)."""
+    B, H, Hkv, N, d = w.B, w.H, w.Hkv, w.N, w.d
+    S = -(-w.L // N)
+    local = B * H * S * 5 * d * N * (N + 1)
+    memory = B * H * S * 4 * 2 * N * d * d + B * Hkv * S * 4 * (4 if w.rule == "delta" else 2) * N * d * d
+    return local + memory
+
+
+def run_backward(args, w: wl.Workload, world: int, rank: int, local: int, dev):
+    """One step = all gradients of one forward of the workload (infini_attn_bwd), with a
+    fixed random upstream gradient; inputs resident on the device, L2 flushed before each
+    step.  The dominant kernel's roofline is against the fp32 FMA rate (CUDA cores)."""
+    import ctypes
+    from compressive_memory_long_b200 import binding
+    host = wl.torch_inputs(w, pin_memory=True)
+    t = {k: (None if x is None else x.to(dev, non_blocking=True)) for k, x in host.items()}
+    g = torch.Generator(device=dev).manual_seed(w.seed + 7)
+    dout = torch.randn(t["q"].shape, device=dev, generator=g).to(t["q"].dtype)
+    dM = 0.1 * torch.randn((w.B, w.Hkv, w.d, w.d), device=dev, generator=g)
+    dz = 0.01 * torch.randn((w.B, w.Hkv, w.d), device=dev, generator=g)
+    outs = [torch.empty_like(t["q"]), torch.empty_like(t["k"]), torch.empty_like(t["v"]),
+            torch.empty((w.H,), device=dev), torch.empty_like(dM), torch.empty_like(dz)]
+    fn = binding.LIB.infini_attn_bwd if w.dtype == "bf16" else binding.LIB.infini_attn_bwd_f32
+    stream = torch.cuda.current_stream(dev)
+    P = lambda x: None if x is None else ctypes.c_void_p(x.data_ptr())
+
+    def step():
+        rc = fn(P(t["q"]), P(t["k"]), P(t["v"]), P(t["beta"]), P(t["M0"]), P(t["z0"]), P(dout),
+                P(dM), P(dz), *(P(x) for x in outs), w.B, w.H, w.Hkv, w.L, w.N, w.d,
+                binding.RULES[w.rule], ctypes.c_void_p(stream.cuda_stream))
+        if rc != 0:
+            raise binding.InfiniError(rc, binding.infini_attn_status_string(rc))
+
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    binding.infini_attn_trace_enable(True)
+    with ClockSampler(local) as clocks:
+        for i in range(args.steps):
+            flush.zero_()
+            starts[i].record(stream)
+            step()
+            ends[i].record(stream)
+        torch.cuda.synchronize(dev)
+    binding.infini_attn_trace_enable(False)
+    barrier(world)
+    kernels = {k: v for k, v in binding.infini_attn_trace_report().items() if isinstance(v, dict)}
+    total_ms = max_over_ranks(float(sum(s_.elapsed_time(e) for s_, e in zip(starts, ends))), world, dev)
+    value = w.tokens * args.steps * world / (total_ms / 1000.0)
+    clk = clocks.summary()
+    peak = fp32_fma_peak_tflops(clk["sm_mhz"] or 1965.0)
+    attn = {k: v for k, v in kernels.items() if k in ("bwd_dq", "bwd_dkdv", "bwd_rows")}
+    attn_ms = sum(v["ms"] for v in attn.values()) / max(1, args.steps)
+    B, H, N, d = w.B, w.H, w.N, w.d
+    S = -(-w.L // N)
+    attn_flops = B * H * S * 2 * d * N * (N + 1) / 2 * (2 + 3 + 2)   # rows: S, PV; dq: S, dP, dS K; dkdv
+    achieved = attn_flops / (attn_ms / 1e3) / 1e12 if attn_ms > 0 else 0.0
+    roof = {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+            "frac": achieved / peak, "traffic": None, "kernel": "bwd_rows + bwd_dq + bwd_dkdv",
+            "kernel_ms": attn_ms, "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 x SM clock",
+            "algorithmic_flops": attn_flops}
+    if rank == 0:
+        line = {
+            "metric": BACKWARD_METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
+            "config": dict(config_of(w), pass_="backward"), "roofline": roof,
+            "cpu_baseline": None, "e2e": None,
+            "gpu_launches": int(sum(v["launches"] for v in kernels.values())),
+            "kernels": kernels, "clocks": clk,
+            "algorithmic_flops_total": backward_flops(w),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
 # ---- our arm ----
 
 def main():
@@ -445,6 +543,8 @@ def main():
                          "kernels' profiles: N = 128 selects the one-tile segment kernel)")
     ap.add_argument("--tail", type=int, default=0,
                     help="append a final segment of this many (< N) tokens to every head")
+    ap.add_argument("--backward", action="store_true",
+                    help="time the backward pass (all gradients of one forward) instead")
     ap.add_argument("--decode", action="store_true",
                     help="time the token-by-token decode step over one segment instead")
     ap.add_argument("--segments", type=int, default=0,
@@ -486,6 +586,8 @@ def main():
 
     if args.decode:
         return run_decode(args, w, world, rank, local, dev)
+    if args.backward:
+        return run_backward(args, w, world, rank, local, dev)
 
     host = wl.torch_inputs(w, pin_memory=True)
     t = {k: (None if x is None else x.to(dev, non_blocking=True)) for k, x in host.items()}

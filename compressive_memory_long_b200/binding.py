@@ -33,6 +33,7 @@ _FWD_ARGS = [_P] * 9 + [_I64] * 6 + [_I, _P]
 _DEC_ARGS = [_P] * 6 + [_I64] + [_P] * 3 + [_I64] * 5 + [_I, _P]
 _FOLD_ARGS = [_P, _P, _I64, _P, _P] + [_I64] * 4 + [_I, _P]
 _STATE_ARGS = [_P] * 6 + [_I64] * 5 + [_I, _P]
+_BWD_ARGS = [_P] * 15 + [_I64] * 6 + [_I, _P]
 SIGNATURES = {
     "infini_attn_fwd": (_FWD_ARGS, _I),
     "infini_attn_fwd_f32": (_FWD_ARGS, _I),
@@ -42,6 +43,8 @@ SIGNATURES = {
     "infini_attn_fold": (_FOLD_ARGS, _I),
     "infini_attn_fold_f32": (_FOLD_ARGS, _I),
     "infini_attn_state": (_STATE_ARGS, _I),
+    "infini_attn_bwd": (_BWD_ARGS, _I),
+    "infini_attn_bwd_f32": (_BWD_ARGS, _I),
     "infini_attn_state_f32": (_STATE_ARGS, _I),
     "infini_attn_workspace_bytes": ([_I64] * 5, _I64),
     "infini_attn_status_string": ([_I], ctypes.c_char_p),
@@ -279,3 +282,40 @@ def state(k, v, M0=None, z0=None, *, N: int, rule="linear", M_out=None, z_out=No
     if rc != 0:
         raise InfiniError(rc, infini_attn_status_string(rc))
     return M_out, z_out
+
+
+def backward(q, k, v, beta, M0, z0, dout, dM=None, dz=None, *, N: int, rule="linear",
+             stream=None):
+    """Gradients of <dout, out> + <dM, M_out> + <dz, z_out> of the forward with these inputs.
+
+    q [B,H,L,d], k/v [B,Hkv,L,d] and dout [B,H,L,d] (bf16 or fp32), beta [H], M0/z0 and dM/dz
+    fp32 or None.  Returns (dq, dk, dv, dbeta, dM0, dz0).
+    """
+    B, H, L, d = q.shape
+    Hkv = k.shape[1]
+    dev = q.device
+    _check(q, "q", q.dtype, (B, H, L, d), dev)
+    _check(k, "k", q.dtype, (B, Hkv, L, d), dev)
+    _check(v, "v", q.dtype, (B, Hkv, L, d), dev)
+    _check(dout, "dout", q.dtype, (B, H, L, d), dev)
+    _check(beta, "beta", torch.float32, (H,), dev)
+    _check(M0, "M0", torch.float32, (B, Hkv, d, d), dev)
+    _check(z0, "z0", torch.float32, (B, Hkv, d), dev)
+    _check(dM, "dM", torch.float32, (B, Hkv, d, d), dev)
+    _check(dz, "dz", torch.float32, (B, Hkv, d), dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dbeta = torch.empty((H,), dtype=torch.float32, device=dev)
+    dM0 = torch.empty((B, Hkv, d, d), dtype=torch.float32, device=dev)
+    dz0 = torch.empty((B, Hkv, d), dtype=torch.float32, device=dev)
+    if q.dtype == torch.bfloat16:
+        fn = LIB.infini_attn_bwd
+    elif q.dtype == torch.float32:
+        fn = LIB.infini_attn_bwd_f32
+    else:
+        raise ValueError(f"unsupported activation dtype {q.dtype}")
+    rc = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(M0), _ptr(z0), _ptr(dout), _ptr(dM),
+            _ptr(dz), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dbeta), _ptr(dM0), _ptr(dz0), B, H, Hkv,
+            L, int(N), d, RULES[rule], _stream_handle(stream))
+    if rc != 0:
+        raise InfiniError(rc, infini_attn_status_string(rc))
+    return dq, dk, dv, dbeta, dM0, dz0

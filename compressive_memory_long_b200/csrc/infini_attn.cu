@@ -21,6 +21,7 @@
 #include "tc_small.cuh"
 #include "tc_pieces.cuh"
 #include "decode.cuh"
+#include "backward.cuh"
 
 #include <cudaTypedefs.h>
 
@@ -111,6 +112,18 @@ bool opt_in_smem(size_t bytes)
         return false;
     done_mask.fetch_or(bit);
     return true;
+}
+
+// SMs of the current device (148 on a B200 if the query fails).
+int sm_count()
+{
+    int sms = 148, dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+        cudaGetLastError();
+        sms = 148;
+    }
+    return sms;
 }
 
 // ---- opt-in launch tracing: a pair of CUDA events on the launch stream around every
@@ -289,7 +302,7 @@ Workspace carve_workspace(void *raw, int64_t units, int64_t d, bool tc_path)
 template <int D>
 int launch_memory_tc(const Problem &p, const __nv_bfloat16 *k, const __nv_bfloat16 *v,
                      const float *M0, const float *z0, const Workspace &ws, float *M_out,
-                     float *z_out, cudaStream_t st)
+                     float *z_out, cudaStream_t st, float *snapMf = nullptr)
 {
     const int64_t chains = p.B * p.Hkv, units = chains * p.S;
     const int S = (int)p.S, N = (int)p.N;
@@ -305,23 +318,25 @@ int launch_memory_tc(const Problem &p, const __nv_bfloat16 *k, const __nv_bfloat
     CUtensorMap mk, mv;
     if (!make_map_bf16_3d(&mk, k, D, p.L, chains, 64) || !make_map_bf16_3d(&mv, v, D, p.L, chains, 64))
         return INFINI_ERR_CUDA;
-    tc::IncrArgs ia{ws.snapZ, ws.Bs, ws.Ahi, ws.Alo, p.L, N, S};
+    // persistent: one CTA per SM (or per item when there are fewer)
+    tc::IncrArgs ia{ws.snapZ, ws.Bs, ws.Ahi, ws.Alo, p.L, N, S, (int)units};
+    const unsigned igrid = (unsigned)std::min<int64_t>(units, sm_count());
     if (delta) {
         using C = tc::IncrCfg<D, true>;
         if (!opt_in_smem<tc::k_mem_incr<D, true>>(C::ALLOC)) return INFINI_ERR_CUDA;
         TRACED("mem_increments", st);
-        tc::k_mem_incr<D, true><<<(unsigned)units, C::THREADS, C::ALLOC, st>>>(mk, mv, ia);
+        tc::k_mem_incr<D, true><<<igrid, C::THREADS, C::ALLOC, st>>>(mk, mv, ia);
     } else {
         using C = tc::IncrCfg<D, false>;
         if (!opt_in_smem<tc::k_mem_incr<D, false>>(C::ALLOC)) return INFINI_ERR_CUDA;
         TRACED("mem_increments", st);
-        tc::k_mem_incr<D, false><<<(unsigned)units, C::THREADS, C::ALLOC, st>>>(mk, mv, ia);
+        tc::k_mem_incr<D, false><<<igrid, C::THREADS, C::ALLOC, st>>>(mk, mv, ia);
     }
     if (!delta) {
         const int64_t n4 = chains * D * D / 4;
         TRACED("mem_prefix", st);
         tc::k_mem_prefix<D><<<(unsigned)((n4 + 255) / 256), 256, 0, st>>>(ws.Bs, M0, ws.snapMb,
-                                                                          M_out, S, chains);
+                                                                          M_out, S, chains, snapMf);
         return INFINI_OK;
     }
     using MC = tc::MChainCfg<D>;
@@ -330,7 +345,7 @@ int launch_memory_tc(const Problem &p, const __nv_bfloat16 *k, const __nv_bfloat
         !make_map_bf16_3d(&mal, ws.Alo, D, D, units, D))
         return INFINI_ERR_CUDA;
     if (!opt_in_smem<tc::k_mem_chain<D>>(MC::ALLOC)) return INFINI_ERR_CUDA;
-    tc::MChainArgs ca{M0, ws.Bs, ws.snapMb, M_out, S};
+    tc::MChainArgs ca{M0, ws.Bs, ws.snapMb, snapMf, M_out, S, 0};
     TRACED("mem_chain", st);
     tc::k_mem_chain<D><<<(unsigned)(chains * (D / MC::CB)), 256, MC::ALLOC, st>>>(mah, mal, ca);
     return INFINI_OK;
@@ -421,16 +436,6 @@ int launch_small_fused(const Problem &p, const __nv_bfloat16 *q, const __nv_bflo
     return INFINI_OK;
 }
 
-int sm_count()
-{
-    int sms = 148, dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
-        cudaGetLastError();
-        sms = 148;
-    }
-    return sms;
-}
 
 // Long heads of 64-token segments: the persistent piece kernel.  Units per piece: about four
 // pieces per CTA across the grid, at most PieceCfg::MAX_UNITS.
@@ -970,6 +975,268 @@ int decode_step(const void *q, const void *k, const void *v, const float *beta, 
     return fold_launch<T>(kc, vc, N, M, z, B, Hkv, N, d, rule, st);   // the segment is complete
 }
 
+// ---- backward pass --------------------------------------------------------------------------
+
+struct BwdPlan {
+    int64_t B, H, Hkv, L, N, d, S, T, chains, units, qtiles;
+    int rule;
+    bool tc;          // bf16 with d in {64, 128}: the memory path runs on the tensor cores
+};
+
+// bf16 activations with d in {64, 128}: the backward's memory recomputation and its
+// reverse delta recurrence use the forward's tensor-core memory kernels.
+template <typename T>
+bool bwd_uses_tc(int64_t d) { return sizeof(T) == 2 && (d == 64 || d == 128); }
+
+// Workspace of one backward call (fp32), in the order carve_bwd lays it out.
+int64_t bwd_workspace_bytes(const BwdPlan &p)
+{
+    const int64_t rows = p.B * p.H * p.L, krows = p.B * p.Hkv * p.L, dd = p.d * p.d;
+    const int64_t floats = p.units * dd * 3 + p.units * p.d * 4 + rows * 4 + rows * p.d +
+                           p.B * p.H * p.S * p.qtiles + krows * p.d * 3 +
+                           (p.tc ? p.units * (p.d + dd + dd) : 0);   // dz, B_s, A_s hi + lo
+    return floats * 4 + 20 * 256;
+}
+
+BwdWs carve_bwd(void *raw, const BwdPlan &p)
+{
+    float *f = static_cast<float *>(raw);
+    auto take = [&](int64_t n) {
+        float *r = f;
+        f += (n + 63) / 64 * 64;          // 256-byte aligned pieces
+        return r;
+    };
+    const int64_t rows = p.B * p.H * p.L, krows = p.B * p.Hkv * p.L, dd = p.d * p.d;
+    BwdWs w;
+    float *snapM = take(p.units * dd), *snapZ = take(p.units * p.d);
+    w.snapM = snapM;
+    w.snapZ = snapZ;
+    w.GM = take(p.units * dd);
+    w.dMs = take(p.units * dd);
+    w.Gz = take(p.units * p.d);
+    w.h = take(p.units * p.d);
+    w.dzs = take(p.units * p.d);
+    w.lse = take(rows);
+    w.Drow = take(rows);
+    w.wsc = take(rows);
+    w.dden = take(rows);
+    w.dq = take(rows * p.d);
+    w.dbeta_part = take(p.B * p.H * p.S * p.qtiles);
+    w.dk = take(krows * p.d);
+    w.dv = take(krows * p.d);
+    w.dsk = take(krows * p.d);
+    return w;
+}
+
+// The tensor-core memory path's buffers of the backward (after carve_bwd's).
+Workspace carve_bwd_tc(void *raw, const BwdPlan &p)
+{
+    const int64_t rows = p.B * p.H * p.L, krows = p.B * p.Hkv * p.L, dd = p.d * p.d;
+    int64_t used = 0;
+    for (int64_t n : {p.units * dd, p.units * p.d, p.units * dd, p.units * dd, p.units * p.d,
+                      p.units * p.d, p.units * p.d, rows, rows, rows, rows, rows * p.d,
+                      p.B * p.H * p.S * p.qtiles, krows * p.d, krows * p.d, krows * p.d})
+        used += (n + 63) / 64 * 64;
+    float *f = static_cast<float *>(raw) + used;
+    Workspace w;
+    w.raw = raw;
+    w.dz = f;
+    w.Bs = w.dz + (p.units * p.d + 63) / 64 * 64;
+    w.Ahi = reinterpret_cast<__nv_bfloat16 *>(w.Bs + p.units * dd);
+    w.Alo = w.Ahi + p.units * dd;
+    return w;
+}
+
+template <typename T, int D>
+int launch_backward(const BwdPlan &p, const T *q, const T *k, const T *v, const float *beta,
+                    const float *M0, const float *z0, const T *dout, const float *dM,
+                    const float *dz, T *dq, T *dk, T *dv, float *dbeta, float *dM0, float *dz0,
+                    void *raw, cudaStream_t st)
+{
+    BwdWs w = carve_bwd(raw, p);
+    float *snapM = const_cast<float *>(w.snapM), *snapZ = const_cast<float *>(w.snapZ);
+    const int S = (int)p.S, N = (int)p.N, T_last = (int)p.T, H = (int)p.H, Hkv = (int)p.Hkv;
+    const int64_t chains = p.chains, units = p.units;
+    const int64_t per = (int64_t)D * D + D;
+    // 1. the memory before every segment (fp32); the final memory goes to scratch (GM, Gz:
+    //    overwritten below)
+    bool tc_mem = false;
+    if constexpr (sizeof(T) == 2 && (D == 64 || D == 128)) {
+        if (p.tc) {
+            Workspace tw = carve_bwd_tc(raw, p);
+            tw.snapZ = snapZ;
+            Problem fp;
+            fp.B = p.B; fp.H = p.H; fp.Hkv = p.Hkv; fp.L = p.L; fp.N = p.N; fp.d = p.d;
+            fp.S = p.S; fp.Lf = p.S * p.N; fp.T = 0; fp.rule = p.rule;
+            const int rc = launch_memory_tc<D>(fp, k, v, M0, z0, tw, w.GM, w.Gz, st, snapM);
+            if (rc != INFINI_OK) return rc;
+            tc_mem = true;
+        }
+    }
+    if (tc_mem) {
+    } else if (p.rule == INFINI_UPDATE_LINEAR) {
+        {
+            TRACED("bwd_state", st);
+            k_linear_increments<T, D><<<(unsigned)units, 256, 0, st>>>(k, v, snapM, snapZ, p.L, N, S,
+                                                                       T_last);
+        }
+        TRACED("bwd_state_scan", st);
+        k_linear_scan<<<(unsigned)((chains * per + 255) / 256), 256, 0, st>>>(
+            snapM, snapZ, nullptr, M0, z0, w.GM, w.Gz, S, D, chains);
+    } else {
+        {
+            TRACED("bwd_state", st);
+            k_state_init<<<(unsigned)((chains * per + 255) / 256), 256, 0, st>>>(M0, z0, snapM, snapZ,
+                                                                               nullptr, S, D, chains);
+        }
+        TRACED("bwd_state_chain", st);
+        k_delta_chain<T, D, 16><<<(unsigned)(chains * (D / 16)), 256, 0, st>>>(
+            k, v, snapM, snapZ, nullptr, w.GM, nullptr, p.L, N, S, T_last);
+    }
+    // 2. row statistics, the retrieval part of dq, the gate's partial sums
+    {
+        const size_t smem = BwdRowsSmem<D>::bytes;
+        if (!opt_in_smem<k_bwd_rows<T, D>>(smem)) return INFINI_ERR_CUDA;
+        TRACED("bwd_rows", st);
+        k_bwd_rows<T, D><<<(unsigned)(p.B * p.H * S * p.qtiles), 256, smem, st>>>(
+            q, k, v, beta, dout, w, p.L, N, S, H, Hkv);
+    }
+    // 3. dq;  4. local dk, dv
+    {
+        const size_t smem = BwdDqSmem<D>::bytes;
+        if (!opt_in_smem<k_bwd_dq<T, D>>(smem) || !opt_in_smem<k_bwd_dkdv<T, D>>(smem))
+            return INFINI_ERR_CUDA;
+        {
+            TRACED("bwd_dq", st);
+            k_bwd_dq<T, D><<<(unsigned)(p.B * p.H * S * p.qtiles), 256, smem, st>>>(
+                q, k, v, beta, dout, w, dq, p.L, N, S, H, Hkv);
+        }
+        TRACED("bwd_dkdv", st);
+        k_bwd_dkdv<T, D><<<(unsigned)(chains * S * p.qtiles), 256, smem, st>>>(
+            q, k, v, beta, dout, w, p.L, N, S, H, Hkv);
+    }
+    // 5. G^M_s, G^z_s;  6. the reverse memory recurrence
+    {
+        TRACED("bwd_gm", st);
+        k_bwd_gm<T, D><<<(unsigned)units, 256, 0, st>>>(q, dout, w, p.L, N, S, H, Hkv);
+    }
+    if (p.rule == INFINI_UPDATE_LINEAR) {
+        TRACED("bwd_mem_rev", st);
+        k_bwd_mlin<<<(unsigned)((chains * D * D + 255) / 256), 256, 0, st>>>(dM, w, dM0, S, D, chains);
+    } else if (tc_mem) {
+        // dM_{s-1} = dM_s + G^M_s - A_s dM_s: the forward recurrence run backwards, with the
+        // forward's A_s; its snapshots are dM_s, its final state dM0 (scratch: B_s, no longer
+        // needed, when the caller does not want it)
+        if constexpr (sizeof(T) == 2 && (D == 64 || D == 128)) {
+            const Workspace tw = carve_bwd_tc(raw, p);
+            using MC = tc::MChainCfg<D>;
+            CUtensorMap mah, mal;
+            if (!make_map_bf16_3d(&mah, tw.Ahi, D, D, units, D) ||
+                !make_map_bf16_3d(&mal, tw.Alo, D, D, units, D))
+                return INFINI_ERR_CUDA;
+            if (!opt_in_smem<tc::k_mem_chain<D>>(MC::ALLOC)) return INFINI_ERR_CUDA;
+            tc::MChainArgs ca{dM, w.GM, nullptr, w.dMs, dM0 ? dM0 : tw.Bs, S, 1};
+            TRACED("bwd_mem_rev", st);
+            tc::k_mem_chain<D><<<(unsigned)(chains * (D / MC::CB)), 256, MC::ALLOC, st>>>(mah, mal, ca);
+        }
+    } else {
+        TRACED("bwd_mem_rev", st);
+        k_bwd_mdelta<T, D, 16><<<(unsigned)(chains * (D / 16)), 256, 0, st>>>(k, dM, w, dM0, p.L, N, S);
+    }
+    // 7. the update's gradients;  8. the reverse z recurrence
+    {
+        const size_t smem = BwdUpdSmem<D>::bytes;
+        if (p.rule == INFINI_UPDATE_LINEAR) {
+            if (!opt_in_smem<k_bwd_update<T, D, false>>(smem)) return INFINI_ERR_CUDA;
+            TRACED("bwd_update", st);
+            k_bwd_update<T, D, false><<<(unsigned)units, 256, smem, st>>>(k, v, w, p.L, N, S);
+        } else {
+            if (!opt_in_smem<k_bwd_update<T, D, true>>(smem)) return INFINI_ERR_CUDA;
+            TRACED("bwd_update", st);
+            k_bwd_update<T, D, true><<<(unsigned)units, 256, smem, st>>>(k, v, w, p.L, N, S);
+        }
+    }
+    {
+        TRACED("bwd_z_rev", st);
+        k_bwd_zrev<<<(unsigned)((chains * D + 255) / 256), 256, 0, st>>>(dz, w, dz0, S, D, chains);
+    }
+    // 9. dk, dv in the activation dtype;  10. dbeta
+    {
+        const int64_t n = p.B * p.Hkv * p.L * D;
+        TRACED("bwd_final", st);
+        k_bwd_final<T, D><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(k, w, dk, dv, p.L, N, S, n);
+    }
+    if (dbeta) {
+        TRACED("bwd_beta", st);
+        k_bwd_beta<<<(unsigned)((p.H + 255) / 256), 256, 0, st>>>(w.dbeta_part, dbeta, (int)p.B, H, S,
+                                                               (int)p.qtiles);
+    }
+    return cudaGetLastError() == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
+}
+
+template <typename T>
+int backward(const void *q, const void *k, const void *v, const float *beta, const float *M0,
+             const float *z0, const void *dout, const float *dM, const float *dz, void *dq,
+             void *dk, void *dv, float *dbeta, float *dM0, float *dz0, int64_t B, int64_t H,
+             int64_t Hkv, int64_t L, int64_t N, int64_t d, int rule, infini_stream_t stream)
+{
+    if (!q || !k || !v || !beta || !dout || !dq || !dk || !dv) return INFINI_ERR_INVALID_ARG;
+    if (B <= 0 || H <= 0 || Hkv <= 0 || L <= 0 || N <= 0 || d <= 0 || H % Hkv != 0)
+        return INFINI_ERR_INVALID_ARG;
+    if (rule != INFINI_UPDATE_LINEAR && rule != INFINI_UPDATE_DELTA) return INFINI_ERR_INVALID_ARG;
+    if (B > (1 << 20) || H > (1 << 16) || L > ((int64_t)1 << 34) || B * H * L > ((int64_t)1 << 40) ||
+        B * H * ((L + 63) / 64) > ((int64_t)1 << 30))
+        return INFINI_ERR_INVALID_ARG;
+    const void *ptrs[] = {q, k, v, beta, M0, z0, dout, dM, dz, dq, dk, dv, dbeta, dM0, dz0};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return INFINI_ERR_INVALID_ARG;
+    const int64_t es = (int64_t)sizeof(T), qb = B * H * L * d * es, kb = B * Hkv * L * d * es;
+    const int64_t mb = B * Hkv * d * d * 4, zb = B * Hkv * d * 4;
+    // outputs overlap no input and no other output
+    const void *ins[] = {q, k, v, beta, M0, z0, dout, dM, dz};
+    const int64_t insz[] = {qb, kb, kb, H * 4, mb, zb, qb, mb, zb};
+    const void *outs[] = {dq, dk, dv, dbeta, dM0, dz0};
+    const int64_t outsz[] = {qb, kb, kb, H * 4, mb, zb};
+    for (int i = 0; i < 6; ++i) {
+        for (int j = 0; j < 9; ++j)
+            if (ranges_overlap(outs[i], outsz[i], ins[j], insz[j])) return INFINI_ERR_INVALID_ARG;
+        for (int j = 0; j < i; ++j)
+            if (ranges_overlap(outs[i], outsz[i], outs[j], outsz[j])) return INFINI_ERR_INVALID_ARG;
+    }
+    if (d != 32 && d != 64 && d != 128) return INFINI_ERR_UNSUPPORTED;
+    if (N % 64 != 0) return INFINI_ERR_UNSUPPORTED;
+    BwdPlan p;
+    p.B = B; p.H = H; p.Hkv = Hkv; p.L = L; p.N = N; p.d = d;
+    p.S = (L + N - 1) / N;
+    p.T = L - (p.S - 1) * N;
+    p.chains = B * Hkv;
+    p.units = p.chains * p.S;
+    p.qtiles = N / 64;
+    p.rule = rule;
+    p.tc = bwd_uses_tc<T>(d);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaGetLastError();
+    if (take_failed_allocation()) return INFINI_ERR_OOM;
+    cudaMemPool_t pool = workspace_pool();
+    if (!pool) return INFINI_ERR_CUDA;
+    void *ws = nullptr;
+    if (cudaMallocFromPoolAsync(&ws, (size_t)bwd_workspace_bytes(p), pool, st) != cudaSuccess) {
+        cudaGetLastError();
+        return INFINI_ERR_OOM;
+    }
+    const T *tq = static_cast<const T *>(q), *tk = static_cast<const T *>(k),
+            *tv = static_cast<const T *>(v), *tdo = static_cast<const T *>(dout);
+    T *gq = static_cast<T *>(dq), *gk = static_cast<T *>(dk), *gv = static_cast<T *>(dv);
+    int rc;
+    switch (d) {
+    case 32: rc = launch_backward<T, 32>(p, tq, tk, tv, beta, M0, z0, tdo, dM, dz, gq, gk, gv, dbeta, dM0, dz0, ws, st); break;
+    case 64: rc = launch_backward<T, 64>(p, tq, tk, tv, beta, M0, z0, tdo, dM, dz, gq, gk, gv, dbeta, dM0, dz0, ws, st); break;
+    default: rc = launch_backward<T, 128>(p, tq, tk, tv, beta, M0, z0, tdo, dM, dz, gq, gk, gv, dbeta, dM0, dz0, ws, st); break;
+    }
+    if (cudaFreeAsync(ws, st) != cudaSuccess && rc == INFINI_OK) rc = INFINI_ERR_CUDA;
+    return rc;
+}
+
 }  // namespace
 }  // namespace infini
 
@@ -991,6 +1258,26 @@ int infini_attn_fwd(const void *q, const void *k, const void *v, const float *be
 {
     return infini::forward<__nv_bfloat16>(q, k, v, beta, M0, z0, out, M_out, z_out, B, H, Hkv,
                                           L, N, d, update_rule, stream);
+}
+
+int infini_attn_bwd(const void *q, const void *k, const void *v, const float *beta,
+                    const float *M0, const float *z0, const void *dout, const float *dM,
+                    const float *dz, void *dq, void *dk, void *dv, float *dbeta, float *dM0,
+                    float *dz0, int64_t B, int64_t H, int64_t Hkv, int64_t L, int64_t N,
+                    int64_t d, int update_rule, infini_stream_t stream)
+{
+    return infini::backward<__nv_bfloat16>(q, k, v, beta, M0, z0, dout, dM, dz, dq, dk, dv, dbeta,
+                                           dM0, dz0, B, H, Hkv, L, N, d, update_rule, stream);
+}
+
+int infini_attn_bwd_f32(const void *q, const void *k, const void *v, const float *beta,
+                        const float *M0, const float *z0, const void *dout, const float *dM,
+                        const float *dz, void *dq, void *dk, void *dv, float *dbeta, float *dM0,
+                        float *dz0, int64_t B, int64_t H, int64_t Hkv, int64_t L, int64_t N,
+                        int64_t d, int update_rule, infini_stream_t stream)
+{
+    return infini::backward<float>(q, k, v, beta, M0, z0, dout, dM, dz, dq, dk, dv, dbeta, dM0,
+                                   dz0, B, H, Hkv, L, N, d, update_rule, stream);
 }
 
 int infini_attn_fwd_f32(const void *q, const void *k, const void *v, const float *beta,

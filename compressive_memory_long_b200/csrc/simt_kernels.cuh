@@ -12,10 +12,11 @@
 // s, snapM[(c * S + s) * d * d ...] and snapZ[(c * S + s) * d ...] hold (M_{s-1}, z_{s-1}),
 // the memory the segment reads.
 //
-// `valid` is the number of tokens a segment really has (N for every full segment).  A
-// final segment shorter than N runs with N rounded up to 64 and valid = its length: the
-// rows past `valid` are never read (they count as a zero key / value whose feature map is
-// 0, not sigma(0)) and never written.
+// `valid` is the number of tokens the LAST segment of a launch really has (N when it is a
+// full one; every earlier segment has N).  A final segment shorter than N runs with its
+// rows past `valid` never read (they count as a zero key / value whose feature map is 0,
+// not sigma(0)) and never written; the segment kernel runs such a segment alone, with N
+// rounded up to 64.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -49,6 +50,7 @@ k_linear_increments(const T *__restrict__ k, const T *__restrict__ v, float *__r
     __shared__ float sV[TK][D + 1];
     const int64_t chain = blockIdx.x / S;
     const int s = blockIdx.x % S;
+    const int vs = s == S - 1 ? valid : N;          // tokens of this segment
     const T *K = k + (chain * L + (int64_t)s * N) * D;
     const T *V = v + (chain * L + (int64_t)s * N) * D;
     const int tid = threadIdx.x, tx = tid % 16, ty = tid / 16;
@@ -63,7 +65,7 @@ k_linear_increments(const T *__restrict__ k, const T *__restrict__ v, float *__r
     for (int t0 = 0; t0 < N; t0 += TK) {
         for (int i = tid; i < TK * D; i += 256) {
             const int t = i / D, c = i % D;
-            const bool in = t0 + t < valid;
+            const bool in = t0 + t < vs;
             sK[t][c] = in ? feature_map(ld_f(K + (int64_t)(t0 + t) * D + c)) : 0.f;
             sV[t][c] = in ? ld_f(V + (int64_t)(t0 + t) * D + c) : 0.f;
         }
@@ -248,6 +250,7 @@ k_delta_chain(const T *__restrict__ k, const T *__restrict__ v, float *snapM,
         }
         const T *K = k + (chain * L + (int64_t)s * N) * D;
         const T *V = v + (chain * L + (int64_t)s * N) * D;
+        const int vs = s == S - 1 ? valid : N;      // tokens of this segment
         float dm[PER];
 #pragma unroll
         for (int p = 0; p < PER; ++p) dm[p] = 0.f;
@@ -256,11 +259,11 @@ k_delta_chain(const T *__restrict__ k, const T *__restrict__ v, float *snapM,
         for (int t0 = 0; t0 < N; t0 += TK) {
             for (int i = tid; i < TK * D; i += 256) {
                 const int t = i / D, c = i % D;
-                sK[t][c] = t0 + t < valid ? feature_map(ld_f(K + (int64_t)(t0 + t) * D + c)) : 0.f;
+                sK[t][c] = t0 + t < vs ? feature_map(ld_f(K + (int64_t)(t0 + t) * D + c)) : 0.f;
             }
             for (int i = tid; i < TK * CB; i += 256) {
                 const int t = i / CB, e = i % CB;
-                sV[t][e] = t0 + t < valid ? ld_f(V + (int64_t)(t0 + t) * D + cb + e) : 0.f;
+                sV[t][e] = t0 + t < vs ? ld_f(V + (int64_t)(t0 + t) * D + cb + e) : 0.f;
             }
             __syncthreads();
             // den_t = sigma(k_t) . z_{s-1}: one warp per token

@@ -112,26 +112,32 @@ template <int D, bool DELTA>
 struct IncrCfg {
     static_assert(D == 64 || D == 128, "tensor-core memory increments: d = 64 or 128");
     static constexpr int CH = 64;                    // tokens per chunk
-    static constexpr int NB = D / 64;                // 64-column boxes of V and of W
+    static constexpr int NB = D / 64;                // 64-column boxes of K, V and W
     static constexpr int BOX = CH * 128;             // 64 rows x 64 bf16 (128-byte rows)
-    static constexpr int ATILE = 2 * BOX;            // sigma: features padded to 128
-    static constexpr int NBB = DELTA ? 3 * NB : NB;  // B boxes: V | W_hi | W_lo
-    static constexpr int OFF_SH = 0;                 // sigma_hi, written over the K tile
-    static constexpr int OFF_SL = ATILE;             // sigma_lo
-    static constexpr int OFF_B = 2 * ATILE;
-    static constexpr int STAGE = 2 * ATILE + NBB * BOX;
-    static constexpr int ST = 2;
-    static constexpr int OFF_Z = ST * STAGE;         // z_{s-1} (delta)
-    static constexpr int OFF_BAR = OFF_Z + 128 * 4;
-    static constexpr int NBAR = 3 * ST + 1;
+    // ring slot (TMA): the K chunk, turned into sigma_hi in place (features padded to 128:
+    // for d = 64 the second box stays zero), then the V chunk
+    static constexpr int RS = 3;
+    static constexpr int OFF_SH = 0;
+    static constexpr int OFF_V = 2 * BOX;
+    static constexpr int SLOT = (2 + NB) * BOX;
+    // operand set (two, alternating by chunk): sigma_lo (padded like sigma_hi), W_hi, W_lo
+    static constexpr int OFF_SL = 0;
+    static constexpr int OFF_WH = 2 * BOX;
+    static constexpr int OFF_WL = OFF_WH + NB * BOX;
+    static constexpr int OSET = DELTA ? (2 + 2 * NB) * BOX : 2 * BOX;
+    static constexpr int OFF_RING = 0;
+    static constexpr int OFF_OPS = RS * SLOT;
+    static constexpr int OFF_BAR = OFF_OPS + 2 * OSET;
+    static constexpr int NBAR = 3 * RS + 2 + 4 + 1;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int BYTES = OFF_MISC + 16;
     static constexpr int ALLOC = BYTES + 1024;
-    static constexpr int NVW = DELTA ? 2 * D : D;    // N of the [V | W_hi] products
-    static constexpr uint32_t TMEM_COLS = NVW <= 64 ? 64 : (NVW <= 128 ? 128 : 256);
-    static constexpr int THREADS = 384;
+    static constexpr int ACC = DELTA ? 2 * D : D;     // accumulator columns: B_s | A_s
+    static constexpr uint32_t TMEM_COLS = 2 * ACC < 32 ? 32 : 2 * ACC;
+    static constexpr int THREADS = 512;
     static constexpr int FPT = D / 4;                // features per worker thread
-    static_assert(STAGE % 1024 == 0 && BOX % 1024 == 0, "operand tiles must be 1024-aligned");
+    static_assert(SLOT % 1024 == 0 && OSET % 1024 == 0, "operand tiles must be 1024-aligned");
+    static_assert(ALLOC <= 232448, "shared memory");
 };
 
 struct IncrArgs {
@@ -140,9 +146,11 @@ struct IncrArgs {
     __nv_bfloat16 *Ahi, *Alo;  // [chains * S, D, D]: A_s split into two bf16 parts (delta)
     int64_t L;
     int N, S;
+    int items;                 // chains * S
 };
 
-enum : int { WI_KV_EMPTY = 501, WI_KV_FULL = 502, WI_A = 503, WI_ACC = 504, WI_DRAIN = 505 };
+enum : int { WI_EMPTY = 501, WI_FULL = 502, WI_OFREE = 503, WI_AREADY = 504, WI_ACCFREE = 505,
+             WI_ACCFULL = 506, WI_DRAIN = 507 };
 
 __device__ __forceinline__ void incr_drain(uint64_t *bar, uint32_t parity)
 {
@@ -155,223 +163,270 @@ __device__ __forceinline__ void incr_drain(uint64_t *bar, uint32_t parity)
     }
 }
 
-// One CTA per (chain, segment).  Warp 0: TMA producer of 64-token K / V chunks (two stages).
-// Warp 1: MMA issuer.  Warps 4-11: four threads per token row turn the K tile into
-// sigma_hi / sigma_lo (in place / beside it) and, for the delta rule, write W = sigma / den
-// (hi, lo) beside V; after the last chunk they read the accumulators (lane i = key feature i)
-// and store row i of B_s (warps 4-7) and of A_s (warps 8-11).
-// TMEM: columns [0, D) accumulate B_s, [D, 2D) A_s.
+// Persistent: CTA b takes items (chain, segment) b, b + grid, ...; every role walks the same
+// schedule of 64-token chunks, numbered g across the CTA's items.
+//   warp 0       TMA producer: K and V chunks into a ring of RS slots, running ahead across
+//                item boundaries
+//   warp 1       MMA issuer: per chunk, acc += sigma_hi^T [V | W_hi | W_lo] + sigma_lo^T
+//                [V | W_hi] into the item's accumulator set (two sets, alternating by item)
+//   warps 4-11   workers: four threads per token row turn K into sigma_hi (in place) and
+//                sigma_lo and, for the delta rule, den = sigma . z_{s-1} and W = sigma / den
+//                (hi, lo) into the chunk's operand set (two sets, alternating by chunk)
+//   warps 12-15  epilogue: lane i of the item's accumulator is key feature i; row i of B_s
+//                (fp32) and of A_s (bf16 hi, lo) to global memory, while the next item's
+//                MMAs fill the other accumulator set
 template <int D, bool DELTA>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(512, 1)
 k_mem_incr(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
            const IncrArgs a)
 {
     using C = IncrCfg<D, DELTA>;
-    constexpr int ST = C::ST;
+    constexpr int RS = C::RS;
     if (__syncthreads_or(threadIdx.x == 0 && wait_status_set())) return;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
-
-    const int64_t cs = blockIdx.x;                 // chain * S + s
-    const int64_t chain = cs / a.S;
-    const int s = (int)(cs % a.S);
-    const int64_t row0 = (int64_t)s * a.N;
-    const int rows = (int)(a.L - row0 < a.N ? a.L - row0 : a.N);
-    const int nch = (rows + C::CH - 1) / C::CH;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-    float *sZ = reinterpret_cast<float *>(smem + C::OFF_Z);
+    uint8_t *ring = smem + C::OFF_RING, *ops = smem + C::OFF_OPS;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
-    uint64_t *kv_full = bars, *kv_empty = bars + ST, *a_ready = bars + 2 * ST;
-    uint64_t *acc_full = bars + 3 * ST;
+    uint64_t *full = bars, *empty = bars + RS, *aready = bars + 2 * RS;
+    uint64_t *ofree = bars + 3 * RS, *accfull = ofree + 2, *accfree = accfull + 2;
+    uint64_t *mma_done = accfree + 2;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
     volatile int *abort = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < ST; ++i) {
-            mbar_init(kv_full + i, 1);
-            mbar_init(kv_empty + i, 1);
-            mbar_init(a_ready + i, 256);
+        for (int i = 0; i < RS; ++i) {
+            mbar_init(full + i, 1);
+            mbar_init(empty + i, 1);
+            mbar_init(aready + i, 256);
         }
-        mbar_init(acc_full, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(ofree + i, 1);
+            mbar_init(accfull + i, 1);
+            mbar_init(accfree + i, 128);
+        }
+        mbar_init(mma_done, 1);
         *abort = 0;
         fence_barrier_init();
     }
+    if (D == 64)    // the padded feature box of every sigma_hi / sigma_lo tile stays zero
+        for (int i = threadIdx.x; i < (RS + 2) * (C::BOX / 16); i += blockDim.x) {
+            const int t = i / (C::BOX / 16), o = i % (C::BOX / 16);
+            uint8_t *base = t < RS ? ring + t * C::SLOT + C::OFF_SH : ops + (t - RS) * C::OSET + C::OFF_SL;
+            reinterpret_cast<uint4 *>(base + C::BOX)[o] = make_uint4(0, 0, 0, 0);
+        }
     if (warp == 1) tmem_alloc(tmem_holder, C::TMEM_COLS);
+    fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t T = *tmem_holder;
+
+    auto item_rows = [&](int item) {
+        const int64_t row0 = (int64_t)(item % a.S) * a.N;
+        return (int)(a.L - row0 < a.N ? a.L - row0 : a.N);
+    };
 
     if (warp == 0) {
         if (lane == 0) {
             // ------------------------------------------------------------ producer
             prefetch_tmap(&tmK);
             prefetch_tmap(&tmV);
-            int issued = 0;
-            for (int g = 0; g < nch; ++g) {
-                const int st = g % ST;
-                if (g >= ST && !mbar_wait_short(kv_empty + st, ((g / ST) - 1) & 1, abort, WI_KV_EMPTY))
-                    break;
-                uint8_t *stage = smem + st * C::STAGE;
-                const int row = (int)row0 + g * C::CH;
-                mbar_arrive_expect_tx(kv_full + st, (uint32_t)(2 * C::NB * C::BOX));
-                for (int b = 0; b < C::NB; ++b) {
-                    tma_load_3d(stage + C::OFF_SH + b * C::BOX, &tmK, kv_full + st, b * 64, row,
-                                (int)chain);
-                    tma_load_3d(stage + C::OFF_B + b * C::BOX, &tmV, kv_full + st, b * 64, row,
-                                (int)chain);
+            int g = 0, issued = 0;
+            bool ok = true;
+            for (int item = blockIdx.x; ok && item < a.items; item += gridDim.x) {
+                const int chain = item / a.S, row0 = (item % a.S) * a.N;
+                const int nch = (item_rows(item) + C::CH - 1) / C::CH;
+                for (int c = 0; c < nch; ++c, ++g) {
+                    const int st = g % RS;
+                    if (g >= RS && !(ok = mbar_wait_short(empty + st, ((g / RS) - 1) & 1, abort, WI_EMPTY)))
+                        break;
+                    uint8_t *slot = ring + st * C::SLOT;
+                    mbar_arrive_expect_tx(full + st, (uint32_t)(2 * C::NB * C::BOX));
+                    for (int b = 0; b < C::NB; ++b) {
+                        tma_load_3d(slot + C::OFF_SH + b * C::BOX, &tmK, full + st, b * 64,
+                                    row0 + c * C::CH, chain);
+                        tma_load_3d(slot + C::OFF_V + b * C::BOX, &tmV, full + st, b * 64,
+                                    row0 + c * C::CH, chain);
+                    }
+                    issued = g + 1;
                 }
-                issued = g + 1;
             }
             if (*abort)
-                for (int g = (issued > ST ? issued - ST : 0); g < issued; ++g)
-                    incr_drain(kv_full + g % ST, (g / ST) & 1);
+                for (int h = (issued > RS ? issued - RS : 0); h < issued; ++h)
+                    incr_drain(full + h % RS, (h / RS) & 1);
         }
     } else if (warp == 1) {
         if (lane == 0) {
             // ------------------------------------------------------------ MMA issuer
-            constexpr uint32_t idVW = idesc_bf16(128, C::NVW, 1, 1);   // sigma^T [V | W_hi]
-            constexpr uint32_t idWl = idesc_bf16(128, D, 1, 1);        // sigma_hi^T W_lo
-            const uint32_t base = smem_u32(smem);
-            for (int g = 0; g < nch; ++g) {
-                const int st = g % ST;
-                if (!mbar_wait_short(a_ready + st, (g / ST) & 1, abort, WI_A)) break;
-                tc_fence_after();
-                const uint32_t sb = base + st * C::STAGE;
+            constexpr uint32_t id = idesc_bf16(128, D, 1, 1);      // both operands MN-major
+            const uint32_t aRing = smem_u32(ring), aOps = smem_u32(ops);
+            int g = 0, j = 0;
+            bool ok = true;
+            for (int item = blockIdx.x; ok && item < a.items; item += gridDim.x, ++j) {
+                const int nch = (item_rows(item) + C::CH - 1) / C::CH;
+                const uint32_t acc = T + (j & 1) * C::ACC;
+                // the epilogue of item j - 2 has read this accumulator set
+                if (j >= 2 && !(ok = mbar_wait_short(accfree + (j & 1), ((j >> 1) - 1) & 1, abort, WI_ACCFREE)))
+                    break;
+                for (int c = 0; c < nch; ++c, ++g) {
+                    const int st = g % RS;
+                    if (!(ok = mbar_wait_short(aready + st, (g / RS) & 1, abort, WI_AREADY))) break;
+                    tc_fence_after();
+                    const uint32_t sl = aRing + st * C::SLOT, os = aOps + (g & 1) * C::OSET;
 #pragma unroll
-                for (int kk = 0; kk < C::CH / 16; ++kk) {       // 16 tokens per step
-                    const uint64_t ah = sdesc_sw128(sb + C::OFF_SH + kk * 2048, C::BOX, 1024);
-                    const uint64_t al = sdesc_sw128(sb + C::OFF_SL + kk * 2048, C::BOX, 1024);
-                    const uint64_t bvw = sdesc_sw128(sb + C::OFF_B + kk * 2048, C::BOX, 1024);
-                    mma_ss(T, ah, bvw, idVW, (g > 0 || kk > 0) ? 1u : 0u);
-                    mma_ss(T, al, bvw, idVW, 1u);
-                    if constexpr (DELTA) {
-                        const uint64_t bwl =
-                            sdesc_sw128(sb + C::OFF_B + 2 * C::NB * C::BOX + kk * 2048, C::BOX, 1024);
-                        mma_ss(T + D, ah, bwl, idWl, 1u);
+                    for (int kk = 0; kk < C::CH / 16; ++kk) {       // 16 tokens per step
+                        const uint32_t k2 = kk * 2048;
+                        const uint64_t ah = sdesc_sw128(sl + C::OFF_SH + k2, C::BOX, 1024);
+                        const uint64_t al = sdesc_sw128(os + C::OFF_SL + k2, C::BOX, 1024);
+                        const uint64_t bv = sdesc_sw128(sl + C::OFF_V + k2, C::BOX, 1024);
+                        const uint32_t first = (c > 0 || kk > 0) ? 1u : 0u;
+                        mma_ss(acc, ah, bv, id, first);
+                        mma_ss(acc, al, bv, id, 1u);
+                        if constexpr (DELTA) {
+                            const uint64_t bwh = sdesc_sw128(os + C::OFF_WH + k2, C::BOX, 1024);
+                            const uint64_t bwl = sdesc_sw128(os + C::OFF_WL + k2, C::BOX, 1024);
+                            mma_ss(acc + D, ah, bwh, id, first);
+                            mma_ss(acc + D, al, bwh, id, 1u);
+                            mma_ss(acc + D, ah, bwl, id, 1u);
+                        }
                     }
+                    mma_commit(empty + st);
+                    mma_commit(ofree + (g & 1));
                 }
-                mma_commit(kv_empty + st);
+                if (ok) mma_commit(accfull + (j & 1));
             }
-            mma_commit(acc_full);
-            incr_drain(acc_full, 0);
+            mma_commit(mma_done);
+            incr_drain(mma_done, 0);
         }
-    } else if (warp >= 4) {
+    } else if (warp >= 4 && warp < 12) {
         // ---------------------------------------------------------------- workers
         const int w = threadIdx.x - 128;            // 0..255
         const int t = w >> 2, q = w & 3;            // token row of the chunk, feature quarter
         const int f0 = q * C::FPT;                  // first feature of this thread
         const int box = f0 >> 6, cq = (f0 & 63) >> 3;
         constexpr int CPT = C::FPT / 8;             // 16-byte chunks per thread
-        if constexpr (DELTA)
-            for (int i = w; i < D; i += 256) sZ[i] = a.snapZ[cs * D + i];
-        if (D == 64)    // the padded feature box of sigma_hi / sigma_lo stays zero
-            for (int i = w; i < ST * 2 * (C::BOX / 16); i += 256) {
-                const int st = i / (2 * (C::BOX / 16)), o = i % (2 * (C::BOX / 16));
-                const int which = o / (C::BOX / 16), oo = o % (C::BOX / 16);
-                reinterpret_cast<uint4 *>(smem + st * C::STAGE + which * C::ATILE + C::BOX)[oo] =
-                    make_uint4(0, 0, 0, 0);
-            }
-        asm volatile("bar.sync 1, 256;" ::: "memory");
-
+        int g = 0, j = 0;
         bool ok = true;
-        for (int g = 0; g < nch; ++g) {
-            const int st = g % ST;
-            if (!(ok = mbar_wait(kv_full + st, (g / ST) & 1, abort, WI_KV_FULL))) break;
-            uint8_t *stage = smem + st * C::STAGE;
-            // rows past the head's L (zero-filled by TMA) carry sigma = 0
-            const uint32_t keep = g * C::CH + t < rows ? 0xFFFFFFFFu : 0u;
-            float sg[C::FPT];
-#pragma unroll
-            for (int i = 0; i < CPT; ++i) {
-                const int off = box * C::BOX + t * 128 + (((cq + i) ^ (t & 7)) << 4);
-                uint4 *ph = reinterpret_cast<uint4 *>(stage + C::OFF_SH + off);
-                const uint4 v = *ph;
-                const uint32_t in[4] = {v.x, v.y, v.z, v.w};
-                uint32_t hi[4], lo[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162 *>(&in[e]);
-                    const float s0 = __uint_as_float(__float_as_uint(elu1(__low2float(x))) & keep);
-                    const float s1 = __uint_as_float(__float_as_uint(elu1(__high2float(x))) & keep);
-                    sg[i * 8 + 2 * e] = s0;
-                    sg[i * 8 + 2 * e + 1] = s1;
-                    const __nv_bfloat162 h = __floats2bfloat162_rn(s0, s1);
-                    hi[e] = *reinterpret_cast<const uint32_t *>(&h);
-                    lo[e] = pack_bf16x2(s0 - __low2float(h), s1 - __high2float(h));
-                }
-                *ph = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-                *reinterpret_cast<uint4 *>(stage + C::OFF_SL + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-            }
+        for (int item = blockIdx.x; ok && item < a.items; item += gridDim.x, ++j) {
+            const int rows = item_rows(item);
+            const int nch = (rows + C::CH - 1) / C::CH;
+            // z_{s-1} at this thread's features (no block-wide barrier: a worker that gives up
+            // on a wait must not leave the others waiting at one)
+            float zr[C::FPT];
             if constexpr (DELTA) {
-                float den = 0.f;
+                const float4 *zp = reinterpret_cast<const float4 *>(a.snapZ + (int64_t)item * D + f0);
 #pragma unroll
-                for (int e = 0; e < C::FPT; ++e) den = fmaf(sg[e], sZ[f0 + e], den);
-                den += __shfl_xor_sync(0xffffffffu, den, 1);
-                den += __shfl_xor_sync(0xffffffffu, den, 2);
-                const float inv = den == 0.f ? 0.f : 1.f / den;
+                for (int e = 0; e < C::FPT / 4; ++e) {
+                    const float4 x = __ldg(zp + e);
+                    zr[4 * e] = x.x;
+                    zr[4 * e + 1] = x.y;
+                    zr[4 * e + 2] = x.z;
+                    zr[4 * e + 3] = x.w;
+                }
+            }
+            for (int c = 0; c < nch; ++c, ++g) {
+                const int st = g % RS;
+                if (!(ok = mbar_wait(full + st, (g / RS) & 1, abort, WI_FULL))) break;
+                if (g >= 2 && !(ok = mbar_wait(ofree + (g & 1), ((g >> 1) - 1) & 1, abort, WI_OFREE)))
+                    break;
+                uint8_t *slot = ring + st * C::SLOT, *os = ops + (g & 1) * C::OSET;
+                // rows past the head's L (zero-filled by TMA) carry sigma = 0
+                const uint32_t keep = c * C::CH + t < rows ? 0xFFFFFFFFu : 0u;
+                float sg[C::FPT];
 #pragma unroll
                 for (int i = 0; i < CPT; ++i) {
                     const int off = box * C::BOX + t * 128 + (((cq + i) ^ (t & 7)) << 4);
+                    uint4 *ph = reinterpret_cast<uint4 *>(slot + C::OFF_SH + off);
+                    const uint4 v = *ph;
+                    const uint32_t in[4] = {v.x, v.y, v.z, v.w};
                     uint32_t hi[4], lo[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const float w0 = sg[i * 8 + 2 * e] * inv, w1 = sg[i * 8 + 2 * e + 1] * inv;
-                        const __nv_bfloat162 h = __floats2bfloat162_rn(w0, w1);
+                        const __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162 *>(&in[e]);
+                        const float s0 = __uint_as_float(__float_as_uint(elu1(__low2float(x))) & keep);
+                        const float s1 = __uint_as_float(__float_as_uint(elu1(__high2float(x))) & keep);
+                        sg[i * 8 + 2 * e] = s0;
+                        sg[i * 8 + 2 * e + 1] = s1;
+                        const __nv_bfloat162 h = __floats2bfloat162_rn(s0, s1);
                         hi[e] = *reinterpret_cast<const uint32_t *>(&h);
-                        lo[e] = pack_bf16x2(w0 - __low2float(h), w1 - __high2float(h));
+                        lo[e] = pack_bf16x2(s0 - __low2float(h), s1 - __high2float(h));
                     }
-                    *reinterpret_cast<uint4 *>(stage + C::OFF_B + C::NB * C::BOX + off) =
-                        make_uint4(hi[0], hi[1], hi[2], hi[3]);
-                    *reinterpret_cast<uint4 *>(stage + C::OFF_B + 2 * C::NB * C::BOX + off) =
-                        make_uint4(lo[0], lo[1], lo[2], lo[3]);
+                    *ph = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                    *reinterpret_cast<uint4 *>(os + C::OFF_SL + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
                 }
+                if constexpr (DELTA) {
+                    float den = 0.f;
+#pragma unroll
+                    for (int e = 0; e < C::FPT; ++e) den = fmaf(sg[e], zr[e], den);
+                    den += __shfl_xor_sync(0xffffffffu, den, 1);
+                    den += __shfl_xor_sync(0xffffffffu, den, 2);
+                    const float inv = den == 0.f ? 0.f : 1.f / den;
+#pragma unroll
+                    for (int i = 0; i < CPT; ++i) {
+                        const int off = box * C::BOX + t * 128 + (((cq + i) ^ (t & 7)) << 4);
+                        uint32_t hi[4], lo[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float w0 = sg[i * 8 + 2 * e] * inv, w1 = sg[i * 8 + 2 * e + 1] * inv;
+                            const __nv_bfloat162 h = __floats2bfloat162_rn(w0, w1);
+                            hi[e] = *reinterpret_cast<const uint32_t *>(&h);
+                            lo[e] = pack_bf16x2(w0 - __low2float(h), w1 - __high2float(h));
+                        }
+                        *reinterpret_cast<uint4 *>(os + C::OFF_WH + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                        *reinterpret_cast<uint4 *>(os + C::OFF_WL + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+                    }
+                }
+                fence_proxy_async_smem();
+                mbar_arrive(aready + st);
             }
-            fence_proxy_async_smem();
-            mbar_arrive(a_ready + st);
         }
-        // ---- epilogue: lane i of the accumulator is key feature i
-        if (ok) ok = mbar_wait(acc_full, 0, abort, WI_ACC);
-        if (ok) {
+    } else if (warp >= 12) {
+        // ---------------------------------------------------------------- epilogue
+        const int i = (warp & 3) * 32 + lane;
+        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+        const bool live = D == 128 || (warp & 3) < 2;      // lanes past d hold nothing
+        int j = 0;
+        for (int item = blockIdx.x; item < a.items; item += gridDim.x, ++j) {
+            if (!mbar_wait(accfull + (j & 1), (j >> 1) & 1, abort, WI_ACCFULL)) break;
             tc_fence_after();
-            const int i = (warp & 3) * 32 + lane;
-            const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-            const bool second = warp >= 8;              // warps 8-11: A_s (delta)
-            if (!second || DELTA) {
-                if (D == 128 || (warp & 3) < 2) {       // lanes past d hold nothing
+            const uint32_t acc = T + (j & 1) * C::ACC;
+            if (live) {
 #pragma unroll 1
-                    for (int c0 = 0; c0 < D; c0 += 32) {
-                        uint32_t r[32];
-                        tmem_ld32(lane_base + T + (second ? D : 0) + c0, r);
-                        tmem_ld_wait();
-                        const int64_t o = (cs * D + i) * D + c0;
-                        if (!second) {
-                            float4 *dst = reinterpret_cast<float4 *>(a.Bs + o);
+                for (int c0 = 0; c0 < C::ACC; c0 += 32) {
+                    uint32_t r[32];
+                    tmem_ld32(lane_base + acc + c0, r);
+                    tmem_ld_wait();
+                    const int col = c0 % D;
+                    const int64_t o = ((int64_t)item * D + i) * D + col;
+                    if (c0 < D) {
+                        float4 *dst = reinterpret_cast<float4 *>(a.Bs + o);
 #pragma unroll
-                            for (int e = 0; e < 8; ++e)
-                                dst[e] = make_float4(__uint_as_float(r[4 * e]), __uint_as_float(r[4 * e + 1]),
-                                                     __uint_as_float(r[4 * e + 2]), __uint_as_float(r[4 * e + 3]));
-                        } else {
-                            uint32_t hi[16], lo[16];
+                        for (int e = 0; e < 8; ++e)
+                            dst[e] = make_float4(__uint_as_float(r[4 * e]), __uint_as_float(r[4 * e + 1]),
+                                                 __uint_as_float(r[4 * e + 2]), __uint_as_float(r[4 * e + 3]));
+                    } else {
+                        uint32_t hi[16], lo[16];
 #pragma unroll
-                            for (int e = 0; e < 16; ++e) {
-                                const float x0 = __uint_as_float(r[2 * e]), x1 = __uint_as_float(r[2 * e + 1]);
-                                const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
-                                hi[e] = *reinterpret_cast<const uint32_t *>(&h);
-                                lo[e] = pack_bf16x2(x0 - __low2float(h), x1 - __high2float(h));
-                            }
-                            uint4 *dh = reinterpret_cast<uint4 *>(a.Ahi + o);
-                            uint4 *dl = reinterpret_cast<uint4 *>(a.Alo + o);
+                        for (int e = 0; e < 16; ++e) {
+                            const float x0 = __uint_as_float(r[2 * e]), x1 = __uint_as_float(r[2 * e + 1]);
+                            const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+                            hi[e] = *reinterpret_cast<const uint32_t *>(&h);
+                            lo[e] = pack_bf16x2(x0 - __low2float(h), x1 - __high2float(h));
+                        }
+                        uint4 *dh = reinterpret_cast<uint4 *>(a.Ahi + o);
+                        uint4 *dl = reinterpret_cast<uint4 *>(a.Alo + o);
 #pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                dh[e] = make_uint4(hi[4 * e], hi[4 * e + 1], hi[4 * e + 2], hi[4 * e + 3]);
-                                dl[e] = make_uint4(lo[4 * e], lo[4 * e + 1], lo[4 * e + 2], lo[4 * e + 3]);
-                            }
+                        for (int e = 0; e < 4; ++e) {
+                            dh[e] = make_uint4(hi[4 * e], hi[4 * e + 1], hi[4 * e + 2], hi[4 * e + 3]);
+                            dl[e] = make_uint4(lo[4 * e], lo[4 * e + 1], lo[4 * e + 2], lo[4 * e + 3]);
                         }
                     }
                 }
             }
+            tc_fence_before();
+            mbar_arrive(accfree + (j & 1));
         }
     }
 
@@ -386,12 +441,13 @@ k_mem_incr(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUte
 // ---------------------------------------------------------------- the serial parts
 
 // Additive rule: M_{s-1} = M0 + sum_{j<s} B_j.  One thread per 4 consecutive elements of a
-// chain's M walks the segments, writing the bf16 snapshot of every M_{s-1} and M_out.  Each
+// chain's M walks the segments, writing the snapshot of every M_{s-1} (bf16 and / or fp32)
+// and M_out.  Each
 // element is read from M0 and written to M_out by the same thread, so they may alias.
 template <int D>
 __global__ void __launch_bounds__(256)
 k_mem_prefix(const float *__restrict__ Bs, const float *M0, __nv_bfloat16 *__restrict__ snapMb,
-             float *M_out, int S, int64_t chains)
+             float *M_out, int S, int64_t chains, float *__restrict__ snapMf = nullptr)
 {
     constexpr int64_t E4 = (int64_t)D * D / 4;
     const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
@@ -399,10 +455,12 @@ k_mem_prefix(const float *__restrict__ Bs, const float *M0, __nv_bfloat16 *__res
     const int64_t chain = i / E4, e = i % E4;
     float4 m = M0 ? reinterpret_cast<const float4 *>(M0)[i] : make_float4(0.f, 0.f, 0.f, 0.f);
     const float4 *b = reinterpret_cast<const float4 *>(Bs) + chain * S * E4 + e;
-    uint2 *snap = reinterpret_cast<uint2 *>(snapMb) + chain * S * E4 + e;
+    uint2 *snap = snapMb ? reinterpret_cast<uint2 *>(snapMb) + chain * S * E4 + e : nullptr;
+    float4 *snapf = snapMf ? reinterpret_cast<float4 *>(snapMf) + chain * S * E4 + e : nullptr;
 #pragma unroll 4
     for (int s = 0; s < S; ++s) {
-        snap[(int64_t)s * E4] = make_uint2(pack_bf16x2(m.x, m.y), pack_bf16x2(m.z, m.w));
+        if (snap) snap[(int64_t)s * E4] = make_uint2(pack_bf16x2(m.x, m.y), pack_bf16x2(m.z, m.w));
+        if (snapf) snapf[(int64_t)s * E4] = m;
         const float4 x = b[(int64_t)s * E4];
         m.x += x.x;
         m.y += x.y;
@@ -419,7 +477,7 @@ struct MChainCfg {
     static constexpr int NK = D / 64;               // 64-wide boxes along the contraction
     static constexpr int ABOX = 128 * 128;          // 128 rows x 64 bf16
     static constexpr int ATILE = NK * ABOX;         // A_hi (or A_lo) of one segment
-    static constexpr int ST = 2;
+    static constexpr int ST = 3;                    // A_s loads run this many segments ahead
     static constexpr int BBOX = CB * 128;           // CB rows x 64 bf16 (K-major M^T)
     static constexpr int BTILE = NK * BBOX;
     static constexpr int OFF_A = 0;                 // per stage: A_hi | A_lo
@@ -430,14 +488,17 @@ struct MChainCfg {
     static constexpr int BYTES = OFF_MISC + 16;
     static constexpr int ALLOC = BYTES + 1024;
     static_assert(OFF_B % 1024 == 0 && BTILE % 1024 == 0, "operand tiles must be 1024-aligned");
+    static_assert(ALLOC <= 232448, "shared memory");
 };
 
 struct MChainArgs {
     const float *M0;           // may be NULL (zeros); may alias M_out exactly
     const float *Bs;           // [chains * S, D, D]
-    __nv_bfloat16 *snapMb;     // [chains * S, D, D]: bf16 M_{s-1}
+    __nv_bfloat16 *snapMb;     // [chains * S, D, D]: bf16 M_{s-1}, or NULL
+    float *snapMf;             // [chains * S, D, D]: fp32 M_{s-1}, or NULL
     float *M_out;
     int S;
+    int reverse;               // walk the segments from the last to the first
 };
 
 enum : int { WM_A_EMPTY = 601, WM_B = 602, WM_A_FULL = 603, WM_D = 604, WM_DRAIN = 605 };
@@ -453,7 +514,9 @@ __device__ __forceinline__ void mchain_drain(uint64_t *bar, uint32_t parity)
     }
 }
 
-// Delta rule: M_s = M_{s-1} + B_s - A_s M_{s-1} in segment order.  One CTA per (chain, 32
+// Delta rule: M_s = M_{s-1} + B_s - A_s M_{s-1} in segment order (with `reverse`, from the
+// last segment to the first: the backward's dM_{s-1} = dM_s + G_s - A_s dM_s, A_s being
+// symmetric; the snapshot of each step is then the gradient after the segment).  One CTA per (chain, 32
 // value columns); column block j of M_s needs only column block j of M_{s-1}.  Warp 0: TMA
 // of A_s (hi and lo parts, K-major, two stages ahead).  Warp 1: MMA issuer, D = A_hi M_hi +
 // A_hi M_lo + A_lo M_hi into 32 TMEM columns.  Warps 4-7: thread i holds row i of the block
@@ -514,7 +577,7 @@ k_mem_chain(const __grid_constant__ CUtensorMap tmAh, const __grid_constant__ CU
                 if (s >= ST && !mbar_wait_short(a_empty + st, ((s / ST) - 1) & 1, abort, WM_A_EMPTY))
                     break;
                 uint8_t *dst = smem + C::OFF_A + st * 2 * C::ATILE;
-                const int slot = (int)(chain * a.S + s);
+                const int slot = (int)(chain * a.S + (a.reverse ? a.S - 1 - s : s));
                 mbar_arrive_expect_tx(a_full + st, (uint32_t)(2 * C::NK * D * 128));
                 for (int b = 0; b < C::NK; ++b) {
                     tma_load_3d(dst + b * C::ABOX, &tmAh, a_full + st, b * 64, 0, slot);
@@ -575,15 +638,23 @@ k_mem_chain(const __grid_constant__ CUtensorMap tmAh, const __grid_constant__ CU
         const int kb = i >> 6, kc = i & 63;
         bool ok = true;
         for (int s = 0; s < a.S; ++s) {
-            const int64_t slot = chain * a.S + s;
+            const int64_t slot = chain * a.S + (a.reverse ? a.S - 1 - s : s);
             if (live) {
-                uint32_t pk[CB / 2];
+                if (a.snapMb) {
+                    uint32_t pk[CB / 2];
 #pragma unroll
-                for (int e = 0; e < CB / 2; ++e) pk[e] = pack_bf16x2(m[2 * e], m[2 * e + 1]);
-                uint4 *dst = reinterpret_cast<uint4 *>(a.snapMb + (slot * D + i) * D + cb);
+                    for (int e = 0; e < CB / 2; ++e) pk[e] = pack_bf16x2(m[2 * e], m[2 * e + 1]);
+                    uint4 *dst = reinterpret_cast<uint4 *>(a.snapMb + (slot * D + i) * D + cb);
 #pragma unroll
-                for (int e = 0; e < CB / 8; ++e)
-                    dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+                    for (int e = 0; e < CB / 8; ++e)
+                        dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+                }
+                if (a.snapMf) {
+                    float4 *dst = reinterpret_cast<float4 *>(a.snapMf + (slot * D + i) * D + cb);
+#pragma unroll
+                    for (int e = 0; e < CB / 4; ++e)
+                        dst[e] = make_float4(m[4 * e], m[4 * e + 1], m[4 * e + 2], m[4 * e + 3]);
+                }
 #pragma unroll
                 for (int j = 0; j < CB; ++j) {
                     const __nv_bfloat16 hi = __float2bfloat16_rn(m[j]);
@@ -602,7 +673,8 @@ k_mem_chain(const __grid_constant__ CUtensorMap tmAh, const __grid_constant__ CU
 #pragma unroll
                 for (int e = 0; e < CB / 4; ++e) bs[e] = src[e];
             }
-            if (!(ok = mbar_wait(d_full, s & 1, abort, WM_D))) break;
+            // on the serial path: probe without the suspend hint
+            if (!(ok = mbar_wait_short(d_full, s & 1, abort, WM_D))) break;
             tc_fence_after();
             uint32_t r[32];
             tmem_ld32(lane_base + T, r);

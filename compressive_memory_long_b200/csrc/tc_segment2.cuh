@@ -8,7 +8,9 @@
 // both read the same K/V tiles, which are loaded once.  Tile B needs key tiles 0..2p+1,
 // tile A 0..2p.  Two softmax warpgroups (A: warps 0-3, B: warps 4-7) work in ping-pong
 // with the tensor core: while one warpgroup turns its S tile into P, the MMA thread
-// (warp 9) runs the other tile's P V and Q K^T.  TMA producer: warp 8; warps 10-11 idle.
+// (warp 9) runs the other tile's P V and Q K^T.  TMA producer: warp 8 (thread 0 issues the
+// first loads right after the barriers exist, ahead of the TMEM allocation and the block
+// barrier); warps 10-11 only lend their registers.
 // The third warpgroup hands registers to the two softmax warpgroups (setmaxnreg), which
 // hold a full 128-score row each.
 //
@@ -64,17 +66,6 @@ __device__ __forceinline__ void seg2_drain(uint64_t *bar, uint32_t parity)
             return;
         }
     }
-}
-
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16])
-{
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
-        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
-        "r"(r[15])
-        : "memory");
 }
 
 template <int D>
@@ -135,6 +126,29 @@ k_segment_tc2(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         mbar_init(mma_done, 1);
         *abort = 0;
         fence_barrier_init();
+        // the first loads go out now, overlapping the TMEM allocation and the block barrier
+        prefetch_tmap(&tmQ);
+        prefetch_tmap(&tmK);
+        prefetch_tmap(&tmV);
+        prefetch_tmap(&tmM);
+        mbar_arrive_expect_tx(q_full, 2 * C::TILE);
+        for (int x = 0; x < 2; ++x)
+            for (int cb = 0; cb < D / 64; ++cb)
+                tma_load_3d(sQ[x] + cb * C::BOX, &tmQ, q_full, cb * 64, s * a.N + p * 256 + x * 128,
+                            (int)bh);
+        for (int j = 0; j < nB && j < ST; ++j) {
+            mbar_arrive_expect_tx(k_full + j, C::TILE);
+            for (int cb = 0; cb < D / 64; ++cb)
+                tma_load_3d(sK + j * C::TILE + cb * C::BOX, &tmK, k_full + j, cb * 64,
+                            s * a.N + j * 128, (int)chain);
+            mbar_arrive_expect_tx(v_full + j, C::TILE);
+            for (int cb = 0; cb < D / 64; ++cb)
+                tma_load_3d(sV + j * C::TILE + cb * C::BOX, &tmV, v_full + j, cb * 64,
+                            s * a.N + j * 128, (int)chain);
+        }
+        mbar_arrive_expect_tx(m_full, C::MBYTES);
+        for (int cb = 0; cb < D / 64; ++cb)
+            tma_load_3d(sM + cb * C::MBOX, &tmM, m_full, cb * 64, 0, (int)(chain * a.S + s));
     }
     if (warp == 9) tmem_alloc(tmem_holder, 512);
     tc_fence_before();
@@ -149,21 +163,10 @@ k_segment_tc2(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       if (warp == 8) {
         if (lane == 0) {
             // ------------------------------------------------------------ producer
-            prefetch_tmap(&tmQ);
-            prefetch_tmap(&tmK);
-            prefetch_tmap(&tmV);
-            prefetch_tmap(&tmM);
-            const int q_row = s * a.N + p * 256;
+            // Q, M and the first ST key / value tiles were issued by thread 0
             const int kv_row0 = s * a.N;
-            mbar_arrive_expect_tx(q_full, 2 * C::TILE);
-            for (int x = 0; x < 2; ++x)
-                for (int cb = 0; cb < D / 64; ++cb)
-                    tma_load_3d(sQ[x] + cb * C::BOX, &tmQ, q_full, cb * 64, q_row + x * 128, (int)bh);
-            mbar_arrive_expect_tx(m_full, C::MBYTES);
-            for (int cb = 0; cb < D / 64; ++cb)
-                tma_load_3d(sM + cb * C::MBOX, &tmM, m_full, cb * 64, 0, (int)(chain * a.S + s));
-            int issued = 0;
-            for (int j = 0; j < nB; ++j) {
+            int issued = nB < ST ? nB : ST;
+            for (int j = issued; j < nB; ++j) {
                 const int st = j % ST;
                 if (j >= ST && !mbar_wait(kv_empty + st, ((j / ST) - 1) & 1, abort, W2_KV_EMPTY))
                     break;
@@ -351,7 +354,7 @@ k_segment_tc2(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         if (ok) ok = mbar_wait(q_full, 0, abort, W2_Q);
         if (ok) {
             tc_fence_after();
-            float den = 0.f;
+            float dp[4] = {0.f, 0.f, 0.f, 0.f};       // sigma(q) . z in four partial sums
             uint8_t *q = sQ[x];
 #pragma unroll
             for (int cb = 0; cb < D / 64; ++cb) {
@@ -367,8 +370,7 @@ k_segment_tc2(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                         x0 = elu1(x0);
                         x1 = elu1(x1);
                         const int c = cb * 64 + ch * 8 + 2 * e;
-                        den = fmaf(x0, sZ[c], den);
-                        den = fmaf(x1, sZ[c + 1], den);
+                        dp[e] = fmaf(x1, sZ[c + 1], fmaf(x0, sZ[c], dp[e]));
                         w[e] = pack_bf16x2(x0, x1);
                     }
                     *ptr = make_uint4(w[0], w[1], w[2], w[3]);
@@ -376,6 +378,7 @@ k_segment_tc2(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             }
             fence_proxy_async_smem();
             mbar_arrive(sq_full + x);
+            const float den = (dp[0] + dp[1]) + (dp[2] + dp[3]);
             if (mbar_wait(r_full + x, 0, abort, W2_R)) {
                 tc_fence_after();
                 const float g = 1.f / (1.f + __expf(-a.beta[h]));

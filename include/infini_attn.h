@@ -97,6 +97,38 @@ INFINI_API int infini_attn_fwd_f32(const void *q, const void *k, const void *v, 
                         int64_t d, int update_rule, infini_stream_t stream);
 
 /*
+ * Backward pass: the gradients of  <dout, out> + <dM, M_out> + <dz, z_out>  of the forward
+ * above (same q, k, v, beta, M0, z0, N, update rule) with respect to every input, through
+ * the local attention, the retrieval, the gate and the memory recurrence of every segment
+ * (AI Wiki "Infini-Attention", "How is an Infini-attention model trained?": gradients flow
+ * through the memory from segment to segment).  A quotient whose denominator is 0 (an
+ * empty memory) is 0 and passes no gradient.
+ *
+ *   dout [B, H, L, d] (activation dtype): gradient of out;  dM [B, Hkv, d, d], dz [B, Hkv, d]
+ *     fp32: gradients of M_out, z_out (NULL = zero)
+ *   dq [B, H, L, d], dk / dv [B, Hkv, L, d] (activation dtype), dbeta [H], dM0 [B, Hkv, d, d],
+ *     dz0 [B, Hkv, d] fp32: written; dbeta, dM0 and dz0 may be NULL (not written)
+ *
+ * infini_attn_bwd takes bf16 activations, infini_attn_bwd_f32 fp32 ones; all arithmetic is
+ * fp32.  Outputs must not overlap any input or each other.  The call recomputes the
+ * forward's memory and softmax statistics itself and allocates its workspace (fp32, about
+ * 4 x (q + 3 k) bytes plus 3 memory snapshots per segment) like the forward.  Shapes,
+ * alignment, streams and errors as for infini_attn_fwd.
+ */
+INFINI_API int infini_attn_bwd(const void *q, const void *k, const void *v, const float *beta,
+                               const float *M0, const float *z0, const void *dout,
+                               const float *dM, const float *dz, void *dq, void *dk, void *dv,
+                               float *dbeta, float *dM0, float *dz0, int64_t B, int64_t H,
+                               int64_t Hkv, int64_t L, int64_t N, int64_t d, int update_rule,
+                               infini_stream_t stream);
+INFINI_API int infini_attn_bwd_f32(const void *q, const void *k, const void *v,
+                                   const float *beta, const float *M0, const float *z0,
+                                   const void *dout, const float *dM, const float *dz, void *dq,
+                                   void *dk, void *dv, float *dbeta, float *dM0, float *dz0,
+                                   int64_t B, int64_t H, int64_t Hkv, int64_t L, int64_t N,
+                                   int64_t d, int update_rule, infini_stream_t stream);
+
+/*
  * The memory after the whole sequence, without the outputs (bf16 keys / values; the _f32
  * variant takes fp32 ones): M_out / z_out exactly as infini_attn_fwd would leave them, from
  * the forward's memory kernels alone.  With M0 = z0 = NULL this is the increment of a

@@ -179,3 +179,29 @@ def call_state(entry="infini_attn_state", B=1, Hkv=2, L=128, N=64, d=64, rule=0,
 ])
 def test_state_argument_errors(entry, kw, status):
     assert call_state(entry, **kw) == status
+
+
+BWD_PTRS = ["q", "k", "v", "beta", "M0", "z0", "dout", "dM", "dz", "dq", "dk", "dv", "dbeta",
+            "dM0", "dz0"]
+
+
+def call_bwd(entry="infini_attn_bwd", B=1, H=2, Hkv=2, L=128, N=64, d=64, rule=0, **ptr):
+    gap = 1 << 32
+    p = {name: BASE + i * gap for i, name in enumerate(BWD_PTRS)}
+    p.update(ptr)
+    a = [None if p[x] is None else ctypes.c_void_p(p[x]) for x in BWD_PTRS]
+    return getattr(binding.LIB, entry)(*a, B, H, Hkv, L, N, d, rule, None)
+
+
+@pytest.mark.parametrize("entry", ["infini_attn_bwd", "infini_attn_bwd_f32"])
+@pytest.mark.parametrize("kw,status", [
+    *[(dict({n: None}), INVALID) for n in ("q", "k", "v", "beta", "dout", "dq", "dk", "dv")],
+    (dict(B=0), INVALID), (dict(H=3, Hkv=2), INVALID), (dict(rule=2), INVALID),
+    (dict(q=BASE + 8), INVALID),
+    (dict(dq=BASE), INVALID),                                # dq on top of q
+    (dict(dk=BASE + (9 << 32) + 64), INVALID),               # dk inside dq
+    (dict(dM0=BASE + (4 << 32)), INVALID),                   # dM0 on top of M0
+    (dict(d=48), UNSUPPORTED), (dict(N=100), UNSUPPORTED),
+])
+def test_backward_argument_errors(entry, kw, status):
+    assert call_bwd(entry, **kw) == status

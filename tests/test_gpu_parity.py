@@ -70,6 +70,9 @@ def run_gpu(w, t=None):
     out, M, z = binding.forward(t["q"], t["k"], t["v"], t["beta"], t["M0"], t["z0"], N=w.N,
                                 rule=w.rule)
     torch.cuda.synchronize()
+    # a bounded wait that gave up anywhere in the launch fails here (and the sticky status is
+    # read and cleared, so later tests start clean)
+    assert binding.infini_attn_device_status() == 0, f"{w.name}: a device wait timed out"
     return out, M, z
 
 
