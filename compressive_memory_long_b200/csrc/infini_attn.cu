@@ -16,7 +16,7 @@
 #include "infini_attn.h"
 #include "simt_kernels.cuh"
 #include "tc_segment.cuh"
-#include "tc_segment2.cuh"
+#include "tc_segment_p.cuh"
 #include "tc_memory.cuh"
 #include "tc_small.cuh"
 #include "tc_pieces.cuh"
@@ -355,15 +355,15 @@ int launch_memory_tc(const Problem &p, const __nv_bfloat16 *k, const __nv_bfloat
 // register count per thread it was compiled with.  Checked once per kernel: a mismatch
 // would leave the growing warpgroups waiting forever, so the one-tile kernel runs instead.
 template <int D>
-bool seg2_registers_match()
+bool segp_registers_match()
 {
     static const bool ok = [] {
         cudaFuncAttributes fa;
-        if (cudaFuncGetAttributes(&fa, tc::k_segment_tc2<D>) != cudaSuccess) {
+        if (cudaFuncGetAttributes(&fa, tc::k_segment_tcp<D>) != cudaSuccess) {
             cudaGetLastError();
             return false;
         }
-        return fa.numRegs == tc::Seg2Cfg<D>::REGS;
+        return fa.numRegs == tc::SegPCfg<D>::REGS;
     }();
     return ok;
 }
@@ -381,12 +381,14 @@ int launch_segment_tc(const Problem &p, const __nv_bfloat16 *q, const __nv_bfloa
         !make_map_bf16_3d(&mm, snapMb, D, D, p.B * p.Hkv * p.S, D))
         return INFINI_ERR_CUDA;
     tc::SegArgs a{beta, snapZ, out, p.L, (int)p.N, (int)p.S, (int)p.H, (int)p.Hkv};
-    if (p.N % 256 == 0 && seg2_registers_match<D>()) {   // two query tiles per CTA
-        using C2 = tc::Seg2Cfg<D>;
-        if (!opt_in_smem<tc::k_segment_tc2<D>>(C2::ALLOC)) return INFINI_ERR_CUDA;
-        const int64_t ctas = p.B * p.H * p.S * (p.N / 256);
+    if (p.N % 256 == 0 && segp_registers_match<D>()) {
+        // persistent, two query tiles per work item: one CTA per SM over balanced units
+        using CP = tc::SegPCfg<D>;
+        if (!opt_in_smem<tc::k_segment_tcp<D>>(CP::ALLOC)) return INFINI_ERR_CUDA;
+        const int64_t units = p.B * p.H * p.S * ((p.N / 256 + 1) / 2);
+        const int64_t ctas = units < sm_count() ? units : sm_count();
         TRACED("segment_tc", st);
-        tc::k_segment_tc2<D><<<(unsigned)ctas, C2::THREADS, C2::ALLOC, st>>>(mq, mk, mv, mm, a);
+        tc::k_segment_tcp<D><<<(unsigned)ctas, CP::THREADS, CP::ALLOC, st>>>(mq, mk, mv, mm, a, units);
         return INFINI_OK;
     }
     if (!opt_in_smem<tc::k_segment_tc<D>>(C::ALLOC)) return INFINI_ERR_CUDA;

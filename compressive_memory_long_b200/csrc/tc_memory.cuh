@@ -149,8 +149,8 @@ struct IncrArgs {
     int items;                 // chains * S
 };
 
-enum : int { WI_EMPTY = 501, WI_FULL = 502, WI_OFREE = 503, WI_AREADY = 504, WI_ACCFREE = 505,
-             WI_ACCFULL = 506, WI_DRAIN = 507 };
+enum : int { WI_EMPTY = 701, WI_FULL = 702, WI_OFREE = 703, WI_AREADY = 704, WI_ACCFREE = 705,
+             WI_ACCFULL = 706, WI_DRAIN = 707 };
 
 __device__ __forceinline__ void incr_drain(uint64_t *bar, uint32_t parity)
 {
@@ -501,7 +501,7 @@ struct MChainArgs {
     int reverse;               // walk the segments from the last to the first
 };
 
-enum : int { WM_A_EMPTY = 601, WM_B = 602, WM_A_FULL = 603, WM_D = 604, WM_DRAIN = 605 };
+enum : int { WM_A_EMPTY = 801, WM_B = 802, WM_A_FULL = 803, WM_D = 804, WM_DRAIN = 805 };
 
 __device__ __forceinline__ void mchain_drain(uint64_t *bar, uint32_t parity)
 {

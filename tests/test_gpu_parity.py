@@ -232,6 +232,23 @@ def test_tensor_core_segment_kernel(rule, d, N, S):
     assert binding.infini_attn_device_status() == 0
 
 
+@pytest.mark.parametrize("rule", ["linear", "delta"])
+def test_tensor_core_segment_kernel_many_items_per_cta(rule):
+    """More work units than SMs (B*H*S*ceil(N/512) = 2*4*17*3 = 408), with N = 1280 (an odd
+    number of 256-row pairs, so one unit per segment holds a single item) and a short 17th
+    segment (300 rows: its items past row 300 are skipped): each CTA of the persistent
+    kernel walks several items, heavy and light."""
+    from compressive_memory_long_b200 import binding
+    w = wl.Workload("tc_many", B=2, H=4, Hkv=2, d=64, N=1280, S=16, tail=300, dtype="bf16",
+                    rule=rule, seed=23, beta_dist=("normal", 0.0, 1.5),
+                    M0_dist=("uniform", 0.0, 0.1), z0_dist=("uniform", 1.0, 2.0))
+    binding.infini_attn_trace_enable(True)
+    check_full(w)
+    binding.infini_attn_trace_enable(False)
+    assert "segment_tc" in binding.infini_attn_trace_report()
+    assert binding.infini_attn_device_status() == 0
+
+
 def test_tensor_core_first_segment_empty_memory():
     """z0 = 0: the first segment's retrieval is exactly 0, so with beta -> +inf the first
     segment's output is exactly 0 and later segments are not."""
