@@ -384,11 +384,15 @@ int launch_segment_tc(const Problem &p, const __nv_bfloat16 *q, const __nv_bfloa
     if (p.N % 256 == 0 && segp_registers_match<D>()) {
         // persistent, two query tiles per work item: one CTA per SM over balanced units
         using CP = tc::SegPCfg<D>;
+        CUtensorMap mo;
+        if (!make_map_bf16_3d(&mo, out, D, p.L, p.B * p.H, 128)) return INFINI_ERR_CUDA;
         if (!opt_in_smem<tc::k_segment_tcp<D>>(CP::ALLOC)) return INFINI_ERR_CUDA;
         const int64_t units = p.B * p.H * p.S * ((p.N / 256 + 1) / 2);
+        if (units >= (int64_t)1 << 31) return INFINI_ERR_UNSUPPORTED;   // beyond any device memory
         const int64_t ctas = units < sm_count() ? units : sm_count();
         TRACED("segment_tc", st);
-        tc::k_segment_tcp<D><<<(unsigned)ctas, CP::THREADS, CP::ALLOC, st>>>(mq, mk, mv, mm, a, units);
+        tc::k_segment_tcp<D><<<(unsigned)ctas, CP::THREADS, CP::ALLOC, st>>>(mq, mk, mv, mm, mo, a,
+                                                                              (uint32_t)units);
         return INFINI_OK;
     }
     if (!opt_in_smem<tc::k_segment_tc<D>>(C::ALLOC)) return INFINI_ERR_CUDA;

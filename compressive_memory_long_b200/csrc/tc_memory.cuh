@@ -120,11 +120,12 @@ struct IncrCfg {
     static constexpr int OFF_SH = 0;
     static constexpr int OFF_V = 2 * BOX;
     static constexpr int SLOT = (2 + NB) * BOX;
-    // operand set (two, alternating by chunk): sigma_lo (padded like sigma_hi), W_hi, W_lo
+    // operand set (two, alternating by chunk): sigma_lo (bf16, padded like sigma_hi) and, for
+    // the delta rule, sigma in f16 (padded the same way) and W' = 2^e sigma / den in f16
     static constexpr int OFF_SL = 0;
-    static constexpr int OFF_WH = 2 * BOX;
-    static constexpr int OFF_WL = OFF_WH + NB * BOX;
-    static constexpr int OSET = DELTA ? (2 + 2 * NB) * BOX : 2 * BOX;
+    static constexpr int OFF_S16 = 2 * BOX;
+    static constexpr int OFF_W16 = 4 * BOX;
+    static constexpr int OSET = DELTA ? (4 + NB) * BOX : 2 * BOX;
     static constexpr int OFF_RING = 0;
     static constexpr int OFF_OPS = RS * SLOT;
     static constexpr int OFF_BAR = OFF_OPS + 2 * OSET;
@@ -149,6 +150,27 @@ struct IncrArgs {
     int items;                 // chains * S
 };
 
+// The scale of W' for the item whose z_{s-1} is z: 2^e with Sigma_f z_f in [2^(e-1), 2^e)
+// (e = 0 when the sum is 0).  Then den_t / 2^e is a z-weighted mean of sigma(k_t) within a
+// factor 2, so W' = 2^e sigma / den is O(1) and fits f16; A_s = 2^-e sigma^T W'.  Workers
+// and epilogue call this on the same z and get the same e (one fixed summation order).
+__device__ __forceinline__ int incr_scale_exp(const float *z, int d)
+{
+    const float4 *z4 = reinterpret_cast<const float4 *>(z);
+    float sum = 0.f;
+    for (int i = 0; i < d / 4; ++i) {
+        const float4 x = __ldg(z4 + i);
+        sum = (((sum + x.x) + x.y) + x.z) + x.w;
+    }
+    if (!(sum > 0.f)) return 0;
+    int e;
+    frexpf(sum, &e);
+    return e < -100 ? -100 : (e > 100 ? 100 : e);
+}
+
+// 2^e as a float (|e| <= 100)
+__device__ __forceinline__ float pow2f(int e) { return __int_as_float((127 + e) << 23); }
+
 enum : int { WI_EMPTY = 701, WI_FULL = 702, WI_OFREE = 703, WI_AREADY = 704, WI_ACCFREE = 705,
              WI_ACCFULL = 706, WI_DRAIN = 707 };
 
@@ -167,14 +189,18 @@ __device__ __forceinline__ void incr_drain(uint64_t *bar, uint32_t parity)
 // schedule of 64-token chunks, numbered g across the CTA's items.
 //   warp 0       TMA producer: K and V chunks into a ring of RS slots, running ahead across
 //                item boundaries
-//   warp 1       MMA issuer: per chunk, acc += sigma_hi^T [V | W_hi | W_lo] + sigma_lo^T
-//                [V | W_hi] into the item's accumulator set (two sets, alternating by item)
+//   warp 1       MMA issuer: per chunk, B += sigma_hi^T V + sigma_lo^T V (bf16 operands) and,
+//                for the delta rule, A' += sigma_f16^T W' (f16 operands), into the item's
+//                accumulator set (two sets, alternating by item)
 //   warps 4-11   workers: four threads per token row turn K into sigma_hi (in place) and
-//                sigma_lo and, for the delta rule, den = sigma . z_{s-1} and W = sigma / den
-//                (hi, lo) into the chunk's operand set (two sets, alternating by chunk)
+//                sigma_lo and, for the delta rule, sigma in f16, den = sigma . z_{s-1} and
+//                W' = 2^e sigma / den in f16 into the chunk's operand set (two sets,
+//                alternating by chunk)
 //   warps 12-15  epilogue: lane i of the item's accumulator is key feature i; row i of B_s
-//                (fp32) and of A_s (bf16 hi, lo) to global memory, while the next item's
-//                MMAs fill the other accumulator set
+//                (fp32) and of A_s = 2^-e A' (bf16 hi, lo) to global memory, while the next
+//                item's MMAs fill the other accumulator set
+// Precision: B_s carries sigma to about 16 bits (hi + lo); A_s, which only scales the
+// correction A_s M_{s-1}, carries sigma and W' to f16's 11 bits.
 template <int D, bool DELTA>
 __global__ void __launch_bounds__(512, 1)
 k_mem_incr(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
@@ -210,12 +236,15 @@ k_mem_incr(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUte
         *abort = 0;
         fence_barrier_init();
     }
-    if (D == 64)    // the padded feature box of every sigma_hi / sigma_lo tile stays zero
-        for (int i = threadIdx.x; i < (RS + 2) * (C::BOX / 16); i += blockDim.x) {
+    if (D == 64) {  // the padded feature box of every sigma tile (hi, lo, f16) stays zero
+        constexpr int NT = RS + (DELTA ? 4 : 2);
+        for (int i = threadIdx.x; i < NT * (C::BOX / 16); i += blockDim.x) {
             const int t = i / (C::BOX / 16), o = i % (C::BOX / 16);
-            uint8_t *base = t < RS ? ring + t * C::SLOT + C::OFF_SH : ops + (t - RS) * C::OSET + C::OFF_SL;
+            uint8_t *base = t < RS ? ring + t * C::SLOT + C::OFF_SH
+                                   : ops + ((t - RS) % 2) * C::OSET + ((t - RS) < 2 ? C::OFF_SL : C::OFF_S16);
             reinterpret_cast<uint4 *>(base + C::BOX)[o] = make_uint4(0, 0, 0, 0);
         }
+    }
     if (warp == 1) tmem_alloc(tmem_holder, C::TMEM_COLS);
     fence_proxy_async_smem();
     tc_fence_before();
@@ -261,6 +290,7 @@ k_mem_incr(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUte
         if (lane == 0) {
             // ------------------------------------------------------------ MMA issuer
             constexpr uint32_t id = idesc_bf16(128, D, 1, 1);      // both operands MN-major
+            constexpr uint32_t id16 = idesc_f16(128, D, 1, 1);
             const uint32_t aRing = smem_u32(ring), aOps = smem_u32(ops);
             int g = 0, j = 0;
             bool ok = true;
@@ -285,11 +315,9 @@ k_mem_incr(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUte
                         mma_ss(acc, ah, bv, id, first);
                         mma_ss(acc, al, bv, id, 1u);
                         if constexpr (DELTA) {
-                            const uint64_t bwh = sdesc_sw128(os + C::OFF_WH + k2, C::BOX, 1024);
-                            const uint64_t bwl = sdesc_sw128(os + C::OFF_WL + k2, C::BOX, 1024);
-                            mma_ss(acc + D, ah, bwh, id, first);
-                            mma_ss(acc + D, al, bwh, id, 1u);
-                            mma_ss(acc + D, ah, bwl, id, 1u);
+                            const uint64_t a16 = sdesc_sw128(os + C::OFF_S16 + k2, C::BOX, 1024);
+                            const uint64_t bw = sdesc_sw128(os + C::OFF_W16 + k2, C::BOX, 1024);
+                            mma_ss(acc + D, a16, bw, id16, first);
                         }
                     }
                     mma_commit(empty + st);
@@ -315,7 +343,9 @@ k_mem_incr(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUte
             // z_{s-1} at this thread's features (no block-wide barrier: a worker that gives up
             // on a wait must not leave the others waiting at one)
             float zr[C::FPT];
+            float wscale = 1.f;
             if constexpr (DELTA) {
+                wscale = pow2f(incr_scale_exp(a.snapZ + (int64_t)item * D, D));
                 const float4 *zp = reinterpret_cast<const float4 *>(a.snapZ + (int64_t)item * D + f0);
 #pragma unroll
                 for (int e = 0; e < C::FPT / 4; ++e) {
@@ -341,7 +371,7 @@ k_mem_incr(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUte
                     uint4 *ph = reinterpret_cast<uint4 *>(slot + C::OFF_SH + off);
                     const uint4 v = *ph;
                     const uint32_t in[4] = {v.x, v.y, v.z, v.w};
-                    uint32_t hi[4], lo[4];
+                    uint32_t hi[4], lo[4], h16[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162 *>(&in[e]);
@@ -352,9 +382,12 @@ k_mem_incr(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUte
                         const __nv_bfloat162 h = __floats2bfloat162_rn(s0, s1);
                         hi[e] = *reinterpret_cast<const uint32_t *>(&h);
                         lo[e] = pack_bf16x2(s0 - __low2float(h), s1 - __high2float(h));
+                        if constexpr (DELTA) h16[e] = pack_f16x2(s0, s1);
                     }
                     *ph = make_uint4(hi[0], hi[1], hi[2], hi[3]);
                     *reinterpret_cast<uint4 *>(os + C::OFF_SL + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+                    if constexpr (DELTA)
+                        *reinterpret_cast<uint4 *>(os + C::OFF_S16 + off) = make_uint4(h16[0], h16[1], h16[2], h16[3]);
                 }
                 if constexpr (DELTA) {
                     float den = 0.f;
@@ -362,20 +395,16 @@ k_mem_incr(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUte
                     for (int e = 0; e < C::FPT; ++e) den = fmaf(sg[e], zr[e], den);
                     den += __shfl_xor_sync(0xffffffffu, den, 1);
                     den += __shfl_xor_sync(0xffffffffu, den, 2);
-                    const float inv = den == 0.f ? 0.f : 1.f / den;
+                    const float inv = den == 0.f ? 0.f : wscale / den;
 #pragma unroll
                     for (int i = 0; i < CPT; ++i) {
                         const int off = box * C::BOX + t * 128 + (((cq + i) ^ (t & 7)) << 4);
-                        uint32_t hi[4], lo[4];
+                        uint32_t w16[4];
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float w0 = sg[i * 8 + 2 * e] * inv, w1 = sg[i * 8 + 2 * e + 1] * inv;
-                            const __nv_bfloat162 h = __floats2bfloat162_rn(w0, w1);
-                            hi[e] = *reinterpret_cast<const uint32_t *>(&h);
-                            lo[e] = pack_bf16x2(w0 - __low2float(h), w1 - __high2float(h));
-                        }
-                        *reinterpret_cast<uint4 *>(os + C::OFF_WH + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-                        *reinterpret_cast<uint4 *>(os + C::OFF_WL + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+                        for (int e = 0; e < 4; ++e)   // W' >= 0; clamped to f16's largest finite value
+                            w16[e] = pack_f16x2(fminf(sg[i * 8 + 2 * e] * inv, 65504.f),
+                                                fminf(sg[i * 8 + 2 * e + 1] * inv, 65504.f));
+                        *reinterpret_cast<uint4 *>(os + C::OFF_W16 + off) = make_uint4(w16[0], w16[1], w16[2], w16[3]);
                     }
                 }
                 fence_proxy_async_smem();
@@ -392,6 +421,7 @@ k_mem_incr(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUte
             if (!mbar_wait(accfull + (j & 1), (j >> 1) & 1, abort, WI_ACCFULL)) break;
             tc_fence_after();
             const uint32_t acc = T + (j & 1) * C::ACC;
+            const float ascale = DELTA ? pow2f(-incr_scale_exp(a.snapZ + (int64_t)item * D, D)) : 1.f;
             if (live) {
 #pragma unroll 1
                 for (int c0 = 0; c0 < C::ACC; c0 += 32) {
@@ -410,7 +440,8 @@ k_mem_incr(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUte
                         uint32_t hi[16], lo[16];
 #pragma unroll
                         for (int e = 0; e < 16; ++e) {
-                            const float x0 = __uint_as_float(r[2 * e]), x1 = __uint_as_float(r[2 * e + 1]);
+                            const float x0 = __uint_as_float(r[2 * e]) * ascale;
+                            const float x1 = __uint_as_float(r[2 * e + 1]) * ascale;
                             const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
                             hi[e] = *reinterpret_cast<const uint32_t *>(&h);
                             lo[e] = pack_bf16x2(x0 - __low2float(h), x1 - __high2float(h));

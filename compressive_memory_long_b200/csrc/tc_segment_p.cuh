@@ -18,11 +18,20 @@
 // tcgen05.mma operations execute in issue order, so P is read before the next S overwrites
 // it.  After the last P V of a tile the retrieval R_X = sigma(Q_X) M_{s-1} reuses S_X.
 //
+// Epilogue: each softmax thread writes its gated output row into a staging buffer in the
+// 128-byte-swizzled layout of a Q tile and one thread writes the tile with a TMA store
+// (full 128-byte lines instead of one 16-byte piece per row and instruction).  Tile A stages
+// in its own Q buffer, tile B in M's buffer at d = 128 (free once R_B has read it; at d = 64
+// M's buffer is too small and tile B stages in its Q buffer).  z_{s-1} arrives in shared
+// memory with M (one bulk copy on the same barrier).  Each item's Q tiles are prefetched
+// into L2 when the producer reaches the item, so their loads, which wait for the buffers,
+// land from L2.
+//
 // Across items: the producer loads the next item's keys and values as soon as ring stages
-// free up, its Q_X once R_X of the current item has read sigma(Q_X), and M once both R
-// have; the issuer starts the next item's S_X once warpgroup X has read O_X and R_X
-// (epi_done), so the next item's loads and first scores overlap the current item's tail.
-// All waits are bounded (tc_common.cuh).
+// free up, Q_A once tile A's output store has read its buffer, Q_B once R_B has read
+// sigma(Q_B), M and z once tile B's store has read M's buffer; the issuer starts the next
+// item's S_X once warpgroup X has read O_X and R_X (epi_done), so the next item's loads and
+// first scores overlap the current item's tail.  All waits are bounded (tc_common.cuh).
 #pragma once
 
 #include "tc_common.cuh"
@@ -50,18 +59,25 @@ struct SegPCfg {
     static constexpr int OFF_K = 2 * TILE;
     static constexpr int OFF_V = OFF_K + STAGES * TILE;
     static constexpr int OFF_M = OFF_V + STAGES * TILE;
-    // q_full[2], m_full, k_full/v_full/kv_empty[ST], s_full/p_full/sq_full/r_full/epi_done[2],
-    // mma_done
-    static constexpr int NBAR = 3 + 3 * STAGES + 2 * 5 + 1;
-    static constexpr int OFF_BAR = OFF_M + MBYTES;
+    static constexpr int OFF_Z = OFF_M + MBYTES;       // z_{s-1}, fp32, loaded with M
+    // q_full[2], m_full, k_full/v_full/kv_empty[ST],
+    // s_full/p_full/sq_full/r_full/epi_done/st_ready/out_free[2], mma_done
+    static constexpr int NBAR = 3 + 3 * STAGES + 2 * 7 + 1;
+    static constexpr int OFF_BAR = OFF_Z + D * 4;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int BYTES = OFF_MISC + 16;
     static constexpr int ALLOC = BYTES + 1024;
+    static_assert(ALLOC <= 227 * 1024, "shared memory per CTA");
+    // the output tile of a query tile is staged in shared memory and written by one TMA store:
+    // tile A through its Q buffer, tile B through M's buffer when it holds a tile (d = 128:
+    // Q_B of the next item need not wait for the store), else through its own Q buffer
+    static constexpr bool B_OUT_IN_M = MBYTES >= TILE;
 };
 
 // wait ids recorded in g_wait_status
 enum : int { WT_KV_EMPTY = 401, WT_Q = 402, WT_K = 403, WT_P = 404, WT_V = 405, WT_S = 406,
-             WT_R = 407, WT_M = 408, WT_SQ = 409, WT_EPI = 410, WT_QFREE = 411, WT_DRAIN = 412 };
+             WT_R = 407, WT_M = 408, WT_SQ = 409, WT_EPI = 410, WT_QFREE = 411, WT_DRAIN = 412,
+             WT_STAGED = 413, WT_MFREE = 414 };
 
 __device__ __forceinline__ void segp_drain(uint64_t *bar, uint32_t parity)
 {
@@ -78,15 +94,15 @@ __device__ __forceinline__ void segp_drain(uint64_t *bar, uint32_t parity)
 // its items are p = npairs-1-j and, when different, p = j.  Items whose first row lies past
 // L (the short last segment) are skipped.  Every role walks the same list.
 struct SegPList {
-    int64_t u;     // current unit
+    uint32_t u;    // current unit (fewer than 2^31 units: the host checks)
     int half;      // 0: its heavier item next, 1: its lighter one
-    __device__ bool next(const SegArgs &a, int64_t units, int &p, int &s, int64_t &bh)
+    __device__ bool next(const SegArgs &a, uint32_t units, int &p, int &s, int64_t &bh)
     {
-        const int npairs = a.N >> 8, nu = (npairs + 1) >> 1;
+        const uint32_t npairs = (uint32_t)a.N >> 8, nu = (npairs + 1) >> 1;
         while (u < units) {
-            const int64_t g = u / nu;
-            const int j = (int)(u - g * nu);
-            const int pp = half == 0 ? npairs - 1 - j : j;
+            const uint32_t g = u / nu;
+            const uint32_t j = u - g * nu;
+            const int pp = (int)(half == 0 ? npairs - 1 - j : j);
             const bool exists = half == 0 || j < npairs - 1 - j;
             if (half == 0) {
                 half = 1;
@@ -95,8 +111,8 @@ struct SegPList {
                 u += gridDim.x;
             }
             if (!exists) continue;
-            const int64_t bb = g / a.S;
-            const int ss = (int)(g - bb * a.S);
+            const uint32_t bb = g / (uint32_t)a.S;
+            const int ss = (int)(g - bb * (uint32_t)a.S);
             if ((int64_t)ss * a.N + pp * 256 >= a.L) continue;
             p = pp;
             s = ss;
@@ -122,11 +138,48 @@ __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b)
     return r;
 }
 
+// sigma(x) = ELU(x) + 1 over the columns [C0, C1) of row r of a Q tile in shared memory
+// (128-byte swizzle, 64-column boxes), written back in place as bf16 (max(x + 1, e^min(x, 0))
+// on packed fp32 pairs, rounded once); returns sigma(q) . z over those columns in fp32.
+template <int C0, int C1, int UNROLL>
+__device__ __forceinline__ float segp_sigma_row(uint8_t *q, int r, const float *sZ)
+{
+    constexpr int BOX = 128 * 128;
+    const uint64_t one2 = f2_pack(1.f, 1.f);
+    const uint64_t log2e2 = f2_pack(1.4426950408889634f, 1.4426950408889634f);
+    const float4 *z4 = reinterpret_cast<const float4 *>(sZ);
+    uint64_t dp2[2] = {0ull, 0ull};
+#pragma unroll UNROLL
+    for (int c0 = C0; c0 < C1; c0 += 8) {
+        const int ch = (c0 & 63) >> 3;
+        uint4 *ptr = reinterpret_cast<uint4 *>(q + (c0 >> 6) * BOX + r * 128 + ((ch ^ (r & 7)) << 4));
+        const uint4 qv = *ptr;
+        const float4 za = z4[c0 >> 2], zb = z4[(c0 >> 2) + 1];
+        const float zz[8] = {za.x, za.y, za.z, za.w, zb.x, zb.y, zb.z, zb.w};
+        uint32_t w[4] = {qv.x, qv.y, qv.z, qv.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float x0 = __uint_as_float(w[e] << 16), x1 = __uint_as_float(w[e] & 0xffff0000u);
+            float a0, a1, p0, p1;
+            f2_unpack(f2_mul(f2_pack(fminf(x0, 0.f), fminf(x1, 0.f)), log2e2), a0, a1);
+            f2_unpack(f2_add(f2_pack(x0, x1), one2), p0, p1);
+            const float s0 = fmaxf(p0, ex2(a0)), s1 = fmaxf(p1, ex2(a1));
+            dp2[e & 1] = f2_fma(f2_pack(s0, s1), f2_pack(zz[2 * e], zz[2 * e + 1]), dp2[e & 1]);
+            w[e] = pack_bf16x2(s0, s1);
+        }
+        *ptr = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    float d0, d1, d2, d3;
+    f2_unpack(dp2[0], d0, d1);
+    f2_unpack(dp2[1], d2, d3);
+    return (d0 + d1) + (d2 + d3);
+}
+
 template <int D>
 __global__ void __launch_bounds__(384, 1)
 k_segment_tcp(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmM,
-              const SegArgs a, const int64_t units)
+              const __grid_constant__ CUtensorMap tmO, const SegArgs a, const uint32_t units)
 {
     using C = SegPCfg<D>;
     constexpr int ST = C::STAGES;
@@ -140,11 +193,13 @@ k_segment_tcp(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     uint8_t *sK = smem + C::OFF_K;
     uint8_t *sV = smem + C::OFF_V;
     uint8_t *sM = smem + C::OFF_M;
+    float *sZ = reinterpret_cast<float *>(smem + C::OFF_Z);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
     uint64_t *q_full = bars, *m_full = bars + 2;
     uint64_t *k_full = bars + 3, *v_full = k_full + ST, *kv_empty = v_full + ST;
     uint64_t *s_full = kv_empty + ST, *p_full = s_full + 2, *sq_full = p_full + 2;
-    uint64_t *r_full = sq_full + 2, *epi_done = r_full + 2, *mma_done = epi_done + 2;
+    uint64_t *r_full = sq_full + 2, *epi_done = r_full + 2, *st_ready = epi_done + 2;
+    uint64_t *out_free = st_ready + 2, *mma_done = out_free + 2;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
     volatile int *abort = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
 
@@ -163,6 +218,8 @@ k_segment_tcp(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             mbar_init(sq_full + x, 128);
             mbar_init(r_full + x, 1);
             mbar_init(epi_done + x, 128);
+            mbar_init(st_ready + x, 128);
+            mbar_init(out_free + x, 1);
         }
         mbar_init(mma_done, 1);
         *abort = 0;
@@ -176,7 +233,7 @@ k_segment_tcp(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     const uint32_t T_S[2] = {tmem, tmem + 128};
     const uint32_t T_O[2] = {tmem + 256, tmem + 256 + D};
 
-    SegPList list{(int64_t)blockIdx.x, 0};
+    SegPList list{blockIdx.x, 0};
     int p, s;
     int64_t bh;
 
@@ -189,18 +246,19 @@ k_segment_tcp(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             prefetch_tmap(&tmK);
             prefetch_tmap(&tmV);
             prefetch_tmap(&tmM);
-            int it = 0, nqb = 0;                 // items begun; Q_B / M loads issued
+            int it = 0, nm = 0;                  // items begun; M loads issued
+            int nq[2] = {0, 0};                  // Q_A / Q_B loads issued
             int64_t g = 0;                       // key/value tiles issued so far
             bool ok = true;
             while (ok && list.next(a, units, p, s, bh)) {
                 const int64_t chain = (bh / a.H) * a.Hkv + (bh % a.H) / group;
                 const int nB = 2 * p + 2;
                 const int q_row = s * a.N + p * 256;
-                // Q_A: sQ[0] holds sigma(Q_A) of the previous item until R_A has read it
-                if (it > 0 && !(ok = mbar_wait(r_full + 0, (it - 1) & 1, abort, WT_QFREE))) break;
-                mbar_arrive_expect_tx(q_full + 0, C::TILE);
-                for (int cb = 0; cb < D / 64; ++cb)
-                    tma_load_3d(sQ[0] + cb * C::BOX, &tmQ, q_full + 0, cb * 64, q_row, (int)bh);
+                // the item's Q tiles into L2 now (its loads wait for the previous item's
+                // buffers; from L2 they then land quickly)
+                for (int x = 0; x < 2; ++x)
+                    for (int cb = 0; cb < D / 64; ++cb)
+                        tma_prefetch_l2_3d(&tmQ, cb * 64, q_row + x * 128, (int)bh);
                 for (int j = 0; ok && j < nB; ++j) {
                     const int st = (int)(g % ST);
                     if (g >= ST && !(ok = mbar_wait_short(kv_empty + st, (uint32_t)((g / ST) - 1) & 1,
@@ -215,30 +273,39 @@ k_segment_tcp(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                         tma_load_3d(sV + st * C::TILE + cb * C::BOX, &tmV, v_full + st, cb * 64,
                                     s * a.N + j * 128, (int)chain);
                     ++g;
-                    // Q_B and M: free once R_B (issued after R_A) of the previous item is done
-                    if (j == 0 && (it == 0 || (ok = mbar_wait(r_full + 1, (it - 1) & 1, abort, WT_QFREE)))) {
-                        mbar_arrive_expect_tx(q_full + 1, C::TILE);
-                        for (int cb = 0; cb < D / 64; ++cb)
-                            tma_load_3d(sQ[1] + cb * C::BOX, &tmQ, q_full + 1, cb * 64, q_row + 128,
-                                        (int)bh);
-                        mbar_arrive_expect_tx(m_full, C::MBYTES);
-                        for (int cb = 0; cb < D / 64; ++cb)
-                            tma_load_3d(sM + cb * C::MBOX, &tmM, m_full, cb * 64, 0,
-                                        (int)(chain * a.S + s));
-                        ++nqb;
-                    }
+                    if (j > 1) continue;
+                    // after the first key/value tile Q_A, whose buffer holds tile A's staged
+                    // output of the previous item until its store has read it; after the
+                    // second Q_B, free once R_B has read sigma(Q_B) (or, when tile B's output
+                    // goes through sQ[1], once that store has read it)
+                    uint64_t *gate = j == 0 ? out_free + 0 : (C::B_OUT_IN_M ? r_full + 1 : out_free + 1);
+                    if (it > 0 && !(ok = mbar_wait(gate, (it - 1) & 1, abort, WT_QFREE))) break;
+                    mbar_arrive_expect_tx(q_full + j, C::TILE);
+                    for (int cb = 0; cb < D / 64; ++cb)
+                        tma_load_3d(sQ[j] + cb * C::BOX, &tmQ, q_full + j, cb * 64, q_row + j * 128, (int)bh);
+                    ++nq[j];
+                }
+                // M_{s-1} and z_{s-1}, needed only by the item's retrieval: sM is free once
+                // R_B has read it (or, when tile B's output goes through sM, once that store
+                // has read it)
+                if (ok && it > 0)
+                    ok = mbar_wait(C::B_OUT_IN_M ? out_free + 1 : r_full + 1, (it - 1) & 1, abort, WT_MFREE);
+                if (ok) {
+                    mbar_arrive_expect_tx(m_full, C::MBYTES + D * 4);
+                    for (int cb = 0; cb < D / 64; ++cb)
+                        tma_load_3d(sM + cb * C::MBOX, &tmM, m_full, cb * 64, 0, (int)(chain * a.S + s));
+                    bulk_load(sZ, a.snapZ + (chain * a.S + s) * (int64_t)D, D * 4, m_full);
+                    ++nm;
                 }
                 ++it;
             }
             if (*abort) {
-                // let every copy this thread issued land before the CTA exits: the Q_A of the
-                // last item begun, its Q_B and M when issued, the last ST key/value tiles
-                // (older tiles completed before their stage was reused)
-                if (it > 0) segp_drain(q_full + 0, (uint32_t)(it - 1) & 1);
-                if (nqb > 0) {
-                    segp_drain(q_full + 1, (uint32_t)(nqb - 1) & 1);
-                    segp_drain(m_full, (uint32_t)(nqb - 1) & 1);
-                }
+                // let every copy this thread issued land before the CTA exits: the last Q_A,
+                // Q_B and M, the last ST key/value tiles (older tiles completed before their
+                // stage was reused)
+                for (int x = 0; x < 2; ++x)
+                    if (nq[x] > 0) segp_drain(q_full + x, (uint32_t)(nq[x] - 1) & 1);
+                if (nm > 0) segp_drain(m_full, (uint32_t)(nm - 1) & 1);
                 for (int64_t t = (g > ST ? g - ST : 0); t < g; ++t) {
                     segp_drain(k_full + t % ST, (uint32_t)(t / ST) & 1);
                     segp_drain(v_full + t % ST, (uint32_t)(t / ST) & 1);
@@ -352,8 +419,6 @@ k_segment_tcp(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         while (ok && list.next(a, units, p, s, bh)) {
             const int qt = 2 * p + x;                     // q tile index inside the segment
             const int nX = 2 * p + 1 + x;                 // key tiles this tile reads
-            const int64_t chain = (bh / a.H) * a.Hkv + (bh % a.H) / group;
-            const float4 *z4 = reinterpret_cast<const float4 *>(a.snapZ + (chain * a.S + s) * (int64_t)D);
             float m_used = -INFINITY, l = 0.f;
             for (int i = 0; i < nX; ++i) {
                 if (!(ok = mbar_wait(s_full + x, (ns + i) & 1, abort, WT_S))) break;
@@ -429,48 +494,21 @@ k_segment_tcp(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             }
             if (!ok) break;
             // sigma(Q_X) over this row, written over Q_X: every Q_X K^T of the item has
-            // completed (its last S was read above).  The q_full wait makes the TMA-written
-            // Q visible to this thread.
+            // completed (its last S was read above).  The q_full and m_full waits make the
+            // TMA-written Q and z_{s-1} visible to this thread.
             if (!(ok = mbar_wait(q_full + x, it & 1, abort, WT_Q))) break;
-            uint64_t dp2[2] = {0ull, 0ull};                // sigma(q) . z in packed partial sums
-            uint8_t *q = sQ[x];
-#pragma unroll
-            for (int cb = 0; cb < D / 64; ++cb) {
-#pragma unroll
-                for (int ch = 0; ch < 8; ++ch) {
-                    uint4 *ptr = reinterpret_cast<uint4 *>(q + cb * C::BOX + r * 128 + ((ch ^ (r & 7)) << 4));
-                    const uint4 qv = *ptr;
-                    const float4 za = __ldg(z4 + cb * 16 + ch * 2), zb = __ldg(z4 + cb * 16 + ch * 2 + 1);
-                    const float zz[8] = {za.x, za.y, za.z, za.w, zb.x, zb.y, zb.z, zb.w};
-                    uint32_t w[4] = {qv.x, qv.y, qv.z, qv.w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        // sigma(x) = max(x + 1, e^min(x, 0)) on a bf16 pair, in fp32
-                        const float x0 = __uint_as_float(w[e] << 16), x1 = __uint_as_float(w[e] & 0xffff0000u);
-                        float a0, a1, p0, p1;
-                        f2_unpack(f2_mul(f2_pack(fminf(x0, 0.f), fminf(x1, 0.f)), log2e2), a0, a1);
-                        f2_unpack(f2_add(f2_pack(x0, x1), one2), p0, p1);
-                        const float s0 = fmaxf(p0, ex2(a0)), s1 = fmaxf(p1, ex2(a1));
-                        dp2[e & 1] = f2_fma(f2_pack(s0, s1), f2_pack(zz[2 * e], zz[2 * e + 1]), dp2[e & 1]);
-                        w[e] = pack_bf16x2(s0, s1);
-                    }
-                    *ptr = make_uint4(w[0], w[1], w[2], w[3]);
-                }
-            }
+            if (!(ok = mbar_wait(m_full, it & 1, abort, WT_M))) break;
+            const float den = segp_sigma_row<0, D, D / 8>(sQ[x], r, sZ);
             fence_proxy_async_smem();
             mbar_arrive(sq_full + x);
-            float d0, d1, d2, d3;
-            f2_unpack(dp2[0], d0, d1);
-            f2_unpack(dp2[1], d2, d3);
-            const float den = (d0 + d1) + (d2 + d3);
             if (!(ok = mbar_wait(r_full + x, it & 1, abort, WT_R))) break;
             tc_fence_after();
             const float gt = 1.f / (1.f + __expf(-a.beta[bh % a.H]));
             const float wl = (1.f - gt) / l;
             const float wm = den == 0.f ? 0.f : gt / den;
-            const int64_t row = (int64_t)s * a.N + (int64_t)qt * 128 + r;
-            const bool live = row < a.L;                     // rows past L: not stored
-            __nv_bfloat16 *orow = a.out + (bh * a.L + row) * D;
+            // the output row goes to the staging buffer in the layout of a Q tile (128-byte
+            // swizzle, 64-column boxes), which is the layout the TMA store reads
+            uint8_t *stage = x == 0 ? sQ[0] : (C::B_OUT_IN_M ? sM : sQ[1]);
 #pragma unroll 1
             for (int c = 0; c < D; c += 32) {
                 uint32_t o[32], rr[32];
@@ -484,15 +522,32 @@ k_segment_tcp(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     const float y1 = fmaf(__uint_as_float(rr[2 * e + 1]), wm, __uint_as_float(o[2 * e + 1]) * wl);
                     pk[e] = pack_bf16x2(y0, y1);
                 }
-                uint4 *dst = reinterpret_cast<uint4 *>(orow + c);
-                if (live)
 #pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+                for (int e = 0; e < 4; ++e) {
+                    const int ch = ((c & 63) >> 3) + e;
+                    *reinterpret_cast<uint4 *>(stage + (c >> 6) * C::BOX + r * 128 + ((ch ^ (r & 7)) << 4)) =
+                        make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+                }
             }
             // O_X and S_X (R_X) have been read: the next item may overwrite them
             tc_fence_before();
             mbar_arrive(epi_done + x);
+            fence_proxy_async_smem();
+            mbar_arrive(st_ready + x);
+            if (r == 0) {
+                // one thread stores the tile once every row is staged (rows past L are not
+                // written: the store clips at the tensor's extent), waits until the store has
+                // read shared memory and releases the buffer to the producer
+                if (!(ok = mbar_wait(st_ready + x, it & 1, abort, WT_STAGED))) break;
+                const int row0 = s * a.N + qt * 128;
+                if (row0 < a.L) {
+                    for (int cb = 0; cb < D / 64; ++cb)
+                        tma_store_3d(&tmO, stage + cb * C::BOX, cb * 64, row0, (int)bh);
+                    bulk_commit();
+                    bulk_wait_read_all();
+                }
+                mbar_arrive(out_free + x);
+            }
             ns += nX;
             ++it;
         }
