@@ -335,6 +335,8 @@ k_mem_incr(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUte
         const int f0 = q * C::FPT;                  // first feature of this thread
         const int box = f0 >> 6, cq = (f0 & 63) >> 3;
         constexpr int CPT = C::FPT / 8;             // 16-byte chunks per thread
+        const uint64_t one2 = f2_pack(1.f, 1.f);
+        const uint64_t log2e2 = f2_pack(1.4426950408889634f, 1.4426950408889634f);
         int g = 0, j = 0;
         bool ok = true;
         for (int item = blockIdx.x; ok && item < a.items; item += gridDim.x, ++j) {
@@ -362,7 +364,9 @@ k_mem_incr(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUte
                 if (g >= 2 && !(ok = mbar_wait(ofree + (g & 1), ((g >> 1) - 1) & 1, abort, WI_OFREE)))
                     break;
                 uint8_t *slot = ring + st * C::SLOT, *os = ops + (g & 1) * C::OSET;
-                // rows past the head's L (zero-filled by TMA) carry sigma = 0
+                // rows past the head's L (zero-filled by TMA) carry sigma = 0 (only a chunk
+                // that reaches past L needs the mask)
+                const bool partial = c * C::CH + C::CH > rows;
                 const uint32_t keep = c * C::CH + t < rows ? 0xFFFFFFFFu : 0u;
                 float sg[C::FPT];
 #pragma unroll
@@ -374,14 +378,24 @@ k_mem_incr(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUte
                     uint32_t hi[4], lo[4], h16[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162 *>(&in[e]);
-                        const float s0 = __uint_as_float(__float_as_uint(elu1(__low2float(x))) & keep);
-                        const float s1 = __uint_as_float(__float_as_uint(elu1(__high2float(x))) & keep);
+                        // sigma = max(x + 1, e^min(x, 0)) on packed fp32 pairs (as elu1)
+                        const float x0 = __uint_as_float(in[e] << 16), x1 = __uint_as_float(in[e] & 0xffff0000u);
+                        float a0, a1, p0, p1;
+                        f2_unpack(f2_mul(f2_pack(fminf(x0, 0.f), fminf(x1, 0.f)), log2e2), a0, a1);
+                        f2_unpack(f2_add(f2_pack(x0, x1), one2), p0, p1);
+                        float s0 = fmaxf(p0, ex2(a0)), s1 = fmaxf(p1, ex2(a1));
+                        if (partial) {
+                            s0 = __uint_as_float(__float_as_uint(s0) & keep);
+                            s1 = __uint_as_float(__float_as_uint(s1) & keep);
+                        }
                         sg[i * 8 + 2 * e] = s0;
                         sg[i * 8 + 2 * e + 1] = s1;
-                        const __nv_bfloat162 h = __floats2bfloat162_rn(s0, s1);
-                        hi[e] = *reinterpret_cast<const uint32_t *>(&h);
-                        lo[e] = pack_bf16x2(s0 - __low2float(h), s1 - __high2float(h));
+                        hi[e] = pack_bf16x2(s0, s1);
+                        float l0, l1;
+                        f2_unpack(f2_sub(f2_pack(s0, s1), f2_pack(__uint_as_float(hi[e] << 16),
+                                                                  __uint_as_float(hi[e] & 0xffff0000u))),
+                                  l0, l1);
+                        lo[e] = pack_bf16x2(l0, l1);
                         if constexpr (DELTA) h16[e] = pack_f16x2(s0, s1);
                     }
                     *ph = make_uint4(hi[0], hi[1], hi[2], hi[3]);
@@ -390,20 +404,29 @@ k_mem_incr(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUte
                         *reinterpret_cast<uint4 *>(os + C::OFF_S16 + off) = make_uint4(h16[0], h16[1], h16[2], h16[3]);
                 }
                 if constexpr (DELTA) {
-                    float den = 0.f;
+                    uint64_t dp2[2] = {0ull, 0ull};
 #pragma unroll
-                    for (int e = 0; e < C::FPT; ++e) den = fmaf(sg[e], zr[e], den);
+                    for (int e = 0; e < C::FPT / 2; ++e)
+                        dp2[e & 1] = f2_fma(f2_pack(sg[2 * e], sg[2 * e + 1]), f2_pack(zr[2 * e], zr[2 * e + 1]),
+                                            dp2[e & 1]);
+                    float d0, d1, d2, d3;
+                    f2_unpack(dp2[0], d0, d1);
+                    f2_unpack(dp2[1], d2, d3);
+                    float den = (d0 + d1) + (d2 + d3);
                     den += __shfl_xor_sync(0xffffffffu, den, 1);
                     den += __shfl_xor_sync(0xffffffffu, den, 2);
                     const float inv = den == 0.f ? 0.f : wscale / den;
+                    const uint64_t inv2 = f2_pack(inv, inv);
 #pragma unroll
                     for (int i = 0; i < CPT; ++i) {
                         const int off = box * C::BOX + t * 128 + (((cq + i) ^ (t & 7)) << 4);
                         uint32_t w16[4];
 #pragma unroll
-                        for (int e = 0; e < 4; ++e)   // W' >= 0; clamped to f16's largest finite value
-                            w16[e] = pack_f16x2(fminf(sg[i * 8 + 2 * e] * inv, 65504.f),
-                                                fminf(sg[i * 8 + 2 * e + 1] * inv, 65504.f));
+                        for (int e = 0; e < 4; ++e) {   // W' >= 0; clamped to f16's largest finite value
+                            float w0, w1;
+                            f2_unpack(f2_mul(f2_pack(sg[i * 8 + 2 * e], sg[i * 8 + 2 * e + 1]), inv2), w0, w1);
+                            w16[e] = pack_f16x2(fminf(w0, 65504.f), fminf(w1, 65504.f));
+                        }
                         *reinterpret_cast<uint4 *>(os + C::OFF_W16 + off) = make_uint4(w16[0], w16[1], w16[2], w16[3]);
                     }
                 }

@@ -131,13 +131,6 @@ __device__ __forceinline__ uint32_t opaque_u32(uint32_t x)
     return x;
 }
 
-__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b)
-{
-    uint64_t r;
-    asm("mul.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-    return r;
-}
-
 // sigma(x) = ELU(x) + 1 over the columns [C0, C1) of row r of a Q tile in shared memory
 // (128-byte swizzle, 64-column boxes), written back in place as bf16 (max(x + 1, e^min(x, 0))
 // on packed fp32 pairs, rounded once); returns sigma(q) . z over those columns in fp32.
