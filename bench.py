@@ -64,6 +64,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 NCU_TRAFFIC_BYTES: dict = {
     ("hf_repro_n64", "small_fused"): 6362112,
     ("n64_bandwidth", "small_pieces"): (1028091000 + 268262400) * 8,
+    ("gqa8b_n2048_delta", "segment_tc"): 413104384 + 238214912,
+    # 4 of 8 segments captured (x 2) and 16 of 512 segments captured (x 32)
+    ("batched_n1024_linear", "segment_tc"): (1701618688 + 515050496) * 2,
+    ("stream1m_n2048_delta", "segment_tc"): (413484800 + 109220352) * 32,
 }
 
 
