@@ -418,19 +418,24 @@ k_small_pieces(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         const int rr = r < 64 ? r : r + 64;                      // row in the sigma(Q) buffer
         uint32_t g = 0, cA = 0, cB = 0;                          // this group's A- / B-steps
         bool ok = true;
-        // sigma of row r of a 128 x 64 tile into row dr of dst (same swizzle: dr % 8 == r % 8).
-        // Not unrolled: with five roles on each SM sub-partition, instruction-cache misses
-        // cost more than the loop overhead.
+        // sigma of row r of a 128 x 64 tile into row dr of dst (same swizzle: dr % 8 == r % 8),
+        // as elu1 on packed fp32 pairs.  Two chunks per iteration: fully unrolled, with five
+        // roles on each SM sub-partition, instruction-cache misses cost more than the loop.
+        const uint64_t one2 = f2_pack(1.f, 1.f);
+        const uint64_t log2e2 = f2_pack(1.4426950408889634f, 1.4426950408889634f);
         auto sigma_row_to = [&](const uint8_t *src, uint8_t *dst, int dr) {
-#pragma unroll 1
+#pragma unroll 2
             for (int ch = 0; ch < 8; ++ch) {
                 const int c = (ch ^ (r & 7)) << 4;
                 const uint4 x = *reinterpret_cast<const uint4 *>(src + r * 128 + c);
                 uint32_t w4[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    __nv_bfloat162 t2 = *reinterpret_cast<__nv_bfloat162 *>(&w4[e]);
-                    w4[e] = pack_bf16x2(elu1(__low2float(t2)), elu1(__high2float(t2)));
+                    const float x0 = __uint_as_float(w4[e] << 16), x1 = __uint_as_float(w4[e] & 0xffff0000u);
+                    float a0, a1, p0, p1;
+                    f2_unpack(f2_mul(f2_pack(fminf(x0, 0.f), fminf(x1, 0.f)), log2e2), a0, a1);
+                    f2_unpack(f2_add(f2_pack(x0, x1), one2), p0, p1);
+                    w4[e] = pack_bf16x2(fmaxf(p0, ex2(a0)), fmaxf(p1, ex2(a1)));
                 }
                 *reinterpret_cast<uint4 *>(dst + dr * 128 + c) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
             }
@@ -513,27 +518,34 @@ k_small_pieces(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                     const float *zz = sZ + (wg * 2 + (r >> 6)) * 64;
                     uint8_t *row = sSQ(wg) + rr * 128;
                     uint4 q4[8];
-                    float den0 = 0.f, den1 = 0.f;
+                    uint64_t dp2[2] = {0ull, 0ull};
+                    const float2 *z2 = reinterpret_cast<const float2 *>(zz);
 #pragma unroll
                     for (int ch = 0; ch < 8; ++ch) {
                         q4[ch] = *reinterpret_cast<const uint4 *>(row + ((ch ^ (rr & 7)) << 4));
                         const uint32_t w4[4] = {q4[ch].x, q4[ch].y, q4[ch].z, q4[ch].w};
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
-                            __nv_bfloat162 t2 = *reinterpret_cast<const __nv_bfloat162 *>(&w4[e]);
-                            den0 = fmaf(__low2float(t2), zz[ch * 8 + 2 * e], den0);
-                            den1 = fmaf(__high2float(t2), zz[ch * 8 + 2 * e + 1], den1);
+                            const float2 zp = z2[ch * 4 + e];
+                            dp2[e & 1] = f2_fma(f2_pack(__uint_as_float(w4[e] << 16), __uint_as_float(w4[e] & 0xffff0000u)),
+                                                f2_pack(zp.x, zp.y), dp2[e & 1]);
                         }
                     }
-                    const float den = den0 + den1;
+                    float d0, d1, d2, d3;
+                    f2_unpack(dp2[0], d0, d1);
+                    f2_unpack(dp2[1], d2, d3);
+                    const float den = (d0 + d1) + (d2 + d3);
                     const float wm = den == 0.f ? 0.f : gate / den;
+                    const uint64_t wm2 = f2_pack(wm, wm);
 #pragma unroll
                     for (int ch = 0; ch < 8; ++ch) {
                         uint32_t w4[4] = {q4[ch].x, q4[ch].y, q4[ch].z, q4[ch].w};
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
-                            __nv_bfloat162 t2 = *reinterpret_cast<__nv_bfloat162 *>(&w4[e]);
-                            w4[e] = pack_bf16x2(__low2float(t2) * wm, __high2float(t2) * wm);
+                            float y0, y1;
+                            f2_unpack(f2_mul(f2_pack(__uint_as_float(w4[e] << 16), __uint_as_float(w4[e] & 0xffff0000u)), wm2),
+                                      y0, y1);
+                            w4[e] = pack_bf16x2(y0, y1);
                         }
                         *reinterpret_cast<uint4 *>(row + ((ch ^ (rr & 7)) << 4)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
                     }
