@@ -243,7 +243,7 @@ template <typename T>
 bool use_small_fused(const Problem &p)
 {
     return sizeof(T) == 2 && p.d == 64 && p.N == 64 && p.rule == INFINI_UPDATE_LINEAR &&
-           p.H == p.Hkv && p.Lf % 128 == 0;
+           p.Lf % 128 == 0;
 }
 
 // Long heads (16 units of 128 tokens or more) go to the persistent piece kernel.
@@ -404,7 +404,7 @@ int launch_segment_tc(const Problem &p, const __nv_bfloat16 *q, const __nv_bfloa
 
 int64_t small_workspace_bytes(const Problem &p)
 {
-    const int64_t chains = p.B * p.Hkv, units = chains * (p.Lf / 128);
+    const int64_t chains = p.B * p.H, units = chains * (p.Lf / 128);
     const int64_t head = ((64 + chains + units) * 4 + 255) / 256 * 256;
     return head + 2 * units * tc::SmallCfg::STATE * 4;
 }
@@ -415,7 +415,7 @@ int launch_small_fused(const Problem &p, const __nv_bfloat16 *q, const __nv_bflo
                        void *ws, cudaStream_t st)
 {
     using C = tc::SmallCfg;
-    const int64_t chains = p.B * p.Hkv, U = p.Lf / 128, units = chains * U;
+    const int64_t chains = p.B * p.H, U = p.Lf / 128, units = chains * U;   // query-head chains
     // workspace: ticket, per-head M0 reader counts, flags (all zeroed here), then the
     // published aggregates / prefixes
     int *ticket = static_cast<int *>(ws);
@@ -428,15 +428,15 @@ int launch_small_fused(const Problem &p, const __nv_bfloat16 *q, const __nv_bflo
     if (cudaMemsetAsync(ws, 0, ints * 4, st) != cudaSuccess) return INFINI_ERR_CUDA;
     CUtensorMap mq, mk, mv;
     if (!make_map_bf16_3d(&mq, q, C::D, p.L, p.B * p.H, 128) ||
-        !make_map_bf16_3d(&mk, k, C::D, p.L, chains, 128) ||
-        !make_map_bf16_3d(&mv, v, C::D, p.L, chains, 128))
+        !make_map_bf16_3d(&mk, k, C::D, p.L, p.B * p.Hkv, 128) ||
+        !make_map_bf16_3d(&mv, v, C::D, p.L, p.B * p.Hkv, 128))
         return INFINI_ERR_CUDA;
     if (!opt_in_smem<tc::k_small_linear_fused>(C::ALLOC)) return INFINI_ERR_CUDA;
     // few units per head: each sums its predecessors' aggregates directly
     const int direct = U <= 64 ? 1 : 0;
     const int in_place = ((M0 && M0 == M_out) || (z0 && z0 == z_out)) ? 1 : 0;
     tc::SmallArgs a{beta, M0, z0, out, M_out, z_out, ticket, m0_done, flags, agg, incl,
-                    p.L, (int)U, (int)p.H, (int)chains, direct, in_place};
+                    p.L, (int)U, (int)p.H, (int)p.Hkv, (int)chains, direct, in_place};
     TRACED("small_fused", st);
     tc::k_small_linear_fused<<<(unsigned)units, 256, C::ALLOC, st>>>(mq, mk, mv, a);
     return INFINI_OK;
@@ -487,12 +487,13 @@ int launch_pieces(const Problem &p, const __nv_bfloat16 *q, const __nv_bfloat16 
     if (cudaMemsetAsync(ws, 0, ints * 4, st) != cudaSuccess) return INFINI_ERR_CUDA;
     CUtensorMap mq, mk, mv;
     if (!make_map_bf16_3d(&mq, q, C::D, p.L, p.B * p.H, 128) ||
-        !make_map_bf16_3d(&mk, k, C::D, p.L, pl.chains, 128) ||
-        !make_map_bf16_3d(&mv, v, C::D, p.L, pl.chains, 128))
+        !make_map_bf16_3d(&mk, k, C::D, p.L, p.B * p.Hkv, 128) ||
+        !make_map_bf16_3d(&mv, v, C::D, p.L, p.B * p.Hkv, 128))
         return INFINI_ERR_CUDA;
     if (!opt_in_smem<tc::k_small_pieces>(C::ALLOC)) return INFINI_ERR_CUDA;
     tc::PieceArgs a{beta, M0, z0, out, M_out, z_out, ticket, flags, agg, incl, p.L,
-                    (int)pl.U, (int)pl.UP, (int)pl.P, (int)p.H, (int)pl.chains, (int)pl.total};
+                    (int)pl.U, (int)pl.UP, (int)pl.P, (int)p.H, (int)p.Hkv, (int)pl.chains,
+                    (int)pl.total};
     const int64_t sms = sm_count();
     const int64_t grid = pl.total < sms ? pl.total : sms;
     TRACED("small_pieces", st);
@@ -507,7 +508,10 @@ int launch_all(const Problem &p, const T *q, const T *k, const T *v, const float
                const Workspace &ws, cudaStream_t st, bool outputs = true)
 {
     if constexpr (sizeof(T) == 2 && D == 64) {
-        if (outputs && use_small_fused<T>(p)) {
+        // grouped query heads with the state updated in place take the general path: a head
+        // of the group could still be reading M0 / z0 when the group's writer replaces them
+        const bool group_in_place = p.H != p.Hkv && ((M0 && M0 == M_out) || (z0 && z0 == z_out));
+        if (outputs && use_small_fused<T>(p) && !group_in_place) {
             const int rc = use_pieces(p)
                 ? launch_pieces(p, q, k, v, beta, M0, z0, out, M_out, z_out, ws.raw, st)
                 : launch_small_fused(p, q, k, v, beta, M0, z0, out, M_out, z_out, ws.raw, st);
@@ -661,8 +665,14 @@ template <typename T>
 int64_t call_workspace_bytes(const Problem &p)
 {
     if (p.S == 0) return 0;
-    if (use_small_fused<T>(p)) return use_pieces(p) ? pieces_workspace_bytes(p) : small_workspace_bytes(p);
     const int64_t units = p.B * p.Hkv * p.S;
+    if (use_small_fused<T>(p)) {
+        const int64_t fused = use_pieces(p) ? pieces_workspace_bytes(p) : small_workspace_bytes(p);
+        if (p.H == p.Hkv) return fused;
+        // grouped heads updated in place take the general (CUDA-core) path: room for both
+        const int64_t general = simt_workspace_bytes(units, p.d);
+        return fused > general ? fused : general;
+    }
     return use_tc<T>(p) ? tc_workspace_bytes(units, p.d, p.rule == INFINI_UPDATE_DELTA)
                         : simt_workspace_bytes(units, p.d);
 }

@@ -25,7 +25,10 @@
 // Pieces are taken by ticket in start order, so a CTA only looks back at pieces taken
 // before its own, by CTAs that are running: no wait can depend on a CTA that has not
 // started.  Every wait is bounded.
-// Layout limits: bf16, d = 64, N = 64, L % 128 == 0, one query head per key/value head.
+// Layout limits: bf16, d = 64, N = 64, L % 128 == 0.  With several query heads per key/value
+// head each query head is a chain of its own (its own pieces, flags and published states);
+// keys, values, M0 and z0 are read through the head's key/value head, and the first query
+// head of a group writes M_out and z_out.
 #pragma once
 
 #include "tc_common.cuh"
@@ -81,8 +84,8 @@ struct PieceArgs {
     int U;                         // units per head
     int UP;                        // units per piece (last piece of a head may be shorter)
     int P;                         // pieces per head
-    int H;
-    int chains;                    // heads (B * H)
+    int H, Hkv;
+    int chains;                    // query heads (B * H)
     int total;                     // chains * P
 };
 
@@ -252,14 +255,15 @@ k_small_pieces(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                 if (t < 0) break;
                 int chain, pc, u0, n;
                 piece_units(t, chain, pc, u0, n);
+                const int kvc = (int)kv_chain(chain, a.H, a.Hkv);
                 // L2 prefetch of the piece's tiles a few steps ahead of the loads (the loads
                 // are limited to two stages in flight, too few to cover HBM latency alone)
                 auto prefetch = [&](int x) {
                     if (x >= 2 * n) return;
                     const int row = (u0 + (x < n ? x : x - n)) * C::TOK;
                     if (x >= n) tma_prefetch_l2_3d(&tmQ, 0, row, chain);
-                    tma_prefetch_l2_3d(&tmK, 0, row, chain);
-                    tma_prefetch_l2_3d(&tmV, 0, row, chain);
+                    tma_prefetch_l2_3d(&tmK, 0, row, kvc);
+                    tma_prefetch_l2_3d(&tmV, 0, row, kvc);
                 };
                 for (int x = 0; x < C::PREFETCH; ++x) prefetch(x);
                 for (int phase = 0; ok && phase < 2; ++phase)
@@ -278,8 +282,8 @@ k_small_pieces(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                         // unit; queries and the B-step's second read are last uses
                         const uint64_t pol = phase ? pol_first : pol_last;
                         if (phase) tma_load_3d_hint(stage_q(w), &tmQ, bar, 0, row, chain, pol);
-                        tma_load_3d_hint(stage_k(w), &tmK, bar, 0, row, chain, pol);
-                        tma_load_3d_hint(stage_v(w), &tmV, bar, 0, row, chain, pol);
+                        tma_load_3d_hint(stage_k(w), &tmK, bar, 0, row, kvc, pol);
+                        tma_load_3d_hint(stage_v(w), &tmV, bar, 0, row, kvc, pol);
                     }
             }
             // nothing may still be landing in shared memory when the CTA exits
@@ -624,6 +628,8 @@ k_small_pieces(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             int chain, pc, u0, n;
             piece_units(t, chain, pc, u0, n);
             const bool last = pc == a.P - 1;
+            const int64_t kvc = kv_chain(chain, a.H, a.Hkv);
+            const bool state_writer = (chain % a.H) % (a.H / a.Hkv) == 0;   // first query head of its group
             g += n;                                                   // A-steps
             // ---- the piece's aggregate, published for later pieces of the head
             if (!(ok = wait_full())) break;
@@ -652,14 +658,14 @@ k_small_pieces(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 #pragma unroll
                 for (int e = 0; e <= D; ++e) ex[e] = 0.f;
                 if (a.M0) {
-                    const float4 *m = reinterpret_cast<const float4 *>(a.M0 + ((int64_t)chain * D + r) * D);
+                    const float4 *m = reinterpret_cast<const float4 *>(a.M0 + (kvc * D + r) * D);
 #pragma unroll
                     for (int q = 0; q < D / 4; ++q) {
                         const float4 x = m[q];
                         ex[4 * q] = x.x; ex[4 * q + 1] = x.y; ex[4 * q + 2] = x.z; ex[4 * q + 3] = x.w;
                     }
                 }
-                if (a.z0) ex[D] = a.z0[(int64_t)chain * D + r];
+                if (a.z0) ex[D] = a.z0[kvc * D + r];
             } else {
                 // thread i watches predecessor pc-1-i; the walk ends at the nearest piece
                 // that has published its inclusive prefix, and every piece after it must
@@ -709,27 +715,33 @@ k_small_pieces(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             // ---- inclusive prefix (or the head's final memory): ex plus the aggregate, which
             // the accumulator still holds (the carry waits for this role before reusing it)
             {
-                float *dst = last ? a.M_out + ((int64_t)chain * D + r) * D
+                // the head's final memory goes to M_out from the first query head of its group
+                // only; the other heads of the group skip it (their incl is never read)
+                float *dst = last ? (state_writer ? a.M_out + (kvc * D + r) * D : nullptr)
                                   : a.incl + (int64_t)t * C::STATE + r * C::ROW;
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     uint32_t x[32];
                     tmem_ld32(tACC + h * 32, x);
                     tmem_ld_wait();
+                    if (dst)
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        const int c = h * 32 + 4 * q;
-                        reinterpret_cast<float4 *>(dst)[h * 8 + q] =
-                            make_float4(ex[c] + __uint_as_float(x[4 * q]), ex[c + 1] + __uint_as_float(x[4 * q + 1]),
-                                        ex[c + 2] + __uint_as_float(x[4 * q + 2]), ex[c + 3] + __uint_as_float(x[4 * q + 3]));
-                    }
+                        for (int q = 0; q < 8; ++q) {
+                            const int c = h * 32 + 4 * q;
+                            reinterpret_cast<float4 *>(dst)[h * 8 + q] =
+                                make_float4(ex[c] + __uint_as_float(x[4 * q]), ex[c + 1] + __uint_as_float(x[4 * q + 1]),
+                                            ex[c + 2] + __uint_as_float(x[4 * q + 2]), ex[c + 3] + __uint_as_float(x[4 * q + 3]));
+                        }
                 }
                 uint32_t zc[16];
                 tmem_ld16(tACC + 64, zc);
                 tmem_ld_wait();
                 const float zi = ex[D] + __uint_as_float(zc[0]);
-                if (last) a.z_out[(int64_t)chain * D + r] = zi;
-                else reinterpret_cast<float4 *>(dst)[D / 4] = make_float4(zi, 0.f, 0.f, 0.f);
+                if (last) {
+                    if (state_writer) a.z_out[kvc * D + r] = zi;
+                } else {
+                    reinterpret_cast<float4 *>(dst)[D / 4] = make_float4(zi, 0.f, 0.f, 0.f);
+                }
             }
             __threadfence();
             asm volatile("bar.sync 1, 64;" ::: "memory");

@@ -20,7 +20,10 @@
 //      (rows of the first segment read R_0, rows of the second R_1), and the gated output.
 // Units take tickets in start order, so a CTA only waits for units that started before it
 // (running or finished): no unit waits on one that cannot run.  Every wait is bounded.
-// Layout limits: bf16, d = 64, N = 64, L % 128 == 0, one query head per key/value head.
+// Layout limits: bf16, d = 64, N = 64, L % 128 == 0.  With several query heads per key/value
+// head each query head is a chain of its own (its own units, flags and published states);
+// keys, values, M0 and z0 are read through the head's key/value head, and the first query
+// head of a group writes M_out and z_out.
 #pragma once
 
 #include "tc_common.cuh"
@@ -63,11 +66,17 @@ struct SmallArgs {
     int *flags;                    // [chains * U], zeroed before the launch
     float *agg, *incl;             // [chains * U, 64, ROW]
     int64_t L;
-    int U, H;
-    int chains;
+    int U, H, Hkv;
+    int chains;                    // query heads, B * H
     int direct;                    // 1: every unit sums M0 and all earlier aggregates itself
-    int in_place;                  // 1: M_out / z_out are the very buffers M0 / z0
+    int in_place;                  // 1: M_out / z_out are the very buffers M0 / z0 (H == Hkv)
 };
+
+// the key/value head of query-head chain c = b * H + h
+__device__ __forceinline__ int64_t kv_chain(int64_t c, int H, int Hkv)
+{
+    return (c / H) * Hkv + (c % H) / (H / Hkv);
+}
 
 enum : int { FLAG_AGG = 1, FLAG_INCL = 2 };
 enum : int { WS_FULL = 501, WS_S = 502, WS_SIG = 503, WS_D = 504, WS_P = 505, WS_O = 506,
@@ -176,14 +185,15 @@ k_small_linear_fused(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         // and the block barrier, so they overlap both
         const int t0 = *s_ticket;
         const int64_t ch = t0 % a.chains;
+        const int64_t kvc = kv_chain(ch, a.H, a.Hkv);
         const int un = t0 / a.chains;
         prefetch_tmap(&tmQ);
         prefetch_tmap(&tmK);
         prefetch_tmap(&tmV);
         mbar_arrive_expect_tx(full, 3 * C::BOX);
         tma_load_3d(sQ, &tmQ, full, 0, un * C::TOK, (int)ch);
-        tma_load_3d(sK, &tmK, full, 0, un * C::TOK, (int)ch);
-        tma_load_3d(sV, &tmV, full, 0, un * C::TOK, (int)ch);
+        tma_load_3d(sK, &tmK, full, 0, un * C::TOK, (int)kvc);
+        tma_load_3d(sV, &tmV, full, 0, un * C::TOK, (int)kvc);
     }
     if (warp == 1) tmem_alloc(tmem_holder, 512);
     tc_fence_before();
@@ -194,7 +204,9 @@ k_small_linear_fused(const __grid_constant__ CUtensorMap tmQ, const __grid_const
     const uint32_t T_D0 = tmem + 320, T_D1 = tmem + 400;
     // tickets interleave heads (unit-major), so every head advances side by side
     const int t = *s_ticket;
-    const int64_t chain = t % a.chains;     // = b * H + h (one query head per kv head)
+    const int64_t chain = t % a.chains;     // = b * H + h
+    const int64_t kvc = kv_chain(chain, a.H, a.Hkv);
+    const bool state_writer = (chain % a.H) % (a.H / a.Hkv) == 0;   // first query head of its group
     const int unit = t / a.chains;
     const int64_t idx = chain * a.U + unit;
 
@@ -400,11 +412,11 @@ k_small_linear_fused(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                     const int row = i / (C::ROW / 4), c4 = i % (C::ROW / 4);
                     if (c4 < D / 4) {
                         if (a.M0) {
-                            const float4 m = *reinterpret_cast<const float4 *>(a.M0 + (chain * D + row) * D + 4 * c4);
+                            const float4 m = *reinterpret_cast<const float4 *>(a.M0 + (kvc * D + row) * D + 4 * c4);
                             ex[k].x += m.x; ex[k].y += m.y; ex[k].z += m.z; ex[k].w += m.w;
                         }
                     } else if (a.z0) {
-                        ex[k].x += a.z0[chain * D + row];
+                        ex[k].x += a.z0[kvc * D + row];
                     }
                 }
             }
@@ -495,14 +507,14 @@ k_small_linear_fused(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                 const int i = r + 128 * k;
                 if (i < C::STATE4) {
                     sEx4[i] = ex[k];
-                    if (unit + 1 == a.U) {                  // the head's final state
+                    if (unit + 1 == a.U && state_writer) {  // the head's final state
                         const float4 g = sAgg4[i];
                         const int row = i / (C::ROW / 4), c4 = i % (C::ROW / 4);
                         if (c4 < D / 4)
-                            reinterpret_cast<float4 *>(a.M_out + (chain * D + row) * D)[c4] =
+                            reinterpret_cast<float4 *>(a.M_out + (kvc * D + row) * D)[c4] =
                                 make_float4(ex[k].x + g.x, ex[k].y + g.y, ex[k].z + g.z, ex[k].w + g.w);
                         else
-                            a.z_out[chain * D + row] = ex[k].x + g.x;
+                            a.z_out[kvc * D + row] = ex[k].x + g.x;
                     }
                     if (!a.direct && unit + 1 < a.U) {      // inclusive prefix for successors
                         const float4 g = sAgg4[i];

@@ -338,6 +338,51 @@ def test_small_pieces_zero_state_and_split():
     assert torch.allclose(M, Mf, rtol=1e-4, atol=1e-3) and torch.allclose(z, zf, rtol=1e-5)
 
 
+@pytest.mark.parametrize("B,H,Hkv,S,kernel", [(2, 4, 2, 4, "small_fused"),
+                                              (1, 6, 2, 16, "small_fused"),
+                                              (1, 8, 2, 66, "small_pieces"),
+                                              (2, 4, 1, 40, "small_pieces")])
+def test_small_fused_grouped_heads(B, H, Hkv, S, kernel):
+    """Several query heads per key/value head on the fused 64-token kernels: each query head
+    is a chain of its own over its group's keys, values and state; the memory is the
+    group's (M_out and z_out match the oracle)."""
+    from compressive_memory_long_b200 import binding
+    w = wl.Workload("small_gqa", B=B, H=H, Hkv=Hkv, d=64, N=64, S=S, dtype="bf16",
+                    rule="linear", seed=51 + S, beta_dist=("normal", 0.0, 1.5),
+                    M0_dist=("uniform", 0.0, 0.1), z0_dist=("uniform", 1.0, 2.0))
+    binding.infini_attn_trace_enable(True)
+    check_full(w)
+    binding.infini_attn_trace_enable(False)
+    assert list(binding.infini_attn_trace_report()) == [kernel]
+    assert binding.infini_attn_device_status() == 0
+
+
+def test_small_grouped_heads_in_place_take_the_general_path():
+    """Grouped heads with M_out = M0: a query head could still be reading M0 while its
+    group's writer replaces it, so the call runs on the general kernels; the results match
+    the oracle and the same call without aliasing."""
+    from compressive_memory_long_b200 import binding
+    w = wl.Workload("small_gqa_inplace", B=1, H=4, Hkv=2, d=64, N=64, S=8, dtype="bf16",
+                    rule="linear", seed=57, beta_dist=("normal", 0.0, 1.0),
+                    M0_dist=("uniform", 0.0, 0.1), z0_dist=("uniform", 1.0, 2.0))
+    t = to_dev(wl.torch_inputs(w))
+    ref_out, ref_M, ref_z = binding.forward(t["q"], t["k"], t["v"], t["beta"], t["M0"], t["z0"],
+                                            N=w.N, rule=w.rule)
+    M, z = t["M0"].clone(), t["z0"].clone()
+    binding.infini_attn_trace_enable(True)
+    out, _, _ = binding.forward(t["q"], t["k"], t["v"], t["beta"], M, z, N=w.N, rule=w.rule,
+                                M_out=M, z_out=z)
+    torch.cuda.synchronize()
+    binding.infini_attn_trace_enable(False)
+    assert "small_fused" not in binding.infini_attn_trace_report()
+    q, k, v, beta, M0, z0 = wl.host_inputs(w)
+    ro, rM, rz = oracle.infini_attn_fwd(q, k, v, beta, M0, z0, N=w.N, rule=w.rule)
+    assert rel_err(out.float().cpu(), ro) <= TOL["bf16"]
+    assert rel_err(M.cpu(), rM) <= TOL["bf16"] and rel_err(ref_M.cpu(), rM) <= TOL["bf16"]
+    assert rel_err(z.cpu()[:, :, None], rz[:, :, None]) <= TOL["bf16"]
+    assert binding.infini_attn_device_status() == 0
+
+
 def test_n64_bandwidth_sampled():
     w = wl.WORKLOADS["n64_bandwidth"]
     check_sampled(w, chains=[(1, 5)], segs=[0, 1, 8191, 16383])

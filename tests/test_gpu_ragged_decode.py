@@ -52,6 +52,10 @@ RAGGED = [
     (make("fused64", B=2, H=4, Hkv=4, d=64, N=64, S=6, tail=37, seed=11), "small_fused", True),
     (make("pieces64", B=1, H=2, Hkv=2, d=64, N=64, S=40, tail=1, state=True, seed=12),
      "small_pieces", True),
+    (make("fused64_gqa", B=1, H=4, Hkv=2, d=64, N=64, S=6, tail=37, state=True, seed=26),
+     "small_fused", True),
+    (make("pieces64_gqa", B=1, H=6, Hkv=3, d=64, N=64, S=34, tail=63, seed=27),
+     "small_pieces", True),
     (make("odd_s64", B=1, H=2, Hkv=2, d=64, N=64, S=3, tail=50, seed=13), "segment_simt", True),
     (make("simt_d32", B=1, H=2, Hkv=2, d=32, N=64, S=2, tail=10, seed=17), "segment_simt", True),
     (make("f32_delta", B=1, H=2, Hkv=2, d=64, N=64, S=2, tail=33, dtype="f32", rule="delta",
