@@ -449,10 +449,39 @@ def backward_flops(w: wl.Workload):
     return local + memory
 
 
+def backward_roofline(w: wl.Workload, kernels: dict, steps: int, clk: dict) -> dict:
+    """The backward's dominant kernel against its own ceiling.  Algorithmic flops per
+    (b, h, segment), one causal product = d N (N + 1): k_bwd_rows recomputes S and P V (2)
+    plus the retrieval's sigma(q) M and dout M^T (4 N d^2), on CUDA cores; the dq kernel S, dP
+    and dS K (3), the dk/dv kernel S^T, dP^T, P^T dout and dS^T Q (4), on the tensor cores for
+    bf16 with N % 128 == 0 (bf16 peak), else on CUDA cores (fp32 FMA peak)."""
+    B, H, N, d = w.B, w.H, w.N, w.d
+    S = -(-w.L // N)
+    prod = B * H * S * d * N * (N + 1)
+    flops = {"bwd_rows": 2 * prod + B * H * S * 4 * N * d * d, "bwd_dq": 3 * prod, "bwd_dkdv": 4 * prod}
+    tensor = w.dtype == "bf16" and d in (64, 128) and N % 128 == 0
+    cand = {k: v for k, v in kernels.items() if k in flops}
+    if not cand:
+        return None
+    dom = max(cand, key=lambda k: cand[k]["ms"])
+    ms = cand[dom]["ms"] / max(1, cand[dom]["launches"]) * (cand[dom]["launches"] / max(1, steps))
+    achieved = flops[dom] / (ms / 1e3) / 1e12 if ms > 0 else 0.0
+    if tensor and dom != "bwd_rows":
+        peaks, src = load_peaks()
+        peak, bound, psrc = peaks["bf16_tflops"], "tensor", f"{src} (burst)"
+    else:
+        peak, bound = fp32_fma_peak_tflops(clk["sm_mhz"] or 1965.0), "alu"
+        psrc = "derived: 148 SMs x 128 fp32 lanes x 2 x SM clock"
+    return {"bound": bound, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+            "frac": achieved / peak, "traffic": None, "kernel": dom, "kernel_ms": ms,
+            "peak_source": psrc, "algorithmic_flops": flops[dom],
+            "kernel_share": cand[dom]["ms"] / sum(v["ms"] for v in kernels.values())}
+
+
 def run_backward(args, w: wl.Workload, world: int, rank: int, local: int, dev):
     """One step = all gradients of one forward of the workload (infini_attn_bwd), with a
     fixed random upstream gradient; inputs resident on the device, L2 flushed before each
-    step.  The dominant kernel's roofline is against the fp32 FMA rate (CUDA cores)."""
+    step.  The roofline is the dominant kernel's (backward_roofline)."""
     import ctypes
     from compressive_memory_long_b200 import binding
     host = wl.torch_inputs(w, pin_memory=True)
@@ -497,17 +526,7 @@ def run_backward(args, w: wl.Workload, world: int, rank: int, local: int, dev):
     total_ms = max_over_ranks(float(sum(s_.elapsed_time(e) for s_, e in zip(starts, ends))), world, dev)
     value = w.tokens * args.steps * world / (total_ms / 1000.0)
     clk = clocks.summary()
-    peak = fp32_fma_peak_tflops(clk["sm_mhz"] or 1965.0)
-    attn = {k: v for k, v in kernels.items() if k in ("bwd_dq", "bwd_dkdv", "bwd_rows")}
-    attn_ms = sum(v["ms"] for v in attn.values()) / max(1, args.steps)
-    B, H, N, d = w.B, w.H, w.N, w.d
-    S = -(-w.L // N)
-    attn_flops = B * H * S * 2 * d * N * (N + 1) / 2 * (2 + 3 + 2)   # rows: S, PV; dq: S, dP, dS K; dkdv
-    achieved = attn_flops / (attn_ms / 1e3) / 1e12 if attn_ms > 0 else 0.0
-    roof = {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-            "frac": achieved / peak, "traffic": None, "kernel": "bwd_rows + bwd_dq + bwd_dkdv",
-            "kernel_ms": attn_ms, "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 x SM clock",
-            "algorithmic_flops": attn_flops}
+    roof = backward_roofline(w, kernels, args.steps, clk)
     if rank == 0:
         line = {
             "metric": BACKWARD_METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,

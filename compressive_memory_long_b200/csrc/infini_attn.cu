@@ -17,6 +17,7 @@
 #include "simt_kernels.cuh"
 #include "tc_segment.cuh"
 #include "tc_segment_p.cuh"
+#include "tc_backward.cuh"
 #include "tc_memory.cuh"
 #include "tc_small.cuh"
 #include "tc_pieces.cuh"
@@ -1117,8 +1118,34 @@ int launch_backward(const BwdPlan &p, const T *q, const T *k, const T *v, const 
         k_bwd_rows<T, D><<<(unsigned)(p.B * p.H * S * p.qtiles), 256, smem, st>>>(
             q, k, v, beta, dout, w, p.L, N, S, H, Hkv);
     }
-    // 3. dq;  4. local dk, dv
-    {
+    // 3. dq;  4. local dk, dv: on the tensor cores for bf16 with 128-row tiles
+    bool tc_attn = false;
+    if constexpr (sizeof(T) == 2 && (D == 64 || D == 128)) {
+        if (p.N % 128 == 0) {
+            using CB = tc::BwdTcCfg<D>;
+            CUtensorMap mq, mk, mv, mo;
+            if (!make_map_bf16_3d(&mq, q, D, p.L, p.B * p.H, 128) ||
+                !make_map_bf16_3d(&mk, k, D, p.L, p.B * p.Hkv, 128) ||
+                !make_map_bf16_3d(&mv, v, D, p.L, p.B * p.Hkv, 128) ||
+                !make_map_bf16_3d(&mo, dout, D, p.L, p.B * p.H, 128))
+                return INFINI_ERR_CUDA;
+            if (!opt_in_smem<tc::k_bwd_dq_tc<D>>(CB::ALLOC_DQ) || !opt_in_smem<tc::k_bwd_dkdv_tc<D>>(CB::ALLOC_KV))
+                return INFINI_ERR_CUDA;
+            tc::BwdTcArgs ta{beta, w.lse, w.Drow, w.dq, reinterpret_cast<__nv_bfloat16 *>(dq), w.dk, w.dv,
+                             p.L, N, S, H, Hkv};
+            const int64_t tiles = p.N / 128;
+            {
+                TRACED("bwd_dq", st);
+                tc::k_bwd_dq_tc<D><<<(unsigned)(p.B * p.H * S * tiles), CB::THREADS, CB::ALLOC_DQ, st>>>(
+                    mq, mk, mv, mo, ta);
+            }
+            TRACED("bwd_dkdv", st);
+            tc::k_bwd_dkdv_tc<D><<<(unsigned)(chains * S * tiles), CB::THREADS, CB::ALLOC_KV, st>>>(
+                mq, mk, mv, mo, ta);
+            tc_attn = true;
+        }
+    }
+    if (!tc_attn) {
         const size_t smem = BwdDqSmem<D>::bytes;
         if (!opt_in_smem<k_bwd_dq<T, D>>(smem) || !opt_in_smem<k_bwd_dkdv<T, D>>(smem))
             return INFINI_ERR_CUDA;

@@ -1,0 +1,503 @@
+// Local-attention part of the backward pass on the tensor cores (sm_100a, bf16, d = 64 or
+// 128, N % 128 == 0).
+//
+// Same arithmetic as k_bwd_dq / k_bwd_dkdv (backward.cuh; AI Wiki "Infini-Attention", "What
+// happens inside the Infini-attention block?", the local causal softmax of each segment):
+// with lse and D_i = dA_dot_i . A_dot_i from k_bwd_rows, g = sigmoid(beta_h),
+//   P = exp2(S log2(e) / sqrt(d) - lse),  dS = P * ((1 - g) dout V^T - D),
+//   dq += dS K / sqrt(d),  dk += dS^T Q / sqrt(d),  dv += (1 - g) P^T dout,
+// over the causal keys of the row's own segment.  P and dS enter the second products as
+// bf16 (the operands of kind::f16), every product accumulates in fp32 in TMEM.
+//
+//   k_bwd_dq_tc    one CTA per (b, h, segment, 128 query rows); per key tile:
+//                  S = Q K^T and dP = dout V^T into TMEM, dS (bf16) over S, dQ += dS K
+//   k_bwd_dkdv_tc  one CTA per (b, kv head, segment, 128 keys), over the group's query
+//                  heads and the query tiles at or after the key tile; per query tile:
+//                  S^T = K Q^T and dP^T = V dout^T, (1 - g) P^T over S^T and dS^T over
+//                  dP^T (bf16), dV += P^T dout, dK += dS^T Q; each key row has one owner
+// Roles: warps 0-3 one thread per row (elementwise work, epilogue); warp 4 loads (TMA; in
+// k_bwd_dkdv_tc its 32 lanes also stage the query tile's lse and D); warp 5 lane 0 issues
+// the MMAs.  All waits are bounded (tc_common.cuh).
+#pragma once
+
+#include "tc_common.cuh"
+
+namespace infini {
+namespace tc {
+
+template <int D>
+struct BwdTcCfg {
+    static_assert(D == 64 || D == 128, "tensor-core backward: d = 64 or 128");
+    static constexpr int THREADS = 192;
+    static constexpr int TILE = 128 * D * 2;          // 128 rows x d bf16
+    static constexpr int BOX = 128 * 128;             // 128 rows x 64 bf16
+    static constexpr int ST = 2;                      // stages of the streamed operands
+    // dq: Q | dout | ST x (K | V);  dkdv: K | V | ST x (Q | dout | lse | D)
+    static constexpr int OFF_A = 0, OFF_B = TILE, OFF_RING = 2 * TILE;
+    static constexpr int RING_DQ = 2 * TILE;
+    static constexpr int RING_KV = 2 * TILE + 2 * 128 * 4;
+    static constexpr int OFF_BAR_DQ = OFF_RING + ST * RING_DQ;
+    static constexpr int OFF_BAR_KV = OFF_RING + ST * RING_KV;
+    static constexpr int NBAR = 3 * ST + 6;
+    static constexpr int ALLOC_DQ = OFF_BAR_DQ + NBAR * 8 + 16 + 1024;
+    static constexpr int ALLOC_KV = OFF_BAR_KV + NBAR * 8 + 16 + 1024;
+    static_assert(ALLOC_DQ <= 227 * 1024 && ALLOC_KV <= 227 * 1024, "shared memory");
+    // TMEM: S (or S^T) [0,128), dP (or dP^T) [128,256), then the accumulators
+    static constexpr uint32_t T_S = 0, T_P = 128, T_A0 = 256, T_A1 = 256 + D;
+};
+
+struct BwdTcArgs {
+    const float *beta;
+    const float *lse, *Drow;      // [B, H, L] from k_bwd_rows
+    const float *dq_mem;          // [B, H, L, D]: the retrieval part of dq
+    __nv_bfloat16 *dq;            // [B, H, L, D] output
+    float *dk, *dv;               // [B, Hkv, L, D]: the local parts (fp32)
+    int64_t L;
+    int N, S, H, Hkv;
+};
+
+enum : int { WB_QF = 901, WB_KF = 902, WB_VF = 903, WB_KVE = 904, WB_SDP = 905, WB_DS = 906,
+             WB_DONE = 907, WB_FULL = 908, WB_EMPTY = 909, WB_DRAIN = 910 };
+
+__device__ __forceinline__ void bwdtc_drain(uint64_t *bar, uint32_t parity)
+{
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity)) {
+        if (clock64() - t0 > spin_limit()) {
+            atomicCAS(&g_wait_status, 0, WB_DRAIN);
+            return;
+        }
+    }
+}
+
+// dq of 128 query rows: the retrieval part (from k_bwd_rows) plus dS K / sqrt(d)
+template <int D>
+__global__ void __launch_bounds__(192, 1)
+k_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+            const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+            const BwdTcArgs a)
+{
+    using C = BwdTcCfg<D>;
+    constexpr int ST = C::ST;
+    if (__syncthreads_or(threadIdx.x == 0 && wait_status_set())) return;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+    const int qtiles = a.N / 128;
+    int64_t bid = blockIdx.x;
+    const int qt = qtiles - 1 - (int)(bid % qtiles);          // the longest rows first
+    bid /= qtiles;
+    const int s = (int)(bid % a.S);
+    const int64_t bh = bid / a.S;
+    const int h = (int)(bh % a.H);
+    const int64_t chain = (bh / a.H) * a.Hkv + h / (a.H / a.Hkv);
+    const int64_t seg0 = (int64_t)s * a.N;
+    const int valid = (int)(a.L - seg0 < a.N ? a.L - seg0 : a.N);
+    const int q0 = qt * 128;
+    if (q0 >= valid) return;
+    const int nk = qt + 1;                                      // key tiles 0..qt
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    uint8_t *sQ = smem + C::OFF_A, *sO = smem + C::OFF_B;
+    auto sK = [&](int st) { return smem + C::OFF_RING + st * C::RING_DQ; };
+    auto sV = [&](int st) { return smem + C::OFF_RING + st * C::RING_DQ + C::TILE; };
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR_DQ);
+    uint64_t *k_full = bars, *v_full = bars + ST, *kv_empty = bars + 2 * ST;
+    uint64_t *q_full = bars + 3 * ST, *sdp_full = q_full + 1, *ds_full = q_full + 2, *dq_done = q_full + 3;
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C::OFF_BAR_DQ + C::NBAR * 8);
+    volatile int *abort = reinterpret_cast<volatile int *>(smem + C::OFF_BAR_DQ + C::NBAR * 8 + 4);
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < ST; ++i) {
+            mbar_init(k_full + i, 1);
+            mbar_init(v_full + i, 1);
+            mbar_init(kv_empty + i, 1);
+        }
+        mbar_init(q_full, 1);
+        mbar_init(sdp_full, 1);
+        mbar_init(ds_full, 128);
+        mbar_init(dq_done, 1);
+        *abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == 5) tmem_alloc(tmem_holder, 512);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+
+    if (warp == 4) {
+        if (lane == 0) {
+            // ---------------------------------------------------------------- loads
+            prefetch_tmap(&tmQ);
+            prefetch_tmap(&tmK);
+            prefetch_tmap(&tmV);
+            prefetch_tmap(&tmO);
+            mbar_arrive_expect_tx(q_full, 2 * C::TILE);
+            for (int cb = 0; cb < D / 64; ++cb) {
+                tma_load_3d(sQ + cb * C::BOX, &tmQ, q_full, cb * 64, (int)(seg0 + q0), (int)bh);
+                tma_load_3d(sO + cb * C::BOX, &tmO, q_full, cb * 64, (int)(seg0 + q0), (int)bh);
+            }
+            int issued = 0;
+            for (int j = 0; j < nk; ++j) {
+                const int st = j % ST;
+                if (j >= ST && !mbar_wait_short(kv_empty + st, ((j / ST) - 1) & 1, abort, WB_KVE)) break;
+                mbar_arrive_expect_tx(k_full + st, C::TILE);
+                for (int cb = 0; cb < D / 64; ++cb)
+                    tma_load_3d(sK(st) + cb * C::BOX, &tmK, k_full + st, cb * 64, (int)(seg0 + j * 128),
+                                (int)chain);
+                mbar_arrive_expect_tx(v_full + st, C::TILE);
+                for (int cb = 0; cb < D / 64; ++cb)
+                    tma_load_3d(sV(st) + cb * C::BOX, &tmV, v_full + st, cb * 64, (int)(seg0 + j * 128),
+                                (int)chain);
+                issued = j + 1;
+            }
+            if (*abort) {
+                bwdtc_drain(q_full, 0);
+                for (int j = (issued > ST ? issued - ST : 0); j < issued; ++j) {
+                    bwdtc_drain(k_full + j % ST, (j / ST) & 1);
+                    bwdtc_drain(v_full + j % ST, (j / ST) & 1);
+                }
+            }
+        }
+    } else if (warp == 5) {
+        if (lane == 0) {
+            // ---------------------------------------------------------------- MMA issuer
+            constexpr uint32_t idS = idesc_bf16(128, 128, 0, 0);
+            constexpr uint32_t idO = idesc_bf16(128, D, 0, 1);
+            const uint32_t aQ = smem_u32(sQ), aO = smem_u32(sO);
+            bool ok = mbar_wait_short(q_full, 0, abort, WB_QF);
+            for (int j = 0; ok && j < nk; ++j) {
+                const int st = j % ST;
+                const uint32_t aK = smem_u32(sK(st)), aV = smem_u32(sV(st));
+                if (!(ok = mbar_wait_short(k_full + st, (j / ST) & 1, abort, WB_KF))) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {        // S = Q K^T
+                    const uint32_t off = (kk >> 2) * C::BOX + (kk & 3) * 32;
+                    mma_ss(tmem + C::T_S, sdesc_sw128(aQ + off, 16, 1024), sdesc_sw128(aK + off, 16, 1024),
+                           idS, kk > 0 ? 1u : 0u);
+                }
+                if (!(ok = mbar_wait_short(v_full + st, (j / ST) & 1, abort, WB_VF))) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {        // dP = dout V^T
+                    const uint32_t off = (kk >> 2) * C::BOX + (kk & 3) * 32;
+                    mma_ss(tmem + C::T_P, sdesc_sw128(aO + off, 16, 1024), sdesc_sw128(aV + off, 16, 1024),
+                           idS, kk > 0 ? 1u : 0u);
+                }
+                mma_commit(sdp_full);
+                if (!(ok = mbar_wait_short(ds_full, j & 1, abort, WB_DS))) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)                 // dQ += dS K (dS in S's columns)
+                    mma_ts(tmem + C::T_A0, tmem + C::T_S + kk * 8, sdesc_sw128(aK + kk * 2048, C::BOX, 1024),
+                           idO, (j > 0 || kk > 0) ? 1u : 0u);
+                mma_commit(kv_empty + st);
+            }
+            mma_commit(dq_done);
+            bwdtc_drain(dq_done, 0);
+        }
+    } else if (warp < 4) {
+        // ---------------------------------------------------------------- rows
+        const int r = threadIdx.x;
+        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        const int64_t row = bh * a.L + seg0 + q0 + r;
+        const bool live = q0 + r < valid;
+        const float lse = live ? a.lse[row] : 0.f, Dr = live ? a.Drow[row] : 0.f;
+        const float c1 = 1.f - 1.f / (1.f + __expf(-a.beta[h]));
+        const float sl2 = rsqrtf((float)D) * 1.4426950408889634f;
+        bool ok = true;
+        for (int j = 0; ok && j < nk; ++j) {
+            if (!(ok = mbar_wait(sdp_full, j & 1, abort, WB_SDP))) break;
+            tc_fence_after();
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                uint32_t sv[2][32], pv[2][32];
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    tmem_ld32(lane_base + tmem + C::T_S + half * 64 + c * 32, sv[c]);
+                    tmem_ld32(lane_base + tmem + C::T_P + half * 64 + c * 32, pv[c]);
+                }
+                tmem_ld_wait();
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        float ds2[2];
+#pragma unroll
+                        for (int u = 0; u < 2; ++u) {
+                            const int col = half * 64 + c * 32 + 2 * e + u;       // key in the tile
+                            const bool vis = live && j * 128 + col < valid && (j < qt || col <= r);
+                            const float p = vis ? ex2(fmaf(__uint_as_float(sv[c][2 * e + u]), sl2, -lse)) : 0.f;
+                            ds2[u] = p * fmaf(c1, __uint_as_float(pv[c][2 * e + u]), -Dr);
+                        }
+                        pk[e] = pack_bf16x2(ds2[0], ds2[1]);
+                    }
+                    tmem_st16(lane_base + tmem + C::T_S + half * 32 + c * 16, pk);
+                }
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(ds_full);
+        }
+        if (ok && mbar_wait(dq_done, 0, abort, WB_DONE)) {
+            tc_fence_after();
+            const float rs = rsqrtf((float)D);
+#pragma unroll 1
+            for (int c = 0; c < D; c += 32) {
+                uint32_t o[32];
+                tmem_ld32(lane_base + tmem + C::T_A0 + c, o);
+                tmem_ld_wait();
+                if (live) {
+                    const float4 *src = reinterpret_cast<const float4 *>(a.dq_mem + row * D + c);
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const float4 m = src[e];
+                        pk[2 * e] = pack_bf16x2(fmaf(__uint_as_float(o[4 * e]), rs, m.x),
+                                                fmaf(__uint_as_float(o[4 * e + 1]), rs, m.y));
+                        pk[2 * e + 1] = pack_bf16x2(fmaf(__uint_as_float(o[4 * e + 2]), rs, m.z),
+                                                    fmaf(__uint_as_float(o[4 * e + 3]), rs, m.w));
+                    }
+                    uint4 *dst = reinterpret_cast<uint4 *>(a.dq + row * D + c);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 5) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// local dk, dv of 128 keys over the group's query heads and the query tiles at or after
+// the key tile
+template <int D>
+__global__ void __launch_bounds__(192, 1)
+k_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+              const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+              const BwdTcArgs a)
+{
+    using C = BwdTcCfg<D>;
+    constexpr int ST = C::ST;
+    if (__syncthreads_or(threadIdx.x == 0 && wait_status_set())) return;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+    const int ktiles = a.N / 128;
+    int64_t bid = blockIdx.x;
+    const int kt = (int)(bid % ktiles);                      // the longest key tiles first
+    bid /= ktiles;
+    const int s = (int)(bid % a.S);
+    const int64_t chain = bid / a.S;                         // b * Hkv + kv head
+    const int G = a.H / a.Hkv;
+    const int64_t bh0 = (chain / a.Hkv) * a.H + (chain % a.Hkv) * G;   // first query head
+    const int64_t seg0 = (int64_t)s * a.N;
+    const int valid = (int)(a.L - seg0 < a.N ? a.L - seg0 : a.N);
+    const int k0 = kt * 128;
+    if (k0 >= valid) return;
+    const int nq = (valid - k0 + 127) / 128;                 // query tiles kt .. kt + nq - 1
+    const int steps = G * nq;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    uint8_t *sK = smem + C::OFF_A, *sV = smem + C::OFF_B;
+    auto sQ = [&](int st) { return smem + C::OFF_RING + st * C::RING_KV; };
+    auto sO = [&](int st) { return smem + C::OFF_RING + st * C::RING_KV + C::TILE; };
+    auto sL = [&](int st) { return reinterpret_cast<float *>(smem + C::OFF_RING + st * C::RING_KV + 2 * C::TILE); };
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR_KV);
+    uint64_t *full = bars, *empty = bars + ST, *kv_full = bars + 3 * ST;
+    uint64_t *sdp_full = kv_full + 1, *ps_full = kv_full + 2, *done = kv_full + 3;
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C::OFF_BAR_KV + C::NBAR * 8);
+    volatile int *abort = reinterpret_cast<volatile int *>(smem + C::OFF_BAR_KV + C::NBAR * 8 + 4);
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < ST; ++i) {
+            mbar_init(full + i, 33);          // the TMA lane's expect_tx + the 32 lanes' lse / D
+            mbar_init(empty + i, 1);
+        }
+        mbar_init(kv_full, 1);
+        mbar_init(sdp_full, 1);
+        mbar_init(ps_full, 128);
+        mbar_init(done, 1);
+        *abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == 5) tmem_alloc(tmem_holder, 512);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+
+    if (warp == 4) {
+        // -------------------------------------------------------------------- loads
+        if (lane == 0) {
+            prefetch_tmap(&tmQ);
+            prefetch_tmap(&tmK);
+            prefetch_tmap(&tmV);
+            prefetch_tmap(&tmO);
+            mbar_arrive_expect_tx(kv_full, 2 * C::TILE);
+            for (int cb = 0; cb < D / 64; ++cb) {
+                tma_load_3d(sK + cb * C::BOX, &tmK, kv_full, cb * 64, (int)(seg0 + k0), (int)chain);
+                tma_load_3d(sV + cb * C::BOX, &tmV, kv_full, cb * 64, (int)(seg0 + k0), (int)chain);
+            }
+        }
+        int issued = 0;
+        bool ok = true;
+        for (int i = 0; i < steps; ++i) {
+            const int st = i % ST;
+            const int64_t bh = bh0 + i / nq;
+            const int q0 = k0 + (i % nq) * 128;
+            if (i >= ST && !(ok = mbar_wait_short(empty + st, ((i / ST) - 1) & 1, abort, WB_EMPTY))) break;
+            if (lane == 0) {
+                mbar_arrive_expect_tx(full + st, 2 * C::TILE);
+                for (int cb = 0; cb < D / 64; ++cb) {
+                    tma_load_3d(sQ(st) + cb * C::BOX, &tmQ, full + st, cb * 64, (int)(seg0 + q0), (int)bh);
+                    tma_load_3d(sO(st) + cb * C::BOX, &tmO, full + st, cb * 64, (int)(seg0 + q0), (int)bh);
+                }
+            }
+            // lse and D of the tile's 128 query rows (0 past the segment's valid rows)
+            float *sl = sL(st);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int jr = lane * 4 + u;
+                const bool in = q0 + jr < valid;
+                const int64_t row = bh * a.L + seg0 + q0 + jr;
+                sl[jr] = in ? a.lse[row] : 0.f;
+                sl[128 + jr] = in ? a.Drow[row] : 0.f;
+            }
+            mbar_arrive(full + st);
+            issued = i + 1;
+        }
+        if (lane == 0 && (*abort || !ok)) {
+            bwdtc_drain(kv_full, 0);
+            for (int i = (issued > ST ? issued - ST : 0); i < issued; ++i) bwdtc_drain(full + i % ST, (i / ST) & 1);
+        }
+    } else if (warp == 5) {
+        if (lane == 0) {
+            // ---------------------------------------------------------------- MMA issuer
+            constexpr uint32_t idS = idesc_bf16(128, 128, 0, 0);
+            constexpr uint32_t idO = idesc_bf16(128, D, 0, 1);
+            const uint32_t aK = smem_u32(sK), aV = smem_u32(sV);
+            bool ok = mbar_wait_short(kv_full, 0, abort, WB_KF);
+            for (int i = 0; ok && i < steps; ++i) {
+                const int st = i % ST;
+                const uint32_t aQ = smem_u32(sQ(st)), aO = smem_u32(sO(st));
+                if (!(ok = mbar_wait_short(full + st, (i / ST) & 1, abort, WB_FULL))) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {        // S^T = K Q^T, dP^T = V dout^T
+                    const uint32_t off = (kk >> 2) * C::BOX + (kk & 3) * 32;
+                    mma_ss(tmem + C::T_S, sdesc_sw128(aK + off, 16, 1024), sdesc_sw128(aQ + off, 16, 1024),
+                           idS, kk > 0 ? 1u : 0u);
+                    mma_ss(tmem + C::T_P, sdesc_sw128(aV + off, 16, 1024), sdesc_sw128(aO + off, 16, 1024),
+                           idS, kk > 0 ? 1u : 0u);
+                }
+                mma_commit(sdp_full);
+                if (!(ok = mbar_wait_short(ps_full, i & 1, abort, WB_DS))) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {               // dV += P^T dout, dK += dS^T Q
+                    const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
+                    mma_ts(tmem + C::T_A0, tmem + C::T_S + kk * 8, sdesc_sw128(aO + kk * 2048, C::BOX, 1024),
+                           idO, acc);
+                    mma_ts(tmem + C::T_A1, tmem + C::T_P + kk * 8, sdesc_sw128(aQ + kk * 2048, C::BOX, 1024),
+                           idO, acc);
+                }
+                mma_commit(empty + st);
+            }
+            mma_commit(done);
+            bwdtc_drain(done, 0);
+        }
+    } else if (warp < 4) {
+        // ---------------------------------------------------------------- key rows
+        const int r = threadIdx.x;                               // key row of the tile
+        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        const bool live = k0 + r < valid;
+        const float sl2 = rsqrtf((float)D) * 1.4426950408889634f;
+        bool ok = true;
+        for (int i = 0; ok && i < steps; ++i) {
+            const int st = i % ST;
+            const int h = (int)((bh0 + i / nq) % a.H);
+            const int qrel = (i % nq) * 128;                     // query tile - key tile, in rows
+            const float c1 = 1.f - 1.f / (1.f + __expf(-a.beta[h]));
+            // the producer's lse / D writes are visible after this wait
+            if (!(ok = mbar_wait(full + st, (i / ST) & 1, abort, WB_FULL))) break;
+            if (!(ok = mbar_wait(sdp_full, i & 1, abort, WB_SDP))) break;
+            tc_fence_after();
+            const float *sl = sL(st);
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                uint32_t sv[2][32], pv[2][32];
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    tmem_ld32(lane_base + tmem + C::T_S + half * 64 + c * 32, sv[c]);
+                    tmem_ld32(lane_base + tmem + C::T_P + half * 64 + c * 32, pv[c]);
+                }
+                tmem_ld_wait();
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    uint32_t pp[16], dd[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        float p2[2], d2[2];
+#pragma unroll
+                        for (int u = 0; u < 2; ++u) {
+                            const int col = half * 64 + c * 32 + 2 * e + u;   // query in the tile
+                            // causal: query row >= key row; rows past the segment's end out
+                            const bool vis = live && (qrel > 0 || col >= r) && k0 + qrel + col < valid;
+                            const float p = vis ? ex2(fmaf(__uint_as_float(sv[c][2 * e + u]), sl2, -sl[col])) : 0.f;
+                            p2[u] = c1 * p;
+                            d2[u] = p * fmaf(c1, __uint_as_float(pv[c][2 * e + u]), -sl[128 + col]);
+                        }
+                        pp[e] = pack_bf16x2(p2[0], p2[1]);
+                        dd[e] = pack_bf16x2(d2[0], d2[1]);
+                    }
+                    tmem_st16(lane_base + tmem + C::T_S + half * 32 + c * 16, pp);
+                    tmem_st16(lane_base + tmem + C::T_P + half * 32 + c * 16, dd);
+                }
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(ps_full);
+        }
+        if (ok && mbar_wait(done, 0, abort, WB_DONE)) {
+            tc_fence_after();
+            const float rs = rsqrtf((float)D);
+            const int64_t krow = chain * a.L + seg0 + k0 + r;
+#pragma unroll 1
+            for (int c = 0; c < D; c += 32) {
+                uint32_t v32[32], k32[32];
+                tmem_ld32(lane_base + tmem + C::T_A0 + c, v32);
+                tmem_ld32(lane_base + tmem + C::T_A1 + c, k32);
+                tmem_ld_wait();
+                if (live) {
+                    float4 *dv = reinterpret_cast<float4 *>(a.dv + krow * D + c);
+                    float4 *dk = reinterpret_cast<float4 *>(a.dk + krow * D + c);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        dv[e] = make_float4(__uint_as_float(v32[4 * e]), __uint_as_float(v32[4 * e + 1]),
+                                            __uint_as_float(v32[4 * e + 2]), __uint_as_float(v32[4 * e + 3]));
+                        dk[e] = make_float4(__uint_as_float(k32[4 * e]) * rs, __uint_as_float(k32[4 * e + 1]) * rs,
+                                            __uint_as_float(k32[4 * e + 2]) * rs, __uint_as_float(k32[4 * e + 3]) * rs);
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 5) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+}  // namespace tc
+}  // namespace infini

@@ -43,6 +43,11 @@ CASES = [
     make("bf16_delta_d128", B=1, H=4, Hkv=2, d=128, N=128, S=2, tail=64, dtype="bf16",
          rule="delta", seed=96),
     make("bf16_lin_d64", B=2, H=2, Hkv=2, d=64, N=64, S=4, dtype="bf16", seed=97),
+    # tensor-core local attention (N % 128 == 0): several key / query tiles, grouped heads,
+    # a short last segment
+    make("bf16_delta_gqa_n256_tail", B=1, H=4, Hkv=2, d=64, N=256, S=2, tail=100, dtype="bf16",
+         rule="delta", seed=98),
+    make("bf16_lin_n384_d128", B=2, H=2, Hkv=1, d=128, N=384, S=2, dtype="bf16", seed=99),
 ]
 
 
