@@ -1011,7 +1011,7 @@ int64_t bwd_workspace_bytes(const BwdPlan &p)
     const int64_t rows = p.B * p.H * p.L, krows = p.B * p.Hkv * p.L, dd = p.d * p.d;
     const int64_t floats = p.units * dd * 3 + p.units * p.d * 4 + rows * 4 + rows * p.d +
                            p.B * p.H * p.S * p.qtiles + krows * p.d * 3 +
-                           (p.tc ? p.units * (p.d + dd + dd) : 0);   // dz, B_s, A_s hi + lo
+                           (p.tc ? p.units * (p.d + dd + dd + dd / 2) : 0);   // dz, B_s, A_s hi + lo, bf16 M
     return floats * 4 + 20 * 256;
 }
 
@@ -1061,6 +1061,7 @@ Workspace carve_bwd_tc(void *raw, const BwdPlan &p)
     w.Bs = w.dz + (p.units * p.d + 63) / 64 * 64;
     w.Ahi = reinterpret_cast<__nv_bfloat16 *>(w.Bs + p.units * dd);
     w.Alo = w.Ahi + p.units * dd;
+    w.snapMb = w.Alo + p.units * dd;                 // bf16 M_{s-1}, for the row statistics
     return w;
 }
 
@@ -1110,8 +1111,30 @@ int launch_backward(const BwdPlan &p, const T *q, const T *k, const T *v, const 
         k_delta_chain<T, D, 16><<<(unsigned)(chains * (D / 16)), 256, 0, st>>>(
             k, v, snapM, snapZ, nullptr, w.GM, nullptr, p.L, N, S, T_last);
     }
-    // 2. row statistics, the retrieval part of dq, the gate's partial sums
-    {
+    // 2. row statistics, the retrieval part of dq, the gate's partial sums: on the tensor
+    //    cores for bf16 with 128-row tiles (the memory path left bf16 snapshots)
+    bool tc_rows = false;
+    if constexpr (sizeof(T) == 2 && (D == 64 || D == 128)) {
+        if (tc_mem && p.N % 128 == 0) {
+            using CR = tc::BwdRowsCfg<D>;
+            Workspace tw = carve_bwd_tc(raw, p);
+            CUtensorMap mq, mk, mv, mo, mm;
+            if (!make_map_bf16_3d(&mq, q, D, p.L, p.B * p.H, 128) ||
+                !make_map_bf16_3d(&mk, k, D, p.L, p.B * p.Hkv, 128) ||
+                !make_map_bf16_3d(&mv, v, D, p.L, p.B * p.Hkv, 128) ||
+                !make_map_bf16_3d(&mo, dout, D, p.L, p.B * p.H, 128) ||
+                !make_map_bf16_3d(&mm, tw.snapMb, D, D, chains * S, D))
+                return INFINI_ERR_CUDA;
+            if (!opt_in_smem<tc::k_bwd_rows_tc<D>>(CR::ALLOC)) return INFINI_ERR_CUDA;
+            tc::BwdRowsArgs ra{beta, snapZ, w.lse, w.Drow, w.wsc, w.dden, w.dq, w.dbeta_part,
+                               p.L, N, S, H, Hkv, (int)p.qtiles};
+            TRACED("bwd_rows", st);
+            tc::k_bwd_rows_tc<D><<<(unsigned)(p.B * p.H * S * (p.N / 128)), 192, CR::ALLOC, st>>>(
+                mq, mk, mv, mo, mm, ra);
+            tc_rows = true;
+        }
+    }
+    if (!tc_rows) {
         const size_t smem = BwdRowsSmem<D>::bytes;
         if (!opt_in_smem<k_bwd_rows<T, D>>(smem)) return INFINI_ERR_CUDA;
         TRACED("bwd_rows", st);

@@ -15,12 +15,18 @@
 //                  heads and the query tiles at or after the key tile; per query tile:
 //                  S^T = K Q^T and dP^T = V dout^T, (1 - g) P^T over S^T and dS^T over
 //                  dP^T (bf16), dV += P^T dout, dK += dS^T Q; each key row has one owner
+//   k_bwd_rows_tc  one CTA per (b, h, segment, 128 query rows): the forward of the rows
+//                  (S = Q K^T, online softmax, O += P V; sigma(Q) over Q, R = sigma(Q) M and
+//                  dout M^T from one bf16 M tile read MN-major and K-major), then per row
+//                  lse, D = (1 - g) dout . A_dot, the retrieval factors g / den and dden, the
+//                  retrieval part of dq and the gate's partial sum
 // Roles: warps 0-3 one thread per row (elementwise work, epilogue); warp 4 loads (TMA; in
 // k_bwd_dkdv_tc its 32 lanes also stage the query tile's lse and D); warp 5 lane 0 issues
 // the MMAs.  All waits are bounded (tc_common.cuh).
 #pragma once
 
 #include "tc_common.cuh"
+#include "tc_segment_p.cuh"
 
 namespace infini {
 namespace tc {
@@ -56,8 +62,36 @@ struct BwdTcArgs {
     int N, S, H, Hkv;
 };
 
+// Outputs of the row statistics (the same buffers as k_bwd_rows writes)
+struct BwdRowsArgs {
+    const float *beta;
+    const float *snapZ;           // [chains * S, D]: z_{s-1}
+    float *lse, *Drow, *wsc, *dden;   // [B, H, L]
+    float *dq_mem;                // [B, H, L, D]
+    float *dbeta_part;            // [B, H, S, qparts]: qparts 64-row parts per segment
+    int64_t L;
+    int N, S, H, Hkv, qparts;
+};
+
+template <int D>
+struct BwdRowsCfg {
+    static constexpr int TILE = 128 * D * 2, BOX = 128 * 128, ST = 2;
+    static constexpr int MBYTES = D * D * 2, MBOX = D * 128;
+    static constexpr int OFF_Q = 0, OFF_O = TILE, OFF_RING = 2 * TILE;      // ring: ST x (K | V)
+    static constexpr int OFF_M = OFF_RING + ST * 2 * TILE;
+    static constexpr int OFF_Z = OFF_M + MBYTES;
+    static constexpr int OFF_RED = OFF_Z + D * 4;     // 4 warp partial sums of the gate term
+    static constexpr int NBAR = 3 * ST + 8;
+    static constexpr int OFF_BAR = OFF_RED + 16;
+    static constexpr int ALLOC = OFF_BAR + NBAR * 8 + 16 + 1024;
+    static_assert(ALLOC <= 227 * 1024, "shared memory");
+    // TMEM: S [0,128), O, R = sigma(Q) M, dout M^T (d columns each)
+    static constexpr uint32_t T_S = 0, T_O = 128, T_R = 128 + D, T_DM = 128 + 2 * D;
+};
+
 enum : int { WB_QF = 901, WB_KF = 902, WB_VF = 903, WB_KVE = 904, WB_SDP = 905, WB_DS = 906,
-             WB_DONE = 907, WB_FULL = 908, WB_EMPTY = 909, WB_DRAIN = 910 };
+             WB_DONE = 907, WB_FULL = 908, WB_EMPTY = 909, WB_DRAIN = 910, WB_MF = 911,
+             WB_SQ = 912, WB_RF = 913, WB_RED = 914 };
 
 __device__ __forceinline__ void bwdtc_drain(uint64_t *bar, uint32_t parity)
 {
@@ -487,6 +521,334 @@ k_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                                             __uint_as_float(k32[4 * e + 2]) * rs, __uint_as_float(k32[4 * e + 3]) * rs);
                     }
                 }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 5) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+
+// the forward of 128 query rows and the backward's row statistics
+template <int D>
+__global__ void __launch_bounds__(192, 1)
+k_bwd_rows_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+              const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+              const __grid_constant__ CUtensorMap tmM, const BwdRowsArgs a)
+{
+    using C = BwdRowsCfg<D>;
+    constexpr int ST = C::ST;
+    if (__syncthreads_or(threadIdx.x == 0 && wait_status_set())) return;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+    const int qtiles = a.N / 128;
+    int64_t bid = blockIdx.x;
+    const int qt = qtiles - 1 - (int)(bid % qtiles);          // the longest rows first
+    bid /= qtiles;
+    const int s = (int)(bid % a.S);
+    const int64_t bh = bid / a.S;
+    const int h = (int)(bh % a.H);
+    const int64_t chain = (bh / a.H) * a.Hkv + h / (a.H / a.Hkv);
+    const int64_t seg0 = (int64_t)s * a.N;
+    const int valid = (int)(a.L - seg0 < a.N ? a.L - seg0 : a.N);
+    const int q0 = qt * 128;
+    float *part = a.dbeta_part + (bh * a.S + s) * a.qparts + 2 * qt;   // two 64-row parts
+    if (q0 >= valid) {
+        if (threadIdx.x < 2) part[threadIdx.x] = 0.f;
+        return;
+    }
+    const int nk = qt + 1;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    uint8_t *sQ = smem + C::OFF_Q, *sO = smem + C::OFF_O, *sM = smem + C::OFF_M;
+    float *sZ = reinterpret_cast<float *>(smem + C::OFF_Z);
+    float *sRed = reinterpret_cast<float *>(smem + C::OFF_RED);
+    auto sK = [&](int st) { return smem + C::OFF_RING + st * 2 * C::TILE; };
+    auto sV = [&](int st) { return smem + C::OFF_RING + st * 2 * C::TILE + C::TILE; };
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
+    uint64_t *k_full = bars, *v_full = bars + ST, *kv_empty = bars + 2 * ST;
+    uint64_t *q_full = bars + 3 * ST, *m_full = q_full + 1, *s_full = q_full + 2, *p_full = q_full + 3;
+    uint64_t *sq_full = q_full + 4, *r_full = q_full + 5, *red_full = q_full + 6, *mma_done = q_full + 7;
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C::OFF_BAR + C::NBAR * 8);
+    volatile int *abort = reinterpret_cast<volatile int *>(smem + C::OFF_BAR + C::NBAR * 8 + 4);
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < ST; ++i) {
+            mbar_init(k_full + i, 1);
+            mbar_init(v_full + i, 1);
+            mbar_init(kv_empty + i, 1);
+        }
+        mbar_init(q_full, 1);
+        mbar_init(m_full, 1);
+        mbar_init(s_full, 1);
+        mbar_init(p_full, 128);
+        mbar_init(sq_full, 128);
+        mbar_init(r_full, 1);
+        mbar_init(red_full, 4);
+        mbar_init(mma_done, 1);
+        *abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == 5) tmem_alloc(tmem_holder, 512);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+
+    if (warp == 4) {
+        if (lane == 0) {
+            // ---------------------------------------------------------------- loads
+            prefetch_tmap(&tmQ);
+            prefetch_tmap(&tmK);
+            prefetch_tmap(&tmV);
+            prefetch_tmap(&tmO);
+            prefetch_tmap(&tmM);
+            mbar_arrive_expect_tx(q_full, 2 * C::TILE);
+            for (int cb = 0; cb < D / 64; ++cb) {
+                tma_load_3d(sQ + cb * C::BOX, &tmQ, q_full, cb * 64, (int)(seg0 + q0), (int)bh);
+                tma_load_3d(sO + cb * C::BOX, &tmO, q_full, cb * 64, (int)(seg0 + q0), (int)bh);
+            }
+            mbar_arrive_expect_tx(m_full, C::MBYTES + D * 4);
+            for (int cb = 0; cb < D / 64; ++cb)
+                tma_load_3d(sM + cb * C::MBOX, &tmM, m_full, cb * 64, 0, (int)(chain * a.S + s));
+            bulk_load(sZ, a.snapZ + (chain * a.S + s) * (int64_t)D, D * 4, m_full);
+            int issued = 0;
+            for (int j = 0; j < nk; ++j) {
+                const int st = j % ST;
+                if (j >= ST && !mbar_wait_short(kv_empty + st, ((j / ST) - 1) & 1, abort, WB_KVE)) break;
+                mbar_arrive_expect_tx(k_full + st, C::TILE);
+                for (int cb = 0; cb < D / 64; ++cb)
+                    tma_load_3d(sK(st) + cb * C::BOX, &tmK, k_full + st, cb * 64, (int)(seg0 + j * 128),
+                                (int)chain);
+                mbar_arrive_expect_tx(v_full + st, C::TILE);
+                for (int cb = 0; cb < D / 64; ++cb)
+                    tma_load_3d(sV(st) + cb * C::BOX, &tmV, v_full + st, cb * 64, (int)(seg0 + j * 128),
+                                (int)chain);
+                issued = j + 1;
+            }
+            if (*abort) {
+                bwdtc_drain(q_full, 0);
+                bwdtc_drain(m_full, 0);
+                for (int j = (issued > ST ? issued - ST : 0); j < issued; ++j) {
+                    bwdtc_drain(k_full + j % ST, (j / ST) & 1);
+                    bwdtc_drain(v_full + j % ST, (j / ST) & 1);
+                }
+            }
+        }
+    } else if (warp == 5) {
+        if (lane == 0) {
+            // ---------------------------------------------------------------- MMA issuer
+            constexpr uint32_t idS = idesc_bf16(128, 128, 0, 0);
+            constexpr uint32_t idO = idesc_bf16(128, D, 0, 1);     // B MN-major (V; M for R)
+            constexpr uint32_t idK = idesc_bf16(128, D, 0, 0);     // B K-major (M for dout M^T)
+            const uint32_t aQ = smem_u32(sQ), aO = smem_u32(sO), aM = smem_u32(sM);
+            bool ok = mbar_wait_short(q_full, 0, abort, WB_QF);
+            for (int j = 0; ok && j < nk; ++j) {
+                const int st = j % ST;
+                const uint32_t aK = smem_u32(sK(st)), aV = smem_u32(sV(st));
+                if (!(ok = mbar_wait_short(k_full + st, (j / ST) & 1, abort, WB_KF))) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {        // S = Q K^T
+                    const uint32_t off = (kk >> 2) * C::BOX + (kk & 3) * 32;
+                    mma_ss(tmem + C::T_S, sdesc_sw128(aQ + off, 16, 1024), sdesc_sw128(aK + off, 16, 1024),
+                           idS, kk > 0 ? 1u : 0u);
+                }
+                mma_commit(s_full);
+                if (!(ok = mbar_wait_short(p_full, j & 1, abort, WB_DS))) break;
+                if (!(ok = mbar_wait_short(v_full + st, (j / ST) & 1, abort, WB_VF))) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)                 // O += P V (P in S's columns)
+                    mma_ts(tmem + C::T_O, tmem + C::T_S + kk * 8, sdesc_sw128(aV + kk * 2048, C::BOX, 1024),
+                           idO, (j > 0 || kk > 0) ? 1u : 0u);
+                mma_commit(kv_empty + st);
+            }
+            if (ok) ok = mbar_wait_short(m_full, 0, abort, WB_MF);
+            if (ok) ok = mbar_wait_short(sq_full, 0, abort, WB_SQ);
+            if (ok) {
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * C::BOX + (kk & 3) * 32;
+                    // R = sigma(Q) M: B = M, rows a (key features) along K, MN-major
+                    mma_ss(tmem + C::T_R, sdesc_sw128(aQ + off, 16, 1024), sdesc_sw128(aM + kk * 2048, C::MBOX, 1024),
+                           idO, kk > 0 ? 1u : 0u);
+                    // dout M^T: B[c][a] = M[a][c], value columns c along K: K-major
+                    mma_ss(tmem + C::T_DM, sdesc_sw128(aO + off, 16, 1024),
+                           sdesc_sw128(aM + (kk >> 2) * C::MBOX + (kk & 3) * 32, 16, 1024), idK, kk > 0 ? 1u : 0u);
+                }
+                mma_commit(r_full);
+            }
+            mma_commit(mma_done);
+            bwdtc_drain(mma_done, 0);
+        }
+    } else if (warp < 4) {
+        // ---------------------------------------------------------------- rows
+        const int r = threadIdx.x;
+        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        const bool live = q0 + r < valid;
+        const float kscale = rsqrtf((float)D) * 1.4426950408889634f;
+        const float g = 1.f / (1.f + __expf(-a.beta[h]));
+        float m_used = -INFINITY, l = 0.f;
+        bool ok = true;
+        for (int j = 0; ok && j < nk; ++j) {
+            if (!(ok = mbar_wait(s_full, j & 1, abort, WB_SDP))) break;
+            tc_fence_after();
+            const bool diag = (j == qt);
+            uint32_t v[4][32];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tmem_ld32(lane_base + tmem + C::T_S + c * 32, v[c]);
+            tmem_ld_wait();
+            if (diag) {
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        if (c * 32 + e > r) v[c][e] = __float_as_uint(-INFINITY);
+            }
+            float pm[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) pm[u] = __uint_as_float(v[0][u]);
+#pragma unroll
+            for (int u = 4; u < 128; u += 2)
+                pm[(u >> 1) & 3] = max3f(pm[(u >> 1) & 3], __uint_as_float(v[u >> 5][u & 31]),
+                                         __uint_as_float(v[u >> 5][(u & 31) + 1]));
+            const float mt = fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3]));
+            const bool resc = (mt - m_used) * kscale > 8.f;
+            float alpha = 1.f;
+            if (resc) {
+                alpha = ex2((m_used - mt) * kscale);
+                m_used = mt;
+                l *= alpha;
+            }
+            if (j > 0 && __any_sync(0xffffffffu, resc)) {
+                // PV(j-1) is complete: the commit behind S(j) covers it
+#pragma unroll 1
+                for (int c = 0; c < D; c += 32) {
+                    uint32_t o[32];
+                    tmem_ld32(lane_base + tmem + C::T_O + c, o);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                    tmem_st32(lane_base + tmem + C::T_O + c, o);
+                }
+            }
+            const float mk = m_used * kscale;
+            const uint64_t ks2 = f2_pack(kscale, kscale), nm2 = f2_pack(-mk, -mk);
+            uint64_t ps2[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    float y0, y1;
+                    f2_unpack(f2_fma(f2_pack(__uint_as_float(v[c][2 * e]), __uint_as_float(v[c][2 * e + 1])),
+                                     ks2, nm2), y0, y1);
+                    const float p0 = ex2(y0), p1 = ex2(y1);
+                    ps2[e & 3] = f2_add(ps2[e & 3], f2_pack(p0, p1));
+                    pk[e] = pack_bf16x2(p0, p1);
+                }
+                tmem_st16(lane_base + tmem + C::T_S + c * 16, pk);
+            }
+            float rsum[8];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) f2_unpack(ps2[u], rsum[2 * u], rsum[2 * u + 1]);
+            l += ((rsum[0] + rsum[1]) + (rsum[2] + rsum[3])) + ((rsum[4] + rsum[5]) + (rsum[6] + rsum[7]));
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(p_full);
+        }
+        // sigma(Q) over this row (every Q K^T has completed) and den = sigma(q) . z
+        float den = 0.f;
+        if (ok) ok = mbar_wait(q_full, 0, abort, WB_QF);
+        if (ok) ok = mbar_wait(m_full, 0, abort, WB_MF);
+        if (ok) {
+            den = segp_sigma_row<0, D, D / 8>(sQ, r, sZ);
+            fence_proxy_async_smem();
+            mbar_arrive(sq_full);
+        }
+        float gm = 0.f;
+        if (ok && (ok = mbar_wait(r_full, 0, abort, WB_RF))) {
+            tc_fence_after();
+            // per row: A_dot = O / l, A_mem = R / den; dd = dout . A_dot, dam = dout . A_mem
+            const float inv_l = 1.f / l;
+            const float inv_den = den == 0.f ? 0.f : 1.f / den;
+            float dd = 0.f, dam = 0.f;
+#pragma unroll 1
+            for (int c = 0; c < D; c += 32) {
+                uint32_t o[32], rr[32];
+                tmem_ld32(lane_base + tmem + C::T_O + c, o);
+                tmem_ld32(lane_base + tmem + C::T_R + c, rr);
+                tmem_ld_wait();
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int ch = ((c & 63) >> 3) + e;
+                    const uint4 x = *reinterpret_cast<const uint4 *>(sO + (c >> 6) * C::BOX + r * 128 + ((ch ^ (r & 7)) << 4));
+                    const uint32_t w4[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const float d0 = __uint_as_float(w4[u] << 16), d1 = __uint_as_float(w4[u] & 0xffff0000u);
+                        const int i0 = 8 * e + 2 * u;
+                        dd = fmaf(d0, __uint_as_float(o[i0]) * inv_l, fmaf(d1, __uint_as_float(o[i0 + 1]) * inv_l, dd));
+                        dam = fmaf(d0, __uint_as_float(rr[i0]) * inv_den, fmaf(d1, __uint_as_float(rr[i0 + 1]) * inv_den, dam));
+                    }
+                }
+            }
+            const float wsc = den == 0.f ? 0.f : g * inv_den;
+            const float ddn = den == 0.f ? 0.f : -g * dam * inv_den;
+            gm = live ? dam - dd : 0.f;
+            const int64_t row = bh * a.L + seg0 + q0 + r;
+            if (live) {
+                a.lse[row] = m_used * kscale + __log2f(l);
+                a.Drow[row] = (1.f - g) * dd;
+                a.wsc[row] = wsc;
+                a.dden[row] = ddn;
+            }
+            // the retrieval part of dq: (wsc dout M^T + dden z) * sigma'(q), sigma' = min(sigma, 1)
+#pragma unroll 1
+            for (int c = 0; c < D; c += 32) {
+                uint32_t dm[32];
+                tmem_ld32(lane_base + tmem + C::T_DM + c, dm);
+                tmem_ld_wait();
+                if (live) {
+                    float4 *dst = reinterpret_cast<float4 *>(a.dq_mem + row * D + c);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int ch = ((c & 63) >> 3) + e;
+                        const uint4 x = *reinterpret_cast<const uint4 *>(sQ + (c >> 6) * C::BOX + r * 128 + ((ch ^ (r & 7)) << 4));
+                        const uint32_t w4[4] = {x.x, x.y, x.z, x.w};
+                        float y[8];
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const float s0 = __uint_as_float(w4[u] << 16), s1 = __uint_as_float(w4[u] & 0xffff0000u);
+                            const int i0 = 8 * e + 2 * u;
+                            y[2 * u] = fmaf(wsc, __uint_as_float(dm[i0]), ddn * sZ[c + i0]) * fminf(s0, 1.f);
+                            y[2 * u + 1] = fmaf(wsc, __uint_as_float(dm[i0 + 1]), ddn * sZ[c + i0 + 1]) * fminf(s1, 1.f);
+                        }
+                        dst[2 * e] = make_float4(y[0], y[1], y[2], y[3]);
+                        dst[2 * e + 1] = make_float4(y[4], y[5], y[6], y[7]);
+                    }
+                }
+            }
+        }
+        // the gate's partial sums: rows 0-63 and 64-127 of the tile, each in a fixed order
+        if (ok) {
+            float t = gm;
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) t += __shfl_xor_sync(0xffffffffu, t, off);
+            if (lane == 0) {
+                sRed[warp] = t;
+                mbar_arrive(red_full);
+            }
+            if (threadIdx.x == 0 && mbar_wait(red_full, 0, abort, WB_RED)) {
+                part[0] = g * (1.f - g) * (sRed[0] + sRed[1]);
+                part[1] = g * (1.f - g) * (sRed[2] + sRed[3]);
             }
         }
     }
