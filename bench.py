@@ -451,22 +451,29 @@ def backward_flops(w: wl.Workload):
 
 def backward_roofline(w: wl.Workload, kernels: dict, steps: int, clk: dict) -> dict:
     """The backward's dominant kernel against its own ceiling.  Algorithmic flops per
-    (b, h, segment), one causal product = d N (N + 1): k_bwd_rows recomputes S and P V (2)
-    plus the retrieval's sigma(q) M and dout M^T (4 N d^2), on CUDA cores; the dq kernel S, dP
-    and dS K (3), the dk/dv kernel S^T, dP^T, P^T dout and dS^T Q (4), on the tensor cores for
-    bf16 with N % 128 == 0 (bf16 peak), else on CUDA cores (fp32 FMA peak)."""
+    (b, h, segment), one causal product = d N (N + 1): the row statistics recompute S and P V
+    (2) plus the retrieval's sigma(q) M and dout M^T (4 N d^2); the dq kernel S, dP and dS K
+    (3); the dk/dv kernel S^T, dP^T, P^T dout and dS^T Q (4); G^M 2 N d^2; the update
+    (per kv head) 8 N d^2 (delta) or 4 N d^2 (linear).  On the tensor cores (bf16 peak) for
+    bf16 with d in {64, 128} and N % 128 == 0 except the update, else on CUDA cores (fp32 FMA
+    peak)."""
     B, H, N, d = w.B, w.H, w.N, w.d
     S = -(-w.L // N)
     prod = B * H * S * d * N * (N + 1)
-    flops = {"bwd_rows": 2 * prod + B * H * S * 4 * N * d * d, "bwd_dq": 3 * prod, "bwd_dkdv": 4 * prod}
+    # G^M_s: one N x d x d product per (b, h, segment); the update: 4 (delta) or 2 (linear)
+    # N x d x d products per (b, kv head, segment)
+    upd = (8 if w.rule == "delta" else 4) * N * d * d * B * w.Hkv * S
+    flops = {"bwd_rows": 2 * prod + B * H * S * 4 * N * d * d, "bwd_dq": 3 * prod, "bwd_dkdv": 4 * prod,
+             "bwd_gm": B * H * S * 2 * N * d * d, "bwd_update": upd}
     tensor = w.dtype == "bf16" and d in (64, 128) and N % 128 == 0
+    on_tc = {"bwd_rows", "bwd_dq", "bwd_dkdv", "bwd_gm"} if tensor else set()
     cand = {k: v for k, v in kernels.items() if k in flops}
     if not cand:
         return None
     dom = max(cand, key=lambda k: cand[k]["ms"])
     ms = cand[dom]["ms"] / max(1, cand[dom]["launches"]) * (cand[dom]["launches"] / max(1, steps))
     achieved = flops[dom] / (ms / 1e3) / 1e12 if ms > 0 else 0.0
-    if tensor and dom != "bwd_rows":
+    if dom in on_tc:
         peaks, src = load_peaks()
         peak, bound, psrc = peaks["bf16_tflops"], "tensor", f"{src} (burst)"
     else:

@@ -1181,8 +1181,24 @@ int launch_backward(const BwdPlan &p, const T *q, const T *k, const T *v, const 
         k_bwd_dkdv<T, D><<<(unsigned)(chains * S * p.qtiles), 256, smem, st>>>(
             q, k, v, beta, dout, w, p.L, N, S, H, Hkv);
     }
-    // 5. G^M_s, G^z_s;  6. the reverse memory recurrence
-    {
+    // 5. G^M_s, G^z_s (on the tensor cores with the tensor-core row statistics);
+    // 6. the reverse memory recurrence
+    bool tc_gm = false;
+    if constexpr (sizeof(T) == 2 && (D == 64 || D == 128)) {
+        if (tc_rows) {
+            using CG = tc::BwdGmCfg<D>;
+            CUtensorMap mq, mo;
+            if (!make_map_bf16_3d(&mq, q, D, p.L, p.B * p.H, 128) ||
+                !make_map_bf16_3d(&mo, dout, D, p.L, p.B * p.H, 128))
+                return INFINI_ERR_CUDA;
+            if (!opt_in_smem<tc::k_bwd_gm_tc<D>>(CG::ALLOC)) return INFINI_ERR_CUDA;
+            tc::BwdGmArgs ga{w.wsc, w.dden, w.GM, w.Gz, p.L, N, S, H, Hkv};
+            TRACED("bwd_gm", st);
+            tc::k_bwd_gm_tc<D><<<(unsigned)units, 192, CG::ALLOC, st>>>(mq, mo, ga);
+            tc_gm = true;
+        }
+    }
+    if (!tc_gm) {
         TRACED("bwd_gm", st);
         k_bwd_gm<T, D><<<(unsigned)units, 256, 0, st>>>(q, dout, w, p.L, N, S, H, Hkv);
     }

@@ -20,6 +20,10 @@
 //                  dout M^T from one bf16 M tile read MN-major and K-major), then per row
 //                  lse, D = (1 - g) dout . A_dot, the retrieval factors g / den and dden, the
 //                  retrieval part of dq and the gate's partial sum
+//   k_bwd_gm_tc    one CTA per (b, kv head, segment): G^M_s = sum over the group's rows of
+//                  (wsc sigma(q))^T dout and G^z_s = sum sigma(q) dden in one product
+//                  [wsc sigma(Q)]^T [dout | dden / wsc] (the extra column is 0 where wsc is:
+//                  dden is 0 there too); wsc sigma(Q) is written over the staged Q tile
 // Roles: warps 0-3 one thread per row (elementwise work, epilogue); warp 4 loads (TMA; in
 // k_bwd_dkdv_tc its 32 lanes also stage the query tile's lse and D); warp 5 lane 0 issues
 // the MMAs.  All waits are bounded (tc_common.cuh).
@@ -87,6 +91,28 @@ struct BwdRowsCfg {
     static_assert(ALLOC <= 227 * 1024, "shared memory");
     // TMEM: S [0,128), O, R = sigma(Q) M, dout M^T (d columns each)
     static constexpr uint32_t T_S = 0, T_O = 128, T_R = 128 + D, T_DM = 128 + 2 * D;
+};
+
+struct BwdGmArgs {
+    const float *wsc, *dden;      // [B, H, L] from the row statistics
+    float *GM, *Gz;               // [chains * S, D, D], [chains * S, D]
+    int64_t L;
+    int N, S, H, Hkv;
+};
+
+template <int D>
+struct BwdGmCfg {
+    static constexpr int BOX = 128 * 128, NB = D / 64, ST = 2;
+    // stage: A = wsc sigma(Q) over Q (features padded to 128 with a zero box at d = 64) |
+    //        dout (NB boxes) | the extra column's box
+    static constexpr int OFF_AQ = 0, OFF_DO = 2 * BOX, OFF_EX = OFF_DO + NB * BOX;
+    static constexpr int STAGE = OFF_EX + BOX;
+    static constexpr int NBAR = 3 * ST + 1;
+    static constexpr int OFF_BAR = ST * STAGE;
+    static constexpr int ALLOC = OFF_BAR + NBAR * 8 + 16 + 1024;
+    static_assert(ALLOC <= 227 * 1024, "shared memory");
+    static constexpr int NACC = D + 16;                    // G^M columns, then the G^z column
+    static constexpr uint32_t TMEM_COLS = NACC <= 128 ? 128 : 256;
 };
 
 enum : int { WB_QF = 901, WB_KF = 902, WB_VF = 903, WB_KVE = 904, WB_SDP = 905, WB_DS = 906,
@@ -858,6 +884,173 @@ k_bwd_rows_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     if (warp == 5) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);
+    }
+}
+
+
+// G^M_s and G^z_s of one (b, kv head, segment)
+template <int D>
+__global__ void __launch_bounds__(192, 1)
+k_bwd_gm_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
+            const BwdGmArgs a)
+{
+    using C = BwdGmCfg<D>;
+    constexpr int ST = C::ST;
+    if (__syncthreads_or(threadIdx.x == 0 && wait_status_set())) return;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+    const int64_t cs = blockIdx.x;                           // chain * S + s
+    const int64_t chain = cs / a.S;
+    const int s = (int)(cs % a.S);
+    const int G = a.H / a.Hkv;
+    const int64_t bh0 = (chain / a.Hkv) * a.H + (chain % a.Hkv) * G;
+    const int64_t seg0 = (int64_t)s * a.N;
+    const int valid = (int)(a.L - seg0 < a.N ? a.L - seg0 : a.N);
+    const int nt = (valid + 127) / 128;                      // 128-row tiles of the segment
+    const int steps = G * nt;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    auto stage = [&](int st) { return smem + st * C::STAGE; };
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
+    uint64_t *full = bars, *ready = bars + ST, *empty = bars + 2 * ST, *done = bars + 3 * ST;
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C::OFF_BAR + C::NBAR * 8);
+    volatile int *abort = reinterpret_cast<volatile int *>(smem + C::OFF_BAR + C::NBAR * 8 + 4);
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < ST; ++i) {
+            mbar_init(full + i, 1);
+            mbar_init(ready + i, 128);
+            mbar_init(empty + i, 1);
+        }
+        mbar_init(done, 1);
+        *abort = 0;
+        fence_barrier_init();
+    }
+    if (D == 64)       // the padded feature box of both stages' A tiles stays zero
+        for (int i = threadIdx.x; i < ST * (C::BOX / 16); i += blockDim.x)
+            reinterpret_cast<uint4 *>(stage(i / (C::BOX / 16)) + C::OFF_AQ + C::BOX)[i % (C::BOX / 16)] =
+                make_uint4(0, 0, 0, 0);
+    if (warp == 5) tmem_alloc(tmem_holder, C::TMEM_COLS);
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+
+    if (warp == 4) {
+        if (lane == 0) {
+            // ---------------------------------------------------------------- loads
+            prefetch_tmap(&tmQ);
+            prefetch_tmap(&tmO);
+            int issued = 0;
+            for (int i = 0; i < steps; ++i) {
+                const int st = i % ST;
+                const int64_t bh = bh0 + i / nt;
+                const int row = (int)(seg0 + (i % nt) * 128);
+                if (i >= ST && !mbar_wait_short(empty + st, ((i / ST) - 1) & 1, abort, WB_EMPTY)) break;
+                mbar_arrive_expect_tx(full + st, 2 * C::NB * C::BOX);
+                for (int cb = 0; cb < C::NB; ++cb) {
+                    tma_load_3d(stage(st) + C::OFF_AQ + cb * C::BOX, &tmQ, full + st, cb * 64, row, (int)bh);
+                    tma_load_3d(stage(st) + C::OFF_DO + cb * C::BOX, &tmO, full + st, cb * 64, row, (int)bh);
+                }
+                issued = i + 1;
+            }
+            if (*abort)
+                for (int i = (issued > ST ? issued - ST : 0); i < issued; ++i)
+                    bwdtc_drain(full + i % ST, (i / ST) & 1);
+        }
+    } else if (warp == 5) {
+        if (lane == 0) {
+            // ---------------------------------------------------------------- MMA issuer
+            constexpr uint32_t id = idesc_bf16(128, C::NACC, 1, 1);    // both operands MN-major
+            bool ok = true;
+            for (int i = 0; ok && i < steps; ++i) {
+                const int st = i % ST;
+                if (!(ok = mbar_wait_short(ready + st, (i / ST) & 1, abort, WB_DS))) break;
+                tc_fence_after();
+                const uint32_t aA = smem_u32(stage(st) + C::OFF_AQ), aB = smem_u32(stage(st) + C::OFF_DO);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)                 // 16 rows per step
+                    mma_ss(tmem, sdesc_sw128(aA + kk * 2048, C::BOX, 1024), sdesc_sw128(aB + kk * 2048, C::BOX, 1024),
+                           id, (i > 0 || kk > 0) ? 1u : 0u);
+                mma_commit(empty + st);
+            }
+            mma_commit(done);
+            bwdtc_drain(done, 0);
+        }
+    } else if (warp < 4) {
+        // ---------------------------------------------------------------- rows
+        const int r = threadIdx.x;
+        bool ok = true;
+        for (int i = 0; ok && i < steps; ++i) {
+            const int st = i % ST;
+            const int64_t bh = bh0 + i / nt;
+            const int t = (i % nt) * 128 + r;                    // row in the segment
+            const bool in = t < valid;
+            const float wsc = in ? a.wsc[bh * a.L + seg0 + t] : 0.f;
+            const float dd = in ? a.dden[bh * a.L + seg0 + t] : 0.f;
+            if (!(ok = mbar_wait(full + st, (i / ST) & 1, abort, WB_FULL))) break;
+            // A row = wsc sigma(q) over the Q row, in place (the TMA wrote it; the wait above
+            // makes it visible); the extra column dden / wsc
+            uint8_t *q = stage(st) + C::OFF_AQ;
+            const uint64_t one2 = f2_pack(1.f, 1.f);
+            const uint64_t log2e2 = f2_pack(1.4426950408889634f, 1.4426950408889634f);
+            const uint64_t w2 = f2_pack(wsc, wsc);
+#pragma unroll 4
+            for (int c0 = 0; c0 < D; c0 += 8) {
+                const int ch = (c0 & 63) >> 3;
+                uint4 *ptr = reinterpret_cast<uint4 *>(q + (c0 >> 6) * C::BOX + r * 128 + ((ch ^ (r & 7)) << 4));
+                const uint4 x = *ptr;
+                uint32_t w4[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float x0 = __uint_as_float(w4[e] << 16), x1 = __uint_as_float(w4[e] & 0xffff0000u);
+                    float a0, a1, p0, p1;
+                    f2_unpack(f2_mul(f2_pack(fminf(x0, 0.f), fminf(x1, 0.f)), log2e2), a0, a1);
+                    f2_unpack(f2_add(f2_pack(x0, x1), one2), p0, p1);
+                    float y0, y1;
+                    f2_unpack(f2_mul(f2_pack(fmaxf(p0, ex2(a0)), fmaxf(p1, ex2(a1))), w2), y0, y1);
+                    w4[e] = pack_bf16x2(y0, y1);
+                }
+                *ptr = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+            }
+            uint8_t *ex = stage(st) + C::OFF_EX + r * 128;
+            const uint32_t e0 = pack_bf16x2(wsc == 0.f ? 0.f : dd / wsc, 0.f);
+            *reinterpret_cast<uint4 *>(ex + ((0 ^ (r & 7)) << 4)) = make_uint4(e0, 0u, 0u, 0u);
+            *reinterpret_cast<uint4 *>(ex + ((1 ^ (r & 7)) << 4)) = make_uint4(0u, 0u, 0u, 0u);
+            fence_proxy_async_smem();
+            mbar_arrive(ready + st);
+        }
+        // lane a of the accumulator is key feature a: row a of G^M and G^z[a]
+        if (ok && mbar_wait(done, 0, abort, WB_DONE)) {
+            tc_fence_after();
+            const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+            const bool live = r < D;
+#pragma unroll 1
+            for (int c = 0; c < C::NACC; c += 16) {
+                uint32_t x[16];
+                tmem_ld16(lane_base + tmem + c, x);
+                tmem_ld_wait();
+                if (live) {
+                    if (c < D) {
+                        float4 *dst = reinterpret_cast<float4 *>(a.GM + (cs * D + r) * D + c);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            dst[e] = make_float4(__uint_as_float(x[4 * e]), __uint_as_float(x[4 * e + 1]),
+                                                 __uint_as_float(x[4 * e + 2]), __uint_as_float(x[4 * e + 3]));
+                    } else {
+                        a.Gz[cs * D + r] = __uint_as_float(x[0]);
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 5) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
     }
 }
 
