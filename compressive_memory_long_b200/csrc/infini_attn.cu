@@ -1226,7 +1226,28 @@ int launch_backward(const BwdPlan &p, const T *q, const T *k, const T *v, const 
         k_bwd_mdelta<T, D, 16><<<(unsigned)(chains * (D / 16)), 256, 0, st>>>(k, dM, w, dM0, p.L, N, S);
     }
     // 7. the update's gradients;  8. the reverse z recurrence
-    {
+    bool tc_upd = false;
+    if constexpr (sizeof(T) == 2 && (D == 64 || D == 128)) {
+        if (tc_mem && p.N % 128 == 0) {
+            using CU = tc::BwdUpdCfg<D>;
+            CUtensorMap mk, mv;
+            if (!make_map_bf16_3d(&mk, k, D, p.L, p.B * p.Hkv, 128) ||
+                !make_map_bf16_3d(&mv, v, D, p.L, p.B * p.Hkv, 128))
+                return INFINI_ERR_CUDA;
+            tc::BwdUpdArgs ua{w.dMs, snapM, snapZ, w.dv, w.dsk, w.h, p.L, N, S};
+            if (p.rule == INFINI_UPDATE_LINEAR) {
+                if (!opt_in_smem<tc::k_bwd_update_tc<D, false>>(CU::ALLOC)) return INFINI_ERR_CUDA;
+                TRACED("bwd_update", st);
+                tc::k_bwd_update_tc<D, false><<<(unsigned)units, 192, CU::ALLOC, st>>>(mk, mv, ua);
+            } else {
+                if (!opt_in_smem<tc::k_bwd_update_tc<D, true>>(CU::ALLOC)) return INFINI_ERR_CUDA;
+                TRACED("bwd_update", st);
+                tc::k_bwd_update_tc<D, true><<<(unsigned)units, 192, CU::ALLOC, st>>>(mk, mv, ua);
+            }
+            tc_upd = true;
+        }
+    }
+    if (!tc_upd) {
         const size_t smem = BwdUpdSmem<D>::bytes;
         if (p.rule == INFINI_UPDATE_LINEAR) {
             if (!opt_in_smem<k_bwd_update<T, D, false>>(smem)) return INFINI_ERR_CUDA;

@@ -24,6 +24,13 @@
 //                  (wsc sigma(q))^T dout and G^z_s = sum sigma(q) dden in one product
 //                  [wsc sigma(Q)]^T [dout | dden / wsc] (the extra column is 0 where wsc is:
 //                  dden is 0 there too); wsc sigma(Q) is written over the staged Q tile
+//   k_bwd_update_tc one CTA per (b, kv head, segment), per 128-token tile: dU = sigma(K) dM_s
+//                  (dv += dU) and, for the delta rule, sigma(K) M_{s-1} = den R; then
+//                  dsigma(k) = U dM_s^T - (dU / den) M_{s-1}^T + dden z with U = v - R,
+//                  dden = dU . R / den, and h_s += sigma(K)^T dden; linear: dsigma(k) = V dM_s^T.
+//                  dM_s and M_{s-1} enter as bf16 hi + lo tiles (read MN-major and K-major):
+//                  one rounding of them is shared by every row, so its error would add up
+//                  coherently in h_s; dden enters as hi + lo columns
 // Roles: warps 0-3 one thread per row (elementwise work, epilogue); warp 4 loads (TMA; in
 // k_bwd_dkdv_tc its 32 lanes also stage the query tile's lse and D); warp 5 lane 0 issues
 // the MMAs.  All waits are bounded (tc_common.cuh).
@@ -115,9 +122,31 @@ struct BwdGmCfg {
     static constexpr uint32_t TMEM_COLS = NACC <= 128 ? 128 : 256;
 };
 
+struct BwdUpdArgs {
+    const float *dMs, *snapM, *snapZ;   // [chains * S, D, D], [chains * S, D, D], [chains * S, D]
+    float *dv, *dsk, *h;                // [B, Hkv, L, D] (+=), [B, Hkv, L, D], [chains * S, D]
+    int64_t L;
+    int N, S;
+};
+
+template <int D>
+struct BwdUpdCfg {
+    static constexpr int BOX = 128 * 128, NB = D / 64, MBOX = D * 128, MBYTES = D * D * 2;
+    // sigma(K) over K (features padded to 128 with a zero box at d = 64), then -dU / den over it
+    // | V, then U | the dden columns' box | dM_s hi, lo | M_{s-1} hi, lo (bf16) | z
+    static constexpr int OFF_K = 0, OFF_V = 2 * BOX, OFF_E = OFF_V + NB * BOX;
+    static constexpr int OFF_DM = OFF_E + BOX, OFF_M = OFF_DM + 2 * MBYTES, OFF_Z = OFF_M + 2 * MBYTES;
+    static constexpr int NBAR = 9;
+    static constexpr int OFF_BAR = OFF_Z + D * 4;
+    static constexpr int ALLOC = OFF_BAR + NBAR * 8 + 16 + 1024;
+    static_assert(ALLOC <= 227 * 1024, "shared memory");
+    // TMEM: dU | sigma(K) M | dsigma(k) (d columns each) | h (16)
+    static constexpr uint32_t T_1 = 0, T_2 = D, T_3 = 2 * D, T_H = 3 * D;
+};
+
 enum : int { WB_QF = 901, WB_KF = 902, WB_VF = 903, WB_KVE = 904, WB_SDP = 905, WB_DS = 906,
              WB_DONE = 907, WB_FULL = 908, WB_EMPTY = 909, WB_DRAIN = 910, WB_MF = 911,
-             WB_SQ = 912, WB_RF = 913, WB_RED = 914 };
+             WB_SQ = 912, WB_RF = 913, WB_RED = 914, WB_UR = 915, WB_P3 = 916 };
 
 __device__ __forceinline__ void bwdtc_drain(uint64_t *bar, uint32_t parity)
 {
@@ -1051,6 +1080,312 @@ k_bwd_gm_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
     if (warp == 5) {
         tc_fence_after();
         tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+
+// the memory update's gradients of one (b, kv head, segment)
+template <int D, bool DELTA>
+__global__ void __launch_bounds__(192, 1)
+k_bwd_update_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                const BwdUpdArgs a)
+{
+    using C = BwdUpdCfg<D>;
+    if (__syncthreads_or(threadIdx.x == 0 && wait_status_set())) return;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+    const int64_t cs = blockIdx.x;                           // chain * S + s
+    const int64_t chain = cs / a.S;
+    const int s = (int)(cs % a.S);
+    const int64_t seg0 = (int64_t)s * a.N;
+    const int valid = (int)(a.L - seg0 < a.N ? a.L - seg0 : a.N);
+    const int nt = (valid + 127) / 128;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    uint8_t *sK = smem + C::OFF_K, *sV = smem + C::OFF_V, *sE = smem + C::OFF_E;
+    uint8_t *sDU = sK;                                       // -dU / den, after h has read sigma(K)
+    uint8_t *sDM = smem + C::OFF_DM, *sM = smem + C::OFF_M;  // hi at +0, lo at +MBYTES
+    float *sz = reinterpret_cast<float *>(smem + C::OFF_Z);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
+    uint64_t *full = bars, *mready = bars + 1, *kready = bars + 2, *p12 = bars + 3, *uready = bars + 4;
+    uint64_t *p3 = bars + 5, *done = bars + 6, *eready = bars + 7, *hdone = bars + 8;
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C::OFF_BAR + C::NBAR * 8);
+    volatile int *abort = reinterpret_cast<volatile int *>(smem + C::OFF_BAR + C::NBAR * 8 + 4);
+
+    if (threadIdx.x == 0) {
+        mbar_init(full, 1);
+        mbar_init(mready, 128);
+        mbar_init(kready, 128);
+        mbar_init(p12, 1);
+        mbar_init(uready, 128);
+        mbar_init(p3, 1);
+        mbar_init(done, 1);
+        mbar_init(eready, 128);
+        mbar_init(hdone, 1);
+        *abort = 0;
+        fence_barrier_init();
+    }
+    if (D == 64)       // the padded feature box of sigma(K) stays zero
+        for (int i = threadIdx.x; i < C::BOX / 16; i += blockDim.x)
+            reinterpret_cast<uint4 *>(sK + C::BOX)[i] = make_uint4(0, 0, 0, 0);
+    if (warp == 5) tmem_alloc(tmem_holder, 512);
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+
+    if (warp == 4) {
+        if (lane == 0) {
+            // ---------------------------------------------------------------- loads
+            prefetch_tmap(&tmK);
+            prefetch_tmap(&tmV);
+            bool ok = true;
+            int issued = 0;
+            for (int i = 0; ok && i < nt; ++i) {
+                // the tile's buffers are free once the previous tile's last products are done
+                if (i > 0 && !(ok = mbar_wait(p3, (i - 1) & 1, abort, WB_P3))) break;
+                mbar_arrive_expect_tx(full, 2 * C::NB * C::BOX);
+                for (int cb = 0; cb < C::NB; ++cb) {
+                    tma_load_3d(sK + cb * C::BOX, &tmK, full, cb * 64, (int)(seg0 + i * 128), (int)chain);
+                    tma_load_3d(sV + cb * C::BOX, &tmV, full, cb * 64, (int)(seg0 + i * 128), (int)chain);
+                }
+                issued = i + 1;
+            }
+            if (*abort && issued > 0) bwdtc_drain(full, (issued - 1) & 1);
+        }
+    } else if (warp == 5) {
+        if (lane == 0) {
+            // ---------------------------------------------------------------- MMA issuer
+            constexpr uint32_t idMN = idesc_bf16(128, D, 0, 1);   // B = dM / M, MN-major
+            constexpr uint32_t idK = idesc_bf16(128, D, 0, 0);    // B = dM^T / M^T, K-major
+            constexpr uint32_t idH = idesc_bf16(128, 16, 1, 1);   // h: A = sigma(K) MN-major
+            const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aDU = smem_u32(sDU), aE = smem_u32(sE);
+            const uint32_t aDM = smem_u32(sDM), aM = smem_u32(sM);
+            constexpr uint32_t LO = C::MBYTES;
+            bool ok = mbar_wait_short(mready, 0, abort, WB_MF);
+            for (int i = 0; ok && i < nt; ++i) {
+                if (!(ok = mbar_wait_short(kready, i & 1, abort, WB_FULL))) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {                 // dU, sigma(K) M: hi + lo parts
+                    const uint32_t off = (kk >> 2) * C::BOX + (kk & 3) * 32;
+                    const uint64_t ak = sdesc_sw128(aK + off, 16, 1024);
+                    mma_ss(tmem + C::T_1, ak, sdesc_sw128(aDM + kk * 2048, C::MBOX, 1024), idMN, kk > 0 ? 1u : 0u);
+                    mma_ss(tmem + C::T_1, ak, sdesc_sw128(aDM + LO + kk * 2048, C::MBOX, 1024), idMN, 1u);
+                    if (DELTA) {
+                        mma_ss(tmem + C::T_2, ak, sdesc_sw128(aM + kk * 2048, C::MBOX, 1024), idMN, kk > 0 ? 1u : 0u);
+                        mma_ss(tmem + C::T_2, ak, sdesc_sw128(aM + LO + kk * 2048, C::MBOX, 1024), idMN, 1u);
+                    }
+                }
+                mma_commit(p12);
+                if (DELTA) {
+                    if (!(ok = mbar_wait_short(eready, i & 1, abort, WB_UR))) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)             // h += sigma(K)^T [dden_hi | dden_lo]
+                        mma_ss(tmem + C::T_H, sdesc_sw128(aK + kk * 2048, C::BOX, 1024),
+                               sdesc_sw128(aE + kk * 2048, C::BOX, 1024), idH, (i > 0 || kk > 0) ? 1u : 0u);
+                    mma_commit(hdone);
+                }
+                if (!(ok = mbar_wait_short(uready, i & 1, abort, WB_UR))) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * C::BOX + (kk & 3) * 32;
+                    const uint32_t boff = (kk >> 2) * C::MBOX + (kk & 3) * 32;
+                    // U dM^T, then (-dU / den) M^T into the same accumulator
+                    mma_ss(tmem + C::T_3, sdesc_sw128(aV + off, 16, 1024), sdesc_sw128(aDM + boff, 16, 1024),
+                           idK, kk > 0 ? 1u : 0u);
+                    if (DELTA)
+                        mma_ss(tmem + C::T_3, sdesc_sw128(aDU + off, 16, 1024), sdesc_sw128(aM + boff, 16, 1024),
+                               idK, 1u);
+                }
+                mma_commit(p3);
+            }
+            mma_commit(done);
+            bwdtc_drain(done, 0);
+        }
+    } else if (warp < 4) {
+        // ---------------------------------------------------------------- rows
+        const int r = threadIdx.x;
+        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        // dM_s and M_{s-1} as bf16 tiles (row r of each), z_{s-1}
+        if (r < D) {
+            const float4 *g4 = reinterpret_cast<const float4 *>(a.dMs + (cs * D + r) * D);
+            const float4 *m4 = reinterpret_cast<const float4 *>(a.snapM + (cs * D + r) * D);
+#pragma unroll
+            for (int c0 = 0; c0 < D; c0 += 8) {
+                const int ch = (c0 & 63) >> 3;
+                const int off = (c0 >> 6) * C::MBOX + r * 128 + ((ch ^ (r & 7)) << 4);
+                // x = hi + lo in two bf16 parts, 8 values at a time
+                auto split = [&](const float4 &x0, const float4 &x1, uint8_t *dst) {
+                    const float v8[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+                    uint32_t hi[4], lo[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        hi[e] = pack_bf16x2(v8[2 * e], v8[2 * e + 1]);
+                        lo[e] = pack_bf16x2(v8[2 * e] - __uint_as_float(hi[e] << 16),
+                                            v8[2 * e + 1] - __uint_as_float(hi[e] & 0xffff0000u));
+                    }
+                    *reinterpret_cast<uint4 *>(dst + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                    *reinterpret_cast<uint4 *>(dst + C::MBYTES + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+                };
+                split(g4[c0 / 4], g4[c0 / 4 + 1], sDM);
+                if (DELTA) split(m4[c0 / 4], m4[c0 / 4 + 1], sM);
+            }
+            sz[r] = DELTA ? a.snapZ[cs * D + r] : 0.f;
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(mready);
+        const uint64_t one2 = f2_pack(1.f, 1.f);
+        const uint64_t log2e2 = f2_pack(1.4426950408889634f, 1.4426950408889634f);
+        bool ok = mbar_wait(mready, 0, abort, WB_MF);       // z visible to every row
+        for (int i = 0; ok && i < nt; ++i) {
+            const int t = i * 128 + r;                           // row in the segment
+            const bool in = t < valid;
+            const uint32_t keep = in ? 0xFFFFFFFFu : 0u;         // rows past the end: sigma = 0
+            if (!(ok = mbar_wait(full, i & 1, abort, WB_FULL))) break;
+            // sigma(k) over the K row, den = sigma(k) . z from the unrounded sigma
+            uint64_t dp2[2] = {0ull, 0ull};
+#pragma unroll 4
+            for (int c0 = 0; c0 < D; c0 += 8) {
+                const int ch = (c0 & 63) >> 3;
+                uint4 *ptr = reinterpret_cast<uint4 *>(sK + (c0 >> 6) * C::BOX + r * 128 + ((ch ^ (r & 7)) << 4));
+                const uint4 x = *ptr;
+                uint32_t w4[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float x0 = __uint_as_float(w4[e] << 16), x1 = __uint_as_float(w4[e] & 0xffff0000u);
+                    float a0, a1, p0, p1;
+                    f2_unpack(f2_mul(f2_pack(fminf(x0, 0.f), fminf(x1, 0.f)), log2e2), a0, a1);
+                    f2_unpack(f2_add(f2_pack(x0, x1), one2), p0, p1);
+                    const float s0 = __uint_as_float(__float_as_uint(fmaxf(p0, ex2(a0))) & keep);
+                    const float s1 = __uint_as_float(__float_as_uint(fmaxf(p1, ex2(a1))) & keep);
+                    if (DELTA) dp2[e & 1] = f2_fma(f2_pack(s0, s1), f2_pack(sz[c0 + 2 * e], sz[c0 + 2 * e + 1]), dp2[e & 1]);
+                    w4[e] = pack_bf16x2(s0, s1);
+                }
+                *ptr = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+            }
+            float d0, d1, d2, d3;
+            f2_unpack(dp2[0], d0, d1);
+            f2_unpack(dp2[1], d2, d3);
+            const float den = (d0 + d1) + (d2 + d3);
+            const float inv = den == 0.f ? 0.f : 1.f / den;
+            fence_proxy_async_smem();
+            mbar_arrive(kready);
+            if (!(ok = mbar_wait(p12, i & 1, abort, WB_SDP))) break;
+            tc_fence_after();
+            const int64_t row = chain * a.L + seg0 + t;
+            // dU_t (dv += dU_t) and, delta, R_t = (sigma(k_t) M) / den, U_t = v_t - R_t written
+            // over V, -dU_t / den over the dU tile, dden_t = dU_t . R_t / den into the column box
+            float dd = 0.f;
+#pragma unroll 1
+            for (int c = 0; c < D; c += 32) {
+                uint32_t du[32], rm[32];
+                tmem_ld32(lane_base + tmem + C::T_1 + c, du);
+                if (DELTA) tmem_ld32(lane_base + tmem + C::T_2 + c, rm);
+                tmem_ld_wait();
+                if (in) {
+                    float4 *dvp = reinterpret_cast<float4 *>(a.dv + row * D + c);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        float4 x = dvp[e];
+                        x.x += __uint_as_float(du[4 * e]);
+                        x.y += __uint_as_float(du[4 * e + 1]);
+                        x.z += __uint_as_float(du[4 * e + 2]);
+                        x.w += __uint_as_float(du[4 * e + 3]);
+                        dvp[e] = x;
+                    }
+                }
+                if (DELTA) {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int ch = ((c & 63) >> 3) + e;
+                        const int off = (c >> 6) * C::BOX + r * 128 + ((ch ^ (r & 7)) << 4);
+                        uint4 *vp = reinterpret_cast<uint4 *>(sV + off);
+                        const uint4 vx = *vp;
+                        const uint32_t v4[4] = {vx.x, vx.y, vx.z, vx.w};
+                        uint32_t u4[4];
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const int i0 = 8 * e + 2 * u;
+                            const float r0 = __uint_as_float(rm[i0]) * inv, r1 = __uint_as_float(rm[i0 + 1]) * inv;
+                            dd = fmaf(__uint_as_float(du[i0]), r0, fmaf(__uint_as_float(du[i0 + 1]), r1, dd));
+                            u4[u] = pack_bf16x2(__uint_as_float(v4[u] << 16) - r0, __uint_as_float(v4[u] & 0xffff0000u) - r1);
+                        }
+                        *vp = make_uint4(u4[0], u4[1], u4[2], u4[3]);
+                    }
+                }
+            }
+            const float dden = DELTA ? dd * inv : 0.f;
+            if (DELTA) {
+                // dden as hi + lo columns; sigma(K) stays until h has read it
+                uint8_t *ex = sE + r * 128;
+                const uint32_t dh = pack_bf16x2(dden, 0.f);
+                const uint32_t dl = pack_bf16x2(0.f, dden - __uint_as_float(dh << 16));
+                *reinterpret_cast<uint4 *>(ex + ((0 ^ (r & 7)) << 4)) = make_uint4(dh | dl, 0u, 0u, 0u);
+                *reinterpret_cast<uint4 *>(ex + ((1 ^ (r & 7)) << 4)) = make_uint4(0u, 0u, 0u, 0u);
+                fence_proxy_async_smem();
+                mbar_arrive(eready);
+                // -dU / den over sigma(K) once h has read it (dU read again from TMEM)
+                if (!(ok = mbar_wait(hdone, i & 1, abort, WB_UR))) break;
+                tc_fence_after();
+#pragma unroll 1
+                for (int c = 0; c < D; c += 32) {
+                    uint32_t du[32];
+                    tmem_ld32(lane_base + tmem + C::T_1 + c, du);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int ch = ((c & 63) >> 3) + e;
+                        const int off = (c >> 6) * C::BOX + r * 128 + ((ch ^ (r & 7)) << 4);
+                        uint32_t n4[4];
+#pragma unroll
+                        for (int u = 0; u < 4; ++u)
+                            n4[u] = pack_bf16x2(-__uint_as_float(du[8 * e + 2 * u]) * inv,
+                                                -__uint_as_float(du[8 * e + 2 * u + 1]) * inv);
+                        *reinterpret_cast<uint4 *>(sDU + off) = make_uint4(n4[0], n4[1], n4[2], n4[3]);
+                    }
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(uready);
+            if (!(ok = mbar_wait(p3, i & 1, abort, WB_P3))) break;
+            tc_fence_after();
+            // dsigma(k_t) = U dM^T - (dU / den) M^T + dden z (without the dz_s term)
+#pragma unroll 1
+            for (int c = 0; c < D; c += 32) {
+                uint32_t x[32];
+                tmem_ld32(lane_base + tmem + C::T_3 + c, x);
+                tmem_ld_wait();
+                if (in) {
+                    float4 *dst = reinterpret_cast<float4 *>(a.dsk + row * D + c);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        dst[e] = make_float4(fmaf(dden, sz[c + 4 * e], __uint_as_float(x[4 * e])),
+                                             fmaf(dden, sz[c + 4 * e + 1], __uint_as_float(x[4 * e + 1])),
+                                             fmaf(dden, sz[c + 4 * e + 2], __uint_as_float(x[4 * e + 2])),
+                                             fmaf(dden, sz[c + 4 * e + 3], __uint_as_float(x[4 * e + 3])));
+                }
+            }
+        }
+        // h_s: lane a of the h accumulator is key feature a
+        if (ok && mbar_wait(done, 0, abort, WB_DONE)) {
+            tc_fence_after();
+            uint32_t x[16];
+            tmem_ld16(lane_base + tmem + C::T_H, x);
+            tmem_ld_wait();
+            if (r < D) a.h[cs * D + r] = DELTA ? __uint_as_float(x[0]) + __uint_as_float(x[1]) : 0.f;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 5) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
     }
 }
 
