@@ -14,7 +14,7 @@
 //   k_zsum      per (chain, segment): dz_s = sum_t sigma(k_t), fp32 on the CUDA cores
 //   k_zscan     per chain: z_{s-1} for every segment (what the segment kernel and den read)
 //   k_mem_incr  per (chain, segment), all at once, on the tensor cores: B_s and (delta) A_s
-//   k_mem_chain delta: per (chain, 32 value columns), the recurrence in segment order, one
+//   k_mem_chain delta: per (chain, 16 value columns), the recurrence in segment order, one
 //               d x d x 32 product per segment on the tensor cores
 //   k_mem_prefix linear: the running sum M0 + sum_{j<s} B_j, elementwise
 // The last two write the bf16 snapshots M_{s-1} the segment kernel reads, and M_out.
@@ -116,7 +116,7 @@ struct IncrCfg {
     static constexpr int BOX = CH * 128;             // 64 rows x 64 bf16 (128-byte rows)
     // ring slot (TMA): the K chunk, turned into sigma_hi in place (features padded to 128:
     // for d = 64 the second box stays zero), then the V chunk
-    static constexpr int RS = 3;
+    static constexpr int RS = 4;
     static constexpr int OFF_SH = 0;
     static constexpr int OFF_V = 2 * BOX;
     static constexpr int SLOT = (2 + NB) * BOX;
@@ -527,7 +527,7 @@ k_mem_prefix(const float *__restrict__ Bs, const float *M0, __nv_bfloat16 *__res
 template <int D>
 struct MChainCfg {
     static_assert(D == 64 || D == 128, "tensor-core delta recurrence: d = 64 or 128");
-    static constexpr int CB = 32;                   // value columns per CTA
+    static constexpr int CB = 16;                   // value columns per CTA
     static constexpr int NK = D / 64;               // 64-wide boxes along the contraction
     static constexpr int ABOX = 128 * 128;          // 128 rows x 64 bf16
     static constexpr int ATILE = NK * ABOX;         // A_hi (or A_lo) of one segment
@@ -570,7 +570,7 @@ __device__ __forceinline__ void mchain_drain(uint64_t *bar, uint32_t parity)
 
 // Delta rule: M_s = M_{s-1} + B_s - A_s M_{s-1} in segment order (with `reverse`, from the
 // last segment to the first: the backward's dM_{s-1} = dM_s + G_s - A_s dM_s, A_s being
-// symmetric; the snapshot of each step is then the gradient after the segment).  One CTA per (chain, 32
+// symmetric; the snapshot of each step is then the gradient after the segment).  One CTA per (chain, 16
 // value columns); column block j of M_s needs only column block j of M_{s-1}.  Warp 0: TMA
 // of A_s (hi and lo parts, K-major, two stages ahead).  Warp 1: MMA issuer, D = A_hi M_hi +
 // A_hi M_lo + A_lo M_hi into 32 TMEM columns.  Warps 4-7: thread i holds row i of the block

@@ -48,6 +48,8 @@ CASES = [
     make("bf16_delta_gqa_n256_tail", B=1, H=4, Hkv=2, d=64, N=256, S=2, tail=100, dtype="bf16",
          rule="delta", seed=98),
     make("bf16_lin_n384_d128", B=2, H=2, Hkv=1, d=128, N=384, S=2, dtype="bf16", seed=99),
+    make("bf16_delta_g4_d128_tail", B=1, H=8, Hkv=2, d=128, N=256, S=3, tail=129, dtype="bf16",
+         rule="delta", seed=100),
 ]
 
 
