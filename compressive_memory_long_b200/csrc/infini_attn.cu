@@ -232,19 +232,22 @@ bool make_map_bf16_3d(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// The tensor-core segment kernel covers bf16 activations, d in {64, 128}, N % 128 == 0.
+// The tensor-core path covers bf16 activations, d in {64, 128}, N % 128 == 0 or N = 64
+// (two 64-token segments per 128-row tile).
 template <typename T>
 bool use_tc(const Problem &p)
 {
-    return sizeof(T) == 2 && (p.d == 64 || p.d == 128) && p.N % 128 == 0;
+    return sizeof(T) == 2 && (p.d == 64 || p.d == 128) && (p.N % 128 == 0 || p.N == 64);
 }
 
-// One launch for 64-token segments under the additive rule (bf16, d = 64, MHA).
+// One launch for 64-token segments under the additive rule (bf16, d = 64): whole 128-token
+// units only, so never a problem whose last segment is short (L < Lf once effective() has
+// made a short tail one more segment).
 template <typename T>
 bool use_small_fused(const Problem &p)
 {
     return sizeof(T) == 2 && p.d == 64 && p.N == 64 && p.rule == INFINI_UPDATE_LINEAR &&
-           p.Lf % 128 == 0;
+           p.Lf % 128 == 0 && p.L >= p.Lf;
 }
 
 // Long heads (16 units of 128 tokens or more) go to the persistent piece kernel.
@@ -397,7 +400,8 @@ int launch_segment_tc(const Problem &p, const __nv_bfloat16 *q, const __nv_bfloa
         return INFINI_OK;
     }
     if (!opt_in_smem<tc::k_segment_tc<D>>(C::ALLOC)) return INFINI_ERR_CUDA;
-    const int64_t ctas = p.B * p.H * p.S * (p.N / 128);
+    // N = 64: one CTA per pair of consecutive segments
+    const int64_t ctas = p.N == 64 ? p.B * p.H * ((p.S + 1) / 2) : p.B * p.H * p.S * (p.N / 128);
     TRACED("segment_tc", st);
     tc::k_segment_tc<D><<<(unsigned)ctas, 256, C::ALLOC, st>>>(mq, mk, mv, mm, a);
     return INFINI_OK;
@@ -415,6 +419,7 @@ int launch_small_fused(const Problem &p, const __nv_bfloat16 *q, const __nv_bflo
                        const float *z0, __nv_bfloat16 *out, float *M_out, float *z_out,
                        void *ws, cudaStream_t st)
 {
+    if (p.L < p.Lf || p.Lf % 128 != 0) return INFINI_ERR_UNSUPPORTED;   // whole 128-token units
     using C = tc::SmallCfg;
     const int64_t chains = p.B * p.H, U = p.Lf / 128, units = chains * U;   // query-head chains
     // workspace: ticket, per-head M0 reader counts, flags (all zeroed here), then the
@@ -477,6 +482,7 @@ int launch_pieces(const Problem &p, const __nv_bfloat16 *q, const __nv_bfloat16 
                   const __nv_bfloat16 *v, const float *beta, const float *M0, const float *z0,
                   __nv_bfloat16 *out, float *M_out, float *z_out, void *ws, cudaStream_t st)
 {
+    if (p.L < p.Lf || p.Lf % 128 != 0) return INFINI_ERR_UNSUPPORTED;   // whole 128-token units
     using C = tc::PieceCfg;
     const PiecePlan pl = piece_plan(p);
     int *ticket = static_cast<int *>(ws);
@@ -632,13 +638,14 @@ int launch_tail(const Problem &p, const T *q, const T *k, const T *v, const floa
 // The problem the kernels run.  On the tensor-core path a final short segment is simply
 // one more segment: TMA fills its rows past L with zeros, the memory kernels leave those
 // rows out of the update (zero sigma(K)), and the segment kernel neither computes tiles
-// that start past L nor stores rows past L.  Elsewhere the CUDA-core tail follows the
-// full segments.
+// that start past L nor stores rows past L.  Elsewhere, and after the fused 64-token
+// kernels (which take whole 128-token units only), the CUDA-core tail follows the full
+// segments.
 template <typename T>
 Problem effective(const Problem &p)
 {
     Problem e = p;
-    if (p.T > 0 && use_tc<T>(p)) {
+    if (p.T > 0 && use_tc<T>(p) && !use_small_fused<T>(p)) {
         e.S = p.S + 1;
         e.Lf = e.S * p.N;
         e.T = 0;
@@ -670,8 +677,8 @@ int64_t call_workspace_bytes(const Problem &p)
     if (use_small_fused<T>(p)) {
         const int64_t fused = use_pieces(p) ? pieces_workspace_bytes(p) : small_workspace_bytes(p);
         if (p.H == p.Hkv) return fused;
-        // grouped heads updated in place take the general (CUDA-core) path: room for both
-        const int64_t general = simt_workspace_bytes(units, p.d);
+        // grouped heads updated in place take the general (tensor-core) path: room for both
+        const int64_t general = tc_workspace_bytes(units, p.d, p.rule == INFINI_UPDATE_DELTA);
         return fused > general ? fused : general;
     }
     return use_tc<T>(p) ? tc_workspace_bytes(units, p.d, p.rule == INFINI_UPDATE_DELTA)

@@ -5,6 +5,11 @@
 //   A_mem = sigma(Q) M_{s-1} / (sigma(Q) . z_{s-1})        (0 where the denominator is 0)
 //   out   = g A_mem + (1 - g) A_dot,  g = sigmoid(beta[h])
 // (AI Wiki "Infini-Attention", "What happens inside the Infini-attention block?").
+// With 64-token segments (N = 64) the 128 rows are two consecutive segments s, s + 1: one
+// key step over the same 128 rows under a block-diagonal causal mask (each segment sees only
+// its own keys), and two retrievals, sigma(Q) M_{s-1} into S0 for the first 64 rows and
+// sigma(Q) M_s into S1 (unused by the single key step) for the others; the second snapshot
+// is loaded into the key ring's second slot, which the single key step leaves free.
 //
 // Roles (256 threads):
 //   warp 0      TMA producer: Q tile, M_{s-1} (bf16 snapshot), K/V tiles through a ring
@@ -42,7 +47,8 @@ struct SegCfg {
     static constexpr int OFF_M = OFF_V + STAGES * TILE;
     static constexpr int OFF_Z = OFF_M + MBYTES;
     static constexpr int NBAR = 2 + 3 * STAGES + 2 + 2 + 4;
-    static constexpr int OFF_BAR = OFF_Z + D * 4;
+    static constexpr int OFF_BAR = OFF_Z + 2 * D * 4;   // z of one segment (two at N = 64)
+    static_assert(STAGES >= 2 && MBYTES <= TILE, "second snapshot in the key ring's slot 1");
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int BYTES = OFF_MISC + 16;
     static constexpr int ALLOC = BYTES + 1024;      // slack to align the base to 1024 B
@@ -86,12 +92,23 @@ k_segment_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
 
-    const int qtiles = a.N / C::BQ;
+    // N = 64: a CTA per pair of segments (s, s + 1); s1 = -1 when the pair has no second
+    const bool pair = a.N == 64;
     int64_t bid = blockIdx.x;
-    const int qt = qtiles - 1 - (int)(bid % qtiles);   // longest rows first
-    bid /= qtiles;
-    const int s = (int)(bid % a.S);
-    bid /= a.S;
+    int qt, s, s1 = -1;
+    if (pair) {
+        const int U = (a.S + 1) / 2;
+        s = 2 * (int)(bid % U);
+        bid /= U;
+        qt = 0;
+        if (s + 1 < a.S) s1 = s + 1;
+    } else {
+        const int qtiles = a.N / C::BQ;
+        qt = qtiles - 1 - (int)(bid % qtiles);   // longest rows first
+        bid /= qtiles;
+        s = (int)(bid % a.S);
+        bid /= a.S;
+    }
     // a last segment shorter than N: tiles past the head's L rows have nothing to do
     if ((int64_t)s * a.N + qt * C::BQ >= a.L) return;
     const int64_t bh = bid;
@@ -154,9 +171,13 @@ k_segment_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
             mbar_arrive_expect_tx(q_full, C::TILE);
             for (int cb = 0; cb < D / 64; ++cb)
                 tma_load_3d(sQ + cb * C::BOX, &tmQ, q_full, cb * 64, q_row, (int)bh);
-            mbar_arrive_expect_tx(m_full, C::MBYTES);
+            mbar_arrive_expect_tx(m_full, (s1 >= 0 ? 2 : 1) * C::MBYTES);
             for (int cb = 0; cb < D / 64; ++cb)
                 tma_load_3d(sM + cb * C::MBOX, &tmM, m_full, cb * 64, 0, (int)(chain * a.S + s));
+            if (s1 >= 0)
+                for (int cb = 0; cb < D / 64; ++cb)
+                    tma_load_3d(sK + C::TILE + cb * C::MBOX, &tmM, m_full, cb * 64, 0,
+                                (int)(chain * a.S + s1));
             int issued = 0;
             for (int j = 0; j < nkv; ++j) {
                 const int st = j % ST;
@@ -222,16 +243,19 @@ k_segment_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
                 if (j > 0) ok = issue_pv(j - 1);
             }
             if (ok) ok = issue_pv(nkv - 1);
-            // retrieval R = sigma(Q) M_{s-1} into S0
+            // retrieval R = sigma(Q) M_{s-1} into S0 (and sigma(Q) M_s into S1 for a pair)
             if (ok) ok = mbar_wait(m_full, 0, abort, W_M);
             if (ok) ok = mbar_wait(sq_full, 0, abort, W_SQ);
             if (ok) {
                 tc_fence_after();
+                for (int x = 0; x < (s1 >= 0 ? 2 : 1); ++x) {
+                    const uint32_t mb = x == 0 ? aM : aK + C::TILE;
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * C::BOX + (kk & 3) * 32;
-                    mma_ss(T_S0, sdesc_sw128(aQ + off, 16, 1024),
-                           sdesc_sw128(aM + kk * 2048, C::MBOX, 1024), idO, kk > 0 ? 1u : 0u);
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t off = (kk >> 2) * C::BOX + (kk & 3) * 32;
+                        mma_ss(x == 0 ? T_S0 : T_S1, sdesc_sw128(aQ + off, 16, 1024),
+                               sdesc_sw128(mb + kk * 2048, C::MBOX, 1024), idO, kk > 0 ? 1u : 0u);
+                    }
                 }
                 mma_commit(r_full);
             }
@@ -244,8 +268,14 @@ k_segment_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
         const int r = threadIdx.x - 128;                 // query row of this thread
         const uint32_t lane_base = (uint32_t)((warp - 4) * 32) << 16;
         const float *zsrc = a.snapZ + (chain * a.S + s) * (int64_t)D;
-        for (int i = r; i < D; i += 128) sZ[i] = zsrc[i];
+        for (int i = r; i < D; i += 128) {
+            sZ[i] = zsrc[i];
+            if (pair) sZ[D + i] = s1 >= 0 ? zsrc[D + i] : 0.f;   // z_s of the pair's second
+        }
         asm volatile("bar.sync 1, 128;" ::: "memory");
+        // the rows of a pair's second segment use its own memory (S1, z_s)
+        const bool second = pair && r >= 64;
+        const float *zr = sZ + (second ? D : 0);
 
         const float kscale = rsqrtf((float)D) * 1.4426950408889634f;
         float m_used = -INFINITY, l = 0.f;
@@ -263,7 +293,7 @@ k_segment_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
             if (j == qt) {                                  // causal mask on the diagonal tile
 #pragma unroll
                 for (int c = 0; c < 128; ++c)
-                    if (c > r) raw[c >> 5][c & 31] = __float_as_uint(-INFINITY);
+                    if (c > r || (second && c < 64)) raw[c >> 5][c & 31] = __float_as_uint(-INFINITY);
             }
             float pm[8];
 #pragma unroll
@@ -331,8 +361,8 @@ k_segment_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
                         x0 = elu1(x0);
                         x1 = elu1(x1);
                         const int c = cb * 64 + ch * 8 + 2 * e;
-                        den = fmaf(x0, sZ[c], den);
-                        den = fmaf(x1, sZ[c + 1], den);
+                        den = fmaf(x0, zr[c], den);
+                        den = fmaf(x1, zr[c + 1], den);
                         w[e] = pack_bf16x2(x0, x1);
                     }
                     *p = make_uint4(w[0], w[1], w[2], w[3]);
@@ -352,7 +382,7 @@ k_segment_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
                 for (int c = 0; c < D; c += 32) {
                     uint32_t o[32], rr[32];
                     tmem_ld32(lane_base + T_O + c, o);
-                    tmem_ld32(lane_base + T_S0 + c, rr);
+                    tmem_ld32(lane_base + (second ? T_S1 : T_S0) + c, rr);
                     tmem_ld_wait();
                     uint32_t pk[16];
 #pragma unroll

@@ -261,6 +261,48 @@ def test_tensor_core_first_segment_empty_memory():
     assert binding.infini_attn_device_status() == 0
 
 
+# ---- 64-token segments on the tensor cores: a pair of segments per 128-row tile ------
+
+@pytest.mark.parametrize("rule", ["linear", "delta"])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("H,Hkv,S", [(4, 4, 6), (8, 2, 5), (2, 1, 1)])
+def test_tensor_core_64_token_segments(rule, d, H, Hkv, S):
+    """N = 64 where the fused additive-rule kernels do not apply (the delta rule, d = 128, or
+    a segment count that is not a whole number of 128-token units): one CTA per pair of
+    segments (block-diagonal causal mask, each half retrieving from its own memory), an odd
+    number of segments (a pair without its second), a single segment; the memory path and
+    the segment kernel both on the tensor cores, no CUDA-core segment kernel."""
+    from compressive_memory_long_b200 import binding
+    w = wl.Workload("tc64", B=2, H=H, Hkv=Hkv, d=d, N=64, S=S, dtype="bf16", rule=rule, seed=31,
+                    beta_dist=("normal", 0.0, 1.5), M0_dist=("uniform", 0.0, 0.1),
+                    z0_dist=("uniform", 1.0, 2.0))
+    fused = rule == "linear" and d == 64 and S % 2 == 0
+    binding.infini_attn_trace_enable(True)
+    check_full(w)
+    binding.infini_attn_trace_enable(False)
+    report = list(binding.infini_attn_trace_report())
+    if fused:
+        assert report in (["small_fused"], ["small_pieces"]), report
+    else:
+        assert "segment_tc" in report and "mem_increments" in report, report
+        assert ("mem_chain" if rule == "delta" else "mem_prefix") in report, report
+        assert not any(n in report for n in ("segment_simt", "delta_chain", "tail_segment")), report
+    assert binding.infini_attn_device_status() == 0
+
+
+def test_tensor_core_64_token_pair_halves_use_their_own_memory():
+    """beta -> +inf (the output is the retrieval alone) and M0 = 0, z0 = 0: the first
+    segment's rows are exactly 0 (empty memory), while the second segment of the same
+    128-row tile retrieves from the memory after the first segment, so its rows are not."""
+    from compressive_memory_long_b200 import binding
+    w = wl.Workload("tc64_halves", B=1, H=2, Hkv=2, d=128, N=64, S=2, dtype="bf16",
+                    rule="delta", seed=32, beta_dist=("normal", 40.0, 0.0))
+    out, _, _ = run_gpu(w)
+    assert torch.count_nonzero(out[:, :, :64]) == 0
+    assert torch.count_nonzero(out[:, :, 64:]) > 0
+    assert binding.infini_attn_device_status() == 0
+
+
 # ---- the fused single-launch path (bf16, linear rule, N = 64, d = 64, MHA) -------------
 
 @pytest.mark.parametrize("S", [2, 4, 6, 16])

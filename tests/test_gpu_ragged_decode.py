@@ -46,8 +46,9 @@ def dev_inputs(w):
 
 
 # (workload, a kernel that must run, whether the CUDA-core tail runs).  On the tensor-core
-# path (bf16, d in {64, 128}, N % 128 == 0) the short segment is one more segment of the
-# tensor-core kernels; elsewhere the CUDA-core tail follows the full segments.
+# path (bf16, d in {64, 128}, N % 128 == 0 or N = 64) the short segment is one more segment
+# of the tensor-core kernels; after the fused 64-token kernels (additive rule, d = 64, whole
+# 128-token units) and elsewhere the CUDA-core tail follows the full segments.
 RAGGED = [
     (make("fused64", B=2, H=4, Hkv=4, d=64, N=64, S=6, tail=37, seed=11), "small_fused", True),
     (make("pieces64", B=1, H=2, Hkv=2, d=64, N=64, S=40, tail=1, state=True, seed=12),
@@ -56,7 +57,11 @@ RAGGED = [
      "small_fused", True),
     (make("pieces64_gqa", B=1, H=6, Hkv=3, d=64, N=64, S=34, tail=63, seed=27),
      "small_pieces", True),
-    (make("odd_s64", B=1, H=2, Hkv=2, d=64, N=64, S=3, tail=50, seed=13), "segment_simt", True),
+    (make("odd_s64", B=1, H=2, Hkv=2, d=64, N=64, S=3, tail=50, seed=13), "segment_tc", False),
+    (make("tc_delta_n64", B=1, H=4, Hkv=2, d=64, N=64, S=5, tail=20, rule="delta", state=True,
+          seed=28), "mem_chain", False),
+    (make("tc_n64_d128", B=2, H=2, Hkv=1, d=128, N=64, S=2, tail=63, seed=29), "segment_tc",
+     False),
     (make("simt_d32", B=1, H=2, Hkv=2, d=32, N=64, S=2, tail=10, seed=17), "segment_simt", True),
     (make("f32_delta", B=1, H=2, Hkv=2, d=64, N=64, S=2, tail=33, dtype="f32", rule="delta",
           state=True, seed=18), "delta_chain", True),
