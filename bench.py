@@ -84,6 +84,15 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+def tensor_peak(peaks: dict, clk: dict):
+    """(peak TFLOP/s, kind) for a tensor-bound kernel: the sustained bf16 figure when the
+    clock record of its timed region shows sw_power_cap active (the loop ran long enough for
+    the power cap to lower the clock), else the burst one."""
+    if "sw_power_cap" in ((clk or {}).get("reasons") or []) and peaks.get("bf16_tflops_sustained"):
+        return peaks["bf16_tflops_sustained"], "sustained: sw_power_cap active in the timed region"
+    return peaks["bf16_tflops"], "burst"
+
+
 # ---- algorithmic work per kernel (flops and bytes; snapshots and re-reads excluded) ----
 
 def algorithmic(w: wl.Workload, kernel: str):
@@ -476,11 +485,9 @@ def backward_roofline(w: wl.Workload, kernels: dict, steps: int, clk: dict) -> d
     frac_burst = None
     if dom in on_tc:
         peaks, src = load_peaks()
-        peak, bound, psrc = peaks["bf16_tflops"], "tensor", f"{src} (burst)"
-        frac_burst = achieved / peak
-        if "sw_power_cap" in (clk.get("reasons") or []) and peaks.get("bf16_tflops_sustained"):
-            peak = peaks["bf16_tflops_sustained"]
-            psrc = f"{src} (sustained: sw_power_cap active in the timed region)"
+        frac_burst = achieved / peaks["bf16_tflops"]
+        peak, kind = tensor_peak(peaks, clk)
+        bound, psrc = "tensor", f"{src} ({kind})"
     else:
         peak, bound = fp32_fma_peak_tflops(clk["sm_mhz"] or 1965.0), "alu"
         psrc = "derived: 148 SMs x 128 fp32 lanes x 2 x SM clock"
@@ -706,9 +713,7 @@ def main():
         # act (sw_power_cap seen during the timed region) is held to the sustained figure, a
         # kernel that ran at full clock to the burst one; both fractions are reported
         burst = peaks["bf16_tflops"]
-        peak = burst
-        if "sw_power_cap" in clocks.summary().get("reasons", []) and peaks.get("bf16_tflops_sustained"):
-            peak, peak_kind = peaks["bf16_tflops_sustained"], "sustained: sw_power_cap active in the timed region"
+        peak, peak_kind = tensor_peak(peaks, clocks.summary())
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak,
                 "unit": "TFLOP/s", "frac": achieved / peak, "frac_of_burst_peak": achieved / burst}
     else:

@@ -21,3 +21,20 @@ def test_bench_rejects_bad_flags(args, needle):
                        text=True, timeout=300)
     assert r.returncode == 2
     assert needle in r.stderr
+
+
+def test_tensor_peak_follows_the_power_cap():
+    """A tensor-bound kernel is held to the sustained bf16 figure only when the clock record
+    of its timed region shows sw_power_cap active; otherwise (no reason, other reasons, no
+    NVML, no sustained figure) to the burst one."""
+    sys.path.insert(0, ROOT)
+    import bench
+    peaks = {"bf16_tflops": 1665.9, "bf16_tflops_sustained": 1414.4, "hbm_gbs": 6544.0}
+    assert bench.tensor_peak(peaks, {"reasons": ["sw_power_cap"]})[0] == 1414.4
+    assert bench.tensor_peak(peaks, {"reasons": ["sw_power_cap", "sync_boost"]})[0] == 1414.4
+    assert bench.tensor_peak(peaks, {"reasons": []}) == (1665.9, "burst")
+    assert bench.tensor_peak(peaks, {"reasons": ["sync_boost"]})[0] == 1665.9
+    assert bench.tensor_peak(peaks, {"reasons": None})[0] == 1665.9
+    assert bench.tensor_peak(peaks, None)[0] == 1665.9
+    no_sustained = {"bf16_tflops": 1590.0, "hbm_gbs": 6650.0}
+    assert bench.tensor_peak(no_sustained, {"reasons": ["sw_power_cap"]})[0] == 1590.0
