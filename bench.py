@@ -57,18 +57,51 @@ FLUSH_BYTES = 256 << 20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from an ncu
-# capture, keyed by (workload, kernel).  Absent: no capture of the current kernel.  The
-# summaries with the commands are under profiles/.  The N = 64 bandwidth, batched and 1M-stream
-# figures are captures of fewer segments scaled to the workload's (traffic grows with the
-# units processed).
-NCU_TRAFFIC_BYTES: dict = {
-    ("hf_repro_n64", "small_fused"): 6362112,
-    ("n64_bandwidth", "small_pieces"): (1028091000 + 268262400) * 8,
-    ("gqa8b_n2048_delta", "segment_tc"): 413104384 + 238214912,
-    # 4 of 8 segments captured (x 2) and 16 of 512 segments captured (x 32)
-    ("batched_n1024_linear", "segment_tc"): (1701618688 + 515050496) * 2,
-    ("stream1m_n2048_delta", "segment_tc"): (413484800 + 109220352) * 32,
+# capture, keyed by (workload, kernel), with a digest of the kernel's source files at the
+# time of the capture: a kernel whose sources have changed since reports no traffic (the
+# counters no longer describe it) until it is captured again.  The summaries with the
+# commands are under profiles/.  The N = 64 bandwidth, batched and 1M-stream figures are
+# captures of fewer segments scaled to the workload's (traffic grows with the units
+# processed).
+KERNEL_SOURCES = {
+    "segment_tc": ("tc_segment_p.cuh", "tc_segment.cuh", "tc_common.cuh"),
+    "small_pieces": ("tc_pieces.cuh", "tc_small.cuh", "tc_common.cuh"),
+    "small_fused": ("tc_small.cuh", "tc_common.cuh"),
 }
+NCU_TRAFFIC_BYTES: dict = {
+    ("hf_repro_n64", "small_fused"): (6364160, "b4076352787a7b26"),
+    # 2048 of 16384 segments captured (x 8)
+    ("n64_bandwidth", "small_pieces"): ((1032990976 + 268926464) * 8, "5c6fb8137091e762"),
+    ("gqa8b_n2048_delta", "segment_tc"): (421510144 + 238118912, "09d83465c9002f40"),
+    # 4 of 8 segments captured (x 2) and 16 of 512 segments captured (x 32)
+    ("batched_n1024_linear", "segment_tc"): ((1704829184 + 515661312) * 2, "09d83465c9002f40"),
+    ("stream1m_n2048_delta", "segment_tc"): ((413263872 + 112340992) * 32, "09d83465c9002f40"),
+}
+
+
+def kernel_digest(kernel: str):
+    """sha256 (first 16 hex digits) of the CUDA sources a kernel is compiled from, or None."""
+    import hashlib
+    files = KERNEL_SOURCES.get(kernel)
+    if not files:
+        return None
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "compressive_memory_long_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def captured_traffic(workload: str, kernel: str):
+    """(bytes per launch or None, note): the captured DRAM traffic when it describes the
+    kernel as built now."""
+    entry = NCU_TRAFFIC_BYTES.get((workload, kernel))
+    if entry is None:
+        return None, "no ncu capture of this kernel on this workload"
+    byts, digest = entry
+    if kernel_digest(kernel) != digest:
+        return None, "stale: the kernel's sources changed since the ncu capture"
+    return byts, "ncu capture of the current kernel"
 
 
 def fp32_fma_peak_tflops(sm_mhz=1965.0, sms=148):
@@ -720,7 +753,7 @@ def main():
         achieved = byts / (dom_ms / 1e3) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm_gbs"]}
-    roof["traffic"] = NCU_TRAFFIC_BYTES.get((w.name, dom))
+    roof["traffic"], roof["traffic_source"] = captured_traffic(w.name, dom)
     roof.update({"kernel": dom, "kernel_ms": dom_ms, "peak_source": f"{peak_src} ({peak_kind})",
                  "algorithmic_flops": flops, "algorithmic_bytes": byts,
                  "kernel_share": kernels[dom]["ms"] / sum(v["ms"] for v in kernels.values())})

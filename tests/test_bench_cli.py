@@ -38,3 +38,22 @@ def test_tensor_peak_follows_the_power_cap():
     assert bench.tensor_peak(peaks, None)[0] == 1665.9
     no_sustained = {"bf16_tflops": 1590.0, "hbm_gbs": 6650.0}
     assert bench.tensor_peak(no_sustained, {"reasons": ["sw_power_cap"]})[0] == 1590.0
+
+
+def test_captured_traffic_is_dropped_once_the_kernel_changes():
+    """The bench line's roofline.traffic comes from an ncu capture recorded with a digest of
+    the kernel's sources: a matching digest gives the bytes, a changed one (the kernel was
+    edited after the capture) or a missing entry gives None."""
+    sys.path.insert(0, ROOT)
+    import bench
+    key = ("test_workload", "segment_tc")
+    try:
+        bench.NCU_TRAFFIC_BYTES[key] = (123456, bench.kernel_digest("segment_tc"))
+        assert bench.captured_traffic(*key)[0] == 123456
+        bench.NCU_TRAFFIC_BYTES[key] = (123456, "0" * 16)
+        byts, note = bench.captured_traffic(*key)
+        assert byts is None and note.startswith("stale")
+    finally:
+        bench.NCU_TRAFFIC_BYTES.pop(key, None)
+    assert bench.captured_traffic(*key)[0] is None
+    assert bench.kernel_digest("no_such_kernel") is None
