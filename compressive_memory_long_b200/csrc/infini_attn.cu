@@ -1119,10 +1119,14 @@ int launch_backward(const BwdPlan &p, const T *q, const T *k, const T *v, const 
             k, v, snapM, snapZ, nullptr, w.GM, nullptr, p.L, N, S, T_last);
     }
     // 2. row statistics, the retrieval part of dq, the gate's partial sums: on the tensor
-    //    cores for bf16 with 128-row tiles (the memory path left bf16 snapshots)
+    //    cores for bf16 with 128-row tiles (the memory path left bf16 snapshots); with
+    //    64-token segments (and in step 3) a tile is a pair of segments: the kernels see
+    //    N = 128 and ceil(S / 2) segments with `pair` set
+    const bool pair = p.N == 64;
+    const int Nt = pair ? 128 : N, St = pair ? (S + 1) / 2 : S;
     bool tc_rows = false;
     if constexpr (sizeof(T) == 2 && (D == 64 || D == 128)) {
-        if (tc_mem && p.N % 128 == 0) {
+        if (tc_mem && (p.N % 128 == 0 || pair)) {
             using CR = tc::BwdRowsCfg<D>;
             Workspace tw = carve_bwd_tc(raw, p);
             CUtensorMap mq, mk, mv, mo, mm;
@@ -1134,9 +1138,9 @@ int launch_backward(const BwdPlan &p, const T *q, const T *k, const T *v, const 
                 return INFINI_ERR_CUDA;
             if (!opt_in_smem<tc::k_bwd_rows_tc<D>>(CR::ALLOC)) return INFINI_ERR_CUDA;
             tc::BwdRowsArgs ra{beta, snapZ, w.lse, w.Drow, w.wsc, w.dden, w.dq, w.dbeta_part,
-                               p.L, N, S, H, Hkv, (int)p.qtiles};
+                               p.L, Nt, St, H, Hkv, (int)p.qtiles, pair ? 1 : 0, S};
             TRACED("bwd_rows", st);
-            tc::k_bwd_rows_tc<D><<<(unsigned)(p.B * p.H * S * (p.N / 128)), 192, CR::ALLOC, st>>>(
+            tc::k_bwd_rows_tc<D><<<(unsigned)(p.B * p.H * St * (Nt / 128)), 192, CR::ALLOC, st>>>(
                 mq, mk, mv, mo, mm, ra);
             tc_rows = true;
         }
@@ -1151,7 +1155,7 @@ int launch_backward(const BwdPlan &p, const T *q, const T *k, const T *v, const 
     // 3. dq;  4. local dk, dv: on the tensor cores for bf16 with 128-row tiles
     bool tc_attn = false;
     if constexpr (sizeof(T) == 2 && (D == 64 || D == 128)) {
-        if (p.N % 128 == 0) {
+        if (p.N % 128 == 0 || pair) {
             using CB = tc::BwdTcCfg<D>;
             CUtensorMap mq, mk, mv, mo;
             if (!make_map_bf16_3d(&mq, q, D, p.L, p.B * p.H, 128) ||
@@ -1162,15 +1166,15 @@ int launch_backward(const BwdPlan &p, const T *q, const T *k, const T *v, const 
             if (!opt_in_smem<tc::k_bwd_dq_tc<D>>(CB::ALLOC_DQ) || !opt_in_smem<tc::k_bwd_dkdv_tc<D>>(CB::ALLOC_KV))
                 return INFINI_ERR_CUDA;
             tc::BwdTcArgs ta{beta, w.lse, w.Drow, w.dq, reinterpret_cast<__nv_bfloat16 *>(dq), w.dk, w.dv,
-                             p.L, N, S, H, Hkv};
-            const int64_t tiles = p.N / 128;
+                             p.L, Nt, St, H, Hkv, pair ? 1 : 0};
+            const int64_t tiles = Nt / 128;
             {
                 TRACED("bwd_dq", st);
-                tc::k_bwd_dq_tc<D><<<(unsigned)(p.B * p.H * S * tiles), CB::THREADS, CB::ALLOC_DQ, st>>>(
+                tc::k_bwd_dq_tc<D><<<(unsigned)(p.B * p.H * St * tiles), CB::THREADS, CB::ALLOC_DQ, st>>>(
                     mq, mk, mv, mo, ta);
             }
             TRACED("bwd_dkdv", st);
-            tc::k_bwd_dkdv_tc<D><<<(unsigned)(chains * S * tiles), CB::THREADS, CB::ALLOC_KV, st>>>(
+            tc::k_bwd_dkdv_tc<D><<<(unsigned)(chains * St * tiles), CB::THREADS, CB::ALLOC_KV, st>>>(
                 mq, mk, mv, mo, ta);
             tc_attn = true;
         }
@@ -1192,7 +1196,7 @@ int launch_backward(const BwdPlan &p, const T *q, const T *k, const T *v, const 
     // 6. the reverse memory recurrence
     bool tc_gm = false;
     if constexpr (sizeof(T) == 2 && (D == 64 || D == 128)) {
-        if (tc_rows) {
+        if (tc_rows && p.N % 128 == 0) {
             using CG = tc::BwdGmCfg<D>;
             CUtensorMap mq, mo;
             if (!make_map_bf16_3d(&mq, q, D, p.L, p.B * p.H, 128) ||

@@ -1,5 +1,8 @@
 // Local-attention part of the backward pass on the tensor cores (sm_100a, bf16, d = 64 or
-// 128, N % 128 == 0).
+// 128, N % 128 == 0; with 64-token segments the row statistics, dq and dk / dv take a pair
+// of segments as one 128-row tile: N = 128 and ceil(S / 2) segments in their arguments,
+// `pair` set, a block-diagonal causal mask, and the row statistics' two halves retrieve
+// from their own segments' memories).
 //
 // Same arithmetic as k_bwd_dq / k_bwd_dkdv (backward.cuh; AI Wiki "Infini-Attention", "What
 // happens inside the Infini-attention block?", the local causal softmax of each segment):
@@ -71,6 +74,7 @@ struct BwdTcArgs {
     float *dk, *dv;               // [B, Hkv, L, D]: the local parts (fp32)
     int64_t L;
     int N, S, H, Hkv;
+    int pair;                     // 1: a tile is two 64-token segments (N = 128 here)
 };
 
 // Outputs of the row statistics (the same buffers as k_bwd_rows writes)
@@ -82,6 +86,8 @@ struct BwdRowsArgs {
     float *dbeta_part;            // [B, H, S, qparts]: qparts 64-row parts per segment
     int64_t L;
     int N, S, H, Hkv, qparts;
+    int pair;                     // 1: a tile is two 64-token segments (N = 128, S = pairs here)
+    int Sr;                       // the real segment count (snapshots, z, dbeta parts) when pair
 };
 
 template <int D>
@@ -90,9 +96,9 @@ struct BwdRowsCfg {
     static constexpr int MBYTES = D * D * 2, MBOX = D * 128;
     static constexpr int OFF_Q = 0, OFF_O = TILE, OFF_RING = 2 * TILE;      // ring: ST x (K | V)
     static constexpr int OFF_M = OFF_RING + ST * 2 * TILE;
-    static constexpr int OFF_Z = OFF_M + MBYTES;
-    static constexpr int OFF_RED = OFF_Z + D * 4;     // 4 warp partial sums of the gate term
-    static constexpr int NBAR = 3 * ST + 8;
+    static constexpr int OFF_Z = OFF_M + MBYTES;      // z of the segment (of both, for a pair)
+    static constexpr int OFF_RED = OFF_Z + 2 * D * 4; // 4 warp partial sums of the gate term
+    static constexpr int NBAR = 3 * ST + 10;
     static constexpr int OFF_BAR = OFF_RED + 16;
     static constexpr int ALLOC = OFF_BAR + NBAR * 8 + 16 + 1024;
     static_assert(ALLOC <= 227 * 1024, "shared memory");
@@ -146,7 +152,7 @@ struct BwdUpdCfg {
 
 enum : int { WB_QF = 901, WB_KF = 902, WB_VF = 903, WB_KVE = 904, WB_SDP = 905, WB_DS = 906,
              WB_DONE = 907, WB_FULL = 908, WB_EMPTY = 909, WB_DRAIN = 910, WB_MF = 911,
-             WB_SQ = 912, WB_RF = 913, WB_RED = 914, WB_UR = 915, WB_P3 = 916 };
+             WB_SQ = 912, WB_RF = 913, WB_RED = 914, WB_UR = 915, WB_P3 = 916, WB_RH = 917 };
 
 __device__ __forceinline__ void bwdtc_drain(uint64_t *bar, uint32_t parity)
 {
@@ -317,7 +323,8 @@ k_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
 #pragma unroll
                         for (int u = 0; u < 2; ++u) {
                             const int col = half * 64 + c * 32 + 2 * e + u;       // key in the tile
-                            const bool vis = live && j * 128 + col < valid && (j < qt || col <= r);
+                            const bool vis = live && j * 128 + col < valid && (j < qt || col <= r) &&
+                                             !(a.pair && (col < 64) != (r < 64));
                             const float p = vis ? ex2(fmaf(__uint_as_float(sv[c][2 * e + u]), sl2, -lse)) : 0.f;
                             ds2[u] = p * fmaf(c1, __uint_as_float(pv[c][2 * e + u]), -Dr);
                         }
@@ -539,7 +546,8 @@ k_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                         for (int u = 0; u < 2; ++u) {
                             const int col = half * 64 + c * 32 + 2 * e + u;   // query in the tile
                             // causal: query row >= key row; rows past the segment's end out
-                            const bool vis = live && (qrel > 0 || col >= r) && k0 + qrel + col < valid;
+                            const bool vis = live && (qrel > 0 || col >= r) && k0 + qrel + col < valid &&
+                                             !(a.pair && (col < 64) != (r < 64));
                             const float p = vis ? ex2(fmaf(__uint_as_float(sv[c][2 * e + u]), sl2, -sl[col])) : 0.f;
                             p2[u] = c1 * p;
                             d2[u] = p * fmaf(c1, __uint_as_float(pv[c][2 * e + u]), -sl[128 + col]);
@@ -612,9 +620,16 @@ k_bwd_rows_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     const int64_t seg0 = (int64_t)s * a.N;
     const int valid = (int)(a.L - seg0 < a.N ? a.L - seg0 : a.N);
     const int q0 = qt * 128;
-    float *part = a.dbeta_part + (bh * a.S + s) * a.qparts + 2 * qt;   // two 64-row parts
+    // a pair: rows 0-63 are segment 2s and read its memory, rows 64-127 segment 2s + 1 (when
+    // it exists); the gate's parts are laid out per real segment
+    const int Ssnap = a.pair ? a.Sr : a.S;
+    const int sA = a.pair ? 2 * s : s;
+    const bool hasB = a.pair && sA + 1 < a.Sr;
+    float *part = a.pair ? a.dbeta_part + bh * a.Sr + sA
+                         : a.dbeta_part + (bh * a.S + s) * a.qparts + 2 * qt;   // two 64-row parts
+    const int nparts = a.pair && !hasB ? 1 : 2;
     if (q0 >= valid) {
-        if (threadIdx.x < 2) part[threadIdx.x] = 0.f;
+        if (threadIdx.x < nparts) part[threadIdx.x] = 0.f;
         return;
     }
     const int nk = qt + 1;
@@ -629,6 +644,9 @@ k_bwd_rows_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     uint64_t *k_full = bars, *v_full = bars + ST, *kv_empty = bars + 2 * ST;
     uint64_t *q_full = bars + 3 * ST, *m_full = q_full + 1, *s_full = q_full + 2, *p_full = q_full + 3;
     uint64_t *sq_full = q_full + 4, *r_full = q_full + 5, *red_full = q_full + 6, *mma_done = q_full + 7;
+    // a pair's second half: its R and dout M^T (r_full2), once the first half's rows have
+    // read theirs from the same TMEM columns (r_half)
+    uint64_t *r_full2 = q_full + 8, *r_half = q_full + 9;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C::OFF_BAR + C::NBAR * 8);
     volatile int *abort = reinterpret_cast<volatile int *>(smem + C::OFF_BAR + C::NBAR * 8 + 4);
 
@@ -646,6 +664,8 @@ k_bwd_rows_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         mbar_init(r_full, 1);
         mbar_init(red_full, 4);
         mbar_init(mma_done, 1);
+        mbar_init(r_full2, 1);
+        mbar_init(r_half, 64);
         *abort = 0;
         fence_barrier_init();
     }
@@ -668,10 +688,15 @@ k_bwd_rows_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 tma_load_3d(sQ + cb * C::BOX, &tmQ, q_full, cb * 64, (int)(seg0 + q0), (int)bh);
                 tma_load_3d(sO + cb * C::BOX, &tmO, q_full, cb * 64, (int)(seg0 + q0), (int)bh);
             }
-            mbar_arrive_expect_tx(m_full, C::MBYTES + D * 4);
-            for (int cb = 0; cb < D / 64; ++cb)
-                tma_load_3d(sM + cb * C::MBOX, &tmM, m_full, cb * 64, 0, (int)(chain * a.S + s));
-            bulk_load(sZ, a.snapZ + (chain * a.S + s) * (int64_t)D, D * 4, m_full);
+            // M_{s-1} (and for a pair's second segment its own memory, in the key ring's second
+            // slot, which the single key tile of a pair leaves free) with z
+            const int nm = hasB ? 2 : 1;
+            mbar_arrive_expect_tx(m_full, nm * (C::MBYTES + D * 4));
+            for (int x = 0; x < nm; ++x)
+                for (int cb = 0; cb < D / 64; ++cb)
+                    tma_load_3d((x ? sK(1) : sM) + cb * C::MBOX, &tmM, m_full, cb * 64, 0,
+                                (int)(chain * Ssnap + sA + x));
+            bulk_load(sZ, a.snapZ + (chain * Ssnap + sA) * (int64_t)D, nm * D * 4, m_full);
             int issued = 0;
             for (int j = 0; j < nk; ++j) {
                 const int st = j % ST;
@@ -740,6 +765,20 @@ k_bwd_rows_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 }
                 mma_commit(r_full);
             }
+            if (ok && hasB) ok = mbar_wait_short(r_half, 0, abort, WB_RH);
+            if (ok && hasB) {
+                tc_fence_after();
+                const uint32_t aM2 = smem_u32(sK(1));
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * C::BOX + (kk & 3) * 32;
+                    mma_ss(tmem + C::T_R, sdesc_sw128(aQ + off, 16, 1024), sdesc_sw128(aM2 + kk * 2048, C::MBOX, 1024),
+                           idO, kk > 0 ? 1u : 0u);
+                    mma_ss(tmem + C::T_DM, sdesc_sw128(aO + off, 16, 1024),
+                           sdesc_sw128(aM2 + (kk >> 2) * C::MBOX + (kk & 3) * 32, 16, 1024), idK, kk > 0 ? 1u : 0u);
+                }
+                mma_commit(r_full2);
+            }
             mma_commit(mma_done);
             bwdtc_drain(mma_done, 0);
         }
@@ -748,6 +787,8 @@ k_bwd_rows_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         const int r = threadIdx.x;
         const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
         const bool live = q0 + r < valid;
+        const bool second = a.pair && r >= 64;                  // a pair's second segment
+        const float *zr = sZ + (second ? D : 0);
         const float kscale = rsqrtf((float)D) * 1.4426950408889634f;
         const float g = 1.f / (1.f + __expf(-a.beta[h]));
         float m_used = -INFINITY, l = 0.f;
@@ -765,7 +806,7 @@ k_bwd_rows_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 for (int c = 0; c < 4; ++c)
 #pragma unroll
                     for (int e = 0; e < 32; ++e)
-                        if (c * 32 + e > r) v[c][e] = __float_as_uint(-INFINITY);
+                        if (c * 32 + e > r || (second && c * 32 + e < 64)) v[c][e] = __float_as_uint(-INFINITY);
             }
             float pm[4];
 #pragma unroll
@@ -824,12 +865,12 @@ k_bwd_rows_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         if (ok) ok = mbar_wait(q_full, 0, abort, WB_QF);
         if (ok) ok = mbar_wait(m_full, 0, abort, WB_MF);
         if (ok) {
-            den = segp_sigma_row<0, D, D / 8>(sQ, r, sZ);
+            den = segp_sigma_row<0, D, D / 8>(sQ, r, zr);
             fence_proxy_async_smem();
             mbar_arrive(sq_full);
         }
         float gm = 0.f;
-        if (ok && (ok = mbar_wait(r_full, 0, abort, WB_RF))) {
+        if (ok && (ok = mbar_wait(second && hasB ? r_full2 : r_full, 0, abort, WB_RF))) {
             tc_fence_after();
             // per row: A_dot = O / l, A_mem = R / den; dd = dout . A_dot, dam = dout . A_mem
             const float inv_l = 1.f / l;
@@ -883,13 +924,18 @@ k_bwd_rows_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                         for (int u = 0; u < 4; ++u) {
                             const float s0 = __uint_as_float(w4[u] << 16), s1 = __uint_as_float(w4[u] & 0xffff0000u);
                             const int i0 = 8 * e + 2 * u;
-                            y[2 * u] = fmaf(wsc, __uint_as_float(dm[i0]), ddn * sZ[c + i0]) * fminf(s0, 1.f);
-                            y[2 * u + 1] = fmaf(wsc, __uint_as_float(dm[i0 + 1]), ddn * sZ[c + i0 + 1]) * fminf(s1, 1.f);
+                            y[2 * u] = fmaf(wsc, __uint_as_float(dm[i0]), ddn * zr[c + i0]) * fminf(s0, 1.f);
+                            y[2 * u + 1] = fmaf(wsc, __uint_as_float(dm[i0 + 1]), ddn * zr[c + i0 + 1]) * fminf(s1, 1.f);
                         }
                         dst[2 * e] = make_float4(y[0], y[1], y[2], y[3]);
                         dst[2 * e + 1] = make_float4(y[4], y[5], y[6], y[7]);
                     }
                 }
+            }
+            if (hasB && !second) {
+                // this row's R and dout M^T have been read: the second half's may replace them
+                tc_fence_before();
+                mbar_arrive(r_half);
             }
         }
         // the gate's partial sums: rows 0-63 and 64-127 of the tile, each in a fixed order
@@ -903,7 +949,7 @@ k_bwd_rows_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             }
             if (threadIdx.x == 0 && mbar_wait(red_full, 0, abort, WB_RED)) {
                 part[0] = g * (1.f - g) * (sRed[0] + sRed[1]);
-                part[1] = g * (1.f - g) * (sRed[2] + sRed[3]);
+                if (nparts > 1) part[1] = g * (1.f - g) * (sRed[2] + sRed[3]);
             }
         }
     }

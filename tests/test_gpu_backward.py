@@ -50,6 +50,12 @@ CASES = [
     make("bf16_lin_n384_d128", B=2, H=2, Hkv=1, d=128, N=384, S=2, dtype="bf16", seed=99),
     make("bf16_delta_g4_d128_tail", B=1, H=8, Hkv=2, d=128, N=256, S=3, tail=129, dtype="bf16",
          rule="delta", seed=100),
+    # 64-token segments on the tensor cores (a pair of segments per 128-row tile, each half
+    # retrieving from its own memory): grouped heads with a short last segment that leaves the
+    # last pair without its second (3 segments), and an odd count of full segments
+    make("bf16_delta_n64_gqa_tail", B=1, H=4, Hkv=2, d=128, N=64, S=2, tail=20, dtype="bf16",
+         rule="delta", seed=101),
+    make("bf16_lin_n64_d128_odd", B=2, H=2, Hkv=1, d=128, N=64, S=5, dtype="bf16", seed=102),
 ]
 
 
