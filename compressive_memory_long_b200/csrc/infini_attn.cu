@@ -1192,11 +1192,13 @@ int launch_backward(const BwdPlan &p, const T *q, const T *k, const T *v, const 
         k_bwd_dkdv<T, D><<<(unsigned)(chains * S * p.qtiles), 256, smem, st>>>(
             q, k, v, beta, dout, w, p.L, N, S, H, Hkv);
     }
-    // 5. G^M_s, G^z_s (on the tensor cores with the tensor-core row statistics);
+    // 5. G^M_s, G^z_s (on the tensor cores with the tensor-core row statistics; a 64-token
+    //    segment is the first half of the 128-row tile these kernels load, its other rows
+    //    count as rows past the segment's end and add nothing);
     // 6. the reverse memory recurrence
     bool tc_gm = false;
     if constexpr (sizeof(T) == 2 && (D == 64 || D == 128)) {
-        if (tc_rows && p.N % 128 == 0) {
+        if (tc_rows && (p.N % 128 == 0 || pair)) {
             using CG = tc::BwdGmCfg<D>;
             CUtensorMap mq, mo;
             if (!make_map_bf16_3d(&mq, q, D, p.L, p.B * p.H, 128) ||
@@ -1236,10 +1238,11 @@ int launch_backward(const BwdPlan &p, const T *q, const T *k, const T *v, const 
         TRACED("bwd_mem_rev", st);
         k_bwd_mdelta<T, D, 16><<<(unsigned)(chains * (D / 16)), 256, 0, st>>>(k, dM, w, dM0, p.L, N, S);
     }
-    // 7. the update's gradients;  8. the reverse z recurrence
+    // 7. the update's gradients (the same half-tile reading at N = 64);  8. the reverse z
+    //    recurrence
     bool tc_upd = false;
     if constexpr (sizeof(T) == 2 && (D == 64 || D == 128)) {
-        if (tc_mem && p.N % 128 == 0) {
+        if (tc_mem && (p.N % 128 == 0 || pair)) {
             using CU = tc::BwdUpdCfg<D>;
             CUtensorMap mk, mv;
             if (!make_map_bf16_3d(&mk, k, D, p.L, p.B * p.Hkv, 128) ||

@@ -2,7 +2,9 @@
 // 128, N % 128 == 0; with 64-token segments the row statistics, dq and dk / dv take a pair
 // of segments as one 128-row tile: N = 128 and ceil(S / 2) segments in their arguments,
 // `pair` set, a block-diagonal causal mask, and the row statistics' two halves retrieve
-// from their own segments' memories).
+// from their own segments' memories; G^M and the update keep one CTA per segment and read
+// a 64-token segment as the first half of the 128-row tile they load, the other half being
+// rows past the segment's end, which they zero).
 //
 // Same arithmetic as k_bwd_dq / k_bwd_dkdv (backward.cuh; AI Wiki "Infini-Attention", "What
 // happens inside the Infini-attention block?", the local causal softmax of each segment):
