@@ -648,7 +648,9 @@ k_bwd_gm(const T *__restrict__ q, const T *__restrict__ dout, BwdWs w, int64_t L
 
 // ---------------------------------------------------------------------------------------
 // Reverse memory recurrence, additive rule: dM_{s-1} = dM_s + G^M_s from dM_{S-1} = dM.
-// One thread per element; dMs[s] = dM_s; dM0 = dM_{-1}.
+// One thread per element; dMs[s] = dM_s; dM0 = dM_{-1}.  The loads of G^M run eight
+// segments ahead of the dependent sums (G^M and dMs never overlap), so a thread keeps eight
+// memory reads in flight instead of one.
 // ---------------------------------------------------------------------------------------
 __global__ void __launch_bounds__(256)
 k_bwd_mlin(const float *dM, BwdWs w, float *dM0, int S, int D, int64_t chains)
@@ -657,11 +659,23 @@ k_bwd_mlin(const float *dM, BwdWs w, float *dM0, int S, int D, int64_t chains)
     const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
     if (i >= chains * DD) return;
     const int64_t chain = i / DD, e = i % DD;
+    const float *__restrict__ gm = w.GM + chain * S * DD + e;
+    float *__restrict__ out = w.dMs + chain * S * DD + e;
     float m = dM ? dM[i] : 0.f;
-    for (int s = S - 1; s >= 0; --s) {
-        const int64_t o = (chain * S + s) * DD + e;
-        w.dMs[o] = m;
-        m += w.GM[o];
+    int s = S - 1;
+    for (; s >= 7; s -= 8) {
+        float g[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) g[u] = gm[(int64_t)(s - u) * DD];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            out[(int64_t)(s - u) * DD] = m;
+            m += g[u];
+        }
+    }
+    for (; s >= 0; --s) {
+        out[(int64_t)s * DD] = m;
+        m += gm[(int64_t)s * DD];
     }
     if (dM0) dM0[i] = m;
 }
@@ -874,21 +888,40 @@ k_bwd_update(const T *__restrict__ k, const T *__restrict__ v, BwdWs w, int64_t 
 
 // ---------------------------------------------------------------------------------------
 // Reverse z recurrence: dz_{s-1} = dz_s + G^z_s + h_s from dz_{S-1} = dz; dzs[s] = dz_s;
-// dz0 = dz_{-1}.  One thread per (chain, feature).
+// dz0 = dz_{-1}.  A block of 32 features x ZREV_CHUNKS threads per (chain, 32 features): each
+// thread sums G^z + h over its chunk of consecutive segments, the chunk totals give every
+// chunk its starting value (the sum over the later chunks), and each thread then walks its
+// chunk backwards writing dz_s.  The summation order is fixed by the chunking.
 // ---------------------------------------------------------------------------------------
-__global__ void __launch_bounds__(256)
+constexpr int ZREV_CHUNKS = 32;
+
+__global__ void __launch_bounds__(32 * ZREV_CHUNKS)
 k_bwd_zrev(const float *dz, BwdWs w, float *dz0, int S, int D, int64_t chains)
 {
-    const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
-    if (i >= chains * D) return;
-    const int64_t chain = i / D, f = i % D;
-    float z = dz ? dz[i] : 0.f;
-    for (int s = S - 1; s >= 0; --s) {
-        const int64_t o = (chain * S + s) * D + f;
-        w.dzs[o] = z;
-        z += w.Gz[o] + w.h[o];
+    __shared__ float tot[ZREV_CHUNKS][32];
+    const int fb = D / 32 > 0 ? D / 32 : 1;                 // 32-feature blocks per chain
+    const int64_t chain = blockIdx.x / fb;
+    const int f = (int)(blockIdx.x % fb) * 32 + (threadIdx.x & 31);
+    const int c = threadIdx.x >> 5;
+    const bool live = f < D;                                // d = 32: one block, all live
+    const int len = (S + ZREV_CHUNKS - 1) / ZREV_CHUNKS;
+    const int s0 = c * len, s1 = s0 + len < S ? s0 + len : S;
+    const float *__restrict__ gz = w.Gz + chain * S * D + f;
+    const float *__restrict__ hh = w.h + chain * S * D + f;
+    float *__restrict__ out = w.dzs + chain * S * D + f;
+    float t = 0.f;
+    if (live)
+        for (int s = s0; s < s1; ++s) t += gz[(int64_t)s * D] + hh[(int64_t)s * D];
+    tot[c][threadIdx.x & 31] = t;
+    __syncthreads();
+    if (!live) return;
+    float z = dz ? dz[chain * D + f] : 0.f;
+    for (int j = ZREV_CHUNKS - 1; j > c; --j) z += tot[j][threadIdx.x & 31];
+    for (int s = s1 - 1; s >= s0; --s) {
+        out[(int64_t)s * D] = z;
+        z += gz[(int64_t)s * D] + hh[(int64_t)s * D];
     }
-    if (dz0) dz0[i] = z;
+    if (c == 0 && dz0) dz0[chain * D + f] = z;
 }
 
 // ---------------------------------------------------------------------------------------

@@ -1275,7 +1275,8 @@ int launch_backward(const BwdPlan &p, const T *q, const T *k, const T *v, const 
     }
     {
         TRACED("bwd_z_rev", st);
-        k_bwd_zrev<<<(unsigned)((chains * D + 255) / 256), 256, 0, st>>>(dz, w, dz0, S, D, chains);
+        k_bwd_zrev<<<(unsigned)(chains * ((D + 31) / 32)), 32 * ZREV_CHUNKS, 0, st>>>(dz, w, dz0, S, D,
+                                                                                     chains);
     }
     // 9. dk, dv in the activation dtype;  10. dbeta
     {
