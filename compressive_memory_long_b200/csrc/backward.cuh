@@ -933,14 +933,40 @@ __global__ void __launch_bounds__(256)
 k_bwd_final(const T *__restrict__ k, BwdWs w, T *__restrict__ dk, T *__restrict__ dv,
             int64_t L, int N, int S, int64_t n)
 {
-    const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    // four consecutive elements of one row per thread (d is a multiple of 4; the workspace
+    // arrays are 256-byte aligned and the activations 16-byte aligned)
+    const int64_t i = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) * 4;
     if (i >= n) return;
     const int64_t row = i / D, a = i % D;
     const int64_t chain = row / L, t = row % L;
     const int s = (int)(t / N);
-    const float ds = w.dsk[i] + w.dzs[(chain * S + s) * D + a];
-    st_f(dk + i, ds * sigma_grad(ld_f(k + i)) + w.dk[i]);
-    st_f(dv + i, w.dv[i]);
+    const float4 ds = *reinterpret_cast<const float4 *>(w.dsk + i);
+    const float4 zs = *reinterpret_cast<const float4 *>(w.dzs + (chain * S + s) * D + a);
+    const float4 lk = *reinterpret_cast<const float4 *>(w.dk + i);
+    const float4 lv = *reinterpret_cast<const float4 *>(w.dv + i);
+    const float g[4] = {ds.x + zs.x, ds.y + zs.y, ds.z + zs.z, ds.w + zs.w};
+    const float l4[4] = {lk.x, lk.y, lk.z, lk.w};
+    const float v4[4] = {lv.x, lv.y, lv.z, lv.w};
+    if constexpr (sizeof(T) == 2) {
+        const uint2 kr = *reinterpret_cast<const uint2 *>(k + i);
+        const float kx[4] = {__uint_as_float(kr.x << 16), __uint_as_float(kr.x & 0xffff0000u),
+                             __uint_as_float(kr.y << 16), __uint_as_float(kr.y & 0xffff0000u)};
+        float o[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) o[u] = g[u] * sigma_grad(kx[u]) + l4[u];
+        __nv_bfloat162 k01 = __floats2bfloat162_rn(o[0], o[1]), k23 = __floats2bfloat162_rn(o[2], o[3]);
+        __nv_bfloat162 v01 = __floats2bfloat162_rn(v4[0], v4[1]), v23 = __floats2bfloat162_rn(v4[2], v4[3]);
+        *reinterpret_cast<uint2 *>(dk + i) = make_uint2(*reinterpret_cast<uint32_t *>(&k01),
+                                                        *reinterpret_cast<uint32_t *>(&k23));
+        *reinterpret_cast<uint2 *>(dv + i) = make_uint2(*reinterpret_cast<uint32_t *>(&v01),
+                                                        *reinterpret_cast<uint32_t *>(&v23));
+    } else {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            st_f(dk + i + u, g[u] * sigma_grad(ld_f(k + i + u)) + l4[u]);
+            st_f(dv + i + u, v4[u]);
+        }
+    }
 }
 
 // dbeta[h] = sum over batches, segments and row tiles of the partial sums (fixed order).

@@ -1282,7 +1282,7 @@ int launch_backward(const BwdPlan &p, const T *q, const T *k, const T *v, const 
     {
         const int64_t n = p.B * p.Hkv * p.L * D;
         TRACED("bwd_final", st);
-        k_bwd_final<T, D><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(k, w, dk, dv, p.L, N, S, n);
+        k_bwd_final<T, D><<<(unsigned)((n / 4 + 255) / 256), 256, 0, st>>>(k, w, dk, dv, p.L, N, S, n);
     }
     if (dbeta) {
         TRACED("bwd_beta", st);
