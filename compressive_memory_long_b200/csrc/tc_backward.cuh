@@ -148,8 +148,10 @@ struct BwdUpdCfg {
     static constexpr int OFF_BAR = OFF_Z + D * 4;
     static constexpr int ALLOC = OFF_BAR + NBAR * 8 + 16 + 1024;
     static_assert(ALLOC <= 227 * 1024, "shared memory");
-    // TMEM: dU | sigma(K) M | dsigma(k) (d columns each) | h (16)
+    // TMEM: dU | sigma(K) M | dsigma(k) (d columns each) | h (16); at d = 64 that fits 256
+    // columns, so two CTAs share an SM (shared memory allows it too)
     static constexpr uint32_t T_1 = 0, T_2 = D, T_3 = 2 * D, T_H = 3 * D;
+    static constexpr uint32_t TMEM_COLS = 3 * D + 16 <= 256 ? 256 : 512;
 };
 
 enum : int { WB_QF = 901, WB_KF = 902, WB_VF = 903, WB_KVE = 904, WB_SDP = 905, WB_DS = 906,
@@ -1176,7 +1178,7 @@ k_bwd_update_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
     if (D == 64)       // the padded feature box of sigma(K) stays zero
         for (int i = threadIdx.x; i < C::BOX / 16; i += blockDim.x)
             reinterpret_cast<uint4 *>(sK + C::BOX)[i] = make_uint4(0, 0, 0, 0);
-    if (warp == 5) tmem_alloc(tmem_holder, 512);
+    if (warp == 5) tmem_alloc(tmem_holder, C::TMEM_COLS);
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -1433,7 +1435,7 @@ k_bwd_update_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
     __syncthreads();
     if (warp == 5) {
         tc_fence_after();
-        tmem_dealloc(tmem, 512);
+        tmem_dealloc(tmem, C::TMEM_COLS);
     }
 }
 
