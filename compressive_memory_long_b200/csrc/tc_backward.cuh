@@ -305,6 +305,7 @@ k_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         const float lse = live ? a.lse[row] : 0.f, Dr = live ? a.Drow[row] : 0.f;
         const float c1 = 1.f - 1.f / (1.f + __expf(-a.beta[h]));
         const float sl2 = rsqrtf((float)D) * 1.4426950408889634f;
+        const int lo = a.pair && r >= 64 ? 64 : 0;             // a pair's second segment: its own keys
         bool ok = true;
         for (int j = 0; ok && j < nk; ++j) {
             if (!(ok = mbar_wait(sdp_full, j & 1, abort, WB_SDP))) break;
@@ -327,8 +328,7 @@ k_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
 #pragma unroll
                         for (int u = 0; u < 2; ++u) {
                             const int col = half * 64 + c * 32 + 2 * e + u;       // key in the tile
-                            const bool vis = live && j * 128 + col < valid && (j < qt || col <= r) &&
-                                             !(a.pair && (col < 64) != (r < 64));
+                            const bool vis = live && j * 128 + col < valid && (j < qt || col <= r) && col >= lo;
                             const float p = vis ? ex2(fmaf(__uint_as_float(sv[c][2 * e + u]), sl2, -lse)) : 0.f;
                             ds2[u] = p * fmaf(c1, __uint_as_float(pv[c][2 * e + u]), -Dr);
                         }
@@ -520,6 +520,7 @@ k_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
         const bool live = k0 + r < valid;
         const float sl2 = rsqrtf((float)D) * 1.4426950408889634f;
+        const int hi = a.pair && r < 64 ? 64 : 128;            // a pair's first segment: its own queries
         bool ok = true;
         for (int i = 0; ok && i < steps; ++i) {
             const int st = i % ST;
@@ -550,8 +551,7 @@ k_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                         for (int u = 0; u < 2; ++u) {
                             const int col = half * 64 + c * 32 + 2 * e + u;   // query in the tile
                             // causal: query row >= key row; rows past the segment's end out
-                            const bool vis = live && (qrel > 0 || col >= r) && k0 + qrel + col < valid &&
-                                             !(a.pair && (col < 64) != (r < 64));
+                            const bool vis = live && (qrel > 0 || col >= r) && k0 + qrel + col < valid && col < hi;
                             const float p = vis ? ex2(fmaf(__uint_as_float(sv[c][2 * e + u]), sl2, -sl[col])) : 0.f;
                             p2[u] = c1 * p;
                             d2[u] = p * fmaf(c1, __uint_as_float(pv[c][2 * e + u]), -sl[128 + col]);
