@@ -793,6 +793,7 @@ k_bwd_rows_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         const bool live = q0 + r < valid;
         const bool second = a.pair && r >= 64;                  // a pair's second segment
         const float *zr = sZ + (second ? D : 0);
+        const int lo = second ? 64 : 0;                          // the first key this row may see
         const float kscale = rsqrtf((float)D) * 1.4426950408889634f;
         const float g = 1.f / (1.f + __expf(-a.beta[h]));
         float m_used = -INFINITY, l = 0.f;
@@ -810,7 +811,7 @@ k_bwd_rows_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 for (int c = 0; c < 4; ++c)
 #pragma unroll
                     for (int e = 0; e < 32; ++e)
-                        if (c * 32 + e > r || (second && c * 32 + e < 64)) v[c][e] = __float_as_uint(-INFINITY);
+                        if (c * 32 + e > r || c * 32 + e < lo) v[c][e] = __float_as_uint(-INFINITY);
             }
             float pm[4];
 #pragma unroll

@@ -276,6 +276,7 @@ k_segment_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
         // the rows of a pair's second segment use its own memory (S1, z_s)
         const bool second = pair && r >= 64;
         const float *zr = sZ + (second ? D : 0);
+        const int lo = second ? 64 : 0;                      // the first key this row may see
 
         const float kscale = rsqrtf((float)D) * 1.4426950408889634f;
         float m_used = -INFINITY, l = 0.f;
@@ -293,7 +294,7 @@ k_segment_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
             if (j == qt) {                                  // causal mask on the diagonal tile
 #pragma unroll
                 for (int c = 0; c < 128; ++c)
-                    if (c > r || (second && c < 64)) raw[c >> 5][c & 31] = __float_as_uint(-INFINITY);
+                    if (c > r || c < lo) raw[c >> 5][c & 31] = __float_as_uint(-INFINITY);
             }
             float pm[8];
 #pragma unroll
