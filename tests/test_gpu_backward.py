@@ -56,6 +56,8 @@ CASES = [
     make("bf16_delta_n64_gqa_tail", B=1, H=4, Hkv=2, d=128, N=64, S=2, tail=20, dtype="bf16",
          rule="delta", seed=101),
     make("bf16_lin_n64_d128_odd", B=2, H=2, Hkv=1, d=128, N=64, S=5, dtype="bf16", seed=102),
+    make("bf16_delta_n64_d64_gqa_odd", B=2, H=4, Hkv=2, d=64, N=64, S=3, dtype="bf16", rule="delta",
+         seed=103),
 ]
 
 
