@@ -104,8 +104,11 @@ struct BwdRowsCfg {
     static constexpr int OFF_BAR = OFF_RED + 16;
     static constexpr int ALLOC = OFF_BAR + NBAR * 8 + 16 + 1024;
     static_assert(ALLOC <= 227 * 1024, "shared memory");
-    // TMEM: S [0,128), O, R = sigma(Q) M, dout M^T (d columns each)
-    static constexpr uint32_t T_S = 0, T_O = 128, T_R = 128 + D, T_DM = 128 + 2 * D;
+    // TMEM: S [0,128), O, R = sigma(Q) M, dout M^T (d columns each).  At d = 64 dout M^T
+    // takes S's first columns (free once the last P V has run: MMAs execute in issue order),
+    // so the kernel fits 256 columns and two CTAs share an SM.
+    static constexpr uint32_t T_S = 0, T_O = 128, T_R = 128 + D, T_DM = D == 64 ? 0 : 128 + 2 * D;
+    static constexpr uint32_t TMEM_COLS = D == 64 ? 256 : 512;
 };
 
 struct BwdGmArgs {
@@ -117,7 +120,10 @@ struct BwdGmArgs {
 
 template <int D>
 struct BwdGmCfg {
-    static constexpr int BOX = 128 * 128, NB = D / 64, ST = 2;
+    // one stage at d = 64: the stage's 64 KB then lets three CTAs share an SM (most d = 64
+    // workloads have one or few steps per CTA); two at d = 128, whose CTAs walk the group's
+    // heads over long segments
+    static constexpr int BOX = 128 * 128, NB = D / 64, ST = D == 64 ? 1 : 2;
     // stage: A = wsc sigma(Q) over Q (features padded to 128 with a zero box at d = 64) |
     //        dout (NB boxes) | the extra column's box
     static constexpr int OFF_AQ = 0, OFF_DO = 2 * BOX, OFF_EX = OFF_DO + NB * BOX;
@@ -601,9 +607,10 @@ k_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
 }
 
 
-// the forward of 128 query rows and the backward's row statistics
+// the forward of 128 query rows and the backward's row statistics (at d = 64 two CTAs per
+// SM: 256 TMEM columns, ~108 KB of shared memory, at most 168 registers)
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(192, D == 64 ? 2 : 1)
 k_bwd_rows_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
               const __grid_constant__ CUtensorMap tmM, const BwdRowsArgs a)
@@ -673,7 +680,7 @@ k_bwd_rows_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         *abort = 0;
         fence_barrier_init();
     }
-    if (warp == 5) tmem_alloc(tmem_holder, 512);
+    if (warp == 5) tmem_alloc(tmem_holder, C::TMEM_COLS);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -963,7 +970,7 @@ k_bwd_rows_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     __syncthreads();
     if (warp == 5) {
         tc_fence_after();
-        tmem_dealloc(tmem, 512);
+        tmem_dealloc(tmem, C::TMEM_COLS);
     }
 }
 
