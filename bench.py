@@ -72,10 +72,10 @@ NCU_TRAFFIC_BYTES: dict = {
     ("hf_repro_n64", "small_fused"): (6364160, "b4076352787a7b26"),
     # 2048 of 16384 segments captured (x 8)
     ("n64_bandwidth", "small_pieces"): ((1032990976 + 268926464) * 8, "5c6fb8137091e762"),
-    ("gqa8b_n2048_delta", "segment_tc"): (421510144 + 238118912, "09d83465c9002f40"),
+    ("gqa8b_n2048_delta", "segment_tc"): (421691904 + 238313216, "e5dbc14c5524c01e"),
     # 4 of 8 segments captured (x 2) and 16 of 512 segments captured (x 32)
-    ("batched_n1024_linear", "segment_tc"): ((1704829184 + 515661312) * 2, "09d83465c9002f40"),
-    ("stream1m_n2048_delta", "segment_tc"): ((413263872 + 112340992) * 32, "09d83465c9002f40"),
+    ("batched_n1024_linear", "segment_tc"): ((1705369856 + 516162816) * 2, "e5dbc14c5524c01e"),
+    ("stream1m_n2048_delta", "segment_tc"): ((412875264 + 113371136) * 32, "e5dbc14c5524c01e"),
 }
 
 

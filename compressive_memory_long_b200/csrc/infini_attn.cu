@@ -339,8 +339,13 @@ int launch_memory_tc(const Problem &p, const __nv_bfloat16 *k, const __nv_bfloat
     if (!delta) {
         const int64_t n4 = chains * D * D / 4;
         TRACED("mem_prefix", st);
-        tc::k_mem_prefix<D><<<(unsigned)((n4 + 255) / 256), 256, 0, st>>>(ws.Bs, M0, ws.snapMb,
-                                                                          M_out, S, chains, snapMf);
+        // many segments: 8 chunks per element walked side by side; few: one walk
+        if (S >= 64)
+            tc::k_mem_prefix<D, 8><<<(unsigned)((n4 + 31) / 32), 256, 0, st>>>(ws.Bs, M0, ws.snapMb, M_out,
+                                                                            S, chains, snapMf);
+        else
+            tc::k_mem_prefix<D, 1><<<(unsigned)((n4 + 255) / 256), 256, 0, st>>>(ws.Bs, M0, ws.snapMb, M_out,
+                                                                              S, chains, snapMf);
         return INFINI_OK;
     }
     using MC = tc::MChainCfg<D>;

@@ -494,25 +494,54 @@ k_mem_incr(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUte
 
 // ---------------------------------------------------------------- the serial parts
 
-// Additive rule: M_{s-1} = M0 + sum_{j<s} B_j.  One thread per 4 consecutive elements of a
-// chain's M walks the segments, writing the snapshot of every M_{s-1} (bf16 and / or fp32)
-// and M_out.  Each
-// element is read from M0 and written to M_out by the same thread, so they may alias.
-template <int D>
+// Additive rule: M_{s-1} = M0 + sum_{j<s} B_j, writing the snapshot of every M_{s-1} (bf16
+// and / or fp32) and M_out.  A block covers 256 / CH groups of 4 consecutive elements of a
+// chain's M with CH threads each: thread c sums B_j over its chunk of consecutive segments,
+// the chunk totals give every chunk its starting value, and the thread then walks its chunk
+// writing the snapshots (the summation order is fixed by the chunking).  Every thread reads
+// its elements of M0 before the block barrier and only the last chunk's thread writes
+// M_out, so M0 and M_out may alias.  CH = 1 (few segments) is a single walk.
+template <int D, int CH>
 __global__ void __launch_bounds__(256)
 k_mem_prefix(const float *__restrict__ Bs, const float *M0, __nv_bfloat16 *__restrict__ snapMb,
              float *M_out, int S, int64_t chains, float *__restrict__ snapMf = nullptr)
 {
     constexpr int64_t E4 = (int64_t)D * D / 4;
-    const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
-    if (i >= chains * E4) return;
-    const int64_t chain = i / E4, e = i % E4;
-    float4 m = M0 ? reinterpret_cast<const float4 *>(M0)[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+    constexpr int COLS = 256 / CH;
+    __shared__ float4 tot[CH][COLS];
+    const int col = threadIdx.x % COLS, c = threadIdx.x / COLS;
+    const int64_t i = blockIdx.x * (int64_t)COLS + col;
+    const bool live = i < chains * E4;
+    const int64_t chain = live ? i / E4 : 0, e = i % E4;
+    const int len = (S + CH - 1) / CH;
+    const int s0 = c * len, s1 = s0 + len < S ? s0 + len : S;
     const float4 *b = reinterpret_cast<const float4 *>(Bs) + chain * S * E4 + e;
+    float4 m = make_float4(0.f, 0.f, 0.f, 0.f), t = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (live) {
+        if (M0) m = reinterpret_cast<const float4 *>(M0)[i];
+#pragma unroll 4
+        for (int s = s0; CH > 1 && s < s1; ++s) {
+            const float4 x = b[(int64_t)s * E4];
+            t.x += x.x;
+            t.y += x.y;
+            t.z += x.z;
+            t.w += x.w;
+        }
+    }
+    tot[c][col] = t;
+    __syncthreads();
+    if (!live) return;
+    for (int j = 0; j < c; ++j) {
+        const float4 x = tot[j][col];
+        m.x += x.x;
+        m.y += x.y;
+        m.z += x.z;
+        m.w += x.w;
+    }
     uint2 *snap = snapMb ? reinterpret_cast<uint2 *>(snapMb) + chain * S * E4 + e : nullptr;
     float4 *snapf = snapMf ? reinterpret_cast<float4 *>(snapMf) + chain * S * E4 + e : nullptr;
 #pragma unroll 4
-    for (int s = 0; s < S; ++s) {
+    for (int s = s0; s < s1; ++s) {
         if (snap) snap[(int64_t)s * E4] = make_uint2(pack_bf16x2(m.x, m.y), pack_bf16x2(m.z, m.w));
         if (snapf) snapf[(int64_t)s * E4] = m;
         const float4 x = b[(int64_t)s * E4];
@@ -521,7 +550,7 @@ k_mem_prefix(const float *__restrict__ Bs, const float *M0, __nv_bfloat16 *__res
         m.z += x.z;
         m.w += x.w;
     }
-    reinterpret_cast<float4 *>(M_out)[i] = m;
+    if (c == CH - 1) reinterpret_cast<float4 *>(M_out)[i] = m;
 }
 
 template <int D>
