@@ -268,8 +268,8 @@ INFINI_API int64_t infini_attn_trace_report(char *buf, int64_t len);
  *   applies, in SM clock cycles (default about 0.5 s at the top clock; cycles <= 0 restores
  *   it).  A wait that reaches it gives up as described for infini_attn_device_status.
  * infini_attn_test_withhold_publish(on): on the current device, the first unit of every head
- *   in the fused 64-token kernel (additive rule, d = 64, N = 64, H == Hkv, at most 64 units
- *   of 128 tokens per head) skips publishing its memory aggregate, so the later units'
+ *   in the fused 64-token kernel (additive rule, d = 64, N = 64, at most 64 units of 128
+ *   tokens per head) skips publishing its memory aggregate, so the later units'
  *   waits for it run out: the call's outputs are then incomplete and
  *   infini_attn_device_status reports INFINI_ERR_TIMEOUT.  Nothing traps or hangs.
  * The last two copy to device variables synchronously (INFINI_ERR_CUDA if that fails); use
