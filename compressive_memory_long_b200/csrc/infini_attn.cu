@@ -311,19 +311,22 @@ int launch_memory_tc(const Problem &p, const __nv_bfloat16 *k, const __nv_bfloat
     const int64_t chains = p.B * p.Hkv, units = chains * p.S;
     const int S = (int)p.S, N = (int)p.N;
     const bool delta = p.rule == INFINI_UPDATE_DELTA;
-    {
+    // the delta rule's increments need z_{s-1}: sum sigma(K) per segment first; the additive
+    // rule's increments kernel sums it itself on the tensor cores and the scan follows
+    if (delta) {
         TRACED("z_sum", st);
         tc::k_zsum<D><<<(unsigned)units, 256, 0, st>>>(k, ws.dz, p.L, N, S);
     }
-    {
+    auto z_scan = [&]() {
         TRACED("z_scan", st);
         tc::k_zscan<D><<<(unsigned)chains, D * 8, 0, st>>>(ws.dz, z0, ws.snapZ, z_out, S);
-    }
+    };
+    if (delta) z_scan();
     CUtensorMap mk, mv;
     if (!make_map_bf16_3d(&mk, k, D, p.L, chains, 64) || !make_map_bf16_3d(&mv, v, D, p.L, chains, 64))
         return INFINI_ERR_CUDA;
     // persistent: one CTA per SM (or per item when there are fewer)
-    tc::IncrArgs ia{ws.snapZ, ws.Bs, ws.Ahi, ws.Alo, p.L, N, S, (int)units};
+    tc::IncrArgs ia{ws.snapZ, ws.Bs, ws.Ahi, ws.Alo, ws.dz, p.L, N, S, (int)units};
     const unsigned igrid = (unsigned)std::min<int64_t>(units, sm_count());
     if (delta) {
         using C = tc::IncrCfg<D, true>;
@@ -337,6 +340,7 @@ int launch_memory_tc(const Problem &p, const __nv_bfloat16 *k, const __nv_bfloat
         tc::k_mem_incr<D, false><<<igrid, C::THREADS, C::ALLOC, st>>>(mk, mv, ia);
     }
     if (!delta) {
+        z_scan();
         const int64_t n4 = chains * D * D / 4;
         TRACED("mem_prefix", st);
         // many segments: 8 chunks per element walked side by side; few: one walk

@@ -11,9 +11,12 @@
 //   M_s = M_{s-1} + B_s - A_s M_{s-1},
 //   B_s = sigma(K_s)^T V_s,   A_s = sigma(K_s)^T diag(1/den) sigma(K_s)   (d x d each).
 // So the contractions over a segment's N tokens leave the serial path:
-//   k_zsum      per (chain, segment): dz_s = sum_t sigma(k_t), fp32 on the CUDA cores
+//   k_zsum      delta: per (chain, segment) dz_s = sum_t sigma(k_t), fp32 on the CUDA cores
 //   k_zscan     per chain: z_{s-1} for every segment (what the segment kernel and den read)
-//   k_mem_incr  per (chain, segment), all at once, on the tensor cores: B_s and (delta) A_s
+//   k_mem_incr  per (chain, segment), all at once, on the tensor cores: B_s and (delta) A_s;
+//               for the additive rule, whose increments do not need z, also dz_s as
+//               sigma(K_s)^T 1 (the same two sigma parts against a tile of ones), so k is
+//               read once on that path and k_zscan follows it
 //   k_mem_chain delta: per (chain, 16 value columns), the recurrence in segment order, one
 //               d x d x 32 product per segment on the tensor cores
 //   k_mem_prefix linear: the running sum M0 + sum_{j<s} B_j, elementwise
@@ -24,7 +27,8 @@
 // cost about 5e-3 of M over 32 segments of 2048 tokens, the split about 3e-6.  The products
 // are sigma_hi [V | W_hi] + sigma_lo [V | W_hi] + sigma_hi W_lo with W = diag(1/den) sigma
 // split the same way (sigma_lo W_lo is below the fp32 rounding of the sums).  In the chain
-// A_s and M_{s-1} are split too (three products).  z is summed in fp32 from sigma itself.
+// A_s and M_{s-1} are split too (three products).  z is summed in fp32: from sigma itself
+// (delta), or from its two bf16 parts in an fp32 accumulator (additive).
 // Rows of a short last segment past L carry sigma = 0 (not sigma(0) = 1): they add nothing.
 // All waits are bounded (tc_common.cuh).
 #pragma once
@@ -128,13 +132,19 @@ struct IncrCfg {
     static constexpr int OSET = DELTA ? (4 + NB) * BOX : 2 * BOX;
     static constexpr int OFF_RING = 0;
     static constexpr int OFF_OPS = RS * SLOT;
-    static constexpr int OFF_BAR = OFF_OPS + 2 * OSET;
+    // additive rule: a K-major tile of ones (16 columns x 64 tokens), the B operand of
+    // sigma(K)^T 1, which gives the segment's sum of sigma(k_t) beside B_s
+    static constexpr int OFF_ONES = OFF_OPS + 2 * OSET;
+    static constexpr int ONES = DELTA ? 0 : 16 * 128;
+    static constexpr int OFF_BAR = OFF_ONES + ONES;
     static constexpr int NBAR = 3 * RS + 2 + 4 + 1;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int BYTES = OFF_MISC + 16;
     static constexpr int ALLOC = BYTES + 1024;
     static constexpr int ACC = DELTA ? 2 * D : D;     // accumulator columns: B_s | A_s
-    static constexpr uint32_t TMEM_COLS = 2 * ACC < 32 ? 32 : 2 * ACC;
+    static constexpr int ZC = DELTA ? 0 : 32;         // additive rule: columns of sigma(K)^T 1
+    static constexpr int T_Z = 2 * ACC;               // those of the two sets follow both B_s
+    static constexpr uint32_t TMEM_COLS = 2 * (ACC + ZC) <= 256 ? 256 : 512;
     static constexpr int THREADS = 512;
     static constexpr int FPT = D / 4;                // features per worker thread
     static_assert(SLOT % 1024 == 0 && OSET % 1024 == 0, "operand tiles must be 1024-aligned");
@@ -145,6 +155,7 @@ struct IncrArgs {
     const float *snapZ;        // [chains * S, D]: z_{s-1} (delta)
     float *Bs;                 // [chains * S, D, D] fp32: sigma(K_s)^T V_s
     __nv_bfloat16 *Ahi, *Alo;  // [chains * S, D, D]: A_s split into two bf16 parts (delta)
+    float *dz;                 // [chains * S, D]: sum of sigma(k_t) over segment s (additive)
     int64_t L;
     int N, S;
     int items;                 // chains * S
@@ -245,6 +256,10 @@ k_mem_incr(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUte
             reinterpret_cast<uint4 *>(base + C::BOX)[o] = make_uint4(0, 0, 0, 0);
         }
     }
+    if constexpr (!DELTA)
+        for (int i = threadIdx.x; i < C::ONES / 16; i += blockDim.x)   // bf16 1.0 everywhere
+            reinterpret_cast<uint4 *>(smem + C::OFF_ONES)[i] =
+                make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
     if (warp == 1) tmem_alloc(tmem_holder, C::TMEM_COLS);
     fence_proxy_async_smem();
     tc_fence_before();
@@ -291,7 +306,9 @@ k_mem_incr(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUte
             // ------------------------------------------------------------ MMA issuer
             constexpr uint32_t id = idesc_bf16(128, D, 1, 1);      // both operands MN-major
             constexpr uint32_t id16 = idesc_f16(128, D, 1, 1);
+            constexpr uint32_t idZ = idesc_bf16(128, 16, 1, 0);     // sigma(K)^T 1, ones K-major
             const uint32_t aRing = smem_u32(ring), aOps = smem_u32(ops);
+            const uint32_t aOnes = smem_u32(smem + C::OFF_ONES);
             int g = 0, j = 0;
             bool ok = true;
             for (int item = blockIdx.x; ok && item < a.items; item += gridDim.x, ++j) {
@@ -314,6 +331,12 @@ k_mem_incr(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUte
                         const uint32_t first = (c > 0 || kk > 0) ? 1u : 0u;
                         mma_ss(acc, ah, bv, id, first);
                         mma_ss(acc, al, bv, id, 1u);
+                        if constexpr (!DELTA) {      // every element of the tile is 1: any K offset
+                            const uint64_t b1 = sdesc_sw128(aOnes + kk * 32, 16, 1024);
+                            const uint32_t accz = T + C::T_Z + (j & 1) * C::ZC;
+                            mma_ss(accz, ah, b1, idZ, first);
+                            mma_ss(accz, al, b1, idZ, 1u);
+                        }
                         if constexpr (DELTA) {
                             const uint64_t a16 = sdesc_sw128(os + C::OFF_S16 + k2, C::BOX, 1024);
                             const uint64_t bw = sdesc_sw128(os + C::OFF_W16 + k2, C::BOX, 1024);
@@ -477,6 +500,12 @@ k_mem_incr(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUte
                             dl[e] = make_uint4(lo[4 * e], lo[4 * e + 1], lo[4 * e + 2], lo[4 * e + 3]);
                         }
                     }
+                }
+                if constexpr (!DELTA) {          // every column holds the same sum
+                    uint32_t r[16];
+                    tmem_ld16(lane_base + T + C::T_Z + (j & 1) * C::ZC, r);
+                    tmem_ld_wait();
+                    a.dz[(int64_t)item * D + i] = __uint_as_float(r[0]);
                 }
             }
             tc_fence_before();
