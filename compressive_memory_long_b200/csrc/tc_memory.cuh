@@ -145,8 +145,10 @@ struct IncrCfg {
     static constexpr int ZC = DELTA ? 0 : 32;         // additive rule: columns of sigma(K)^T 1
     static constexpr int T_Z = 2 * ACC;               // those of the two sets follow both B_s
     static constexpr uint32_t TMEM_COLS = 2 * (ACC + ZC) <= 256 ? 256 : 512;
-    static constexpr int THREADS = 512;
-    static constexpr int FPT = D / 4;                // features per worker thread
+    static constexpr int THREADS = 768;
+    static constexpr int WORKERS = 512;              // 16 warps: eight threads per token row
+    static constexpr int FPT = D / 8;                // features per worker thread: one 16-byte
+                                                     // chunk of each 64-feature box
     static_assert(SLOT % 1024 == 0 && OSET % 1024 == 0, "operand tiles must be 1024-aligned");
     static_assert(ALLOC <= 232448, "shared memory");
 };
@@ -179,6 +181,15 @@ __device__ __forceinline__ int incr_scale_exp(const float *z, int d)
     return e < -100 ? -100 : (e > 100 ? 100 : e);
 }
 
+// Two floats to f16x2 (lo in the lower half), values past f16's range clamped to its largest
+// finite value by the conversion itself
+__device__ __forceinline__ uint32_t pack_f16x2_sat(float lo, float hi)
+{
+    uint32_t r;
+    asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
 // 2^e as a float (|e| <= 100)
 __device__ __forceinline__ float pow2f(int e) { return __int_as_float((127 + e) << 23); }
 
@@ -203,17 +214,17 @@ __device__ __forceinline__ void incr_drain(uint64_t *bar, uint32_t parity)
 //   warp 1       MMA issuer: per chunk, B += sigma_hi^T V + sigma_lo^T V (bf16 operands) and,
 //                for the delta rule, A' += sigma_f16^T W' (f16 operands), into the item's
 //                accumulator set (two sets, alternating by item)
-//   warps 4-11   workers: four threads per token row turn K into sigma_hi (in place) and
+//   warps 4-19   workers: eight threads per token row turn K into sigma_hi (in place) and
 //                sigma_lo and, for the delta rule, sigma in f16, den = sigma . z_{s-1} and
 //                W' = 2^e sigma / den in f16 into the chunk's operand set (two sets,
 //                alternating by chunk)
-//   warps 12-15  epilogue: lane i of the item's accumulator is key feature i; row i of B_s
+//   warps 20-23  epilogue: lane i of the item's accumulator is key feature i; row i of B_s
 //                (fp32) and of A_s = 2^-e A' (bf16 hi, lo) to global memory, while the next
 //                item's MMAs fill the other accumulator set
 // Precision: B_s carries sigma to about 16 bits (hi + lo); A_s, which only scales the
 // correction A_s M_{s-1}, carries sigma and W' to f16's 11 bits.
 template <int D, bool DELTA>
-__global__ void __launch_bounds__(512, 1)
+__global__ void __launch_bounds__(768, 1)
 k_mem_incr(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
            const IncrArgs a)
 {
@@ -236,7 +247,7 @@ k_mem_incr(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUte
         for (int i = 0; i < RS; ++i) {
             mbar_init(full + i, 1);
             mbar_init(empty + i, 1);
-            mbar_init(aready + i, 256);
+            mbar_init(aready + i, C::WORKERS);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(ofree + i, 1);
@@ -351,13 +362,13 @@ k_mem_incr(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUte
             mma_commit(mma_done);
             incr_drain(mma_done, 0);
         }
-    } else if (warp >= 4 && warp < 12) {
+    } else if (warp >= 4 && warp < 20) {
         // ---------------------------------------------------------------- workers
-        const int w = threadIdx.x - 128;            // 0..255
-        const int t = w >> 2, q = w & 3;            // token row of the chunk, feature quarter
-        const int f0 = q * C::FPT;                  // first feature of this thread
-        const int box = f0 >> 6, cq = (f0 & 63) >> 3;
-        constexpr int CPT = C::FPT / 8;             // 16-byte chunks per thread
+        const int w = threadIdx.x - 128;            // 0..511
+        // token row of the chunk; the thread's 16-byte chunk q of every 64-feature box
+        // (features 64 i + 8 q + e), so the eight threads of a row cover its 128 bytes per box
+        const int t = w >> 3, q = w & 7;
+        constexpr int CPT = C::NB;                  // 16-byte chunks per thread
         const uint64_t one2 = f2_pack(1.f, 1.f);
         const uint64_t log2e2 = f2_pack(1.4426950408889634f, 1.4426950408889634f);
         int g = 0, j = 0;
@@ -371,10 +382,10 @@ k_mem_incr(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUte
             float wscale = 1.f;
             if constexpr (DELTA) {
                 wscale = pow2f(incr_scale_exp(a.snapZ + (int64_t)item * D, D));
-                const float4 *zp = reinterpret_cast<const float4 *>(a.snapZ + (int64_t)item * D + f0);
+                const float *zi = a.snapZ + (int64_t)item * D + 8 * q;
 #pragma unroll
                 for (int e = 0; e < C::FPT / 4; ++e) {
-                    const float4 x = __ldg(zp + e);
+                    const float4 x = __ldg(reinterpret_cast<const float4 *>(zi + (e >> 1) * 64) + (e & 1));
                     zr[4 * e] = x.x;
                     zr[4 * e + 1] = x.y;
                     zr[4 * e + 2] = x.z;
@@ -394,7 +405,7 @@ k_mem_incr(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUte
                 float sg[C::FPT];
 #pragma unroll
                 for (int i = 0; i < CPT; ++i) {
-                    const int off = box * C::BOX + t * 128 + (((cq + i) ^ (t & 7)) << 4);
+                    const int off = i * C::BOX + t * 128 + ((q ^ (t & 7)) << 4);
                     uint4 *ph = reinterpret_cast<uint4 *>(slot + C::OFF_SH + off);
                     const uint4 v = *ph;
                     const uint32_t in[4] = {v.x, v.y, v.z, v.w};
@@ -438,17 +449,18 @@ k_mem_incr(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUte
                     float den = (d0 + d1) + (d2 + d3);
                     den += __shfl_xor_sync(0xffffffffu, den, 1);
                     den += __shfl_xor_sync(0xffffffffu, den, 2);
+                    den += __shfl_xor_sync(0xffffffffu, den, 4);
                     const float inv = den == 0.f ? 0.f : wscale / den;
                     const uint64_t inv2 = f2_pack(inv, inv);
 #pragma unroll
                     for (int i = 0; i < CPT; ++i) {
-                        const int off = box * C::BOX + t * 128 + (((cq + i) ^ (t & 7)) << 4);
+                        const int off = i * C::BOX + t * 128 + ((q ^ (t & 7)) << 4);
                         uint32_t w16[4];
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {   // W' >= 0; clamped to f16's largest finite value
                             float w0, w1;
                             f2_unpack(f2_mul(f2_pack(sg[i * 8 + 2 * e], sg[i * 8 + 2 * e + 1]), inv2), w0, w1);
-                            w16[e] = pack_f16x2(fminf(w0, 65504.f), fminf(w1, 65504.f));
+                            w16[e] = pack_f16x2_sat(w0, w1);
                         }
                         *reinterpret_cast<uint4 *>(os + C::OFF_W16 + off) = make_uint4(w16[0], w16[1], w16[2], w16[3]);
                     }
@@ -457,7 +469,7 @@ k_mem_incr(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUte
                 mbar_arrive(aready + st);
             }
         }
-    } else if (warp >= 12) {
+    } else if (warp >= 20) {
         // ---------------------------------------------------------------- epilogue
         const int i = (warp & 3) * 32 + lane;
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
