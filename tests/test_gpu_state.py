@@ -79,3 +79,34 @@ def test_two_chunk_split_through_the_library(N, cut):
     errs = (rel_err(got, ro), rel_err(M_final.cpu(), rM),
             rel_err(z_final.cpu()[:, :, None], rz[:, :, None]))
     assert max(errs) <= TOL["bf16"], errs
+
+
+@pytest.mark.parametrize("rule", ["linear", "delta"])
+def test_memory_path_kernels_and_z_precision(rule):
+    """The tensor-core memory path launches what its rule needs: the delta rule's increments
+    need z_{s-1}, so the separate sigma(K) sum and the z scan run before them; the additive
+    rule's increments kernel forms the segment sums itself (sigma(K)^T 1 from sigma's two bf16
+    parts into an fp32 accumulator) and only the scan follows.  Either way z keeps about 16
+    bits of sigma: its error is held to 5e-5, far inside the bf16 bound."""
+    from compressive_memory_long_b200 import binding
+    w = make(f"zpath_{rule}", B=2, H=4, Hkv=2, d=128, N=256, S=3, tail=90, rule=rule,
+             state=True, seed=68)
+    t = {k: (None if x is None else x.cuda()) for k, x in wl.torch_inputs(w).items()}
+    binding.infini_attn_trace_enable(True)
+    out, M, z = binding.forward(t["q"], t["k"], t["v"], t["beta"], t["M0"], t["z0"], N=w.N,
+                                rule=w.rule)
+    torch.cuda.synchronize()
+    binding.infini_attn_trace_enable(False)
+    names = set(binding.infini_attn_trace_report())
+    want = ({"z_sum", "z_scan", "mem_increments", "mem_chain"} if rule == "delta"
+            else {"mem_increments", "z_scan", "mem_prefix"})
+    assert want <= names, names
+    assert ("z_sum" in names) == (rule == "delta"), names
+    q, k, v, beta, M0, z0 = wl.host_inputs(w)
+    ro, rM, rz = oracle.infini_attn_fwd(q, k, v, beta, M0, z0, N=w.N, rule=w.rule)
+    ez = rel_err(z.cpu()[:, :, None], rz[:, :, None])
+    errs = (rel_err(out.float().cpu(), ro), rel_err(M.cpu(), rM), ez)
+    print(f"PARITY {w.name}: out {errs[0]:.2e} M {errs[1]:.2e} z {ez:.2e}")
+    assert max(errs) <= TOL["bf16"], f"{w.name}: out/M/z rel err {errs}"
+    assert ez <= 5e-5, f"{w.name}: z rel err {ez}"
+    assert binding.infini_attn_device_status() == 0
