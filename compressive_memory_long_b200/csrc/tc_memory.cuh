@@ -56,22 +56,28 @@ k_zsum(const __nv_bfloat16 *__restrict__ k, float *__restrict__ dz, int64_t L, i
     const int64_t row0 = (int64_t)s * N;
     const int rows = (int)(L - row0 < N ? L - row0 : N);
     const uint4 *src = reinterpret_cast<const uint4 *>(k + (chain * L + row0) * D) + ch;
-    float acc[8];
+    // sigma = max(x + 1, e^min(x, 0)) (as elu1) with the multiply, the add and the sums on
+    // packed fp32 pairs: the pass is bound by its instruction issue, not by HBM
+    const uint64_t one2 = f2_pack(1.f, 1.f);
+    const uint64_t log2e2 = f2_pack(1.4426950408889634f, 1.4426950408889634f);
+    uint64_t acc[4];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+    for (int e = 0; e < 4; ++e) acc[e] = f2_pack(0.f, 0.f);
 #pragma unroll 4
     for (int r = rl; r < rows; r += RL) {
         const uint4 v = __ldg(src + (int64_t)r * CHK);
         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            const __nv_bfloat162 t = *reinterpret_cast<const __nv_bfloat162 *>(&w[e]);
-            acc[2 * e] += elu1(__low2float(t));
-            acc[2 * e + 1] += elu1(__high2float(t));
+            const float x0 = __uint_as_float(w[e] << 16), x1 = __uint_as_float(w[e] & 0xffff0000u);
+            float a0, a1, p0, p1;
+            f2_unpack(f2_mul(f2_pack(fminf(x0, 0.f), fminf(x1, 0.f)), log2e2), a0, a1);
+            f2_unpack(f2_add(f2_pack(x0, x1), one2), p0, p1);
+            acc[e] = f2_add(acc[e], f2_pack(fmaxf(p0, ex2(a0)), fmaxf(p1, ex2(a1))));
         }
     }
 #pragma unroll
-    for (int e = 0; e < 8; ++e) part[rl][ch * 8 + e] = acc[e];
+    for (int e = 0; e < 4; ++e) f2_unpack(acc[e], part[rl][ch * 8 + 2 * e], part[rl][ch * 8 + 2 * e + 1]);
     __syncthreads();
     for (int f = threadIdx.x; f < D; f += 256) {
         float t = 0.f;
