@@ -608,11 +608,14 @@ struct MChainCfg {
     static constexpr int ABOX = 128 * 128;          // 128 rows x 64 bf16
     static constexpr int ATILE = NK * ABOX;         // A_hi (or A_lo) of one segment
     static constexpr int ST = 3;                    // A_s loads run this many segments ahead
-    static constexpr int BBOX = CB * 128;           // CB rows x 64 bf16 (K-major M^T)
+    // per 64-wide box along the contraction, K-major: rows 0..CB-1 M^T hi, rows CB..2CB-1
+    // M^T lo, so one N = 2 CB product takes A_hi against both parts
+    static constexpr int BBOX = 2 * CB * 128;
     static constexpr int BTILE = NK * BBOX;
+    static_assert(CB % 8 == 0, "the lo rows keep the hi rows' swizzle phase");
     static constexpr int OFF_A = 0;                 // per stage: A_hi | A_lo
-    static constexpr int OFF_B = ST * 2 * ATILE;    // M^T hi | M^T lo
-    static constexpr int OFF_BAR = OFF_B + 2 * BTILE;
+    static constexpr int OFF_B = ST * 2 * ATILE;    // [M^T hi ; M^T lo] per box
+    static constexpr int OFF_BAR = OFF_B + BTILE;
     static constexpr int NBAR = 2 * ST + 3;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int BYTES = OFF_MISC + 16;
@@ -648,8 +651,9 @@ __device__ __forceinline__ void mchain_drain(uint64_t *bar, uint32_t parity)
 // last segment to the first: the backward's dM_{s-1} = dM_s + G_s - A_s dM_s, A_s being
 // symmetric; the snapshot of each step is then the gradient after the segment).  One CTA per (chain, 16
 // value columns); column block j of M_s needs only column block j of M_{s-1}.  Warp 0: TMA
-// of A_s (hi and lo parts, K-major, two stages ahead).  Warp 1: MMA issuer, D = A_hi M_hi +
-// A_hi M_lo + A_lo M_hi into 32 TMEM columns.  Warps 4-7: thread i holds row i of the block
+// of A_s (hi and lo parts, K-major, two stages ahead).  Warp 1: MMA issuer, per 16-wide step
+// of the contraction A_hi [M_hi | M_lo] (one N = 32 product into 32 TMEM columns) and A_lo M_hi
+// into the first 16; the threads add the two halves: D = A_hi M_hi + A_lo M_hi + A_hi M_lo.  Warps 4-7: thread i holds row i of the block
 // in fp32 registers, writes the snapshot and the M^T hi / lo operand, then applies
 // M += B_s - D.  d = 64 runs as 128 rows with zero rows 64..127 of A.
 template <int D>
@@ -721,23 +725,25 @@ k_mem_chain(const __grid_constant__ CUtensorMap tmAh, const __grid_constant__ CU
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            constexpr uint32_t id = idesc_bf16(128, CB, 0, 0);
-            const uint32_t aA = smem_u32(smem + C::OFF_A), aB = smem_u32(smem + C::OFF_B);
+            // columns 0..CB-1: A_hi M_hi + A_lo M_hi; columns CB..2CB-1: A_hi M_lo
+            constexpr uint32_t id2 = idesc_bf16(128, 2 * CB, 0, 0);
+            constexpr uint32_t id1 = idesc_bf16(128, CB, 0, 0);
+            // descriptors of the tiles' bases; an offset (a multiple of 16 bytes inside shared
+            // memory) adds to the address field without carrying out of it
+            const uint64_t dA = sdesc_sw128(smem_u32(smem + C::OFF_A), 16, 1024);
+            const uint64_t dB = sdesc_sw128(smem_u32(smem + C::OFF_B), 16, 1024);
             for (int s = 0; s < a.S; ++s) {
                 const int st = s % ST;
                 if (!mbar_wait_short(b_ready, s & 1, abort, WM_B)) break;
                 if (!mbar_wait_short(a_full + st, (s / ST) & 1, abort, WM_A_FULL)) break;
                 tc_fence_after();
-                const uint32_t ah = aA + st * 2 * C::ATILE, al = ah + C::ATILE;
+                const uint32_t ah = st * 2 * C::ATILE, al = ah + C::ATILE;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t ao = (kk >> 2) * C::ABOX + (kk & 3) * 32;
-                    const uint32_t bo = (kk >> 2) * C::BBOX + (kk & 3) * 32;
-                    const uint64_t dah = sdesc_sw128(ah + ao, 16, 1024);
-                    const uint64_t dbh = sdesc_sw128(aB + bo, 16, 1024);
-                    mma_ss(T, dah, dbh, id, kk > 0 ? 1u : 0u);
-                    mma_ss(T, dah, sdesc_sw128(aB + C::BTILE + bo, 16, 1024), id, 1u);
-                    mma_ss(T, sdesc_sw128(al + ao, 16, 1024), dbh, id, 1u);
+                    const uint64_t db = dB + (((kk >> 2) * C::BBOX + (kk & 3) * 32) >> 4);
+                    mma_ss(T, dA + ((ah + ao) >> 4), db, id2, kk > 0 ? 1u : 0u);
+                    mma_ss(T, dA + ((al + ao) >> 4), db, id1, 1u);
                 }
                 mma_commit(a_empty + st);
                 mma_commit(d_full);
@@ -791,7 +797,7 @@ k_mem_chain(const __grid_constant__ CUtensorMap tmAh, const __grid_constant__ CU
                     const __nv_bfloat16 lo = __float2bfloat16_rn(m[j] - __bfloat162float(hi));
                     const int o = kb * C::BBOX + j * 128 + ((((kc >> 3) ^ (j & 7))) << 4) + (kc & 7) * 2;
                     *reinterpret_cast<__nv_bfloat16 *>(sB + o) = hi;
-                    *reinterpret_cast<__nv_bfloat16 *>(sB + C::BTILE + o) = lo;
+                    *reinterpret_cast<__nv_bfloat16 *>(sB + CB * 128 + o) = lo;
                 }
             }
             fence_proxy_async_smem();
@@ -812,10 +818,11 @@ k_mem_chain(const __grid_constant__ CUtensorMap tmAh, const __grid_constant__ CU
             if (live) {
 #pragma unroll
                 for (int e = 0; e < CB / 4; ++e) {
-                    m[4 * e] += bs[e].x - __uint_as_float(r[4 * e]);
-                    m[4 * e + 1] += bs[e].y - __uint_as_float(r[4 * e + 1]);
-                    m[4 * e + 2] += bs[e].z - __uint_as_float(r[4 * e + 2]);
-                    m[4 * e + 3] += bs[e].w - __uint_as_float(r[4 * e + 3]);
+                    const uint32_t *d0 = r + 4 * e, *d1 = r + CB + 4 * e;
+                    m[4 * e] += bs[e].x - (__uint_as_float(d0[0]) + __uint_as_float(d1[0]));
+                    m[4 * e + 1] += bs[e].y - (__uint_as_float(d0[1]) + __uint_as_float(d1[1]));
+                    m[4 * e + 2] += bs[e].z - (__uint_as_float(d0[2]) + __uint_as_float(d1[2]));
+                    m[4 * e + 3] += bs[e].w - (__uint_as_float(d0[3]) + __uint_as_float(d1[3]));
                 }
             }
             tc_fence_before();
