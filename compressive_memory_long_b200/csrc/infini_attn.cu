@@ -360,7 +360,7 @@ int launch_memory_tc(const Problem &p, const __nv_bfloat16 *k, const __nv_bfloat
     if (!opt_in_smem<tc::k_mem_chain<D>>(MC::ALLOC)) return INFINI_ERR_CUDA;
     tc::MChainArgs ca{M0, ws.Bs, ws.snapMb, snapMf, M_out, S, 0};
     TRACED("mem_chain", st);
-    tc::k_mem_chain<D><<<(unsigned)(chains * (D / MC::CB)), 256, MC::ALLOC, st>>>(mah, mal, ca);
+    tc::k_mem_chain<D><<<(unsigned)(chains * (D / MC::CB)), MC::THREADS, MC::ALLOC, st>>>(mah, mal, ca);
     return INFINI_OK;
 }
 
@@ -1241,7 +1241,7 @@ int launch_backward(const BwdPlan &p, const T *q, const T *k, const T *v, const 
             if (!opt_in_smem<tc::k_mem_chain<D>>(MC::ALLOC)) return INFINI_ERR_CUDA;
             tc::MChainArgs ca{dM, w.GM, nullptr, w.dMs, dM0 ? dM0 : tw.Bs, S, 1};
             TRACED("bwd_mem_rev", st);
-            tc::k_mem_chain<D><<<(unsigned)(chains * (D / MC::CB)), 256, MC::ALLOC, st>>>(mah, mal, ca);
+            tc::k_mem_chain<D><<<(unsigned)(chains * (D / MC::CB)), MC::THREADS, MC::ALLOC, st>>>(mah, mal, ca);
         }
     } else {
         TRACED("bwd_mem_rev", st);

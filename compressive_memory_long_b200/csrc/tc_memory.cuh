@@ -604,6 +604,7 @@ template <int D>
 struct MChainCfg {
     static_assert(D == 64 || D == 128, "tensor-core delta recurrence: d = 64 or 128");
     static constexpr int CB = 16;                   // value columns per CTA
+    static constexpr int THREADS = 384;             // TMA, MMA, 2 idle, 8 update warps
     static constexpr int NK = D / 64;               // 64-wide boxes along the contraction
     static constexpr int ABOX = 128 * 128;          // 128 rows x 64 bf16
     static constexpr int ATILE = NK * ABOX;         // A_hi (or A_lo) of one segment
@@ -634,6 +635,15 @@ struct MChainArgs {
     int reverse;               // walk the segments from the last to the first
 };
 
+// 32 lanes x 8 consecutive 32-bit columns (warp-uniform address): thread t gets lane base + t
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8])
+{
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                   "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr));
+}
+
 enum : int { WM_A_EMPTY = 801, WM_B = 802, WM_A_FULL = 803, WM_D = 804, WM_DRAIN = 805 };
 
 __device__ __forceinline__ void mchain_drain(uint64_t *bar, uint32_t parity)
@@ -653,11 +663,13 @@ __device__ __forceinline__ void mchain_drain(uint64_t *bar, uint32_t parity)
 // value columns); column block j of M_s needs only column block j of M_{s-1}.  Warp 0: TMA
 // of A_s (hi and lo parts, K-major, two stages ahead).  Warp 1: MMA issuer, per 16-wide step
 // of the contraction A_hi [M_hi | M_lo] (one N = 32 product into 32 TMEM columns) and A_lo M_hi
-// into the first 16; the threads add the two halves: D = A_hi M_hi + A_lo M_hi + A_hi M_lo.  Warps 4-7: thread i holds row i of the block
-// in fp32 registers, writes the snapshot and the M^T hi / lo operand, then applies
-// M += B_s - D.  d = 64 runs as 128 rows with zero rows 64..127 of A.
+// into the first 16; the threads add the two halves: D = A_hi M_hi + A_lo M_hi + A_hi M_lo.
+// Warps 4-11: two threads per row i of the block, eight columns each, in fp32 registers;
+// each writes its part of the M^T hi / lo operand, signals the issuer, then (while the
+// products run) stores the snapshot and loads B_s, and applies M += B_s - D.  d = 64 runs
+// as 128 rows with zero rows 64..127 of A.
 template <int D>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(384, 1)
 k_mem_chain(const __grid_constant__ CUtensorMap tmAh, const __grid_constant__ CUtensorMap tmAl,
             const MChainArgs a)
 {
@@ -682,14 +694,14 @@ k_mem_chain(const __grid_constant__ CUtensorMap tmAh, const __grid_constant__ CU
             mbar_init(a_full + i, 1);
             mbar_init(a_empty + i, 1);
         }
-        mbar_init(b_ready, 128);
+        mbar_init(b_ready, 256);
         mbar_init(d_full, 1);
         mbar_init(mma_done, 1);
         *abort = 0;
         fence_barrier_init();
     }
     if (D == 64)   // rows 64..127 of every A tile stay zero (the loads fill rows 0..63)
-        for (int i = threadIdx.x; i < ST * 2 * (C::ABOX / 32); i += 256) {
+        for (int i = threadIdx.x; i < ST * 2 * (C::ABOX / 32); i += blockDim.x) {
             const int t = i / (C::ABOX / 32), o = i % (C::ABOX / 32);
             reinterpret_cast<uint4 *>(smem + C::OFF_A + t * C::ATILE + C::ABOX / 2)[o] =
                 make_uint4(0, 0, 0, 0);
@@ -752,17 +764,19 @@ k_mem_chain(const __grid_constant__ CUtensorMap tmAh, const __grid_constant__ CU
             mchain_drain(mma_done, 0);
         }
     } else if (warp >= 4) {
-        const int i = threadIdx.x - 128;            // row of M (key feature), TMEM lane
+        const int i = (threadIdx.x - 128) & 127;    // row of M (key feature), TMEM lane
+        constexpr int CH = CB / 2;                  // two threads per row, CH columns each
+        const int c0 = ((threadIdx.x - 128) >> 7) * CH;
         const bool live = i < D;
-        const uint32_t lane_base = (uint32_t)((warp - 4) * 32) << 16;
+        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
         uint8_t *sB = smem + C::OFF_B;
-        float m[CB];
+        float m[CH];
 #pragma unroll
-        for (int j = 0; j < CB; ++j) m[j] = 0.f;
+        for (int j = 0; j < CH; ++j) m[j] = 0.f;
         if (live && a.M0) {
-            const float4 *src = reinterpret_cast<const float4 *>(a.M0 + (chain * D + i) * D + cb);
+            const float4 *src = reinterpret_cast<const float4 *>(a.M0 + (chain * D + i) * D + cb + c0);
 #pragma unroll
-            for (int e = 0; e < CB / 4; ++e) {
+            for (int e = 0; e < CH / 4; ++e) {
                 const float4 x = src[e];
                 m[4 * e] = x.x;
                 m[4 * e + 1] = x.y;
@@ -776,25 +790,11 @@ k_mem_chain(const __grid_constant__ CUtensorMap tmAh, const __grid_constant__ CU
         for (int s = 0; s < a.S; ++s) {
             const int64_t slot = chain * a.S + (a.reverse ? a.S - 1 - s : s);
             if (live) {
-                if (a.snapMb) {
-                    uint32_t pk[CB / 2];
 #pragma unroll
-                    for (int e = 0; e < CB / 2; ++e) pk[e] = pack_bf16x2(m[2 * e], m[2 * e + 1]);
-                    uint4 *dst = reinterpret_cast<uint4 *>(a.snapMb + (slot * D + i) * D + cb);
-#pragma unroll
-                    for (int e = 0; e < CB / 8; ++e)
-                        dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
-                }
-                if (a.snapMf) {
-                    float4 *dst = reinterpret_cast<float4 *>(a.snapMf + (slot * D + i) * D + cb);
-#pragma unroll
-                    for (int e = 0; e < CB / 4; ++e)
-                        dst[e] = make_float4(m[4 * e], m[4 * e + 1], m[4 * e + 2], m[4 * e + 3]);
-                }
-#pragma unroll
-                for (int j = 0; j < CB; ++j) {
-                    const __nv_bfloat16 hi = __float2bfloat16_rn(m[j]);
-                    const __nv_bfloat16 lo = __float2bfloat16_rn(m[j] - __bfloat162float(hi));
+                for (int jj = 0; jj < CH; ++jj) {
+                    const int j = c0 + jj;
+                    const __nv_bfloat16 hi = __float2bfloat16_rn(m[jj]);
+                    const __nv_bfloat16 lo = __float2bfloat16_rn(m[jj] - __bfloat162float(hi));
                     const int o = kb * C::BBOX + j * 128 + ((((kc >> 3) ^ (j & 7))) << 4) + (kc & 7) * 2;
                     *reinterpret_cast<__nv_bfloat16 *>(sB + o) = hi;
                     *reinterpret_cast<__nv_bfloat16 *>(sB + CB * 128 + o) = lo;
@@ -803,22 +803,41 @@ k_mem_chain(const __grid_constant__ CUtensorMap tmAh, const __grid_constant__ CU
             fence_proxy_async_smem();
             tc_fence_before();
             mbar_arrive(b_ready);
-            float4 bs[CB / 4];
+            // off the serial path, while the products run: the snapshot M_{s-1} and B_s
+            float4 bs[CH / 4];
             if (live) {
-                const float4 *src = reinterpret_cast<const float4 *>(a.Bs + (slot * D + i) * D + cb);
+                if (a.snapMb) {
+                    uint32_t pk[CH / 2];
 #pragma unroll
-                for (int e = 0; e < CB / 4; ++e) bs[e] = src[e];
+                    for (int e = 0; e < CH / 2; ++e) pk[e] = pack_bf16x2(m[2 * e], m[2 * e + 1]);
+                    uint4 *dst = reinterpret_cast<uint4 *>(a.snapMb + (slot * D + i) * D + cb + c0);
+#pragma unroll
+                    for (int e = 0; e < CH / 8; ++e)
+                        dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+                }
+                if (a.snapMf) {
+                    float4 *dst = reinterpret_cast<float4 *>(a.snapMf + (slot * D + i) * D + cb + c0);
+#pragma unroll
+                    for (int e = 0; e < CH / 4; ++e)
+                        dst[e] = make_float4(m[4 * e], m[4 * e + 1], m[4 * e + 2], m[4 * e + 3]);
+                }
+                const float4 *src = reinterpret_cast<const float4 *>(a.Bs + (slot * D + i) * D + cb + c0);
+#pragma unroll
+                for (int e = 0; e < CH / 4; ++e) bs[e] = src[e];
             }
             // on the serial path: probe without the suspend hint
             if (!(ok = mbar_wait_short(d_full, s & 1, abort, WM_D))) break;
             tc_fence_after();
-            uint32_t r[32];
-            tmem_ld32(lane_base + T, r);
+            // this thread's columns of both halves (c0 is uniform across the warp)
+            uint32_t r0[CH], r1[CH];
+            static_assert(CH == 8, "one tmem_ld8 per half");
+            tmem_ld8(lane_base + T + c0, r0);
+            tmem_ld8(lane_base + T + CB + c0, r1);
             tmem_ld_wait();
             if (live) {
 #pragma unroll
-                for (int e = 0; e < CB / 4; ++e) {
-                    const uint32_t *d0 = r + 4 * e, *d1 = r + CB + 4 * e;
+                for (int e = 0; e < CH / 4; ++e) {
+                    const uint32_t *d0 = r0 + 4 * e, *d1 = r1 + 4 * e;
                     m[4 * e] += bs[e].x - (__uint_as_float(d0[0]) + __uint_as_float(d1[0]));
                     m[4 * e + 1] += bs[e].y - (__uint_as_float(d0[1]) + __uint_as_float(d1[1]));
                     m[4 * e + 2] += bs[e].z - (__uint_as_float(d0[2]) + __uint_as_float(d1[2]));
@@ -828,9 +847,9 @@ k_mem_chain(const __grid_constant__ CUtensorMap tmAh, const __grid_constant__ CU
             tc_fence_before();
         }
         if (ok && live) {
-            float4 *dst = reinterpret_cast<float4 *>(a.M_out + (chain * D + i) * D + cb);
+            float4 *dst = reinterpret_cast<float4 *>(a.M_out + (chain * D + i) * D + cb + c0);
 #pragma unroll
-            for (int e = 0; e < CB / 4; ++e)
+            for (int e = 0; e < CH / 4; ++e)
                 dst[e] = make_float4(m[4 * e], m[4 * e + 1], m[4 * e + 2], m[4 * e + 3]);
         }
     }
