@@ -63,17 +63,26 @@ k_zsum(const __nv_bfloat16 *__restrict__ k, float *__restrict__ dz, int64_t L, i
     uint64_t acc[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) acc[e] = f2_pack(0.f, 0.f);
-#pragma unroll 4
-    for (int r = rl; r < rows; r += RL) {
-        const uint4 v = __ldg(src + (int64_t)r * CHK);
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    // U rows per thread in flight: with few segments (one CTA each) the grid is small and
+    // the loads in flight per thread set the bandwidth
+    constexpr int U = 8;
+    for (int r0 = rl; r0 < rows; r0 += U * RL) {
+        uint4 v[U];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const float x0 = __uint_as_float(w[e] << 16), x1 = __uint_as_float(w[e] & 0xffff0000u);
-            float a0, a1, p0, p1;
-            f2_unpack(f2_mul(f2_pack(fminf(x0, 0.f), fminf(x1, 0.f)), log2e2), a0, a1);
-            f2_unpack(f2_add(f2_pack(x0, x1), one2), p0, p1);
-            acc[e] = f2_add(acc[e], f2_pack(fmaxf(p0, ex2(a0)), fmaxf(p1, ex2(a1))));
+        for (int u = 0; u < U; ++u)
+            if (r0 + u * RL < rows) v[u] = __ldg(src + (int64_t)(r0 + u * RL) * CHK);
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            if (r0 + u * RL >= rows) break;
+            const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float x0 = __uint_as_float(w[e] << 16), x1 = __uint_as_float(w[e] & 0xffff0000u);
+                float a0, a1, p0, p1;
+                f2_unpack(f2_mul(f2_pack(fminf(x0, 0.f), fminf(x1, 0.f)), log2e2), a0, a1);
+                f2_unpack(f2_add(f2_pack(x0, x1), one2), p0, p1);
+                acc[e] = f2_add(acc[e], f2_pack(fmaxf(p0, ex2(a0)), fmaxf(p1, ex2(a1))));
+            }
         }
     }
 #pragma unroll
